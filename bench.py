@@ -1,0 +1,440 @@
+"""Benchmark: paged decode attention KV-read GB/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ragged]
+                    [--impl ours|reference] [--partition -1] [--algo auto|simt|tensor]
+
+One step = one decode step of one attention layer over the whole batch: the
+append of the step's new tokens (pa_reshape_and_cache, plus copy-on-write
+copies where the workload has them) followed by pa_decode (split-K +
+log-sum-exp merge where partitions apply).  The default workload is the
+continuous-batching ragged trace: 7B-GQA heads (32 q / 8 KV, head_dim 128),
+fp16 KV, batch 64, lengths U[16, 4096] growing by one per step for 128 steps,
+sequences finishing with p = 0.02 and being replaced by new ones of
+U[16, 512] tokens.  Steps beyond 128 replay the trace from its start (same
+kernels, same byte counts).
+
+value = algorithmic KV-read bytes of the timed decode steps / device time of
+those steps (CUDA events around the whole step: append + decode + merge),
+inputs resident in HBM.  The KV pool (1.1 GB) and the bytes read per step
+(218-498 MB) are larger than the 126 MB L2, so no flush is needed between
+steps.  e2e = the same metric through the C ABI with the per-step inputs in
+pinned host memory copied in and the outputs copied out inside the timed
+region.  For N > 1 (torchrun) every rank runs an independent replica on its
+own GPU (the decode path has no exchange step); value = bytes of all ranks /
+max over ranks of the device time.
+
+--impl reference times the CPU oracle (the fp64 C reference of the same
+computation) on a bounded sample of the same workload, on rank 0 only.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); decode tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOADS = {
+    "ragged": "continuous-batching ragged decode: 7B-GQA 32 q / 8 KV heads, head_dim 128, fp16 KV, "
+              "batch 64, lengths U[16,4096], 128 steps of +1 token, finish p=0.02, "
+              "new sequences U[16,512]",
+    "gqa_b8": "7B-GQA decode: 32 q / 8 KV heads, head_dim 128, fp16, batch 8, all lengths 1024",
+    "long": "long context: 7B-GQA heads, fp16, batch 16, all lengths 8192, split-K 512",
+    "long_int8": "long context: 7B-GQA heads, int8 KV (per-(block, KV head) scales), fp16 q/out, "
+                 "batch 16, all lengths 8192, split-K 512",
+    "mha_prefix": "MHA 32/32 heads, head_dim 128, fp16, batch 16, shared 1000-token prefix with "
+                  "copy-on-write + private suffix U[64,1048]",
+}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=512)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ragged")
+    ap.add_argument("--partition", type=int, default=-1)
+    ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+def load_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def make_workload(name):
+    from paged_kv_cache_395_b200 import workloads as W
+    if name == "ragged":
+        return W.ragged(), False, 256
+    if name == "gqa_b8":
+        return W.gqa_b8(), False, 256
+    if name == "long":
+        return W.long(), False, 512
+    if name == "long_int8":
+        return W.long(), True, 512
+    if name == "mha_prefix":
+        return W.mha_prefix(), False, 256
+    raise ValueError(name)
+
+
+def step_bytes(w, int8):
+    from paged_kv_cache_395_b200 import workloads as W
+    out = []
+    for ops in w.steps:
+        dec = [o for o in ops if isinstance(o, W.Decode)][0]
+        out.append(W.decode_kv_bytes(dec, w, 1 if int8 else None))
+    return out
+
+
+def step_tokens(w):
+    from paged_kv_cache_395_b200 import workloads as W
+    return [int([o for o in ops if isinstance(o, W.Decode)][0].q.shape[0]) for ops in w.steps]
+
+
+class ClockSampler:
+    """Poll NVML (the data nvidia-smi prints) during the timed region."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index, period=0.002):
+        self.samples, self.reasons, self.max_mhz, self.ok = [], 0, None, False
+        self.period = period
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report it, do not guess
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        names = [n for n, b in self.REASONS.items() if self.reasons & b]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def cpu_baseline(w, int8, seconds, host_caches=None):
+    """The oracle as it stands, on this host's cores, over whole decode steps
+    of the workload replayed in order until ``seconds`` of work are done."""
+    import oracle
+    from paged_kv_cache_395_b200 import workloads as W
+    N, H, bs, d = w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim
+    kc = np.zeros((N, H, bs, d), dtype=w.storage_dtype())
+    vc = np.zeros_like(kc)
+    for op in w.setup:
+        oracle.reshape_and_cache(op.k, op.v, kc, vc, op.slot_mapping)
+    ks = vs = None
+    if int8:
+        kc, ks = oracle.quantize_int8(kc)
+        vc, vs = oracle.quantize_int8(vc)
+    threads = oracle.nthreads_default()
+    done_bytes, t_work, nsteps, ntok = 0, 0.0, 0, 0
+    for si, ops in enumerate(w.steps):
+        for op in ops:
+            if isinstance(op, W.Reshape) and not int8:
+                oracle.reshape_and_cache(op.k, op.v, kc, vc, op.slot_mapping)
+            elif isinstance(op, W.Copy) and op.pairs.size and not int8:
+                oracle.block_copy(kc, vc, op.pairs)
+            elif isinstance(op, W.Decode):
+                t0 = time.perf_counter()
+                oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs,
+                              nthreads=threads)
+                t_work += time.perf_counter() - t0
+                done_bytes += W.decode_kv_bytes(op, w, 1 if int8 else None)
+                ntok += op.q.shape[0]
+                nsteps += 1
+        if t_work >= seconds:
+            break
+    return {"value": done_bytes / t_work / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{nsteps} whole decode step(s) of the workload in trace order "
+                      f"({ntok} sequence decodes, all heads), fp64 C oracle, {t_work:.2f} s",
+            "tokens_per_s": ntok / t_work}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    from paged_kv_cache_395_b200 import workloads as W
+    w, int8, _ = make_workload(args.workload)
+    N, H, bs, d = w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim
+    kc = np.zeros((N, H, bs, d), dtype=w.storage_dtype())
+    vc = np.zeros_like(kc)
+    for op in w.setup:
+        oracle.reshape_and_cache(op.k, op.v, kc, vc, op.slot_mapping)
+    ks = vs = None
+    if int8:
+        kc, ks = oracle.quantize_int8(kc)
+        vc, vs = oracle.quantize_int8(vc)
+    threads = oracle.nthreads_default()
+    # each step: the trace's step i % T, a bounded sample of one sequence (all heads)
+    decs = [[o for o in ops if isinstance(o, W.Decode)][0] for ops in w.steps]
+    T = len(decs)
+
+    def one(i):
+        op = decs[i % T]
+        b = i % op.q.shape[0]
+        bh = np.array([[b, h] for h in range(w.num_q_heads)], dtype=np.int32)
+        oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs, bh=bh,
+                      nthreads=threads)
+        L = int(max(op.seq_lens[b], 0))
+        E = 1 if int8 else w.elem_size
+        return L * w.num_kv_heads * w.head_dim * 2 * E
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    nbytes = sum(one(args.warmup + i) for i in range(args.steps))
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOADS[args.workload], "name": args.workload},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": "per step: one sequence (all query heads) of trace step "
+                                   "i mod T, fp64 C oracle"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_setup(args)
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+
+    import torch
+    from paged_kv_cache_395_b200 import pa, runner
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    algo = {"auto": pa.PA_ALGO_AUTO, "simt": pa.PA_ALGO_SIMT, "tensor": pa.PA_ALGO_TENSOR}[args.algo]
+    w, int8, default_part = make_workload(args.workload)
+    part = args.partition if args.partition != -1 else -1
+    dw = runner.DeviceWorkload(w, fill_nan=False)
+    dw.run_setup()
+    if int8:
+        dw.quantize_int8()
+    stream = torch.cuda.current_stream()
+    calls = runner.StepCalls(dw, part, int8, algo, stream)
+    T = len(w.steps)
+    sbytes = step_bytes(w, int8)
+    stoks = step_tokens(w)
+    torch.cuda.synchronize()
+
+    # ---- device-resident timing --------------------------------------------------------
+    for i in range(args.warmup):
+        calls.run(i % T)
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    cur = [0]
+
+    def mark(before):
+        ev[cur[0]][0 if before else 1].record(stream)
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for j in range(K):
+            cur[0] = j
+            calls.run((args.warmup + j) % T, mark)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    dec_ms = sum(a.elapsed_time(b) for a, b in ev)
+    idx = [(args.warmup + j) % T for j in range(K)]
+    bytes_rank = sum(sbytes[i] for i in idx)
+    toks_rank = sum(stoks[i] for i in idx)
+    launches = sum(calls.launches[i] for i in idx)
+    ms_max = ms
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    total_bytes = bytes_rank * world
+    value = total_bytes / (ms_max * 1e-3) / 1e9
+    peak, peak_kind = load_peak()
+    achieved = bytes_rank / (dec_ms * 1e-3) / 1e9
+
+    # ---- end to end through the C ABI with host buffers ------------------------------------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = time_e2e(dw, w, int8, part, algo, args, T, sbytes, stream, dist)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8" if int8 else "f16", "data": "synthetic",
+        "config": {"workload": WORKLOADS[args.workload], "name": args.workload,
+                   "partition_size": 256 if part == -1 else part, "algo": args.algo,
+                   "l2": "inputs larger than L2: KV pool and per-step reads exceed 126 MB, no flush",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "decode_tokens_per_s": toks_rank * world / (ms_max * 1e-3),
+        "hbm_frac_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
+        "hbm_frac_of_" + peak_kind: value / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "pa_decode (decode kernel + merge kernel when split)",
+                     "peak_kind": peak_kind},
+        "gpu_launches": launches,
+        "clocks": clk.report(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, int8, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def time_e2e(dw, w, int8, part, algo, args, T, sbytes, stream, dist):
+    """Per step: one pinned host -> device copy of the step's inputs (new k/v,
+    slots, copy pairs, q, block tables, seq_lens, packed in one buffer), the
+    library calls, and one device -> host copy of the decode output."""
+    import torch
+    from paged_kv_cache_395_b200 import runner
+
+    packs, h2d, d2h = [], [], []
+    for i in range(T):
+        tensors = [t for op in dw.steps[i] for t in op[1:] if isinstance(t, torch.Tensor)]
+        outs = [op[-1] for op in dw.steps[i] if op[0] == "decode"]
+        ins = [t for t in tensors if not any(t is o for o in outs)]
+        offs, n = [], 0
+        for t in ins:
+            offs.append(n)
+            n += (t.numel() * t.element_size() + 255) // 256 * 256
+        host = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+        for t, o in zip(ins, offs):
+            nb = t.numel() * t.element_size()
+            host[o:o + nb].copy_(t.contiguous().view(torch.uint8).view(-1).cpu())
+        dev = torch.empty(n, dtype=torch.uint8, device="cuda")
+        views = {}
+        for t, o in zip(ins, offs):
+            nb = t.numel() * t.element_size()
+            views[id(t)] = dev[o:o + nb].view(t.dtype).view(t.shape)
+        out = outs[0]
+        host_out = torch.empty(out.numel() * out.element_size(), dtype=torch.uint8, pin_memory=True)
+        packs.append((host, dev, views, out, host_out))
+        h2d.append(n)
+        d2h.append(host_out.numel())
+    # library calls that read the staging buffers
+    staged = runner.DeviceWorkload.__new__(runner.DeviceWorkload)
+    staged.__dict__.update(dw.__dict__)
+    staged.steps = {}
+    for i in range(T):
+        views = packs[i][2]
+        staged.steps[i] = [tuple(views.get(id(x), x) if isinstance(x, torch.Tensor) else x
+                                 for x in op) for op in dw.steps[i]]
+    calls = runner.StepCalls(staged, part, int8, algo, stream)
+    K = args.steps
+    for i in range(args.warmup):
+        host, dev, _, out, host_out = packs[i % T]
+        dev.copy_(host, non_blocking=True)
+        calls.run(i % T)
+        host_out.copy_(out.view(torch.uint8).view(-1), non_blocking=True)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    nbytes, hb, db = 0, 0, 0
+    for j in range(K):
+        i = (args.warmup + j) % T
+        host, dev, _, out, host_out = packs[i]
+        dev.copy_(host, non_blocking=True)
+        calls.run(i)
+        host_out.copy_(out.view(torch.uint8).view(-1), non_blocking=True)
+        nbytes += sbytes[i]
+        hb += h2d[i]
+        db += d2h[i]
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    world = 1
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        world = dist.get_world_size()
+    return {"value": nbytes * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": hb // K, "d2h_bytes_per_step": db // K, "ms_per_step": ms / K}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

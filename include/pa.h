@@ -1,0 +1,191 @@
+/*
+ * pa.h -- paged single-token decode attention on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The KV cache of one attention layer lives in a pool of fixed-size physical
+ * blocks of PA_BLOCK_SIZE tokens.  Each sequence owns a block table that maps
+ * its logical block i to a physical block; blocks need not be contiguous and
+ * the kernels walk the table in order without gathering the blocks
+ * (lqnn.cn/news/235768 section 3.2; chanyi.net.cn/article/49 section 三).
+ * Query heads share KV heads under GQA/MQA: query head h reads KV head
+ * h / (num_q_heads / num_kv_heads) (lqnn.cn/news/235768 section 4.2).
+ *
+ * Memory layouts (row-major, innermost last):
+ *   key_cache, value_cache  [num_blocks][num_kv_heads][PA_BLOCK_SIZE][head_dim]
+ *   k_scales, v_scales      [num_blocks][num_kv_heads]  fp32 (int8 caches only)
+ *   q, out                  [num_seqs][num_q_heads][head_dim]
+ *   block_tables            [num_seqs][max_blocks_per_seq]  int32
+ *   seq_lens                [num_seqs]  int32
+ *   slot_mapping            [num_tokens]  int64, slot = block * PA_BLOCK_SIZE + offset
+ *
+ * Ownership: the caller allocates and owns every buffer, including the split-K
+ * workspace.  The library allocates no memory and keeps no per-call state.
+ * Every pointer argument is a DEVICE pointer except `p` (pa_decode_params) and
+ * the host-side out-parameters of pa_get_error_flags.  Every call is
+ * asynchronous on `stream` and never synchronises the host, except
+ * pa_get_error_flags.
+ *
+ * Errors: host-checkable problems are reported by the return value before any
+ * launch (nothing is launched then).  A failed launch returns PA_ERR_CUDA.
+ * Data errors found on the device (a block id outside [0, num_blocks) in a
+ * table entry that is read, a slot outside the pool, a copy pair outside the
+ * pool, a bounded wait that gave up) never trap: the offending item is
+ * skipped and a bit is set in a per-device error word, read with
+ * pa_get_error_flags.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *pa_stream_t;
+
+enum pa_status {
+    PA_OK = 0,
+    PA_ERR_NULL = -1,        /* a required pointer is NULL */
+    PA_ERR_SHAPE = -2,       /* a size is negative/zero where it must be positive, or inconsistent */
+    PA_ERR_DTYPE = -3,       /* unknown dtype or unsupported q/KV dtype pair */
+    PA_ERR_UNSUPPORTED = -4, /* valid but not built: block_size != 16, head_dim, group size */
+    PA_ERR_WORKSPACE = -5,   /* split-K workspace missing or smaller than pa_decode_workspace_size */
+    PA_ERR_CUDA = -6,        /* a CUDA launch or query failed */
+    PA_ERR_ALIGN = -7        /* a buffer is not aligned as documented */
+};
+
+enum pa_dtype { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_I8 = 3 };
+
+/* Kernel family for pa_decode.  AUTO picks the fastest built one. */
+enum pa_algo { PA_ALGO_AUTO = 0, PA_ALGO_SIMT = 1, PA_ALGO_TENSOR = 2 };
+
+/* Bits of the per-device error word (pa_get_error_flags). */
+enum pa_error_flag {
+    PA_EFLAG_BAD_BLOCK = 1,   /* a block table entry read by pa_decode was outside the pool */
+    PA_EFLAG_BAD_SLOT = 2,    /* a slot_mapping entry was >= num_blocks * PA_BLOCK_SIZE */
+    PA_EFLAG_BAD_PAIR = 4,    /* a pa_block_copy pair was outside the pool */
+    PA_EFLAG_WAIT_TIMEOUT = 8 /* a bounded wait on an asynchronous copy gave up */
+};
+
+#define PA_BLOCK_SIZE 16
+
+/*
+ * Append new tokens to the paged cache (lqnn.cn/news/235768 section 2.2:
+ * the new token's k, v are written at position cache_len before attention).
+ *
+ * For every token i with s = slot_mapping[i] >= 0, every KV head h:
+ *   key_cache  [s / 16][h][s % 16][:] = k[i * k_token_stride + h * head_dim + :]
+ *   value_cache[s / 16][h][s % 16][:] = v[i * v_token_stride + h * head_dim + :]
+ * A bit-exact copy.  s < 0 marks padding and is skipped; s >= num_blocks * 16
+ * sets PA_EFLAG_BAD_SLOT and is skipped.  Strides are in elements.  Slots
+ * must be distinct (two tokens writing one slot race).
+ * dtype: PA_F32, PA_F16 or PA_BF16 (PA_I8 caches are written by
+ * pa_quantize_int8, so PA_I8 returns PA_ERR_UNSUPPORTED).
+ * Any alignment works; 16-byte aligned rows are copied with 16-byte vectors.
+ */
+int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *value_cache,
+                         const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int64_t num_blocks, int dtype,
+                         int64_t k_token_stride, int64_t v_token_stride, pa_stream_t stream);
+
+typedef struct pa_decode_params {
+    int num_seqs;            /* B >= 0 */
+    int num_q_heads;         /* H_q, a multiple of num_kv_heads */
+    int num_kv_heads;        /* H_kv; group size G = H_q / H_kv must be 1, 2, 4 or 8 */
+    int head_dim;            /* 64 or 128 */
+    int block_size;          /* must be PA_BLOCK_SIZE */
+    int max_blocks_per_seq;  /* row stride of block_tables */
+    int64_t num_blocks;      /* physical blocks in the pool */
+    int max_seq_len;         /* >= every seq_lens[b]; sizes the split-K grid and workspace.
+                                Tokens beyond max_seq_len or max_blocks_per_seq * 16 are ignored. */
+    int q_dtype;             /* dtype of q and out: PA_F32, PA_F16 or PA_BF16 */
+    int kv_dtype;            /* PA_F32 (q PA_F32), PA_F16 (q PA_F16), PA_BF16 (q PA_BF16),
+                                or PA_I8 (q PA_F16 or PA_BF16) */
+    const float *k_scales;   /* PA_I8 only: [num_blocks][num_kv_heads], else NULL */
+    const float *v_scales;
+    int partition_size;      /* 0: one pass, one CTA per (sequence, KV head), no workspace.
+                                > 0: split-K, partitions of this many tokens (a multiple of
+                                16), then a log-sum-exp merge; needs the workspace.
+                                -1: the library picks (may use split-K; needs the workspace). */
+    int algo;                /* enum pa_algo */
+    void *workspace;         /* device scratch, >= pa_decode_workspace_size(p) bytes,
+                                16-byte aligned; NULL allowed when that size is 0 */
+    size_t workspace_bytes;
+} pa_decode_params;
+
+/*
+ * Bytes of device workspace pa_decode needs for these parameters (0 for
+ * partition_size == 0).  Depends only on num_seqs, num_q_heads, num_kv_heads,
+ * head_dim, max_seq_len and partition_size.  Returns 0 for invalid params.
+ */
+size_t pa_decode_workspace_size(const pa_decode_params *p);
+
+/*
+ * Single-token decode attention over the paged cache
+ * (lqnn.cn/news/235768 sections 1.2 and 2.2; chanyi.net.cn/article/49 section 四):
+ *
+ *   out[b][h][:] = sum_t softmax_t(scale * q[b][h] . K[b][t]) V[b][t]
+ *
+ * over the logical tokens t = 0 .. seq_lens[b]-1 of sequence b, where token t
+ * is slot t % 16 of physical block block_tables[b][t / 16], KV head
+ * h / (H_q / H_kv).  seq_lens include the token being decoded, which must
+ * already be in the cache.  int8 caches are dequantised as x = q8 * scale of
+ * its (block, KV head).  The softmax runs online in fp32 and K/V products
+ * accumulate in fp32; out is rounded once to q_dtype.  seq_lens[b] <= 0 gives
+ * a zero row.  Only the first ceil(seq_lens[b] / 16) entries of a table row
+ * are read.  With partition_size > 0 the sequence is cut into partitions whose
+ * normalised partial outputs and log-sum-exp go to the workspace and are
+ * merged: out = sum_p exp(lse_p - M) o_p / sum_p exp(lse_p - M).
+ * Result does not depend on where the physical blocks sit.
+ */
+int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *seq_lens, float scale,
+              const pa_decode_params *p, pa_stream_t stream);
+
+/*
+ * Copy-on-write block copy (chanyi.net.cn/article/49 section 三: shared prefix
+ * blocks are copied only when a sequence diverges).  For each pair
+ * (src = pairs[2i], dst = pairs[2i+1]) the whole physical block -- every KV
+ * head and all 16 slots -- of key_cache and of value_cache is copied byte for
+ * byte, and k_scales/v_scales[dst][:] = [src][:] when those are non-NULL.
+ * A dst must not appear twice or also as a src (the copies run in parallel).
+ * Pairs outside [0, num_blocks) set PA_EFLAG_BAD_PAIR and are skipped.
+ * dtype: any pa_dtype.
+ */
+int pa_block_copy(void *key_cache, void *value_cache, float *k_scales, float *v_scales,
+                  const int64_t *src_dst_pairs, int64_t num_pairs, int num_kv_heads,
+                  int head_dim, int block_size, int64_t num_blocks, int dtype,
+                  pa_stream_t stream);
+
+/*
+ * 8-bit KV with one scale per group (lqnn.cn/news/235768 section 4.1), the
+ * group being one (block, KV head) tile of 16 * head_dim values.  For each of
+ * the first num_blocks blocks and each KV head, in IEEE fp32:
+ *   a = max |x|,  s = a / 127,  q8 = clamp(round_half_even(x / s), -127, 127)
+ * a == 0 gives s = 0 and q8 = 0.  src_cache: [num_blocks][H_kv][16][head_dim]
+ * of src_dtype (PA_F32, PA_F16 or PA_BF16); dst_cache int8 of the same shape;
+ * scales [num_blocks][H_kv].  Call once for K and once for V.
+ */
+int pa_quantize_int8(const void *src_cache, int src_dtype, int8_t *dst_cache, float *scales,
+                     int64_t num_blocks, int num_kv_heads, int head_dim, int block_size,
+                     pa_stream_t stream);
+
+/*
+ * Read the calling thread's current device's error word into *flags
+ * (pa_error_flag bits); synchronises `stream` first.  reset != 0 clears it.
+ */
+int pa_get_error_flags(unsigned int *flags, int reset, pa_stream_t stream);
+
+/* Static description of a status code. */
+const char *pa_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

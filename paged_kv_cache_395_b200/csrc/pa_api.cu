@@ -1,0 +1,211 @@
+// C-ABI entry points: argument validation, then dispatch to the kernels.
+// Every check that can be made on the host is made here, before any launch.
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+bool set_smem_attr_once(const void *kernel, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<const void *, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kernel, dev})) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    done.insert({kernel, dev});
+    return true;
+}
+
+static int elem_size(int dt) {
+    switch (dt) {
+    case PA_F32: return 4;
+    case PA_F16: return 2;
+    case PA_BF16: return 2;
+    case PA_I8: return 1;
+    default: return 0;
+    }
+}
+
+// Checks shared by pa_decode and pa_decode_workspace_size.  Fills the partition
+// size actually used (auto resolved) and the partition count.
+static int check_decode_params(const pa_decode_params *p, int *part, int *max_parts) {
+    if (!p) return PA_ERR_NULL;
+    if (p->num_seqs < 0 || p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->head_dim <= 0 ||
+        p->max_blocks_per_seq <= 0 || p->num_blocks <= 0 || p->max_seq_len < 0)
+        return PA_ERR_SHAPE;
+    if (p->num_q_heads % p->num_kv_heads) return PA_ERR_SHAPE;
+    if (p->block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
+    if (!elem_size(p->q_dtype) || !elem_size(p->kv_dtype) || p->q_dtype == PA_I8) return PA_ERR_DTYPE;
+    const int G = p->num_q_heads / p->num_kv_heads;
+    if (!decode_simt_supported(p->q_dtype, p->kv_dtype, p->head_dim, G)) {
+        const bool pair_ok = (p->q_dtype == p->kv_dtype) || p->kv_dtype == PA_I8;
+        if (!pair_ok || (p->kv_dtype == PA_I8 && p->q_dtype == PA_F32)) return PA_ERR_DTYPE;
+        return PA_ERR_UNSUPPORTED;
+    }
+    if (p->num_seqs > 65535 || p->num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (p->algo < PA_ALGO_AUTO || p->algo > PA_ALGO_TENSOR) return PA_ERR_UNSUPPORTED;
+    int ps = p->partition_size;
+    if (ps < -1 || (ps > 0 && ps % PA_BLOCK_SIZE)) return PA_ERR_SHAPE;
+    const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
+                            ? p->max_seq_len
+                            : p->max_blocks_per_seq * PA_BLOCK_SIZE;
+    if (ps == -1) ps = 256;
+    if (ps > 0 && max_len <= ps) ps = 0;  // one partition: no split needed
+    *part = ps;
+    *max_parts = ps > 0 ? (max_len + ps - 1) / ps : 1;
+    if (*max_parts > 65535) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+int pa_version(void) { return 100; }
+
+const char *pa_status_string(int status) {
+    switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_NULL: return "a required pointer is NULL";
+    case PA_ERR_SHAPE: return "invalid or inconsistent size";
+    case PA_ERR_DTYPE: return "unknown or unsupported dtype combination";
+    case PA_ERR_UNSUPPORTED: return "valid but unsupported configuration";
+    case PA_ERR_WORKSPACE: return "split-K workspace missing or too small";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_ALIGN: return "buffer not aligned as required";
+    default: return "unknown status";
+    }
+}
+
+int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *value_cache,
+                         const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int64_t num_blocks, int dtype,
+                         int64_t k_token_stride, int64_t v_token_stride, pa_stream_t stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0) return PA_ERR_SHAPE;
+    if (block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
+    const int E = elem_size(dtype);
+    if (!E) return PA_ERR_DTYPE;
+    if (dtype == PA_I8) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL;
+    if (k_token_stride < (int64_t)num_kv_heads * head_dim || v_token_stride < (int64_t)num_kv_heads * head_dim)
+        return PA_ERR_SHAPE;
+    if (num_tokens > 2147483647LL) return PA_ERR_UNSUPPORTED;
+    return launch_reshape_and_cache(k, v, key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads,
+                                    head_dim, num_blocks, E, k_token_stride, v_token_stride,
+                                    (cudaStream_t)stream);
+}
+
+int pa_block_copy(void *key_cache, void *value_cache, float *k_scales, float *v_scales,
+                  const int64_t *src_dst_pairs, int64_t num_pairs, int num_kv_heads, int head_dim,
+                  int block_size, int64_t num_blocks, int dtype, pa_stream_t stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0) return PA_ERR_SHAPE;
+    if (block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
+    const int E = elem_size(dtype);
+    if (!E) return PA_ERR_DTYPE;
+    if (num_pairs == 0) return PA_OK;
+    if (!key_cache || !value_cache || !src_dst_pairs) return PA_ERR_NULL;
+    if ((k_scales == nullptr) != (v_scales == nullptr)) return PA_ERR_NULL;
+    if (num_pairs > 2147483647LL) return PA_ERR_UNSUPPORTED;
+    return launch_block_copy(key_cache, value_cache, k_scales, v_scales, src_dst_pairs, num_pairs,
+                             num_kv_heads, head_dim, num_blocks, E, (cudaStream_t)stream);
+}
+
+int pa_quantize_int8(const void *src_cache, int src_dtype, int8_t *dst_cache, float *scales,
+                     int64_t num_blocks, int num_kv_heads, int head_dim, int block_size,
+                     pa_stream_t stream) {
+    if (num_blocks < 0 || num_kv_heads <= 0 || head_dim <= 0) return PA_ERR_SHAPE;
+    if (block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
+    if (src_dtype != PA_F32 && src_dtype != PA_F16 && src_dtype != PA_BF16) return PA_ERR_DTYPE;
+    if (num_blocks == 0) return PA_OK;
+    if (!src_cache || !dst_cache || !scales) return PA_ERR_NULL;
+    if (num_blocks * num_kv_heads > 2147483647LL) return PA_ERR_UNSUPPORTED;
+    return launch_quantize_int8(src_cache, src_dtype, dst_cache, scales, num_blocks, num_kv_heads, head_dim,
+                                (cudaStream_t)stream);
+}
+
+size_t pa_decode_workspace_size(const pa_decode_params *p) {
+    int part = 0, mp = 0;
+    if (check_decode_params(p, &part, &mp) != PA_OK) return 0;
+    return decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->head_dim,
+                                  p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
+                                      ? p->max_seq_len
+                                      : p->max_blocks_per_seq * PA_BLOCK_SIZE,
+                                  part);
+}
+
+int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *seq_lens, float scale,
+              const pa_decode_params *p, pa_stream_t stream) {
+    int part = 0, mp = 0;
+    int rc = check_decode_params(p, &part, &mp);
+    if (rc != PA_OK) return rc;
+    if (p->num_seqs == 0) return PA_OK;
+    if (!out || !q || !key_cache || !value_cache || !block_tables || !seq_lens) return PA_ERR_NULL;
+    if (p->kv_dtype == PA_I8 && (!p->k_scales || !p->v_scales)) return PA_ERR_NULL;
+    if (((uintptr_t)key_cache | (uintptr_t)value_cache) % 16) return PA_ERR_ALIGN;
+    const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
+                            ? p->max_seq_len
+                            : p->max_blocks_per_seq * PA_BLOCK_SIZE;
+    const size_t need = decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->head_dim, max_len, part);
+    if (need > 0 && (!p->workspace || p->workspace_bytes < need)) return PA_ERR_WORKSPACE;
+    if (need > 0 && (uintptr_t)p->workspace % 16) return PA_ERR_ALIGN;
+
+    DecodeArgs a{};
+    a.out = out;
+    a.q = q;
+    a.kc = key_cache;
+    a.vc = value_cache;
+    a.ks = p->k_scales;
+    a.vs = p->v_scales;
+    a.tables = block_tables;
+    a.lens = seq_lens;
+    a.scale_log2 = scale * kLog2e;
+    a.B = p->num_seqs;
+    a.Hq = p->num_q_heads;
+    a.Hkv = p->num_kv_heads;
+    a.D = p->head_dim;
+    a.G = p->num_q_heads / p->num_kv_heads;
+    a.mbps = p->max_blocks_per_seq;
+    a.N = p->num_blocks;
+    a.max_len = max_len;
+    a.q_dtype = p->q_dtype;
+    a.kv_dtype = p->kv_dtype;
+    a.part = part;
+    a.max_parts = mp;
+    if (need > 0) {
+        const size_t o_bytes = (size_t)a.B * a.Hq * mp * a.D * sizeof(float);
+        a.ws_o = reinterpret_cast<float *>(p->workspace);
+        a.ws_lse = reinterpret_cast<float *>(reinterpret_cast<char *>(p->workspace) + ((o_bytes + 255) / 256) * 256);
+    }
+    if (max_len == 0) {
+        // every row is zero: the one-pass kernel writes zeros for seq_len <= 0
+        a.part = 0;
+        a.max_parts = 1;
+    }
+    return launch_decode_simt(a, (cudaStream_t)stream);
+}
+
+int pa_get_error_flags(unsigned int *flags, int reset, pa_stream_t stream) {
+    if (!flags) return PA_ERR_NULL;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
+    int (*const words[])(unsigned int *, bool) = {error_word_cache_ops, error_word_decode_simt};
+    unsigned int all = 0;
+    for (auto w : words) {
+        unsigned int f = 0;
+        if (w(&f, reset != 0) != PA_OK) return PA_ERR_CUDA;
+        all |= f;
+    }
+    *flags = all;
+    return PA_OK;
+}
+
+}  // extern "C"

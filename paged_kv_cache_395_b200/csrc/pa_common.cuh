@@ -1,0 +1,205 @@
+// Shared device helpers for the paged decode library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+constexpr int kBlockSize = PA_BLOCK_SIZE;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Error word (pa_error_flag bits).  Each translation unit that includes this
+// header gets its own copy on every device; PA_ERROR_WORD_ACCESSOR(name) defines
+// the host function that reads (and optionally clears) the copy of its unit,
+// and pa_get_error_flags ORs them.
+static __device__ unsigned int g_error_flags = 0;
+
+__device__ __forceinline__ void raise_flag(unsigned int bit) { atomicOr(&g_error_flags, bit); }
+
+#define PA_ERROR_WORD_ACCESSOR(name)                                                        \
+    int name(unsigned int *flags, bool reset) {                                             \
+        if (cudaMemcpyFromSymbol(flags, g_error_flags, sizeof(unsigned int)) != cudaSuccess) \
+            return PA_ERR_CUDA;                                                             \
+        if (reset) {                                                                        \
+            const unsigned int zero = 0;                                                    \
+            if (cudaMemcpyToSymbol(g_error_flags, &zero, sizeof(unsigned int)) != cudaSuccess) \
+                return PA_ERR_CUDA;                                                         \
+        }                                                                                   \
+        return PA_OK;                                                                       \
+    }
+
+// ---------------------------------------------------------------------------
+// element types
+// ---------------------------------------------------------------------------
+template <typename T> struct Cvt;
+template <> struct Cvt<float> {
+    static __device__ __forceinline__ float to_f(float x) { return x; }
+    static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct Cvt<__half> {
+    static __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+    static __device__ __forceinline__ __half from_f(float x) { return __float2half_rn(x); }
+};
+template <> struct Cvt<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+template <> struct Cvt<int8_t> {
+    static __device__ __forceinline__ float to_f(int8_t x) { return (float)x; }
+};
+
+// Convert N consecutive elements held in registers (as raw 32-bit words) to float.
+template <typename T, int N>
+__device__ __forceinline__ void to_float(const uint32_t *w, float *f);
+
+template <int N>
+__device__ __forceinline__ void to_float_f32(const uint32_t *w, float *f) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) f[i] = __uint_as_float(w[i]);
+}
+template <> __device__ __forceinline__ void to_float<float, 4>(const uint32_t *w, float *f) { to_float_f32<4>(w, f); }
+template <> __device__ __forceinline__ void to_float<float, 8>(const uint32_t *w, float *f) { to_float_f32<8>(w, f); }
+template <> __device__ __forceinline__ void to_float<float, 16>(const uint32_t *w, float *f) { to_float_f32<16>(w, f); }
+template <> __device__ __forceinline__ void to_float<float, 2>(const uint32_t *w, float *f) { to_float_f32<2>(w, f); }
+
+template <int N>
+__device__ __forceinline__ void to_float_h(const uint32_t *w, float *f) {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+        __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
+        float2 x = __half22float2(h);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+template <> __device__ __forceinline__ void to_float<__half, 2>(const uint32_t *w, float *f) { to_float_h<2>(w, f); }
+template <> __device__ __forceinline__ void to_float<__half, 4>(const uint32_t *w, float *f) { to_float_h<4>(w, f); }
+template <> __device__ __forceinline__ void to_float<__half, 8>(const uint32_t *w, float *f) { to_float_h<8>(w, f); }
+template <> __device__ __forceinline__ void to_float<__half, 16>(const uint32_t *w, float *f) { to_float_h<16>(w, f); }
+
+template <int N>
+__device__ __forceinline__ void to_float_b(const uint32_t *w, float *f) {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+        // bf16 is the top half of an fp32: shift / mask, no rounding involved.
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+template <> __device__ __forceinline__ void to_float<__nv_bfloat16, 2>(const uint32_t *w, float *f) { to_float_b<2>(w, f); }
+template <> __device__ __forceinline__ void to_float<__nv_bfloat16, 4>(const uint32_t *w, float *f) { to_float_b<4>(w, f); }
+template <> __device__ __forceinline__ void to_float<__nv_bfloat16, 8>(const uint32_t *w, float *f) { to_float_b<8>(w, f); }
+template <> __device__ __forceinline__ void to_float<__nv_bfloat16, 16>(const uint32_t *w, float *f) { to_float_b<16>(w, f); }
+
+template <int N>
+__device__ __forceinline__ void to_float_i8(const uint32_t *w, float *f) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) f[i] = (float)(int8_t)((w[i / 4] >> (8 * (i % 4))) & 0xff);
+}
+template <> __device__ __forceinline__ void to_float<int8_t, 2>(const uint32_t *w, float *f) { to_float_i8<2>(w, f); }
+template <> __device__ __forceinline__ void to_float<int8_t, 4>(const uint32_t *w, float *f) { to_float_i8<4>(w, f); }
+template <> __device__ __forceinline__ void to_float<int8_t, 8>(const uint32_t *w, float *f) { to_float_i8<8>(w, f); }
+template <> __device__ __forceinline__ void to_float<int8_t, 16>(const uint32_t *w, float *f) { to_float_i8<16>(w, f); }
+
+// Load BYTES bytes (2, 4, 8, 16, 32 or 64; naturally aligned) from shared memory into words.
+template <int BYTES>
+__device__ __forceinline__ void lds(const void *p, uint32_t *w) {
+    if constexpr (BYTES == 2) {
+        w[0] = *reinterpret_cast<const uint16_t *>(p);
+    } else if constexpr (BYTES == 4) {
+        w[0] = *reinterpret_cast<const uint32_t *>(p);
+    } else if constexpr (BYTES == 8) {
+        uint2 v = *reinterpret_cast<const uint2 *>(p);
+        w[0] = v.x; w[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < BYTES / 16; ++i) {
+            uint4 v = reinterpret_cast<const uint4 *>(p)[i];
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk asynchronous copy (TMA, non-tensor form)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Order this thread's earlier generic-proxy shared-memory accesses before later
+// async-proxy (bulk copy) accesses to the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase with the given parity to complete.  Gives up after about
+// one second (a copy that never lands), raises PA_EFLAG_WAIT_TIMEOUT and
+// returns false; the caller then abandons its remaining work.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63) == 63 && global_timer_ns() - t0 > 1000000000ull) {
+            raise_flag(PA_EFLAG_WAIT_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Global -> shared bulk copy of `bytes` (multiple of 16, both addresses 16-byte
+// aligned), completing `bytes` transactions on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace pa

@@ -1,0 +1,61 @@
+// Launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+template <int N> struct VecT;
+template <> struct VecT<16> { using type = uint4; };
+template <> struct VecT<8> { using type = uint2; };
+template <> struct VecT<4> { using type = uint32_t; };
+template <> struct VecT<2> { using type = uint16_t; };
+template <> struct VecT<1> { using type = uint8_t; };
+
+int launch_reshape_and_cache(const void *k, const void *v, void *kc, void *vc,
+                             const int64_t *slots, int64_t T, int H, int D, int64_t N, int E,
+                             int64_t k_stride, int64_t v_stride, cudaStream_t st);
+int launch_block_copy(void *kc, void *vc, float *ks, float *vs, const int64_t *pairs, int64_t n,
+                      int H, int D, int64_t N, int E, cudaStream_t st);
+int launch_quantize_int8(const void *src, int src_dtype, int8_t *dst, float *scales, int64_t N,
+                         int H, int D, cudaStream_t st);
+
+// Everything pa_decode needs after validation.
+struct DecodeArgs {
+    void *out;
+    const void *q;
+    const void *kc;
+    const void *vc;
+    const float *ks;
+    const float *vs;
+    const int32_t *tables;
+    const int32_t *lens;
+    float scale_log2;        // scale * log2(e): scores are kept in the log2 domain
+    int B, Hq, Hkv, D, G;
+    int mbps;                // max_blocks_per_seq
+    int64_t N;               // num_blocks
+    int max_len;             // effective bound on seq_lens
+    int q_dtype, kv_dtype;
+    int part;                // partition size in tokens (0 = one pass)
+    int max_parts;           // ceil(max_len / part) when part > 0
+    float *ws_o;             // [B][Hq][max_parts][D]
+    float *ws_lse;           // [B][Hq][max_parts]  (log2 domain)
+};
+
+// Per-translation-unit error words (see PA_ERROR_WORD_ACCESSOR).
+int error_word_cache_ops(unsigned int *flags, bool reset);
+int error_word_decode_simt(unsigned int *flags, bool reset);
+
+// Raise a kernel's dynamic shared-memory limit on the current device, once per
+// (kernel, device).  Thread-safe; returns false if CUDA refuses.
+bool set_smem_attr_once(const void *kernel, int bytes);
+
+size_t decode_workspace_bytes(int B, int Hq, int D, int max_len, int part);
+int launch_decode_simt(const DecodeArgs &a, cudaStream_t st);
+int launch_merge(const DecodeArgs &a, cudaStream_t st);
+bool decode_simt_supported(int q_dtype, int kv_dtype, int D, int G);
+
+}  // namespace pa

@@ -1,0 +1,134 @@
+"""The C-ABI library on the host (no GPU needed): it loads, exports every
+function include/pa.h declares, and rejects invalid arguments with the
+documented status codes before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_395_b200 import pa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(pa_[a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_expected_entry_points():
+    names = header_functions()
+    for n in ("pa_reshape_and_cache", "pa_decode", "pa_block_copy", "pa_decode_workspace_size"):
+        assert n in names
+    assert set(names) == set(pa.EXPORTED)
+
+
+@pytest.mark.parametrize("name", header_functions())
+def test_library_exports(name):
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    assert getattr(lib, name) is not None
+
+
+def test_status_strings_and_version():
+    assert pa.lib.pa_status_string(0) == b"ok"
+    for s in range(-7, 0):
+        assert pa.lib.pa_status_string(s) != b"unknown status"
+    assert pa.version() >= 100
+
+
+def params(**kw):
+    p = pa.PaDecodeParams()
+    base = dict(num_seqs=2, num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                max_blocks_per_seq=4, num_blocks=8, max_seq_len=64, q_dtype=pa.PA_F16,
+                kv_dtype=pa.PA_F16, partition_size=0, algo=0)
+    base.update(kw)
+    for k, v in base.items():
+        setattr(p, k, v)
+    return p
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails validation
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=96), pa.PA_ERR_UNSUPPORTED),
+    (dict(head_dim=0), pa.PA_ERR_SHAPE),
+    (dict(block_size=32), pa.PA_ERR_UNSUPPORTED),
+    (dict(num_q_heads=6, num_kv_heads=4), pa.PA_ERR_SHAPE),
+    (dict(num_q_heads=6, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),   # G = 3
+    (dict(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F16), pa.PA_ERR_DTYPE),
+    (dict(q_dtype=pa.PA_I8, kv_dtype=pa.PA_I8), pa.PA_ERR_DTYPE),
+    (dict(q_dtype=9), pa.PA_ERR_DTYPE),
+    (dict(partition_size=24), pa.PA_ERR_SHAPE),
+    (dict(partition_size=-2), pa.PA_ERR_SHAPE),
+    (dict(num_seqs=-1), pa.PA_ERR_SHAPE),
+    (dict(algo=7), pa.PA_ERR_UNSUPPORTED),
+])
+def test_decode_rejects_bad_params(kw, status):
+    p = params(**kw)
+    rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
+    assert rc == status
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_decode_null_and_workspace_checks():
+    p = params()
+    rc = pa.lib.pa_decode(None, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
+    assert rc == pa.PA_ERR_NULL
+    rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), None, None)
+    assert rc == pa.PA_ERR_NULL
+    p = params(kv_dtype=pa.PA_I8)  # int8 without scales
+    rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
+    assert rc == pa.PA_ERR_NULL
+    p = params(partition_size=16)  # split-K without a workspace
+    need = pa.lib.pa_decode_workspace_size(ctypes.byref(p))
+    # 2 seqs x 8 heads x 4 partitions x (128 + 1) floats, each part rounded up to 256 B
+    assert need == 2 * 8 * 4 * 128 * 4 + 256
+    rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
+    assert rc == pa.PA_ERR_WORKSPACE
+    p.workspace, p.workspace_bytes = 0x1000, need - 1
+    rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
+    assert rc == pa.PA_ERR_WORKSPACE
+    p = params()
+    rc = pa.lib.pa_decode(FAKE, FAKE, ctypes.c_void_p(0x1008), FAKE, FAKE, FAKE, ctypes.c_float(0.1),
+                          ctypes.byref(p), None)
+    assert rc == pa.PA_ERR_ALIGN
+    # a partition as long as the longest sequence needs no workspace
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(params(partition_size=64))) == 0
+    # empty batch is a no-op
+    assert pa.lib.pa_decode(None, None, None, None, None, None, ctypes.c_float(0.1),
+                            ctypes.byref(params(num_seqs=0)), None) == pa.PA_OK
+
+
+def test_cache_ops_reject_bad_args():
+    L = pa.lib
+    assert L.pa_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 32, 8, pa.PA_F16, 128, 128, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, pa.PA_I8, 128, 128, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 11, 128, 128, None) == pa.PA_ERR_DTYPE
+    assert L.pa_reshape_and_cache(None, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, pa.PA_F16, 128, 128, None) == pa.PA_ERR_NULL
+    assert L.pa_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, pa.PA_F16, 100, 128, None) == pa.PA_ERR_SHAPE
+    assert L.pa_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 64, 16, 8, pa.PA_F16, 128, 128, None) == pa.PA_ERR_SHAPE
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 0, 2, 64, 16, 8, pa.PA_F16, 128, 128, None) == pa.PA_OK
+    assert L.pa_block_copy(FAKE, FAKE, None, None, FAKE, 1, 2, 64, 8, 8, pa.PA_F16, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_block_copy(FAKE, None, None, None, FAKE, 1, 2, 64, 16, 8, pa.PA_F16, None) == pa.PA_ERR_NULL
+    assert L.pa_block_copy(FAKE, FAKE, FAKE, None, FAKE, 1, 2, 64, 16, 8, pa.PA_I8, None) == pa.PA_ERR_NULL
+    assert L.pa_block_copy(None, None, None, None, None, 0, 2, 64, 16, 8, pa.PA_F16, None) == pa.PA_OK
+    assert L.pa_quantize_int8(FAKE, pa.PA_I8, FAKE, FAKE, 4, 2, 64, 16, None) == pa.PA_ERR_DTYPE
+    assert L.pa_quantize_int8(FAKE, pa.PA_F16, None, FAKE, 4, 2, 64, 16, None) == pa.PA_ERR_NULL
+    assert L.pa_quantize_int8(FAKE, pa.PA_F16, FAKE, FAKE, 4, 2, 64, 8, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_get_error_flags(None, 0, None) == pa.PA_ERR_NULL
+
+
+def test_product_path_does_not_touch_oracle():
+    """The package never imports the oracle (it is test infrastructure)."""
+    pkg = os.path.join(ROOT, "paged_kv_cache_395_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, flags=re.M), f
+                assert not re.search(r"#include\s*[<\"][^>\"]*oracle", src), f
+                assert "liboracle" not in src and "pa_oracle" not in src, f

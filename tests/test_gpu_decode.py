@@ -1,0 +1,206 @@
+"""GPU paged decode against the oracle, element by element, plus invariants.
+
+Every case runs through the C ABI (paged_kv_cache_395_b200.pa).  Tolerance:
+|err| <= 2e-3 + 2e-3 |ref| for fp16/bf16 outputs (fp32 accumulation), and
+1e-5 + 1e-5 |ref| for the fp32 case; int8 caches are compared with the oracle
+dequantising the same int8 values and scales in fp64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_395_b200 import pa, runner, workloads as W
+
+from .gpu_util import assert_close, bits
+from .oracle_replay import replay
+
+pytestmark = pytest.mark.gpu
+
+ALGOS = [pa.PA_ALGO_SIMT, pa.PA_ALGO_AUTO]
+PARTS = [0, 16, 32, 256, -1]
+
+
+@pytest.fixture(autouse=True)
+def _clear_flags():
+    pa.pa_get_error_flags(reset=True)
+    yield
+    assert pa.pa_get_error_flags(reset=True) == 0
+
+
+def run_gpu(w, partition_size=0, algo=pa.PA_ALGO_AUTO, int8=False, dw=None):
+    dw = dw or runner.DeviceWorkload(w)
+    dw.run_setup()
+    if int8:
+        dw.quantize_int8()
+    outs = {}
+    for i in range(len(w.steps)):
+        o = dw.run_step(i, partition_size, int8=int8, algo=algo)
+        outs[i] = o.clone()
+    torch.cuda.synchronize()
+    return outs, dw
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("part", [0, 16, -1])
+def test_tiny_fp32(algo, part):
+    w = W.tiny()
+    ref, _, _ = replay(w)
+    got, _ = run_gpu(w, part, algo)
+    assert_close(got[0], ref[0], "float32", "tiny")
+
+
+CASES = {
+    # lengths hit 1, a full block, block + 1, a ragged tail, several partitions
+    "g4_d128_f16": dict(lens=[1, 16, 17, 100, 513, 1000], num_q_heads=32, num_kv_heads=8,
+                        head_dim=128, dtype="float16"),
+    "g8_d128_bf16": dict(lens=[33, 300, 2, 129], num_q_heads=16, num_kv_heads=2, head_dim=128,
+                         dtype="bfloat16"),
+    "g1_d128_f16": dict(lens=[15, 64, 257], num_q_heads=4, num_kv_heads=4, head_dim=128,
+                        dtype="float16"),
+    "g2_d64_f16": dict(lens=[31, 48, 7, 600], num_q_heads=8, num_kv_heads=4, head_dim=64,
+                       dtype="float16"),
+    "g4_d64_bf16": dict(lens=[5, 77, 256], num_q_heads=8, num_kv_heads=2, head_dim=64,
+                        dtype="bfloat16"),
+    "g8_d64_f32": dict(lens=[3, 45], num_q_heads=8, num_kv_heads=1, head_dim=64, dtype="float32"),
+    "sharp_softmax": dict(lens=[200, 37], num_q_heads=8, num_kv_heads=2, head_dim=128,
+                          dtype="float16", q_scale=6.0),
+}
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("part", PARTS)
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_random_cases(case, part, algo):
+    w = W.random_case(seed=sorted(CASES).index(case) + 100, **CASES[case])
+    ref, _, _ = replay(w)
+    got, _ = run_gpu(w, part, algo)
+    assert_close(got[0], ref[0], w.dtype, case)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("part", [0, 32, -1])
+@pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
+def test_int8_random(qdt, part, algo):
+    w = W.random_case([1, 17, 96, 400], num_q_heads=16, num_kv_heads=4, head_dim=128, dtype=qdt,
+                      seed=4)
+    dw = runner.DeviceWorkload(w)
+    got, dw = run_gpu(w, part, algo, int8=True, dw=dw)
+    # the oracle dequantises the very same int8 values and scales
+    kc8, vc8 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
+    ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
+    op = w.steps[0][0]
+    ref = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
+    assert_close(got[0], ref, qdt, "int8")
+
+
+def test_zero_length_and_empty_batch():
+    w = W.random_case([0, 5, 0, 40], num_q_heads=8, num_kv_heads=2, head_dim=64, dtype="float16")
+    ref, _, _ = replay(w)
+    for part in (0, 16):
+        got, _ = run_gpu(w, part)
+        assert_close(got[0], ref[0], "float16", "zero length")
+        assert torch.count_nonzero(got[0][0]) == 0 and torch.count_nonzero(got[0][2]) == 0
+    # B = 0 is a no-op
+    q = torch.empty((0, 8, 64), dtype=torch.float16, device="cuda")
+    kc = torch.zeros((4, 2, 16, 64), dtype=torch.float16, device="cuda")
+    bt = torch.zeros((0, 1), dtype=torch.int32, device="cuda")
+    sl = torch.zeros((0,), dtype=torch.int32, device="cuda")
+    pa.pa_decode(torch.empty_like(q), q, kc, kc, bt, sl, 0.125, 0)
+
+
+def test_permutation_invariance_bitwise():
+    """Moving the physical blocks leaves the GPU output bit-identical."""
+    w = W.random_case([70, 300, 17], num_q_heads=32, num_kv_heads=8, head_dim=128, seed=9)
+    for part in (0, 32):
+        got, dw = run_gpu(w, part)
+        sigma = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(1)).cuda()
+        kc2 = torch.empty_like(dw.kc)
+        vc2 = torch.empty_like(dw.vc)
+        kc2[sigma] = dw.kc
+        vc2[sigma] = dw.vc
+        _, q, bt, sl, mx, out = dw.steps[0][-1]
+        bt2 = bt.clone()
+        valid = bt2 >= 0
+        bt2[valid] = sigma[bt2[valid].long()].int()
+        out2 = torch.empty_like(out)
+        ws = dw.workspace_for(dw.steps[0][-1], part)
+        pa.pa_decode(out2, q, kc2, vc2, bt2, sl, w.scale, mx, partition_size=part, workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(out2), bits(got[0])), f"part={part}"
+
+
+def test_deterministic_and_split_matches_single():
+    w = W.random_case([900, 1500, 64], num_q_heads=32, num_kv_heads=8, head_dim=128, seed=10)
+    a, _ = run_gpu(w, 0)
+    b, _ = run_gpu(w, 0)
+    assert np.array_equal(bits(a[0]), bits(b[0]))
+    c, _ = run_gpu(w, 128)
+    d, _ = run_gpu(w, 128)
+    assert np.array_equal(bits(c[0]), bits(d[0]))
+    ref, _, _ = replay(w)
+    assert_close(c[0], ref[0], "float16", "split")
+    assert_close(a[0], ref[0], "float16", "single")
+
+
+def test_bad_block_id_flagged():
+    """A table entry outside the pool is skipped by the kernel's own bounds
+    check (no memory access) and reported in the error word."""
+    w = W.random_case([40, 20], num_q_heads=8, num_kv_heads=2, head_dim=64, seed=2)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    _, q, bt, sl, mx, out = dw.steps[0][-1]
+    bt[1, 0] = w.num_blocks + 5
+    pa.pa_decode(out, q, dw.kc, dw.vc, bt, sl, w.scale, mx)
+    assert pa.pa_get_error_flags(reset=True) == pa.PA_EFLAG_BAD_BLOCK
+
+
+# -- the study's workloads at full size ---------------------------------------------------
+def test_gqa_b8_full():
+    w = W.gqa_b8()
+    ref, _, _ = replay(w)
+    for part in (0, -1, 128):
+        got, _ = run_gpu(w, part)
+        assert_close(got[0], ref[0], "float16", f"gqa_b8 part={part}")
+
+
+@pytest.mark.slow
+def test_long_fp16_and_int8_full():
+    w = W.long()
+    ref, kc, vc = replay(w, fill_nan=False)
+    got, dw = run_gpu(w, 512)
+    assert_close(got[0], ref[0], "float16", "long fp16")
+    got8, dw = run_gpu(w, 512, int8=True, dw=runner.DeviceWorkload(w, fill_nan=False))
+    kc8, ks = oracle.quantize_int8(kc)
+    vc8, vs = oracle.quantize_int8(vc)
+    assert np.array_equal(bits(dw.kc8), kc8.view(np.uint8)) and np.array_equal(bits(dw.k_scales), ks.view(np.uint8))
+    op = w.steps[0][0]
+    ref8 = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
+    assert_close(got8[0], ref8, "float16", "long int8")
+
+
+def test_mha_prefix_full():
+    w = W.mha_prefix()
+    ref, kc, vc = replay(w)
+    got, dw = run_gpu(w, -1)
+    assert_close(got[0], ref[0], "float16", "mha_prefix")
+    # after copy-on-write the shared prefix blocks are unchanged and the caches match bit for bit
+    assert np.array_equal(bits(dw.kc), kc.view(np.uint8))
+
+
+@pytest.mark.slow
+def test_ragged_full_trace():
+    """The continuous-batching trace in the benchmark's launch configuration:
+    all 128 steps on the GPU, oracle decode on 8 sampled steps, caches bit-exact."""
+    w = W.ragged()
+    sample = {0, 1, 2, 31, 64, 100, 126, 127}
+    ref, kc, vc = replay(w, want=lambda s: s in sample)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    for i in range(len(w.steps)):
+        out = dw.run_step(i, -1)
+        if i in sample:
+            assert_close(out, ref[i], "float16", f"ragged step {i}")
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(dw.kc), kc.view(np.uint8))
+    assert np.array_equal(bits(dw.vc), vc.view(np.uint8))
