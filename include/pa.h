@@ -108,10 +108,15 @@ typedef struct pa_decode_params {
     int partition_size;      /* 0: one pass, one CTA per (sequence, KV head), no workspace.
                                 > 0: split-K, partitions of this many tokens (a multiple of
                                 16), then a log-sum-exp merge; needs the workspace.
-                                -1: the library picks (may use split-K; needs the workspace). */
+                                -1: the library picks from num_seqs, num_kv_heads and
+                                max_seq_len (64..512 tokens, or one pass when max_seq_len
+                                fits one partition). */
     int algo;                /* enum pa_algo */
     void *workspace;         /* device scratch, >= pa_decode_workspace_size(p) bytes,
-                                16-byte aligned; NULL allowed when that size is 0 */
+                                16-byte aligned; NULL allowed when that size is 0.  Must be
+                                zero-filled once before its first use; every call leaves it
+                                ready for the next (its merge counters back at zero).  Calls
+                                that share a workspace must not overlap on the device. */
     size_t workspace_bytes;
 } pa_decode_params;
 

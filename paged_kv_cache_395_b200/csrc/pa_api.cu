@@ -32,6 +32,20 @@ static int elem_size(int dt) {
     }
 }
 
+// Partition size for partition_size == -1.  The persistent kernel runs
+// 148 SMs x 2 CTAs x 4 warps = 1184 warp workers on B200; aim for at least
+// four (sequence, partition, KV head) items per worker, counting every
+// sequence at max_len, with partitions of 64..512 tokens.  Depends only on
+// the arguments, so pa_decode_workspace_size agrees with pa_decode.
+static int auto_partition(int B, int Hkv, int max_len) {
+    const int64_t want = 4 * 1184;
+    for (int ps = 512; ps >= 64; ps >>= 1) {
+        const int64_t items = (int64_t)B * Hkv * ((max_len + ps - 1) / ps);
+        if (items >= want) return ps;
+    }
+    return 64;
+}
+
 // Checks shared by pa_decode and pa_decode_workspace_size.  Fills the partition
 // size actually used (auto resolved) and the partition count.
 static int check_decode_params(const pa_decode_params *p, int *part, int *max_parts) {
@@ -55,7 +69,7 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
     const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
                             ? p->max_seq_len
                             : p->max_blocks_per_seq * PA_BLOCK_SIZE;
-    if (ps == -1) ps = 256;
+    if (ps == -1) ps = auto_partition(p->num_seqs, p->num_kv_heads, max_len);
     if (ps > 0 && max_len <= ps) ps = 0;  // one partition: no split needed
     *part = ps;
     *max_parts = ps > 0 ? (max_len + ps - 1) / ps : 1;
@@ -135,7 +149,7 @@ int pa_quantize_int8(const void *src_cache, int src_dtype, int8_t *dst_cache, fl
 size_t pa_decode_workspace_size(const pa_decode_params *p) {
     int part = 0, mp = 0;
     if (check_decode_params(p, &part, &mp) != PA_OK) return 0;
-    return decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->head_dim,
+    return decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->num_kv_heads, p->head_dim,
                                   p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
                                       ? p->max_seq_len
                                       : p->max_blocks_per_seq * PA_BLOCK_SIZE,
@@ -155,7 +169,8 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
                             ? p->max_seq_len
                             : p->max_blocks_per_seq * PA_BLOCK_SIZE;
-    const size_t need = decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->head_dim, max_len, part);
+    const size_t need = decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->num_kv_heads, p->head_dim,
+                                               max_len, part);
     if (need > 0 && (!p->workspace || p->workspace_bytes < need)) return PA_ERR_WORKSPACE;
     if (need > 0 && (uintptr_t)p->workspace % 16) return PA_ERR_ALIGN;
 
@@ -182,22 +197,31 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     a.part = part;
     a.max_parts = mp;
     if (need > 0) {
-        const size_t o_bytes = (size_t)a.B * a.Hq * mp * a.D * sizeof(float);
-        a.ws_o = reinterpret_cast<float *>(p->workspace);
-        a.ws_lse = reinterpret_cast<float *>(reinterpret_cast<char *>(p->workspace) + ((o_bytes + 255) / 256) * 256);
+        auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+        const size_t o_bytes = up((size_t)a.B * a.Hq * mp * a.D * sizeof(float));
+        const size_t l_bytes = up((size_t)a.B * a.Hq * mp * sizeof(float));
+        char *ws = reinterpret_cast<char *>(p->workspace);
+        a.ws_o = reinterpret_cast<float *>(ws);
+        a.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
+        a.counters = reinterpret_cast<int *>(ws + o_bytes + l_bytes);
     }
     if (max_len == 0) {
         // every row is zero: the one-pass kernel writes zeros for seq_len <= 0
         a.part = 0;
         a.max_parts = 1;
     }
+    const bool tc_ok = decode_tc_supported(a.q_dtype, a.kv_dtype, a.D, a.G, a.B);
+    if (p->algo == PA_ALGO_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
+    if (p->algo == PA_ALGO_TENSOR || (p->algo == PA_ALGO_AUTO && tc_ok))
+        return launch_decode_tc(a, (cudaStream_t)stream);
     return launch_decode_simt(a, (cudaStream_t)stream);
 }
 
 int pa_get_error_flags(unsigned int *flags, int reset, pa_stream_t stream) {
     if (!flags) return PA_ERR_NULL;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
-    int (*const words[])(unsigned int *, bool) = {error_word_cache_ops, error_word_decode_simt};
+    int (*const words[])(unsigned int *, bool) = {error_word_cache_ops, error_word_decode_simt,
+                                                  error_word_decode_tc};
     unsigned int all = 0;
     for (auto w : words) {
         unsigned int f = 0;

@@ -330,12 +330,14 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
     }
 }
 
-size_t decode_workspace_bytes(int B, int Hq, int D, int max_len, int part) {
-    if (part <= 0 || max_len <= 0) return 0;
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int part) {
+    if (part <= 0 || max_len <= part) return 0;
     const size_t mp = (size_t)((max_len + part - 1) / part);
     const size_t o = (size_t)B * Hq * mp * D * sizeof(float);
     const size_t lse = (size_t)B * Hq * mp * sizeof(float);
-    return ((o + 255) / 256) * 256 + ((lse + 255) / 256) * 256;
+    const size_t cnt = (size_t)B * Hkv * sizeof(int);
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    return up(o) + up(lse) + up(cnt);
 }
 
 template <typename TQ, typename TKV, int D, int G>

@@ -43,17 +43,22 @@ struct DecodeArgs {
     int max_parts;           // ceil(max_len / part) when part > 0
     float *ws_o;             // [B][Hq][max_parts][D]
     float *ws_lse;           // [B][Hq][max_parts]  (log2 domain)
+    int *counters;           // [B][Hkv] merge tickets, zero between calls
 };
 
 // Per-translation-unit error words (see PA_ERROR_WORD_ACCESSOR).
 int error_word_cache_ops(unsigned int *flags, bool reset);
 int error_word_decode_simt(unsigned int *flags, bool reset);
+int error_word_decode_tc(unsigned int *flags, bool reset);
 
 // Raise a kernel's dynamic shared-memory limit on the current device, once per
 // (kernel, device).  Thread-safe; returns false if CUDA refuses.
 bool set_smem_attr_once(const void *kernel, int bytes);
 
-size_t decode_workspace_bytes(int B, int Hq, int D, int max_len, int part);
+// Workspace layout for split-K: ws_o | ws_lse | counters, each 256-byte aligned.
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int part);
+int launch_decode_tc(const DecodeArgs &a, cudaStream_t st);
+bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B);
 int launch_decode_simt(const DecodeArgs &a, cudaStream_t st);
 int launch_merge(const DecodeArgs &a, cudaStream_t st);
 bool decode_simt_supported(int q_dtype, int kv_dtype, int D, int G);

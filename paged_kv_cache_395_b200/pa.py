@@ -161,9 +161,10 @@ def pa_decode_workspace_size(q, key_cache, block_tables, max_seq_len, partition_
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor | None:
+    """Split-K workspace; zero-filled, as pa_decode requires before first use."""
     if nbytes == 0:
         return None
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
 def pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max_seq_len,

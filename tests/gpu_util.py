@@ -2,8 +2,11 @@
 import numpy as np
 import torch
 
-# the benchmark spec tolerance for fp16/bf16 attention outputs with fp32 accumulation
-TOL = {"float16": (2e-3, 2e-3), "bfloat16": (2e-3, 2e-3), "float32": (1e-5, 1e-5)}
+# Tolerance for attention outputs with fp32 accumulation: |err| <= 2e-3 + 2e-3 |ref|
+# for fp16 and bf16.  A bf16 output is rounded once to 8 significant bits, which
+# alone can move it by 2^-8 |ref| (more than 2e-3 |ref|), so bf16 adds that unit
+# roundoff to the relative term.  fp32 outputs: 1e-5 + 1e-5 |ref|.
+TOL = {"float16": (2e-3, 2e-3), "bfloat16": (2e-3, 2e-3 + 2.0 ** -8), "float32": (1e-5, 1e-5)}
 
 
 def gpu_f64(t: torch.Tensor) -> np.ndarray:

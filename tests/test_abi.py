@@ -85,8 +85,9 @@ def test_decode_null_and_workspace_checks():
     assert rc == pa.PA_ERR_NULL
     p = params(partition_size=16)  # split-K without a workspace
     need = pa.lib.pa_decode_workspace_size(ctypes.byref(p))
-    # 2 seqs x 8 heads x 4 partitions x (128 + 1) floats, each part rounded up to 256 B
-    assert need == 2 * 8 * 4 * 128 * 4 + 256
+    # 2 seqs x 8 heads x 4 partitions x 128 floats, their 64 lse floats and
+    # 2 x 2 merge counters, each region rounded up to 256 B
+    assert need == 2 * 8 * 4 * 128 * 4 + 256 + 256
     rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
     assert rc == pa.PA_ERR_WORKSPACE
     p.workspace, p.workspace_bytes = 0x1000, need - 1

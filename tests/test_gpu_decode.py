@@ -17,7 +17,12 @@ from .oracle_replay import replay
 
 pytestmark = pytest.mark.gpu
 
-ALGOS = [pa.PA_ALGO_SIMT, pa.PA_ALGO_AUTO]
+ALGOS = [pa.PA_ALGO_SIMT, pa.PA_ALGO_TENSOR, pa.PA_ALGO_AUTO]
+
+
+def algo_ok(algo, dtype):
+    """The tensor-core family covers fp16/bf16 q with a cache of the same dtype."""
+    return algo != pa.PA_ALGO_TENSOR or dtype in ("float16", "bfloat16")
 PARTS = [0, 16, 32, 256, -1]
 
 
@@ -41,7 +46,7 @@ def run_gpu(w, partition_size=0, algo=pa.PA_ALGO_AUTO, int8=False, dw=None):
     return outs, dw
 
 
-@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_AUTO])
 @pytest.mark.parametrize("part", [0, 16, -1])
 def test_tiny_fp32(algo, part):
     w = W.tiny()
@@ -72,13 +77,15 @@ CASES = {
 @pytest.mark.parametrize("part", PARTS)
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_random_cases(case, part, algo):
+    if not algo_ok(algo, CASES[case]["dtype"]):
+        pytest.skip("fp32 has no tensor-core path")
     w = W.random_case(seed=sorted(CASES).index(case) + 100, **CASES[case])
     ref, _, _ = replay(w)
     got, _ = run_gpu(w, part, algo)
     assert_close(got[0], ref[0], w.dtype, case)
 
 
-@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_AUTO])
 @pytest.mark.parametrize("part", [0, 32, -1])
 @pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
 def test_int8_random(qdt, part, algo):
@@ -92,6 +99,46 @@ def test_int8_random(qdt, part, algo):
     op = w.steps[0][0]
     ref = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
     assert_close(got[0], ref, qdt, "int8")
+
+
+def test_tensor_path_rejects_unsupported():
+    w = W.random_case([20], num_q_heads=4, num_kv_heads=2, head_dim=64, dtype="float32")
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    _, q, bt, sl, mx, out = dw.steps[0][-1]
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode(out, q, dw.kc, dw.vc, bt, sl, w.scale, mx, algo=pa.PA_ALGO_TENSOR)
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_TENSOR])
+def test_long_one_pass_and_many_partitions(algo):
+    """One pass over 40 blocks (more than one 32-entry table chunk) and a split
+    into 70 partitions, both against the oracle."""
+    w = W.random_case([640, 1120, 33], num_q_heads=16, num_kv_heads=4, head_dim=128, seed=12)
+    ref, _, _ = replay(w)
+    for part in (0, 16, 512):
+        got, _ = run_gpu(w, part, algo)
+        assert_close(got[0], ref[0], "float16", f"part={part}")
+
+
+def test_workspace_reused_across_calls():
+    """The merge counters return to zero, so one workspace serves many calls."""
+    w = W.random_case([300, 77, 513], num_q_heads=32, num_kv_heads=8, head_dim=128, seed=13)
+    ref, _, _ = replay(w)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    op = dw.steps[0][-1]
+    ws = dw.workspace_for(op, 32)
+    _, q, bt, sl, mx, out = op
+    for _ in range(5):
+        out.zero_()
+        pa.pa_decode(out, q, dw.kc, dw.vc, bt, sl, w.scale, mx, partition_size=32, workspace=ws,
+                     algo=pa.PA_ALGO_TENSOR)
+        assert_close(out, ref[0], "float16", "reuse")
+    # the last region holds the 3 x 8 merge counters (rounded up to 256 bytes)
+    torch.cuda.synchronize()
+    assert ws[-256:].count_nonzero().item() == 0
 
 
 def test_zero_length_and_empty_batch():
