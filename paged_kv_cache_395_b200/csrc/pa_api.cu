@@ -77,6 +77,58 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
     return PA_OK;
 }
 
+static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Which kernel family runs and what workspace it needs.
+struct Plan {
+    bool tc;
+    int part, max_parts;  // CUDA-core family: per-sequence partitions
+    int tc_chunk;         // tensor-core family: see DecodeArgs::tc_chunk
+    int64_t tc_slots;     // tensor-core family: partial-result slots
+    int max_len;
+    size_t bytes;
+};
+
+static int make_plan(const pa_decode_params *p, Plan *pl) {
+    int part = 0, mp = 0;
+    const int rc = check_decode_params(p, &part, &mp);
+    if (rc != PA_OK) return rc;
+    const int G = p->num_q_heads / p->num_kv_heads;
+    const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
+                            ? p->max_seq_len
+                            : p->max_blocks_per_seq * PA_BLOCK_SIZE;
+    const bool tc_ok = decode_tc_supported(p->q_dtype, p->kv_dtype, p->head_dim, G, p->num_seqs) &&
+                       p->num_blocks * p->num_kv_heads * PA_BLOCK_SIZE <= 2147483647LL;
+    if (p->algo == PA_ALGO_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
+    *pl = Plan{};
+    pl->max_len = max_len;
+    pl->tc = p->algo == PA_ALGO_TENSOR || (p->algo == PA_ALGO_AUTO && tc_ok);
+    if (!pl->tc) {
+        pl->part = part;
+        pl->max_parts = mp;
+        pl->bytes = decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->num_kv_heads, p->head_dim, max_len, part);
+        return PA_OK;
+    }
+    if (p->partition_size == 0 || max_len == 0) {
+        pl->tc_chunk = -1;  // one warp per (sequence, KV head) row, no workspace
+        return PA_OK;
+    }
+    const int64_t tmax = (int64_t)p->num_seqs * p->num_kv_heads * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
+    int64_t nchunks;
+    if (p->partition_size > 0) {
+        pl->tc_chunk = p->partition_size / PA_BLOCK_SIZE;
+        nchunks = (tmax + pl->tc_chunk - 1) / pl->tc_chunk;
+    } else {
+        pl->tc_chunk = 0;
+        nchunks = tmax < kTcMaxChunks ? tmax : kTcMaxChunks;
+    }
+    pl->tc_slots = 2 * nchunks;
+    pl->bytes = up256((size_t)pl->tc_slots * G * p->head_dim * sizeof(float)) +
+                up256((size_t)pl->tc_slots * G * sizeof(float)) +
+                up256((size_t)p->num_seqs * p->num_kv_heads * sizeof(int));
+    return PA_OK;
+}
+
 }  // namespace pa
 
 using namespace pa;
@@ -147,32 +199,23 @@ int pa_quantize_int8(const void *src_cache, int src_dtype, int8_t *dst_cache, fl
 }
 
 size_t pa_decode_workspace_size(const pa_decode_params *p) {
-    int part = 0, mp = 0;
-    if (check_decode_params(p, &part, &mp) != PA_OK) return 0;
-    return decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->num_kv_heads, p->head_dim,
-                                  p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
-                                      ? p->max_seq_len
-                                      : p->max_blocks_per_seq * PA_BLOCK_SIZE,
-                                  part);
+    Plan pl;
+    if (make_plan(p, &pl) != PA_OK) return 0;
+    return pl.bytes;
 }
 
 int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
               const int32_t *block_tables, const int32_t *seq_lens, float scale,
               const pa_decode_params *p, pa_stream_t stream) {
-    int part = 0, mp = 0;
-    int rc = check_decode_params(p, &part, &mp);
+    Plan pl;
+    const int rc = make_plan(p, &pl);
     if (rc != PA_OK) return rc;
     if (p->num_seqs == 0) return PA_OK;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !seq_lens) return PA_ERR_NULL;
     if (p->kv_dtype == PA_I8 && (!p->k_scales || !p->v_scales)) return PA_ERR_NULL;
     if (((uintptr_t)key_cache | (uintptr_t)value_cache) % 16) return PA_ERR_ALIGN;
-    const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
-                            ? p->max_seq_len
-                            : p->max_blocks_per_seq * PA_BLOCK_SIZE;
-    const size_t need = decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->num_kv_heads, p->head_dim,
-                                               max_len, part);
-    if (need > 0 && (!p->workspace || p->workspace_bytes < need)) return PA_ERR_WORKSPACE;
-    if (need > 0 && (uintptr_t)p->workspace % 16) return PA_ERR_ALIGN;
+    if (pl.bytes > 0 && (!p->workspace || p->workspace_bytes < pl.bytes)) return PA_ERR_WORKSPACE;
+    if (pl.bytes > 0 && (uintptr_t)p->workspace % 16) return PA_ERR_ALIGN;
 
     DecodeArgs a{};
     a.out = out;
@@ -191,29 +234,37 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     a.G = p->num_q_heads / p->num_kv_heads;
     a.mbps = p->max_blocks_per_seq;
     a.N = p->num_blocks;
-    a.max_len = max_len;
+    a.max_len = pl.max_len;
     a.q_dtype = p->q_dtype;
     a.kv_dtype = p->kv_dtype;
-    a.part = part;
-    a.max_parts = mp;
-    if (need > 0) {
-        auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-        const size_t o_bytes = up((size_t)a.B * a.Hq * mp * a.D * sizeof(float));
-        const size_t l_bytes = up((size_t)a.B * a.Hq * mp * sizeof(float));
-        char *ws = reinterpret_cast<char *>(p->workspace);
+    char *ws = reinterpret_cast<char *>(p->workspace);
+    if (pl.tc) {
+        a.part = 0;
+        a.max_parts = 1;
+        a.tc_chunk = pl.tc_chunk;
+        if (pl.bytes > 0) {
+            const size_t o_bytes = up256((size_t)pl.tc_slots * a.G * a.D * sizeof(float));
+            const size_t l_bytes = up256((size_t)pl.tc_slots * a.G * sizeof(float));
+            a.ws_o = reinterpret_cast<float *>(ws);
+            a.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
+            a.counters = reinterpret_cast<int *>(ws + o_bytes + l_bytes);
+        }
+        return launch_decode_tc(a, (cudaStream_t)stream);
+    }
+    a.part = pl.part;
+    a.max_parts = pl.max_parts;
+    if (pl.bytes > 0) {
+        const size_t o_bytes = up256((size_t)a.B * a.Hq * pl.max_parts * a.D * sizeof(float));
+        const size_t l_bytes = up256((size_t)a.B * a.Hq * pl.max_parts * sizeof(float));
         a.ws_o = reinterpret_cast<float *>(ws);
         a.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
         a.counters = reinterpret_cast<int *>(ws + o_bytes + l_bytes);
     }
-    if (max_len == 0) {
+    if (pl.max_len == 0) {
         // every row is zero: the one-pass kernel writes zeros for seq_len <= 0
         a.part = 0;
         a.max_parts = 1;
     }
-    const bool tc_ok = decode_tc_supported(a.q_dtype, a.kv_dtype, a.D, a.G, a.B);
-    if (p->algo == PA_ALGO_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
-    if (p->algo == PA_ALGO_TENSOR || (p->algo == PA_ALGO_AUTO && tc_ok))
-        return launch_decode_tc(a, (cudaStream_t)stream);
     return launch_decode_simt(a, (cudaStream_t)stream);
 }
 

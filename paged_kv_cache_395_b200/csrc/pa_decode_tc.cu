@@ -31,6 +31,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 #include <unordered_map>
 
 #include "pa_common.cuh"
@@ -109,16 +110,37 @@ struct TcCfg {
     static constexpr int STAGE = 2 * TILE;        // K tile, then V tile
     static constexpr int KSTEPS = D / 16;         // QK k-steps
     static constexpr int MTILES = D / 16;         // PV m-tiles
+    static constexpr int DPL = D / 32;            // dims per lane in the merge
     static constexpr int RING = NW * S * STAGE;
     static constexpr int BAR_OFF = RING;
-    static constexpr int BLK_OFF = BAR_OFF + NW * S * 8;
-    static constexpr int CUM_OFF = BLK_OFF + NW * S * 4;
-    static constexpr int MAX_B = 4096;
+    static constexpr int OK_OFF = BAR_OFF + NW * S * 8;
+    static constexpr int CUM_OFF = OK_OFF + NW * S * 4;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (B + 1) * 4; }
 };
 
-struct Item {
-    int b, kvh, part, L, t0, nblk, ntok_last, nparts;
+// One contiguous run of blocks of one (sequence, KV head) row.
+struct Seg {
+    int b, kvh, L, nb;  // row: sequence, KV head, tokens, blocks
+    int j0, j1;         // this segment: blocks [j0, j1) of the row
+    int64_t fr;         // index of the row's first block in the concatenated stream
+    int ch;             // chunk that holds the segment (-1: whole-row mode)
+};
+
+// Walks the ranges of one warp (chunks w, w+W, ... or rows w, w+W, ...) and
+// cuts them into segments at row boundaries.
+struct SegIter {
+    int k;
+    int64_t f, fend;
+    int ch;
+    bool done;
+};
+
+// Consecutive table entries of one segment, read 32 at a time (lane l holds
+// entry o + l as a TMA row coordinate, -2 for a block id outside the pool).
+struct Win {
+    Seg sg;
+    int o, n;
+    bool valid;
 };
 
 // Physical address of the 16-byte chunk `chunk` (0 .. D/8-1) of row `row`
@@ -139,77 +161,148 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+template <int N> struct FVec;
+template <> struct FVec<4> {
+    using type = float4;
+    static __device__ __forceinline__ float4 ld(const float *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
+    static __device__ __forceinline__ void fma(float (&a)[4], float w, float4 v) {
+        a[0] = fmaf(w, v.x, a[0]); a[1] = fmaf(w, v.y, a[1]); a[2] = fmaf(w, v.z, a[2]); a[3] = fmaf(w, v.w, a[3]);
+    }
+};
+template <> struct FVec<2> {
+    using type = float2;
+    static __device__ __forceinline__ float2 ld(const float *p) { return __ldcg(reinterpret_cast<const float2 *>(p)); }
+    static __device__ __forceinline__ void fma(float (&a)[2], float w, float2 v) {
+        a[0] = fmaf(w, v.x, a[0]); a[1] = fmaf(w, v.y, a[1]);
+    }
+};
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                         const __grid_constant__ CUtensorMap tmV,
                                                         const DecodeArgs a) {
     using C = TcCfg<D>;
     constexpr int NW = C::NW, S = C::S;
+    constexpr bool SPLIT_P = sizeof(T) == 2 && !std::is_same<T, __half>::value;  // bf16: P = hi + lo
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
-    int *blk_ids = reinterpret_cast<int *>(smem + C::BLK_OFF);
+    int *stage_ok = reinterpret_cast<int *>(smem + C::OK_OFF);
     int *cum = reinterpret_cast<int *>(smem + C::CUM_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int B = a.B;
-    const int P = a.part;  // > 0: partition size; 0: one partition per sequence
+    const int B = a.B, Hkv = a.Hkv;
 
-    // ---- partitions per sequence -> exclusive prefix sum in cum[0..B] ------------
+    // ---- blocks per sequence -> exclusive prefix sum cum[0..B] ------------------------
+    auto eff_len = [&](int b) { return min(min(a.lens[b], a.max_len), a.mbps * kBlockSize); };
     {
         __shared__ int wsum[NW];
         const int per = (B + C::THREADS - 1) / C::THREADS;
         const int lo = min(B, tid * per), hi = min(B, lo + per);
         int s = 0;
         for (int b = lo; b < hi; ++b) {
-            int L = min(min(a.lens[b], a.max_len), a.mbps * kBlockSize);
-            s += (L <= 0 || P == 0) ? 1 : (L + P - 1) / P;
+            const int L = eff_len(b);
+            s += L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
         }
         int x = s;  // inclusive warp scan
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int y = __shfl_up_sync(0xffffffffu, x, o);
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
         if (lane == 31) wsum[warp] = x;
         __syncthreads();
-        int base = 0;
-        for (int w = 0; w < warp; ++w) base += wsum[w];
-        int run = base + x - s;
+        int run = x - s;
+        for (int w = 0; w < warp; ++w) run += wsum[w];
         for (int b = lo; b < hi; ++b) {
             cum[b] = run;
-            int L = min(min(a.lens[b], a.max_len), a.mbps * kBlockSize);
-            run += (L <= 0 || P == 0) ? 1 : (L + P - 1) / P;
+            const int L = eff_len(b);
+            run += L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
         }
         if (tid == C::THREADS - 1) cum[B] = run;
         __syncthreads();
     }
-    const int total_items = cum[B] * a.Hkv;
+    const int64_t total = (int64_t)cum[B] * Hkv;  // blocks of all rows
+    const int gw = blockIdx.x * NW + warp;
+    const int W = gridDim.x * NW;
+    const bool rows_mode = a.tc_chunk < 0;
+    int64_t cb = 1;  // blocks per chunk
+    if (!rows_mode) {
+        const int64_t wc = min(W, kTcMaxChunks);
+        const int64_t bal = (total + wc - 1) / wc;
+        cb = a.tc_chunk > 0 ? a.tc_chunk : (bal > kTcMinChunk ? bal : kTcMinChunk);
+    }
+    const int64_t nchunks = rows_mode ? 0 : (total + cb - 1) / cb;
 
-    auto item_at = [&](int it) -> Item {
-        Item r;
-        const int u = it / a.Hkv;
-        r.kvh = it - u * a.Hkv;
-        int lo = 0, hi = B;  // largest b with cum[b] <= u
+    // rows of sequences with no token produce zeros
+    for (int r = gw; r < B * Hkv; r += W) {
+        const int b = r / Hkv;
+        if (cum[b + 1] == cum[b]) {
+            T *o = reinterpret_cast<T *>(a.out) + ((size_t)b * a.Hq + (size_t)(r % Hkv) * G) * D;
+            for (int i = lane; i < G * D; i += 32) o[i] = Cvt<T>::from_f(0.f);
+        }
+    }
+
+    auto locate = [&](int64_t f, Seg &sg) {
+        int lo = 0, hi = B;  // largest b with cum[b] * Hkv <= f
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (cum[mid] <= u) lo = mid; else hi = mid;
+            if ((int64_t)cum[mid] * Hkv <= f) lo = mid; else hi = mid;
         }
-        r.b = lo;
-        r.part = u - cum[lo];
-        r.L = min(min(a.lens[lo], a.max_len), a.mbps * kBlockSize);
-        const int Pe = P > 0 ? P : max(r.L, 1);
-        r.t0 = r.part * Pe;
-        const int t1 = min(r.L, r.t0 + Pe);
-        r.nblk = r.L > 0 ? (t1 - r.t0 + kBlockSize - 1) / kBlockSize : 0;
-        r.ntok_last = r.L > 0 ? t1 - r.t0 - (r.nblk - 1) * kBlockSize : 0;
-        r.nparts = r.L > 0 ? (r.L + Pe - 1) / Pe : 1;
-        return r;
+        sg.b = lo;
+        sg.nb = cum[lo + 1] - cum[lo];
+        const int64_t off = f - (int64_t)cum[lo] * Hkv;
+        sg.kvh = (int)(off / sg.nb);
+        sg.j0 = (int)(off - (int64_t)sg.kvh * sg.nb);
+        sg.fr = (int64_t)cum[lo] * Hkv + (int64_t)sg.kvh * sg.nb;
+        sg.L = eff_len(lo);
+    };
+    auto range = [&](SegIter &it) -> bool {
+        if (rows_mode) {
+            for (;; ++it.k) {
+                const int64_t r = (int64_t)gw + (int64_t)it.k * W;
+                if (r >= (int64_t)B * Hkv) return false;
+                const int b = (int)(r / Hkv), kvh = (int)(r % Hkv);
+                const int nb = cum[b + 1] - cum[b];
+                if (nb > 0) {
+                    it.f = (int64_t)cum[b] * Hkv + (int64_t)kvh * nb;
+                    it.fend = it.f + nb;
+                    it.ch = -1;
+                    return true;
+                }
+            }
+        }
+        const int64_t ch = (int64_t)gw + (int64_t)it.k * W;
+        if (ch >= nchunks) return false;
+        it.f = ch * cb;
+        it.fend = min(total, it.f + cb);
+        it.ch = (int)ch;
+        return true;
+    };
+    auto it_init = [&](SegIter &it) {
+        it.k = 0;
+        it.done = !range(it);
+    };
+    auto next_seg = [&](SegIter &it, Seg &sg) -> bool {
+        if (it.done) return false;
+        if (it.f >= it.fend) {
+            ++it.k;
+            if (!range(it)) {
+                it.done = true;
+                return false;
+            }
+        }
+        locate(it.f, sg);
+        const int64_t end = min(it.fend, sg.fr + sg.nb);
+        sg.j1 = sg.j0 + (int)(end - it.f);
+        sg.ch = it.ch;
+        it.f = end;
+        return true;
     };
 
     uint64_t *my_bars = bars + warp * S;
-    int *my_blk = blk_ids + warp * S;
+    int *my_ok = stage_ok + warp * S;
     const uint32_t ring = smem_addr(smem) + warp * S * C::STAGE;
     if (lane == 0) {
 #pragma unroll
@@ -218,94 +311,117 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
     }
     __syncwarp();
 
-    const int gw = blockIdx.x * NW + warp;
-    const int W = gridDim.x * NW;
-
-    // ---- producer: the warp's stream of blocks, S blocks ahead of the consumer ----
-    // Lane l holds table entry (p_j & ~31) + l of the producer's item: a
-    // coalesced load of 32 entries, read out with a shuffle per block.
-    int p_item = gw, p_j = 0, p_k = 0, p_tab = -1;
-    Item pi{};
-    auto p_load_tab = [&]() {
-        const int idx = (p_j & ~31) + lane;
-        p_tab = idx < pi.nblk ? a.tables[(size_t)pi.b * a.mbps + pi.t0 / kBlockSize + idx] : -1;
-    };
-    auto p_enter = [&]() {  // position the producer on the next item that has blocks
-        while (p_item < total_items) {
-            pi = item_at(p_item);
-            if (pi.nblk > 0) break;
-            p_item += W;
+    // ---- producer: TMA for the warp's block stream, S blocks ahead of the consumer ----
+    SegIter pit;
+    it_init(pit);
+    auto win_first = [&](Win &w) {
+        Seg sg;
+        w.valid = next_seg(pit, sg);
+        if (w.valid) {
+            w.sg = sg;
+            w.o = 0;
+            w.n = min(32, sg.j1 - sg.j0);
         }
-        if (p_item < total_items) p_load_tab();
     };
-    p_enter();
+    auto win_after = [&](const Win &cur, Win &w) {
+        if (!cur.valid) {
+            w.valid = false;
+            return;
+        }
+        const int len = cur.sg.j1 - cur.sg.j0;
+        if (cur.o + 32 < len) {
+            w = cur;
+            w.o = cur.o + 32;
+            w.n = min(32, len - w.o);
+        } else {
+            win_first(w);
+        }
+    };
+    auto win_load = [&](const Win &w) -> int {
+        if (!w.valid || lane >= w.n) return -1;
+        const int pb = a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
+        if (pb < 0 || (int64_t)pb >= a.N) return -2;
+        return (pb * Hkv + w.sg.kvh) * kBlockSize;
+    };
+    Win pc, pn;
+    win_first(pc);
+    win_after(pc, pn);
+    int p_y = win_load(pc), p_y_next = win_load(pn);
+    int p_i = 0, p_k = 0;
     auto refill = [&]() {
-        if (p_item >= total_items) return;
-        const int pb = __shfl_sync(0xffffffffu, p_tab, p_j & 31);
+        if (!pc.valid) return;
+        const int y = __shfl_sync(0xffffffffu, p_y, p_i);
         if (lane == 0) {
             const int s = p_k % S;
             uint64_t *bar = &my_bars[s];
-            if (pb < 0 || (int64_t)pb >= a.N) {
-                my_blk[s] = -1;
+            if (y < 0) {
+                my_ok[s] = 0;
                 raise_flag(PA_EFLAG_BAD_BLOCK);
                 mbar_arrive(bar);
             } else {
-                my_blk[s] = pb;
+                my_ok[s] = 1;
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, C::STAGE);
-                const int row = (pb * a.Hkv + pi.kvh) * kBlockSize;
                 const uint32_t dst = ring + s * C::STAGE;
 #pragma unroll
                 for (int bx = 0; bx < C::BOXES; ++bx) {
-                    tma_load_2d(dst + bx * C::BOX_BYTES, &tmK, bx * 64, row, smem_addr(bar));
-                    tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * 64, row, smem_addr(bar));
+                    tma_load_2d(dst + bx * C::BOX_BYTES, &tmK, bx * 64, y, smem_addr(bar));
+                    tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * 64, y, smem_addr(bar));
                 }
             }
         }
         ++p_k;
-        if (++p_j == pi.nblk) {
-            p_j = 0;
-            p_item += W;
-            p_enter();
-        } else if ((p_j & 31) == 0) {
-            p_load_tab();
+        if (++p_i == pc.n) {
+            p_i = 0;
+            pc = pn;
+            p_y = p_y_next;
+            win_after(pc, pn);
+            p_y_next = win_load(pn);
         }
     };
 #pragma unroll
     for (int i = 0; i < S; ++i) refill();
 
+    // ---- consumer ------------------------------------------------------------------------
     const int g = lane >> 2, c = lane & 3;  // mma fragment coordinates
-    const int h0 = 2 * c, h1 = 2 * c + 1;  // the two heads of this thread's S^T / O^T columns
-    int c_k = 0;
-    bool alive = true;
-
-    for (int it = gw; it < total_items && alive; it += W) {
-        const Item ci = item_at(it);
-        T *out = reinterpret_cast<T *>(a.out) + ((size_t)ci.b * a.Hq + (size_t)ci.kvh * G) * D;
-        if (ci.L <= 0) {
-            for (int i = lane; i < G * D; i += 32) out[i] = Cvt<T>::from_f(0.f);
-            continue;
-        }
-        // B fragments of Q^T: k = dims, n = heads (rows >= G are zero padding)
-        uint32_t bq[C::KSTEPS][2];
-        {
-            const T *qp = reinterpret_cast<const T *>(a.q) + ((size_t)ci.b * a.Hq + (size_t)ci.kvh * G) * D;
+    const int h0 = 2 * c, h1 = 2 * c + 1;  // heads of this thread's S^T / O^T columns
+    auto load_q = [&](const Seg &sg, uint32_t (&bq)[C::KSTEPS][2]) {
+        const T *qp = reinterpret_cast<const T *>(a.q) + ((size_t)sg.b * a.Hq + (size_t)sg.kvh * G) * D;
 #pragma unroll
-            for (int s = 0; s < C::KSTEPS; ++s) {
-                if (g < G) {
-                    bq[s][0] = *reinterpret_cast<const uint32_t *>(qp + g * D + 16 * s + 2 * c);
-                    bq[s][1] = *reinterpret_cast<const uint32_t *>(qp + g * D + 16 * s + 2 * c + 8);
-                } else {
-                    bq[s][0] = bq[s][1] = 0u;
-                }
+        for (int s = 0; s < C::KSTEPS; ++s) {
+            if (g < G) {
+                bq[s][0] = *reinterpret_cast<const uint32_t *>(qp + g * D + 16 * s + 2 * c);
+                bq[s][1] = *reinterpret_cast<const uint32_t *>(qp + g * D + 16 * s + 2 * c + 8);
+            } else {
+                bq[s][0] = bq[s][1] = 0u;
             }
         }
+    };
+
+    SegIter cit;
+    it_init(cit);
+    Seg cs;
+    bool have = next_seg(cit, cs);
+    uint32_t bq[C::KSTEPS][2];
+    if (have) load_q(cs, bq);
+    int c_k = 0;
+    while (have) {
+        // the next segment's q is fetched now and lands while this one runs
+        SegIter nit = cit;
+        Seg ns;
+        const bool have_next = next_seg(nit, ns);
+        uint32_t bqn[C::KSTEPS][2];
+        if (have_next) load_q(ns, bqn);
+
+        const int len = cs.j1 - cs.j0;
+        const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;  // tokens in the row's last block
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         float o[C::MTILES][4];
 #pragma unroll
         for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
-        for (int j = 0; j < ci.nblk; ++j) {
+        bool alive = true;
+        for (int j = 0; j < len; ++j) {
             const int s = c_k % S;
             const uint32_t parity = (c_k / S) & 1;
             int ok = lane == 0 ? (int)mbar_wait(&my_bars[s], parity) : 0;
@@ -315,20 +431,19 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
                 break;
             }
             if (lane != 0) mbar_wait(&my_bars[s], parity);
-            const int pb = my_blk[s];
-            const int ntok = (j == ci.nblk - 1) ? ci.ntok_last : kBlockSize;
+            const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
             const uint32_t tK = ring + s * C::STAGE;
             const uint32_t tV = tK + C::TILE;
-            if (pb >= 0) {
+            if (my_ok[s]) {
                 if (ntok < kBlockSize) {
                     // rows past the sequence end hold stale data (possibly NaN/Inf):
                     // zero those V rows so that 0-probability tokens add exactly 0
-                    unsigned char *vrow = smem + (tV - smem_addr(smem));
+                    unsigned char *vt = smem + (tV - smem_addr(smem));
                     const int nrow = kBlockSize - ntok;
                     for (int i = lane; i < nrow * C::BOXES * 8; i += 32) {
                         const int r = ntok + i / (C::BOXES * 8);
                         const int rem = i % (C::BOXES * 8);
-                        *reinterpret_cast<uint4 *>(vrow + (rem >> 3) * 2048 + r * 128 + (rem & 7) * 16) =
+                        *reinterpret_cast<uint4 *>(vt + (rem >> 3) * C::BOX_BYTES + r * 128 + (rem & 7) * 16) =
                             make_uint4(0, 0, 0, 0);
                     }
                     fence_proxy_async_smem();  // before the stage is refilled by TMA
@@ -340,12 +455,10 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
                 for (int ks = 0; ks < C::KSTEPS; ++ks) {
                     uint32_t af[4];
                     const int mi = lane >> 3, r = lane & 7;
-                    const int row = r + ((mi & 1) << 3);
-                    const int chunk = 2 * ks + (mi >> 1);
-                    ldsm_x4(af, tile_chunk(tK, row, chunk));
+                    ldsm_x4(af, tile_chunk(tK, r + ((mi & 1) << 3), 2 * ks + (mi >> 1)));
                     Mma<T>::mma(sc, af, bq[ks][0], bq[ks][1]);
                 }
-                // ---- online softmax (log2 domain); rows g and g+8 are tokens, columns heads
+                // ---- online softmax (log2 domain): rows g, g+8 are tokens, columns heads
                 const bool v0 = g < ntok, v1 = g + 8 < ntok;
                 const float s0 = v0 ? sc[0] * a.scale_log2 : -INFINITY;
                 const float s1 = v0 ? sc[1] * a.scale_log2 : -INFINITY;
@@ -374,18 +487,27 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
                         o[i][3] *= al1;
                     }
                 }
-                // ---- P^T fragments (k = tokens, n = heads) by transposing the S^T layout
-                const uint32_t pb0 = movm_t(Mma<T>::pack(p0, p1));  // tokens 0-7
-                const uint32_t pb1 = movm_t(Mma<T>::pack(p2, p3));  // tokens 8-15
+                // ---- P^T fragments (k = tokens, n = heads): transpose the S^T layout
+                const uint32_t ph01 = Mma<T>::pack(p0, p1), ph23 = Mma<T>::pack(p2, p3);
+                const uint32_t pb0 = movm_t(ph01);  // tokens 0-7
+                const uint32_t pb1 = movm_t(ph23);  // tokens 8-15
+                uint32_t pl0 = 0, pl1 = 0;
+                if constexpr (SPLIT_P) {
+                    // bf16 keeps 8 significant bits; the remainder p - hi goes in a second
+                    // bf16 operand so that P enters the product to ~16 bits
+                    const float r0 = __uint_as_float(ph01 << 16), r1 = __uint_as_float(ph01 & 0xffff0000u);
+                    const float r2 = __uint_as_float(ph23 << 16), r3 = __uint_as_float(ph23 & 0xffff0000u);
+                    pl0 = movm_t(Mma<T>::pack(p0 - r0, p1 - r1));
+                    pl1 = movm_t(Mma<T>::pack(p2 - r2, p3 - r3));
+                }
                 // ---- O^T += V^T . P^T
 #pragma unroll
                 for (int i = 0; i < C::MTILES; ++i) {
                     uint32_t af[4];
                     const int mi = lane >> 3, r = lane & 7;
-                    const int row = r + ((mi >> 1) << 3);
-                    const int chunk = 2 * i + (mi & 1);
-                    ldsm_x4_t(af, tile_chunk(tV, row, chunk));
+                    ldsm_x4_t(af, tile_chunk(tV, r + ((mi >> 1) << 3), 2 * i + (mi & 1)));
                     Mma<T>::mma(o[i], af, pb0, pb1);
+                    if constexpr (SPLIT_P) Mma<T>::mma(o[i], af, pl0, pl1);
                 }
             }
             __syncwarp();
@@ -394,14 +516,15 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
         }
         if (!alive) break;
 
-        // ---- finish the item
+        // ---- finish the segment
 #pragma unroll
         for (int msk = 4; msk < 32; msk <<= 1) {
             l0 += __shfl_xor_sync(0xffffffffu, l0, msk);
             l1 += __shfl_xor_sync(0xffffffffu, l1, msk);
         }
         const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-        if (ci.nparts == 1) {
+        T *out = reinterpret_cast<T *>(a.out) + ((size_t)cs.b * a.Hq + (size_t)cs.kvh * G) * D;
+        if (cs.j0 == 0 && cs.j1 == cs.nb) {  // the whole row: final output
 #pragma unroll
             for (int i = 0; i < C::MTILES; ++i) {
                 const int d0 = 16 * i + g, d1 = d0 + 8;
@@ -414,54 +537,84 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
                     out[h1 * D + d1] = Cvt<T>::from_f(o[i][3] * inv1);
                 }
             }
-            continue;
-        }
-        const size_t row0 = ((size_t)ci.b * a.Hq + (size_t)ci.kvh * G) * a.max_parts;
+        } else {
+            // Partial of a row cut by chunk boundaries: chunk ch holds at most two
+            // partial segments, its first (slot 2ch) and its last (slot 2ch+1).
+            const int64_t ch_first = cs.fr / cb, ch_last = (cs.fr + cs.nb - 1) / cb;
+            auto slot_of = [&](int64_t ch) -> int64_t {
+                return 2 * ch + ((ch == ch_first && cs.fr > ch * cb) ? 1 : 0);
+            };
+            const int64_t sl = slot_of(cs.ch);
 #pragma unroll
-        for (int i = 0; i < C::MTILES; ++i) {
-            const int d0 = 16 * i + g, d1 = d0 + 8;
-            if (h0 < G) {
-                float *w = a.ws_o + (row0 + (size_t)h0 * a.max_parts + ci.part) * D;
-                w[d0] = o[i][0] * inv0;
-                w[d1] = o[i][2] * inv0;
+            for (int i = 0; i < C::MTILES; ++i) {
+                const int d0 = 16 * i + g, d1 = d0 + 8;
+                if (h0 < G) {
+                    float *w = a.ws_o + (sl * G + h0) * D;
+                    w[d0] = o[i][0] * inv0;
+                    w[d1] = o[i][2] * inv0;
+                }
+                if (h1 < G) {
+                    float *w = a.ws_o + (sl * G + h1) * D;
+                    w[d0] = o[i][1] * inv1;
+                    w[d1] = o[i][3] * inv1;
+                }
             }
-            if (h1 < G) {
-                float *w = a.ws_o + (row0 + (size_t)h1 * a.max_parts + ci.part) * D;
-                w[d0] = o[i][1] * inv1;
-                w[d1] = o[i][3] * inv1;
+            if (g == 0) {
+                if (h0 < G) a.ws_lse[sl * G + h0] = m0 + log2f(l0);
+                if (h1 < G) a.ws_lse[sl * G + h1] = m1 + log2f(l1);
+            }
+            __threadfence();
+            __syncwarp();
+            int *ticket = a.counters + (size_t)cs.b * Hkv + cs.kvh;
+            int old = 0;
+            if (lane == 0) old = atomicAdd(ticket, 1);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            const int nseg = (int)(ch_last - ch_first + 1);
+            if (old == nseg - 1) {
+                // last segment of the row to finish: merge all of them
+                //   out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M)
+                __threadfence();
+                using V = FVec<C::DPL>;
+                for (int h = 0; h < G; ++h) {
+                    float M = -INFINITY;
+                    for (int i = lane; i < nseg; i += 32) M = fmaxf(M, __ldcg(a.ws_lse + slot_of(ch_first + i) * G + h));
+                    M = warp_max(M);
+                    float acc[C::DPL];
+#pragma unroll
+                    for (int e = 0; e < C::DPL; ++e) acc[e] = 0.f;
+                    float wpart = 0.f;
+                    for (int i0 = 0; i0 < nseg; i0 += 32) {
+                        const int i = i0 + lane;
+                        float wl = 0.f;
+                        int64_t sll = 0;
+                        if (i < nseg) {
+                            sll = slot_of(ch_first + i);
+                            wl = fast_exp2(__ldcg(a.ws_lse + sll * G + h) - M);
+                        }
+                        wpart += wl;
+                        const int cnt = min(32, nseg - i0);
+#pragma unroll 4
+                        for (int t = 0; t < cnt; ++t) {
+                            const float w = __shfl_sync(0xffffffffu, wl, t);
+                            const int64_t st = __shfl_sync(0xffffffffu, sll, t);
+                            V::fma(acc, w, V::ld(a.ws_o + (st * G + h) * D + lane * C::DPL));
+                        }
+                    }
+                    const float inv = 1.f / warp_sum(wpart);
+#pragma unroll
+                    for (int e = 0; e < C::DPL; ++e) out[h * D + lane * C::DPL + e] = Cvt<T>::from_f(acc[e] * inv);
+                }
+                if (lane == 0) *ticket = 0;  // the workspace is left as it was found
             }
         }
-        if (g == 0) {
-            if (h0 < G) a.ws_lse[row0 + (size_t)h0 * a.max_parts + ci.part] = m0 + log2f(l0);
-            if (h1 < G) a.ws_lse[row0 + (size_t)h1 * a.max_parts + ci.part] = m1 + log2f(l1);
+        cit = nit;
+        cs = ns;
+        have = have_next;
+#pragma unroll
+        for (int s = 0; s < C::KSTEPS; ++s) {
+            bq[s][0] = bqn[s][0];
+            bq[s][1] = bqn[s][1];
         }
-        __threadfence();
-        __syncwarp();
-        int *ticket = a.counters + (size_t)ci.b * a.Hkv + ci.kvh;
-        int old = 0;
-        if (lane == 0) old = atomicAdd(ticket, 1);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old != ci.nparts - 1) continue;
-        // ---- last partition of (b, kvh): merge every partition of its G heads
-        __threadfence();
-        for (int h = 0; h < G; ++h) {
-            const float *lse = a.ws_lse + row0 + (size_t)h * a.max_parts;
-            const float *op = a.ws_o + (row0 + (size_t)h * a.max_parts) * D;
-            float M = -INFINITY;
-            for (int p = lane; p < ci.nparts; p += 32) M = fmaxf(M, __ldcg(lse + p));
-            M = warp_max(M);
-            float Ssum = 0.f;
-            for (int p = lane; p < ci.nparts; p += 32) Ssum += fast_exp2(__ldcg(lse + p) - M);
-            Ssum = warp_sum(Ssum);
-            const float inv = 1.f / Ssum;
-            for (int d = lane; d < D; d += 32) {
-                float acc = 0.f;
-                for (int p = 0; p < ci.nparts; ++p)
-                    acc = fmaf(fast_exp2(__ldcg(lse + p) - M), __ldcg(op + (size_t)p * D + d), acc);
-                out[h * D + d] = Cvt<T>::from_f(acc * inv);
-            }
-        }
-        if (lane == 0) *ticket = 0;  // the workspace is left as it was found
     }
 }
 
@@ -527,7 +680,7 @@ static bool cache_tensor_map(CUtensorMap *m, const void *base, int64_t rows, int
 
 bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
     return (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype && (D == 64 || D == 128) &&
-           (G == 1 || G == 2 || G == 4 || G == 8) && B <= TcCfg<128>::MAX_B;
+           (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
 }
 
 template <typename T, int D, int G>
@@ -535,7 +688,7 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     using C = TcCfg<D>;
     auto kern = decode_tc_kernel<T, D, G>;
     const int smem = C::smem_bytes(a.B);
-    if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(C::MAX_B))) return PA_ERR_CUDA;
+    if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
     CUtensorMap tk, tv;
     const int64_t rows = a.N * a.Hkv * kBlockSize;
     if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
@@ -546,11 +699,11 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::THREADS, smem) != cudaSuccess)
         return PA_ERR_CUDA;
     per_sm = per_sm < 1 ? 1 : per_sm;
-    // an upper bound on the items: every sequence at max_len
-    const int64_t parts = a.part > 0 ? a.max_parts : 1;
-    const int64_t items = (int64_t)a.B * a.Hkv * parts;
+    // persistent grid: every resident warp is a worker, but no more warps than
+    // there are blocks to read (every sequence at max_len)
+    const int64_t blocks = (int64_t)a.B * a.Hkv * ((a.max_len + kBlockSize - 1) / kBlockSize);
     int64_t ctas = (int64_t)sms * per_sm;
-    const int64_t need = (items + C::NW - 1) / C::NW;
+    const int64_t need = (blocks + C::NW - 1) / C::NW;
     if (need < ctas) ctas = need;
     if (ctas < 1) ctas = 1;
     kern<<<(unsigned)ctas, C::THREADS, smem, st>>>(tk, tv, a);

@@ -44,7 +44,16 @@ struct DecodeArgs {
     float *ws_o;             // [B][Hq][max_parts][D]
     float *ws_lse;           // [B][Hq][max_parts]  (log2 domain)
     int *counters;           // [B][Hkv] merge tickets, zero between calls
+    int tc_chunk;            // tensor-core schedule: blocks per chunk, 0 = balanced auto,
+                             // -1 = whole rows (one pass)
 };
+
+// Tensor-core schedule limits: the auto schedule cuts the block stream into at
+// most kTcMaxChunks chunks of at least kTcMinChunk blocks; the per-CTA prefix
+// sum holds at most kTcMaxB sequences.
+constexpr int kTcMaxChunks = 2048;
+constexpr int kTcMinChunk = 4;
+constexpr int kTcMaxB = 4096;
 
 // Per-translation-unit error words (see PA_ERROR_WORD_ACCESSOR).
 int error_word_cache_ops(unsigned int *flags, bool reset);

@@ -83,22 +83,35 @@ def test_decode_null_and_workspace_checks():
     p = params(kv_dtype=pa.PA_I8)  # int8 without scales
     rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
     assert rc == pa.PA_ERR_NULL
-    p = params(partition_size=16)  # split-K without a workspace
+    p = params(partition_size=16, algo=pa.PA_ALGO_SIMT)  # split-K without a workspace
     need = pa.lib.pa_decode_workspace_size(ctypes.byref(p))
-    # 2 seqs x 8 heads x 4 partitions x 128 floats, their 64 lse floats and
-    # 2 x 2 merge counters, each region rounded up to 256 B
+    # CUDA-core family: 2 seqs x 8 heads x 4 partitions x 128 floats, their 64 lse
+    # floats and 2 x 2 merge counters, each region rounded up to 256 B
     assert need == 2 * 8 * 4 * 128 * 4 + 256 + 256
     rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
     assert rc == pa.PA_ERR_WORKSPACE
     p.workspace, p.workspace_bytes = 0x1000, need - 1
     rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
     assert rc == pa.PA_ERR_WORKSPACE
+    # tensor-core family: 2 x 2 rows x 4 blocks = 16 blocks in chunks of 1 block ->
+    # 32 partial slots of 4 heads x (128 + 1) floats, plus the counters
+    p = params(partition_size=16, algo=pa.PA_ALGO_TENSOR)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == 32 * 4 * 128 * 4 + 512 + 256
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(params(partition_size=0, algo=pa.PA_ALGO_TENSOR))) == 0
+    # auto partitioning on the tensor-core family: at most 2048 chunks
+    p = params(partition_size=-1, algo=pa.PA_ALGO_TENSOR, num_seqs=64, max_blocks_per_seq=264,
+               max_seq_len=4224)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == 4096 * 4 * 128 * 4 + 4096 * 4 * 4 + 512
+    # the tensor-core family needs fp16/bf16 q and cache
+    p = params(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32, algo=pa.PA_ALGO_TENSOR)
+    assert pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p),
+                            None) == pa.PA_ERR_UNSUPPORTED
     p = params()
     rc = pa.lib.pa_decode(FAKE, FAKE, ctypes.c_void_p(0x1008), FAKE, FAKE, FAKE, ctypes.c_float(0.1),
                           ctypes.byref(p), None)
     assert rc == pa.PA_ERR_ALIGN
-    # a partition as long as the longest sequence needs no workspace
-    assert pa.lib.pa_decode_workspace_size(ctypes.byref(params(partition_size=64))) == 0
+    # a partition as long as the longest sequence needs no workspace (CUDA-core family)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(params(partition_size=64, algo=pa.PA_ALGO_SIMT))) == 0
     # empty batch is a no-op
     assert pa.lib.pa_decode(None, None, None, None, None, None, ctypes.c_float(0.1),
                             ctypes.byref(params(num_seqs=0)), None) == pa.PA_OK
