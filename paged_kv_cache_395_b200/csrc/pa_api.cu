@@ -119,13 +119,16 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
         pl->tc_chunk = p->partition_size / PA_BLOCK_SIZE;
         nchunks = (tmax + pl->tc_chunk - 1) / pl->tc_chunk;
     } else {
+        // guided schedule: at most kTcMaxChunks static chunks and twice as many claimed ones
         pl->tc_chunk = 0;
-        nchunks = tmax < kTcMaxChunks ? tmax : kTcMaxChunks;
+        nchunks = tmax < 3 * (int64_t)kTcMaxChunks + 1 ? tmax : 3 * (int64_t)kTcMaxChunks + 1;
     }
     pl->tc_slots = 2 * nchunks;
+    // partial outputs and lse of two segments per chunk, then one merge ticket
+    // per (sequence, KV head) row and the chunk-claim and finished-warp counters
     pl->bytes = up256((size_t)pl->tc_slots * G * p->head_dim * sizeof(float)) +
                 up256((size_t)pl->tc_slots * G * sizeof(float)) +
-                up256((size_t)p->num_seqs * p->num_kv_heads * sizeof(int));
+                up256(((size_t)p->num_seqs * p->num_kv_heads + 2) * sizeof(int));
     return PA_OK;
 }
 
@@ -238,6 +241,14 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     a.q_dtype = p->q_dtype;
     a.kv_dtype = p->kv_dtype;
     char *ws = reinterpret_cast<char *>(p->workspace);
+    if (pl.tc && (uintptr_t)q % 16) {
+        if (p->algo == PA_ALGO_TENSOR) return PA_ERR_ALIGN;
+        // the tensor-core family reads q rows with 16-byte bulk copies; a q that is not
+        // 16-byte aligned goes to the CUDA-core family, which needs its own plan
+        pa_decode_params p2 = *p;
+        p2.algo = PA_ALGO_SIMT;
+        return pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, &p2, stream);
+    }
     if (pl.tc) {
         a.part = 0;
         a.max_parts = 1;

@@ -198,6 +198,14 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Same, with shared-memory addresses given as 32-bit shared-window offsets.
+__device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }

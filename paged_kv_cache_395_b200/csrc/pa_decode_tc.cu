@@ -56,7 +56,7 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
 }
 __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
     uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
     return y;
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
@@ -76,7 +76,7 @@ template <> struct Mma<__half> {
         return r;
     }
     static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-        asm volatile(
+        asm(
             "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
             : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
             : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -89,7 +89,7 @@ template <> struct Mma<__nv_bfloat16> {
         return r;
     }
     static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-        asm volatile(
+        asm(
             "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
             : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
             : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -99,11 +99,18 @@ template <> struct Mma<__nv_bfloat16> {
 // ---------------------------------------------------------------------------
 // configuration
 // ---------------------------------------------------------------------------
+#ifndef PA_TC_WARPS
+#define PA_TC_WARPS 4
+#endif
+#ifndef PA_TC_STAGES
+#define PA_TC_STAGES 3
+#endif
+
 template <int D>
 struct TcCfg {
-    static constexpr int NW = 4;
+    static constexpr int NW = PA_TC_WARPS;        // warps (independent workers) per CTA
     static constexpr int THREADS = NW * 32;
-    static constexpr int S = 3;                   // ring stages per warp
+    static constexpr int S = PA_TC_STAGES;        // ring stages per warp
     static constexpr int BOXES = D / 64;          // 64-element (128-byte) boxes per row
     static constexpr int BOX_BYTES = 16 * 128;    // one box of a tile
     static constexpr int TILE = BOXES * BOX_BYTES;
@@ -114,8 +121,11 @@ struct TcCfg {
     static constexpr int RING = NW * S * STAGE;
     static constexpr int BAR_OFF = RING;
     static constexpr int OK_OFF = BAR_OFF + NW * S * 8;
-    static constexpr int CUM_OFF = OK_OFF + NW * S * 4;
-    static int smem_bytes(int B) { return 1024 + CUM_OFF + (B + 1) * 4; }
+    static constexpr int RQ = 8;                         // per-warp ring of range chunk ids
+    static constexpr int RQ_OFF = OK_OFF + NW * S * 4;
+    static constexpr int CUM_OFF = RQ_OFF + NW * RQ * 4;
+    static_assert(S < RQ, "the producer runs at most S ranges ahead");
+    static int smem_bytes(int B) { return 1024 + CUM_OFF + (2 * B + 2) * 4; }
 };
 
 // One contiguous run of blocks of one (sequence, KV head) row.
@@ -126,11 +136,10 @@ struct Seg {
     int ch;             // chunk that holds the segment (-1: whole-row mode)
 };
 
-// Walks the ranges of one warp (chunks w, w+W, ... or rows w, w+W, ...) and
-// cuts them into segments at row boundaries.
+// Walks the ranges of one warp and cuts them into segments at row boundaries.
 struct SegIter {
-    int k;
-    int64_t f, fend;
+    int k;              // range counter
+    int64_t f, fend;    // position and end in the concatenated stream
     int ch;
     bool done;
 };
@@ -143,11 +152,34 @@ struct Win {
     bool valid;
 };
 
+// Chunk layout of the concatenated block stream (guided schedule): n0 chunks
+// of c0 blocks, one per warp, then chunks of c1 blocks that warps claim in
+// order from a counter.  Uniform chunks when c0 == c1.
+struct Chunks {
+    int64_t total, c0, n0, c1, n;
+    __device__ int64_t start(int64_t ch) const { return ch < n0 ? ch * c0 : n0 * c0 + (ch - n0) * c1; }
+    __device__ int64_t end(int64_t ch) const {
+        const int64_t e = ch < n0 ? (ch + 1) * c0 : n0 * c0 + (ch - n0 + 1) * c1;
+        return e < total ? e : total;
+    }
+    __device__ int64_t of(int64_t f) const { return f < n0 * c0 ? f / c0 : n0 + (f - n0 * c0) / c1; }
+};
+
 // Physical address of the 16-byte chunk `chunk` (0 .. D/8-1) of row `row`
 // (0..15) of a swizzled tile: box = chunk / 8, and inside the 1024-byte
 // aligned box the chunk index is XORed with row % 8 (128-byte swizzle).
 __device__ __forceinline__ uint32_t tile_chunk(uint32_t tile, int row, int chunk) {
     return tile + (chunk >> 3) * 2048 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
+}
+
+// Ticket increment with acquire-release semantics at GPU scope: the warp's
+// partial-result stores (ordered before lane 0 by __syncwarp) are released
+// with it, and the warp that draws the last ticket acquires every other
+// segment's partial.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -165,22 +197,18 @@ template <int N> struct FVec;
 template <> struct FVec<4> {
     using type = float4;
     static __device__ __forceinline__ float4 ld(const float *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
-    static __device__ __forceinline__ void fma(float (&a)[4], float w, float4 v) {
-        a[0] = fmaf(w, v.x, a[0]); a[1] = fmaf(w, v.y, a[1]); a[2] = fmaf(w, v.z, a[2]); a[3] = fmaf(w, v.w, a[3]);
-    }
+    static __device__ __forceinline__ float get(const float4 &v, int e) { return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w; }
 };
 template <> struct FVec<2> {
     using type = float2;
     static __device__ __forceinline__ float2 ld(const float *p) { return __ldcg(reinterpret_cast<const float2 *>(p)); }
-    static __device__ __forceinline__ void fma(float (&a)[2], float w, float2 v) {
-        a[0] = fmaf(w, v.x, a[0]); a[1] = fmaf(w, v.y, a[1]);
-    }
+    static __device__ __forceinline__ float get(const float2 &v, int e) { return e == 0 ? v.x : v.y; }
 };
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                        const __grid_constant__ CUtensorMap tmV,
-                                                        const DecodeArgs a) {
+__global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                     const __grid_constant__ CUtensorMap tmV,
+                                                                     const DecodeArgs a) {
     using C = TcCfg<D>;
     constexpr int NW = C::NW, S = C::S;
     constexpr bool SPLIT_P = sizeof(T) == 2 && !std::is_same<T, __half>::value;  // bf16: P = hi + lo
@@ -189,20 +217,22 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     int *stage_ok = reinterpret_cast<int *>(smem + C::OK_OFF);
-    int *cum = reinterpret_cast<int *>(smem + C::CUM_OFF);
+    int *rq_all = reinterpret_cast<int *>(smem + C::RQ_OFF);
+    int *cum = reinterpret_cast<int *>(smem + C::CUM_OFF);  // [B + 1] blocks before sequence b
+    int *lens = cum + a.B + 1;                                // [B] effective lengths
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = a.B, Hkv = a.Hkv;
 
-    // ---- blocks per sequence -> exclusive prefix sum cum[0..B] ------------------------
-    auto eff_len = [&](int b) { return min(min(a.lens[b], a.max_len), a.mbps * kBlockSize); };
+    // ---- effective lengths and blocks per sequence -> exclusive prefix sum cum[0..B] ----
     {
         __shared__ int wsum[NW];
         const int per = (B + C::THREADS - 1) / C::THREADS;
         const int lo = min(B, tid * per), hi = min(B, lo + per);
         int s = 0;
         for (int b = lo; b < hi; ++b) {
-            const int L = eff_len(b);
+            const int L = min(min(a.lens[b], a.max_len), a.mbps * kBlockSize);
+            lens[b] = L;
             s += L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
         }
         int x = s;  // inclusive warp scan
@@ -217,7 +247,7 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
         for (int w = 0; w < warp; ++w) run += wsum[w];
         for (int b = lo; b < hi; ++b) {
             cum[b] = run;
-            const int L = eff_len(b);
+            const int L = lens[b];
             run += L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
         }
         if (tid == C::THREADS - 1) cum[B] = run;
@@ -227,13 +257,28 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
     const int gw = blockIdx.x * NW + warp;
     const int W = gridDim.x * NW;
     const bool rows_mode = a.tc_chunk < 0;
-    int64_t cb = 1;  // blocks per chunk
+
+    Chunks ck{total, 1, 0, 1, 0};
     if (!rows_mode) {
         const int64_t wc = min(W, kTcMaxChunks);
-        const int64_t bal = (total + wc - 1) / wc;
-        cb = a.tc_chunk > 0 ? a.tc_chunk : (bal > kTcMinChunk ? bal : kTcMinChunk);
+        if (a.tc_chunk > 0) {
+            ck.c0 = ck.c1 = a.tc_chunk;
+        } else {
+            // about 60% of the stream in one static chunk per warp, the rest in
+            // claimed chunks of about a third of a warp's share (guided schedule)
+            const int64_t c0 = (total * 6) / (10 * wc);
+            ck.c0 = c0 > kTcMinChunk ? c0 : kTcMinChunk;
+            const int64_t n0 = min(wc, (total + ck.c0 - 1) / ck.c0);
+            const int64_t rest = total - n0 * ck.c0 > 0 ? total - n0 * ck.c0 : 0;
+            const int64_t c1 = (rest + 2 * wc - 1) / (2 * wc);
+            ck.c1 = c1 > kTcMinChunk ? c1 : kTcMinChunk;
+        }
+        ck.n0 = min((int64_t)min(W, kTcMaxChunks), (total + ck.c0 - 1) / ck.c0);
+        const int64_t rest = total - ck.n0 * ck.c0 > 0 ? total - ck.n0 * ck.c0 : 0;
+        ck.n = ck.n0 + (rest + ck.c1 - 1) / ck.c1;
     }
-    const int64_t nchunks = rows_mode ? 0 : (total + cb - 1) / cb;
+    int *work = a.counters + (size_t)B * Hkv;  // next claimed chunk (minus n0)
+    int *done = work + 1;                       // warps that have finished
 
     // rows of sequences with no token produce zeros
     for (int r = gw; r < B * Hkv; r += W) {
@@ -256,9 +301,40 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
         sg.kvh = (int)(off / sg.nb);
         sg.j0 = (int)(off - (int64_t)sg.kvh * sg.nb);
         sg.fr = (int64_t)cum[lo] * Hkv + (int64_t)sg.kvh * sg.nb;
-        sg.L = eff_len(lo);
+        sg.L = lens[lo];
     };
-    auto range = [&](SegIter &it) -> bool {
+
+    // ---- range schedule: rows w, w+W, ... (one pass) or chunks (static, then claimed)
+    int *rq = rq_all + warp * C::RQ;  // chunk of the warp's range k is rq[k % RQ]
+    // Claims: lane 0 asks the counter for the next chunk as soon as the producer
+    // enters a range; the answer is read only when that range ends, so the
+    // atomic's latency is hidden behind a whole range of copies.
+    int p_claim_raw = 0;
+    bool p_claim_pending = false;
+    auto producer_chunk = [&](int k) -> int {
+        int ch;
+        if (k == 0 && gw < ck.n0) {
+            ch = gw;  // phase 0: one static chunk per warp
+        } else {
+            if (!p_claim_pending && lane == 0) p_claim_raw = atomicAdd(work, 1);
+            const int cl = __shfl_sync(0xffffffffu, p_claim_raw, 0);
+            ch = (int64_t)ck.n0 + cl < ck.n ? (int)(ck.n0 + cl) : -1;
+        }
+        p_claim_pending = false;
+        if (ch >= 0) {
+            if (lane == 0) p_claim_raw = atomicAdd(work, 1);
+            p_claim_pending = true;
+        }
+        if (lane == 0) rq[k % C::RQ] = ch;
+        return ch;
+    };
+    auto set_range = [&](SegIter &it, int64_t ch) {
+        it.f = ck.start(ch);
+        it.fend = ck.end(ch);
+        it.ch = (int)ch;
+    };
+    // producer iterator: claims chunks
+    auto p_range = [&](SegIter &it) -> bool {
         if (rows_mode) {
             for (;; ++it.k) {
                 const int64_t r = (int64_t)gw + (int64_t)it.k * W;
@@ -273,22 +349,37 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
                 }
             }
         }
-        const int64_t ch = (int64_t)gw + (int64_t)it.k * W;
-        if (ch >= nchunks) return false;
-        it.f = ch * cb;
-        it.fend = min(total, it.f + cb);
-        it.ch = (int)ch;
+        const int ch = producer_chunk(it.k);
+        if (ch < 0) return false;
+        set_range(it, ch);
         return true;
     };
-    auto it_init = [&](SegIter &it) {
-        it.k = 0;
-        it.done = !range(it);
+    // consumer iterator: replays the producer's chunks from rq (the producer is ahead)
+    auto c_range = [&](SegIter &it) -> bool {
+        if (rows_mode) {
+            for (;; ++it.k) {
+                const int64_t r = (int64_t)gw + (int64_t)it.k * W;
+                if (r >= (int64_t)B * Hkv) return false;
+                const int b = (int)(r / Hkv), kvh = (int)(r % Hkv);
+                const int nb = cum[b + 1] - cum[b];
+                if (nb > 0) {
+                    it.f = (int64_t)cum[b] * Hkv + (int64_t)kvh * nb;
+                    it.fend = it.f + nb;
+                    it.ch = -1;
+                    return true;
+                }
+            }
+        }
+        const int ch = rq[it.k % C::RQ];
+        if (ch < 0) return false;
+        set_range(it, ch);
+        return true;
     };
-    auto next_seg = [&](SegIter &it, Seg &sg) -> bool {
+    auto next_seg = [&](SegIter &it, Seg &sg, bool producer) -> bool {
         if (it.done) return false;
         if (it.f >= it.fend) {
             ++it.k;
-            if (!range(it)) {
+            if (!(producer ? p_range(it) : c_range(it))) {
                 it.done = true;
                 return false;
             }
@@ -312,11 +403,11 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
     __syncwarp();
 
     // ---- producer: TMA for the warp's block stream, S blocks ahead of the consumer ----
-    SegIter pit;
-    it_init(pit);
+    SegIter pit{0, 0, 0, -1, false};
+    pit.done = !p_range(pit);
     auto win_first = [&](Win &w) {
         Seg sg;
-        w.valid = next_seg(pit, sg);
+        w.valid = next_seg(pit, sg, true);
         if (w.valid) {
             w.sg = sg;
             w.o = 0;
@@ -360,7 +451,6 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
                 mbar_arrive(bar);
             } else {
                 my_ok[s] = 1;
-                fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, C::STAGE);
                 const uint32_t dst = ring + s * C::STAGE;
 #pragma unroll
@@ -381,6 +471,7 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
     };
 #pragma unroll
     for (int i = 0; i < S; ++i) refill();
+    __syncwarp();
 
     // ---- consumer ------------------------------------------------------------------------
     const int g = lane >> 2, c = lane & 3;  // mma fragment coordinates
@@ -398,20 +489,116 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
         }
     };
 
-    SegIter cit;
-    it_init(cit);
+    SegIter cit{0, 0, 0, -1, false};
+    cit.done = !c_range(cit);
     Seg cs;
-    bool have = next_seg(cit, cs);
+    bool have = next_seg(cit, cs, false);
     uint32_t bq[C::KSTEPS][2];
     if (have) load_q(cs, bq);
     int c_k = 0;
-    while (have) {
-        // the next segment's q is fetched now and lands while this one runs
+    bool alive = true;
+    // Pending ticket: the last partial's ticket is read one segment later, so the
+    // atomic's round trip never stalls the warp.
+    int pend_old = 0;
+    bool pend = false;
+    int pend_b = 0, pend_kvh = 0, pend_nb = 0;
+    int64_t pend_fr = 0;
+    auto merge_row = [&](int b, int kvh, int64_t fr, int nb) {
+        // Last segment of the row to finish: merge all of them,
+        //   out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M),
+        // loading the lse values and partial outputs of up to NB segments at once.
+        const int64_t ch_first = ck.of(fr), ch_last = ck.of(fr + nb - 1);
+        const int nseg = (int)(ch_last - ch_first + 1);
+        auto slot_of = [&](int64_t ch) -> int {
+            return (int)(2 * ch + ((ch == ch_first && fr > ck.start(ch)) ? 1 : 0));
+        };
+        T *out = reinterpret_cast<T *>(a.out) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
+        constexpr int NB = 4;  // segments per batch (NB * G <= 32 lanes hold their lse)
+        using V = FVec<C::DPL>;
+        float Mh[G], Sh[G], acc[G][C::DPL];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            Mh[h] = -INFINITY;
+            Sh[h] = 0.f;
+#pragma unroll
+            for (int e = 0; e < C::DPL; ++e) acc[h][e] = 0.f;
+        }
+        for (int i0 = 0; i0 < nseg; i0 += NB) {
+            const int nbat = min(NB, nseg - i0);
+            const int li = lane / G, lh = lane % G;  // lane holds lse of (segment li, head lh)
+            int sl_l = 0;
+            float lse_l = -INFINITY;
+            if (li < nbat) {
+                sl_l = slot_of(ch_first + i0 + li);
+                lse_l = __ldcg(a.ws_lse + (size_t)sl_l * G + lh);
+            }
+            int sls[NB];
+#pragma unroll
+            for (int i = 0; i < NB; ++i) sls[i] = __shfl_sync(0xffffffffu, sl_l, i * G);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                typename V::type v[NB];
+#pragma unroll
+                for (int i = 0; i < NB; ++i)
+                    if (i < nbat) v[i] = V::ld(a.ws_o + ((size_t)sls[i] * G + h) * D + lane * C::DPL);
+                float bm = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < NB; ++i) {
+                    const float x = __shfl_sync(0xffffffffu, lse_l, i * G + h);
+                    if (i < nbat) bm = fmaxf(bm, x);
+                }
+                const float mn = fmaxf(Mh[h], bm);
+                const float f = Mh[h] == -INFINITY ? 0.f : fast_exp2(Mh[h] - mn);
+                Sh[h] *= f;
+#pragma unroll
+                for (int e = 0; e < C::DPL; ++e) acc[h][e] *= f;
+#pragma unroll
+                for (int i = 0; i < NB; ++i) {
+                    const float x = __shfl_sync(0xffffffffu, lse_l, i * G + h);
+                    if (i < nbat) {
+                        const float w = fast_exp2(x - mn);
+                        Sh[h] += w;
+#pragma unroll
+                        for (int e = 0; e < C::DPL; ++e) acc[h][e] = fmaf(w, V::get(v[i], e), acc[h][e]);
+                    }
+                }
+                Mh[h] = mn;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float inv = 1.f / Sh[h];
+#pragma unroll
+            for (int e = 0; e < C::DPL; ++e) out[h * D + lane * C::DPL + e] = Cvt<T>::from_f(acc[h][e] * inv);
+        }
+        if (lane == 0) a.counters[(size_t)b * Hkv + kvh] = 0;  // the workspace is left as it was found
+    };
+    auto resolve = [&]() {
+        if (!pend) return;
+        pend = false;
+        const int old = __shfl_sync(0xffffffffu, pend_old, 0);
+        __syncwarp();
+        const int nseg = (int)(ck.of(pend_fr + pend_nb - 1) - ck.of(pend_fr) + 1);
+        if (old == nseg - 1) merge_row(pend_b, pend_kvh, pend_fr, pend_nb);
+    };
+
+    while (have && alive) {
+        // The next segment's q is fetched early and lands while this one runs: now
+        // when that segment is in the same range or the producer has already claimed
+        // the next range, else as soon as the producer gets there (block loop).
         SegIter nit = cit;
         Seg ns;
-        const bool have_next = next_seg(nit, ns);
+        bool have_next = false, next_known = false;
         uint32_t bqn[C::KSTEPS][2];
-        if (have_next) load_q(ns, bqn);
+        auto try_peek = [&]() {
+            if (next_known || !(cit.f < cit.fend || pit.k > cit.k || pit.done)) return;
+            __syncwarp();  // lane 0 may just have written the next range's chunk to rq
+            next_known = true;
+            nit = cit;
+            have_next = next_seg(nit, ns, false);
+            if (have_next) load_q(ns, bqn);
+        };
+        try_peek();
 
         const int len = cs.j1 - cs.j0;
         const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;  // tokens in the row's last block
@@ -420,7 +607,6 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
 #pragma unroll
         for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
-        bool alive = true;
         for (int j = 0; j < len; ++j) {
             const int s = c_k % S;
             const uint32_t parity = (c_k / S) & 1;
@@ -449,15 +635,24 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
                     fence_proxy_async_smem();  // before the stage is refilled by TMA
                     __syncwarp();
                 }
-                // ---- S^T = K . Q^T
-                float sc[4] = {0.f, 0.f, 0.f, 0.f};
+                // ---- fragments: K (A of S^T), then V^T (A of O^T), all issued up front
+                const int mi = lane >> 3, r8 = lane & 7;
+                uint32_t kf[C::KSTEPS][4], vf[C::MTILES][4];
 #pragma unroll
-                for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                    uint32_t af[4];
-                    const int mi = lane >> 3, r = lane & 7;
-                    ldsm_x4(af, tile_chunk(tK, r + ((mi & 1) << 3), 2 * ks + (mi >> 1)));
-                    Mma<T>::mma(sc, af, bq[ks][0], bq[ks][1]);
-                }
+                for (int ks = 0; ks < C::KSTEPS; ++ks)
+                    ldsm_x4(kf[ks], tile_chunk(tK, r8 + ((mi & 1) << 3), 2 * ks + (mi >> 1)));
+#pragma unroll
+                for (int i = 0; i < C::MTILES; ++i)
+                    ldsm_x4_t(vf[i], tile_chunk(tV, r8 + ((mi >> 1) << 3), 2 * i + (mi & 1)));
+                // ---- S^T = K . Q^T, four independent accumulator chains
+                float sa[4][4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) sa[u][0] = sa[u][1] = sa[u][2] = sa[u][3] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < C::KSTEPS; ++ks) Mma<T>::mma(sa[ks & 3], kf[ks], bq[ks][0], bq[ks][1]);
+                float sc[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[e] = (sa[0][e] + sa[1][e]) + (sa[2][e] + sa[3][e]);
                 // ---- online softmax (log2 domain): rows g, g+8 are tokens, columns heads
                 const bool v0 = g < ntok, v1 = g + 8 < ntok;
                 const float s0 = v0 ? sc[0] * a.scale_log2 : -INFINITY;
@@ -503,18 +698,17 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
                 // ---- O^T += V^T . P^T
 #pragma unroll
                 for (int i = 0; i < C::MTILES; ++i) {
-                    uint32_t af[4];
-                    const int mi = lane >> 3, r = lane & 7;
-                    ldsm_x4_t(af, tile_chunk(tV, r + ((mi >> 1) << 3), 2 * i + (mi & 1)));
-                    Mma<T>::mma(o[i], af, pb0, pb1);
-                    if constexpr (SPLIT_P) Mma<T>::mma(o[i], af, pl0, pl1);
+                    Mma<T>::mma(o[i], vf[i], pb0, pb1);
+                    if constexpr (SPLIT_P) Mma<T>::mma(o[i], vf[i], pl0, pl1);
                 }
             }
             __syncwarp();
             refill();
             ++c_k;
+            try_peek();
         }
         if (!alive) break;
+        try_peek();
 
         // ---- finish the segment
 #pragma unroll
@@ -540,72 +734,42 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
         } else {
             // Partial of a row cut by chunk boundaries: chunk ch holds at most two
             // partial segments, its first (slot 2ch) and its last (slot 2ch+1).
-            const int64_t ch_first = cs.fr / cb, ch_last = (cs.fr + cs.nb - 1) / cb;
-            auto slot_of = [&](int64_t ch) -> int64_t {
-                return 2 * ch + ((ch == ch_first && cs.fr > ch * cb) ? 1 : 0);
+            const int64_t ch_first = ck.of(cs.fr), ch_last = ck.of(cs.fr + cs.nb - 1);
+            auto slot_of = [&](int64_t ch) -> int {
+                return (int)(2 * ch + ((ch == ch_first && cs.fr > ck.start(ch)) ? 1 : 0));
             };
-            const int64_t sl = slot_of(cs.ch);
+            const int sl = slot_of(cs.ch);
 #pragma unroll
             for (int i = 0; i < C::MTILES; ++i) {
                 const int d0 = 16 * i + g, d1 = d0 + 8;
                 if (h0 < G) {
-                    float *w = a.ws_o + (sl * G + h0) * D;
+                    float *w = a.ws_o + ((size_t)sl * G + h0) * D;
                     w[d0] = o[i][0] * inv0;
                     w[d1] = o[i][2] * inv0;
                 }
                 if (h1 < G) {
-                    float *w = a.ws_o + (sl * G + h1) * D;
+                    float *w = a.ws_o + ((size_t)sl * G + h1) * D;
                     w[d0] = o[i][1] * inv1;
                     w[d1] = o[i][3] * inv1;
                 }
             }
             if (g == 0) {
-                if (h0 < G) a.ws_lse[sl * G + h0] = m0 + log2f(l0);
-                if (h1 < G) a.ws_lse[sl * G + h1] = m1 + log2f(l1);
+                if (h0 < G) a.ws_lse[(size_t)sl * G + h0] = m0 + log2f(l0);
+                if (h1 < G) a.ws_lse[(size_t)sl * G + h1] = m1 + log2f(l1);
             }
-            __threadfence();
             __syncwarp();
-            int *ticket = a.counters + (size_t)cs.b * Hkv + cs.kvh;
-            int old = 0;
-            if (lane == 0) old = atomicAdd(ticket, 1);
-            old = __shfl_sync(0xffffffffu, old, 0);
-            const int nseg = (int)(ch_last - ch_first + 1);
-            if (old == nseg - 1) {
-                // last segment of the row to finish: merge all of them
-                //   out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M)
-                __threadfence();
-                using V = FVec<C::DPL>;
-                for (int h = 0; h < G; ++h) {
-                    float M = -INFINITY;
-                    for (int i = lane; i < nseg; i += 32) M = fmaxf(M, __ldcg(a.ws_lse + slot_of(ch_first + i) * G + h));
-                    M = warp_max(M);
-                    float acc[C::DPL];
-#pragma unroll
-                    for (int e = 0; e < C::DPL; ++e) acc[e] = 0.f;
-                    float wpart = 0.f;
-                    for (int i0 = 0; i0 < nseg; i0 += 32) {
-                        const int i = i0 + lane;
-                        float wl = 0.f;
-                        int64_t sll = 0;
-                        if (i < nseg) {
-                            sll = slot_of(ch_first + i);
-                            wl = fast_exp2(__ldcg(a.ws_lse + sll * G + h) - M);
-                        }
-                        wpart += wl;
-                        const int cnt = min(32, nseg - i0);
-#pragma unroll 4
-                        for (int t = 0; t < cnt; ++t) {
-                            const float w = __shfl_sync(0xffffffffu, wl, t);
-                            const int64_t st = __shfl_sync(0xffffffffu, sll, t);
-                            V::fma(acc, w, V::ld(a.ws_o + (st * G + h) * D + lane * C::DPL));
-                        }
-                    }
-                    const float inv = 1.f / warp_sum(wpart);
-#pragma unroll
-                    for (int e = 0; e < C::DPL; ++e) out[h * D + lane * C::DPL + e] = Cvt<T>::from_f(acc[e] * inv);
-                }
-                if (lane == 0) *ticket = 0;  // the workspace is left as it was found
-            }
+            resolve();
+            if (lane == 0) pend_old = atom_add_acq_rel_gpu(a.counters + (size_t)cs.b * Hkv + cs.kvh, 1);
+            pend = true;
+            pend_b = cs.b;
+            pend_kvh = cs.kvh;
+            pend_fr = cs.fr;
+            pend_nb = cs.nb;
+        }
+        if (!next_known) {  // cannot happen once the producer is past this range; kept for safety
+            nit = cit;
+            have_next = next_seg(nit, ns, false);
+            if (have_next) load_q(ns, bqn);
         }
         cit = nit;
         cs = ns;
@@ -614,6 +778,21 @@ __global__ void __launch_bounds__(128) decode_tc_kernel(const __grid_constant__ 
         for (int s = 0; s < C::KSTEPS; ++s) {
             bq[s][0] = bqn[s][0];
             bq[s][1] = bqn[s][1];
+        }
+    }
+    resolve();
+
+    // ---- the last warp to finish puts the chunk counters back to zero
+    if (!rows_mode) {
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence();
+            last = atomicAdd(done, 1) == W - 1;
+            if (last) {
+                *work = 0;
+                *done = 0;
+            }
         }
     }
 }
@@ -689,6 +868,7 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     auto kern = decode_tc_kernel<T, D, G>;
     const int smem = C::smem_bytes(a.B);
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
+    if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are fetched with bulk copies
     CUtensorMap tk, tv;
     const int64_t rows = a.N * a.Hkv * kBlockSize;
     if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
