@@ -119,16 +119,16 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
         pl->tc_chunk = p->partition_size / PA_BLOCK_SIZE;
         nchunks = (tmax + pl->tc_chunk - 1) / pl->tc_chunk;
     } else {
-        // guided schedule: at most kTcMaxChunks static chunks and twice as many claimed ones
+        // one chunk per warp of the grid: at most kTcMaxChunks
         pl->tc_chunk = 0;
-        nchunks = tmax < 3 * (int64_t)kTcMaxChunks + 1 ? tmax : 3 * (int64_t)kTcMaxChunks + 1;
+        nchunks = tmax < kTcMaxChunks ? tmax : kTcMaxChunks;
     }
     pl->tc_slots = 2 * nchunks;
     // partial outputs and lse of two segments per chunk, then one merge ticket
-    // per (sequence, KV head) row and the chunk-claim and finished-warp counters
+    // per (sequence, KV head) row
     pl->bytes = up256((size_t)pl->tc_slots * G * p->head_dim * sizeof(float)) +
                 up256((size_t)pl->tc_slots * G * sizeof(float)) +
-                up256(((size_t)p->num_seqs * p->num_kv_heads + 2) * sizeof(int));
+                up256((size_t)p->num_seqs * p->num_kv_heads * sizeof(int));
     return PA_OK;
 }
 

@@ -30,7 +30,9 @@
 // and resets the counter to zero (no waiting on other warps).
 #include <cudaTypedefs.h>
 
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <type_traits>
 #include <unordered_map>
 
@@ -103,7 +105,13 @@ template <> struct Mma<__nv_bfloat16> {
 #define PA_TC_WARPS 4
 #endif
 #ifndef PA_TC_STAGES
-#define PA_TC_STAGES 3
+#define PA_TC_STAGES 2
+#endif
+#ifndef PA_TC_HOIST_V
+#define PA_TC_HOIST_V 1
+#endif
+#ifndef PA_TC_MIN_CTAS
+#define PA_TC_MIN_CTAS 1
 #endif
 
 template <int D>
@@ -121,10 +129,7 @@ struct TcCfg {
     static constexpr int RING = NW * S * STAGE;
     static constexpr int BAR_OFF = RING;
     static constexpr int OK_OFF = BAR_OFF + NW * S * 8;
-    static constexpr int RQ = 8;                         // per-warp ring of range chunk ids
-    static constexpr int RQ_OFF = OK_OFF + NW * S * 4;
-    static constexpr int CUM_OFF = RQ_OFF + NW * RQ * 4;
-    static_assert(S < RQ, "the producer runs at most S ranges ahead");
+    static constexpr int CUM_OFF = OK_OFF + NW * S * 4;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (2 * B + 2) * 4; }
 };
 
@@ -152,17 +157,13 @@ struct Win {
     bool valid;
 };
 
-// Chunk layout of the concatenated block stream (guided schedule): n0 chunks
-// of c0 blocks, one per warp, then chunks of c1 blocks that warps claim in
-// order from a counter.  Uniform chunks when c0 == c1.
+// Chunks of the concatenated block stream: n chunks of c blocks (the last one
+// shorter); warp w takes chunks w, w + W, w + 2W, ...
 struct Chunks {
-    int64_t total, c0, n0, c1, n;
-    __device__ int64_t start(int64_t ch) const { return ch < n0 ? ch * c0 : n0 * c0 + (ch - n0) * c1; }
-    __device__ int64_t end(int64_t ch) const {
-        const int64_t e = ch < n0 ? (ch + 1) * c0 : n0 * c0 + (ch - n0 + 1) * c1;
-        return e < total ? e : total;
-    }
-    __device__ int64_t of(int64_t f) const { return f < n0 * c0 ? f / c0 : n0 + (f - n0 * c0) / c1; }
+    int64_t total, c, n;
+    __device__ int64_t start(int64_t ch) const { return ch * c; }
+    __device__ int64_t end(int64_t ch) const { return (ch + 1) * c < total ? (ch + 1) * c : total; }
+    __device__ int64_t of(int64_t f) const { return f / c; }
 };
 
 // Physical address of the 16-byte chunk `chunk` (0 .. D/8-1) of row `row`
@@ -206,7 +207,7 @@ template <> struct FVec<2> {
 };
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
                                                                      const DecodeArgs a) {
     using C = TcCfg<D>;
@@ -217,7 +218,6 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     int *stage_ok = reinterpret_cast<int *>(smem + C::OK_OFF);
-    int *rq_all = reinterpret_cast<int *>(smem + C::RQ_OFF);
     int *cum = reinterpret_cast<int *>(smem + C::CUM_OFF);  // [B + 1] blocks before sequence b
     int *lens = cum + a.B + 1;                                // [B] effective lengths
 
@@ -258,27 +258,20 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
     const int W = gridDim.x * NW;
     const bool rows_mode = a.tc_chunk < 0;
 
-    Chunks ck{total, 1, 0, 1, 0};
+    // Static schedule: by default one chunk of ceil(total / W) blocks (at least
+    // kTcMinChunk) per warp, so every warp reads the same number of blocks;
+    // partition_size > 0 fixes the chunk length instead.
+    Chunks ck{total, 1, 0};
     if (!rows_mode) {
-        const int64_t wc = min(W, kTcMaxChunks);
         if (a.tc_chunk > 0) {
-            ck.c0 = ck.c1 = a.tc_chunk;
+            ck.c = a.tc_chunk;
         } else {
-            // about 60% of the stream in one static chunk per warp, the rest in
-            // claimed chunks of about a third of a warp's share (guided schedule)
-            const int64_t c0 = (total * 6) / (10 * wc);
-            ck.c0 = c0 > kTcMinChunk ? c0 : kTcMinChunk;
-            const int64_t n0 = min(wc, (total + ck.c0 - 1) / ck.c0);
-            const int64_t rest = total - n0 * ck.c0 > 0 ? total - n0 * ck.c0 : 0;
-            const int64_t c1 = (rest + 2 * wc - 1) / (2 * wc);
-            ck.c1 = c1 > kTcMinChunk ? c1 : kTcMinChunk;
+            const int64_t wc = min(W, kTcMaxChunks);
+            const int64_t c = (total + wc - 1) / wc;
+            ck.c = c > kTcMinChunk ? c : kTcMinChunk;
         }
-        ck.n0 = min((int64_t)min(W, kTcMaxChunks), (total + ck.c0 - 1) / ck.c0);
-        const int64_t rest = total - ck.n0 * ck.c0 > 0 ? total - ck.n0 * ck.c0 : 0;
-        ck.n = ck.n0 + (rest + ck.c1 - 1) / ck.c1;
+        ck.n = (total + ck.c - 1) / ck.c;
     }
-    int *work = a.counters + (size_t)B * Hkv;  // next claimed chunk (minus n0)
-    int *done = work + 1;                       // warps that have finished
 
     // rows of sequences with no token produce zeros
     for (int r = gw; r < B * Hkv; r += W) {
@@ -304,37 +297,13 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
         sg.L = lens[lo];
     };
 
-    // ---- range schedule: rows w, w+W, ... (one pass) or chunks (static, then claimed)
-    int *rq = rq_all + warp * C::RQ;  // chunk of the warp's range k is rq[k % RQ]
-    // Claims: lane 0 asks the counter for the next chunk as soon as the producer
-    // enters a range; the answer is read only when that range ends, so the
-    // atomic's latency is hidden behind a whole range of copies.
-    int p_claim_raw = 0;
-    bool p_claim_pending = false;
-    auto producer_chunk = [&](int k) -> int {
-        int ch;
-        if (k == 0 && gw < ck.n0) {
-            ch = gw;  // phase 0: one static chunk per warp
-        } else {
-            if (!p_claim_pending && lane == 0) p_claim_raw = atomicAdd(work, 1);
-            const int cl = __shfl_sync(0xffffffffu, p_claim_raw, 0);
-            ch = (int64_t)ck.n0 + cl < ck.n ? (int)(ck.n0 + cl) : -1;
-        }
-        p_claim_pending = false;
-        if (ch >= 0) {
-            if (lane == 0) p_claim_raw = atomicAdd(work, 1);
-            p_claim_pending = true;
-        }
-        if (lane == 0) rq[k % C::RQ] = ch;
-        return ch;
-    };
+    // ---- range schedule: rows w, w+W, ... (one pass) or chunks w, w+W, ...
     auto set_range = [&](SegIter &it, int64_t ch) {
         it.f = ck.start(ch);
         it.fend = ck.end(ch);
         it.ch = (int)ch;
     };
-    // producer iterator: claims chunks
-    auto p_range = [&](SegIter &it) -> bool {
+    auto range = [&](SegIter &it) -> bool {
         if (rows_mode) {
             for (;; ++it.k) {
                 const int64_t r = (int64_t)gw + (int64_t)it.k * W;
@@ -349,37 +318,16 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
                 }
             }
         }
-        const int ch = producer_chunk(it.k);
-        if (ch < 0) return false;
+        const int64_t ch = (int64_t)gw + (int64_t)it.k * W;
+        if (ch >= ck.n) return false;
         set_range(it, ch);
         return true;
     };
-    // consumer iterator: replays the producer's chunks from rq (the producer is ahead)
-    auto c_range = [&](SegIter &it) -> bool {
-        if (rows_mode) {
-            for (;; ++it.k) {
-                const int64_t r = (int64_t)gw + (int64_t)it.k * W;
-                if (r >= (int64_t)B * Hkv) return false;
-                const int b = (int)(r / Hkv), kvh = (int)(r % Hkv);
-                const int nb = cum[b + 1] - cum[b];
-                if (nb > 0) {
-                    it.f = (int64_t)cum[b] * Hkv + (int64_t)kvh * nb;
-                    it.fend = it.f + nb;
-                    it.ch = -1;
-                    return true;
-                }
-            }
-        }
-        const int ch = rq[it.k % C::RQ];
-        if (ch < 0) return false;
-        set_range(it, ch);
-        return true;
-    };
-    auto next_seg = [&](SegIter &it, Seg &sg, bool producer) -> bool {
+    auto next_seg = [&](SegIter &it, Seg &sg) -> bool {
         if (it.done) return false;
         if (it.f >= it.fend) {
             ++it.k;
-            if (!(producer ? p_range(it) : c_range(it))) {
+            if (!range(it)) {
                 it.done = true;
                 return false;
             }
@@ -404,10 +352,10 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
 
     // ---- producer: TMA for the warp's block stream, S blocks ahead of the consumer ----
     SegIter pit{0, 0, 0, -1, false};
-    pit.done = !p_range(pit);
+    pit.done = !range(pit);
     auto win_first = [&](Win &w) {
         Seg sg;
-        w.valid = next_seg(pit, sg, true);
+        w.valid = next_seg(pit, sg);
         if (w.valid) {
             w.sg = sg;
             w.o = 0;
@@ -490,9 +438,9 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
     };
 
     SegIter cit{0, 0, 0, -1, false};
-    cit.done = !c_range(cit);
+    cit.done = !range(cit);
     Seg cs;
-    bool have = next_seg(cit, cs, false);
+    bool have = next_seg(cit, cs);
     uint32_t bq[C::KSTEPS][2];
     if (have) load_q(cs, bq);
     int c_k = 0;
@@ -583,22 +531,12 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
     };
 
     while (have && alive) {
-        // The next segment's q is fetched early and lands while this one runs: now
-        // when that segment is in the same range or the producer has already claimed
-        // the next range, else as soon as the producer gets there (block loop).
+        // the next segment's q is fetched now and lands while this one runs
         SegIter nit = cit;
         Seg ns;
-        bool have_next = false, next_known = false;
         uint32_t bqn[C::KSTEPS][2];
-        auto try_peek = [&]() {
-            if (next_known || !(cit.f < cit.fend || pit.k > cit.k || pit.done)) return;
-            __syncwarp();  // lane 0 may just have written the next range's chunk to rq
-            next_known = true;
-            nit = cit;
-            have_next = next_seg(nit, ns, false);
-            if (have_next) load_q(ns, bqn);
-        };
-        try_peek();
+        const bool have_next = next_seg(nit, ns);
+        if (have_next) load_q(ns, bqn);
 
         const int len = cs.j1 - cs.j0;
         const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;  // tokens in the row's last block
@@ -637,13 +575,15 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
                 }
                 // ---- fragments: K (A of S^T), then V^T (A of O^T), all issued up front
                 const int mi = lane >> 3, r8 = lane & 7;
-                uint32_t kf[C::KSTEPS][4], vf[C::MTILES][4];
+                uint32_t kf[C::KSTEPS][4], vf[PA_TC_HOIST_V ? C::MTILES : 1][4];
 #pragma unroll
                 for (int ks = 0; ks < C::KSTEPS; ++ks)
                     ldsm_x4(kf[ks], tile_chunk(tK, r8 + ((mi & 1) << 3), 2 * ks + (mi >> 1)));
+                if constexpr (PA_TC_HOIST_V) {
 #pragma unroll
-                for (int i = 0; i < C::MTILES; ++i)
-                    ldsm_x4_t(vf[i], tile_chunk(tV, r8 + ((mi >> 1) << 3), 2 * i + (mi & 1)));
+                    for (int i = 0; i < C::MTILES; ++i)
+                        ldsm_x4_t(vf[i], tile_chunk(tV, r8 + ((mi >> 1) << 3), 2 * i + (mi & 1)));
+                }
                 // ---- S^T = K . Q^T, four independent accumulator chains
                 float sa[4][4];
 #pragma unroll
@@ -698,17 +638,18 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
                 // ---- O^T += V^T . P^T
 #pragma unroll
                 for (int i = 0; i < C::MTILES; ++i) {
-                    Mma<T>::mma(o[i], vf[i], pb0, pb1);
-                    if constexpr (SPLIT_P) Mma<T>::mma(o[i], vf[i], pl0, pl1);
+                    const int vi = PA_TC_HOIST_V ? i : 0;
+                    if constexpr (!PA_TC_HOIST_V)
+                        ldsm_x4_t(vf[vi], tile_chunk(tV, r8 + ((mi >> 1) << 3), 2 * i + (mi & 1)));
+                    Mma<T>::mma(o[i], vf[vi], pb0, pb1);
+                    if constexpr (SPLIT_P) Mma<T>::mma(o[i], vf[vi], pl0, pl1);
                 }
             }
             __syncwarp();
             refill();
             ++c_k;
-            try_peek();
         }
         if (!alive) break;
-        try_peek();
 
         // ---- finish the segment
 #pragma unroll
@@ -766,11 +707,6 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
             pend_fr = cs.fr;
             pend_nb = cs.nb;
         }
-        if (!next_known) {  // cannot happen once the producer is past this range; kept for safety
-            nit = cit;
-            have_next = next_seg(nit, ns, false);
-            if (have_next) load_q(ns, bqn);
-        }
         cit = nit;
         cs = ns;
         have = have_next;
@@ -781,20 +717,6 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32) decode_tc_kernel(const __gri
         }
     }
     resolve();
-
-    // ---- the last warp to finish puts the chunk counters back to zero
-    if (!rows_mode) {
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-            __threadfence();
-            last = atomicAdd(done, 1) == W - 1;
-            if (last) {
-                *work = 0;
-                *done = 0;
-            }
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -857,6 +779,35 @@ static bool cache_tensor_map(CUtensorMap *m, const void *base, int64_t rows, int
     return true;
 }
 
+// SM count and resident CTAs per SM for (kernel, device, dynamic shared memory),
+// queried once: the occupancy query costs microseconds of host time per call.
+static bool launch_shape(const void *kernel, int threads, int smem, int *sms, int *per_sm) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void *, int, int>, std::pair<int, int>> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const auto key = std::make_tuple(kernel, dev, smem);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) {
+            *sms = it->second.first;
+            *per_sm = it->second.second;
+            return true;
+        }
+    }
+    int s = 0, p = 0;
+    if (cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p, kernel, threads, smem) != cudaSuccess)
+        return false;
+    p = p < 1 ? 1 : p;
+    std::lock_guard<std::mutex> lock(mu);
+    cache[key] = {s, p};
+    *sms = s;
+    *per_sm = p;
+    return true;
+}
+
 bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
     return (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype && (D == 64 || D == 128) &&
            (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
@@ -873,12 +824,8 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     const int64_t rows = a.N * a.Hkv * kBlockSize;
     if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
         return PA_ERR_CUDA;
-    int dev = 0, sms = 0, per_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::THREADS, smem) != cudaSuccess)
-        return PA_ERR_CUDA;
-    per_sm = per_sm < 1 ? 1 : per_sm;
+    int sms = 0, per_sm = 0;
+    if (!launch_shape(reinterpret_cast<const void *>(kern), C::THREADS, smem, &sms, &per_sm)) return PA_ERR_CUDA;
     // persistent grid: every resident warp is a worker, but no more warps than
     // there are blocks to read (every sequence at max_len)
     const int64_t blocks = (int64_t)a.B * a.Hkv * ((a.max_len + kBlockSize - 1) / kBlockSize);

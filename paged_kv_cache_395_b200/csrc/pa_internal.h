@@ -48,12 +48,14 @@ struct DecodeArgs {
                              // -1 = whole rows (one pass)
 };
 
-// Tensor-core schedule limits: the auto (guided) schedule cuts the block stream
-// into at most kTcMaxChunks static chunks plus at most twice as many claimed
-// ones, each of at least kTcMinChunk blocks; the per-CTA prefix sum holds at
-// most kTcMaxB sequences.
+// Tensor-core schedule limits: the auto schedule cuts the block stream into at
+// most kTcMaxChunks chunks (one per warp of the grid) of at least kTcMinChunk
+// blocks; the per-CTA prefix sum holds at most kTcMaxB sequences.
 constexpr int kTcMaxChunks = 2048;
-constexpr int kTcMinChunk = 16;
+#ifndef PA_TC_MIN_CHUNK
+#define PA_TC_MIN_CHUNK 8
+#endif
+constexpr int kTcMinChunk = PA_TC_MIN_CHUNK;
 constexpr int kTcMaxB = 4096;
 
 // Per-translation-unit error words (see PA_ERROR_WORD_ACCESSOR).

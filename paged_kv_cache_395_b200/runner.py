@@ -170,6 +170,14 @@ class StepCalls:
             self.calls[i] = calls
             self.launches[i] = launches
 
+    def run_decode_only(self, i):
+        """Issue only the decode call of step i (kernel timing)."""
+        for name, fn, args in self.calls[i]:
+            if name == "decode":
+                rc = fn(*args)
+                if rc != 0:
+                    raise pa.PaError(rc, name)
+
     def run(self, i, on_decode=None):
         """Issue step i; ``on_decode(before: bool)`` brackets the decode call."""
         for name, fn, args in self.calls[i]:
