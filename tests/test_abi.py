@@ -98,14 +98,14 @@ def test_decode_null_and_workspace_checks():
     p = params(partition_size=16, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == 32 * 4 * 128 * 4 + 512 + 256
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(params(partition_size=0, algo=pa.PA_ALGO_TENSOR))) == 0
-    # auto (guided) schedule on the tensor-core family: at most 3 x 2048 + 1 chunks,
-    # two partial slots each; 64 x 2 row tickets + 2 schedule counters
+    # auto schedule on the tensor-core family: at most 2048 chunks (one per warp),
+    # two partial slots each; then 64 x 2 row tickets
     p = params(partition_size=-1, algo=pa.PA_ALGO_TENSOR, num_seqs=64, max_blocks_per_seq=264,
                max_seq_len=4224)
-    slots = 2 * (3 * 2048 + 1)
+    slots = 2 * 2048
     up = lambda x: (x + 255) // 256 * 256
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == \
-        up(slots * 4 * 128 * 4) + up(slots * 4 * 4) + up((64 * 2 + 2) * 4)
+        up(slots * 4 * 128 * 4) + up(slots * 4 * 4) + up(64 * 2 * 4)
     # the tensor-core family needs fp16/bf16 q and cache
     p = params(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p),
