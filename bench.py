@@ -343,7 +343,7 @@ def main(argv=None):
         "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i8" if int8 else "f16", "data": "synthetic",
         "config": {"workload": WORKLOADS[args.workload], "name": args.workload,
-                   "partition_size": 256 if part == -1 else part, "algo": args.algo,
+                   "partition_size": "library picks (-1)" if part == -1 else part, "algo": args.algo,
                    "l2": "inputs larger than L2: KV pool and per-step reads exceed 126 MB, no flush",
                    "timing": "CUDA events around the K steps issued back to back",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},

@@ -17,17 +17,24 @@
 // (cp.async.bulk.tensor, 64-element boxes), so the ldmatrix reads of 8 rows x
 // 16 bytes hit 8 different bank groups.
 //
-// Scheduling: a persistent grid; every warp is an independent worker.  Work
-// items are (sequence, partition of `part` tokens, KV head); warp w takes
-// items w, w + W, w + 2W, ... (W = warps in the grid).  Each warp owns a
-// 3-stage ring, refilled one block ahead per consumed block, and the refill
-// runs straight on into the warp's next item, so the copy stream does not
-// drain between items.  A single-partition item writes its output directly.
-// Otherwise it writes its normalised partial output and log2-sum-exp to the
-// workspace and takes a ticket from a per-(sequence, KV head) counter; the
-// warp that takes the last ticket merges all partitions
+// Scheduling: a persistent grid; every warp is an independent worker with its
+// own 2-stage ring of (K tile, V tile) stages and its own mbarriers.  The
+// (sequence, KV head) rows are laid end to end as one stream of blocks (row
+// order: sequence, then KV head; total = sum_b ceil(L_b / 16) * H_kv blocks).
+// With partition_size == 0 warp w takes whole rows w, w + W, ... (W = warps in
+// the grid).  Otherwise the stream is cut into chunks of c blocks -- by default
+// c = ceil(total / W) (at least 8), so every warp reads the same number of
+// blocks whatever the length mix; partition_size > 0 fixes c = partition/16 --
+// and warp w takes chunks w, w + W, ...  A chunk is walked segment by segment
+// (a segment = the part of one row inside the chunk); the producer side of the
+// warp keeps issuing TMA for the next blocks across segment and chunk ends, so
+// the copy stream does not drain.  A segment that is a whole row writes the
+// output directly.  A cut segment is a partial: its normalised output and
+// log2-sum-exp go to workspace slot 2*chunk (first segment of the chunk) or
+// 2*chunk + 1 (last), and it takes a ticket from a per-row counter; the warp
+// that takes the last ticket merges the row's partials
 //   out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M)
-// and resets the counter to zero (no waiting on other warps).
+// and resets the counter to zero.  No warp ever waits for another.
 #include <cudaTypedefs.h>
 
 #include <map>
@@ -819,7 +826,7 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     auto kern = decode_tc_kernel<T, D, G>;
     const int smem = C::smem_bytes(a.B);
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
-    if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are fetched with bulk copies
+    if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are read as aligned 32-bit pairs
     CUtensorMap tk, tv;
     const int64_t rows = a.N * a.Hkv * kBlockSize;
     if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
