@@ -27,8 +27,10 @@ max over ranks of the device time.
 computation) on a bounded sample of the same workload, on rank 0 only.
 """
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -42,6 +44,31 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); decode tokens/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of the decode kernel from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum of the two captured launches, trace steps 8 and 9 of the
+# ragged workload), per algorithmic byte; the summary is profiles/decode_tc_ragged.md.
+# It holds only for the kernel code it was taken on (hash of the source without
+# comments); after any code change the bench reports null until it is taken again.
+NCU_TRAFFIC = {
+    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "7151f0ec1a012d51",
+               "per_alg_byte": (475345920 + 4564480 + 462447872 + 5231616) / (472969728 + 459894508)},
+}
+
+
+def code_hash(path):
+    s = open(path).read()
+    s = re.sub(r"/\*.*?\*/", " ", s, flags=re.S)
+    s = re.sub(r"//[^\n]*", " ", s)
+    return hashlib.sha256(" ".join(s.split()).encode()).hexdigest()[:16]
+
+
+def traffic_per_launch(workload, algo, partition, mean_alg_bytes):
+    t = NCU_TRAFFIC.get(workload)
+    if t is None or algo == "simt" or partition != -1 or code_hash(os.path.join(ROOT, t["source"])) != t["code"]:
+        return None
+    return t["per_alg_byte"] * mean_alg_bytes
+
 
 WORKLOADS = {
     "ragged": "continuous-batching ragged decode: 7B-GQA 32 q / 8 KV heads, head_dim 128, fp16 KV, "
@@ -351,7 +378,9 @@ def main(argv=None):
         "hbm_frac_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "hbm_frac_of_" + peak_kind: value / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": traffic_per_launch(args.workload, args.algo, part, bytes_rank / K),
+                     "traffic_unit": "bytes per decode launch (ncu DRAM read + write, scaled)",
                      "kernel": "pa_decode: the K steps' decode calls issued back to back",
                      "peak_kind": peak_kind},
         "gpu_launches": launches,
