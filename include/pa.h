@@ -18,7 +18,8 @@
  *   slot_mapping            [num_tokens]  int64, slot = block * PA_BLOCK_SIZE + offset
  *
  * Ownership: the caller allocates and owns every buffer, including the split-K
- * workspace.  The library allocates no memory and keeps no per-call state.
+ * workspace.  The library allocates no memory and keeps no per-call state
+ * (pa_decode_fixed_scratch uses a fixed area compiled into the library).
  * Every pointer argument is a DEVICE pointer except `p` (pa_decode_params) and
  * the host-side out-parameters of pa_get_error_flags.  Every call is
  * asynchronous on `stream` and never synchronises the host, except
@@ -148,6 +149,30 @@ size_t pa_decode_workspace_size(const pa_decode_params *p);
 int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
               const int32_t *block_tables, const int32_t *seq_lens, float scale,
               const pa_decode_params *p, pa_stream_t stream);
+
+/*
+ * pa_decode without a caller workspace.  No counterpart in the paper: it is an
+ * addition of this library for callers that cannot allocate device memory
+ * where they decode -- an engine that has given all free device memory to its
+ * KV block pool up front, or a host integration with no device allocator of
+ * its own.  Same arguments, same result and same errors as pa_decode; the
+ * split-K workspace fields of `p` are ignored and a scratch area of
+ * PA_FIXED_SCRATCH_BYTES compiled into the library (one per device) is used
+ * instead.  The library allocates nothing.
+ *
+ *  - Parameters whose pa_decode_workspace_size exceeds PA_FIXED_SCRATCH_BYTES
+ *    return PA_ERR_WORKSPACE and launch nothing.
+ *  - The first call on a device sets the area up: it looks up its address,
+ *    zero-fills it on `stream` and synchronises `stream`.  Make that first call
+ *    before any stream capture.
+ *  - All calls on one device share the area: calls that overlap on the device
+ *    (different streams, or host threads without ordering) race on it.  Issue
+ *    them in one stream order.
+ */
+#define PA_FIXED_SCRATCH_BYTES ((size_t)32 << 20)
+int pa_decode_fixed_scratch(void *out, const void *q, const void *key_cache, const void *value_cache,
+                            const int32_t *block_tables, const int32_t *seq_lens, float scale,
+                            const pa_decode_params *p, pa_stream_t stream);
 
 /*
  * Copy-on-write block copy (chanyi.net.cn/article/49 section 三: shared prefix

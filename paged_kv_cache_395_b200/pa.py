@@ -64,6 +64,7 @@ def _load():
     P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
     L.pa_reshape_and_cache.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, i64, i64, P]
     L.pa_decode.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), P]
+    L.pa_decode_fixed_scratch.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), P]
     L.pa_decode_workspace_size.argtypes = [ctypes.POINTER(PaDecodeParams)]
     L.pa_decode_workspace_size.restype = ctypes.c_size_t
     L.pa_block_copy.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, P]
@@ -72,8 +73,8 @@ def _load():
     L.pa_status_string.argtypes = [i32]
     L.pa_status_string.restype = ctypes.c_char_p
     L.pa_version.argtypes = []
-    for n in ("pa_reshape_and_cache", "pa_decode", "pa_block_copy", "pa_quantize_int8",
-              "pa_get_error_flags", "pa_version"):
+    for n in ("pa_reshape_and_cache", "pa_decode", "pa_decode_fixed_scratch", "pa_block_copy",
+              "pa_quantize_int8", "pa_get_error_flags", "pa_version"):
         getattr(L, n).restype = i32
     return L
 
@@ -81,8 +82,9 @@ def _load():
 lib = _load()
 
 # the C-ABI symbols include/pa.h declares
-EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_block_copy",
-            "pa_quantize_int8", "pa_get_error_flags", "pa_status_string", "pa_version")
+EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_fixed_scratch",
+            "pa_block_copy", "pa_quantize_int8", "pa_get_error_flags", "pa_status_string", "pa_version")
+FIXED_SCRATCH_BYTES = 32 << 20  # PA_FIXED_SCRATCH_BYTES
 
 
 class PaError(RuntimeError):
@@ -186,6 +188,29 @@ def pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max
     _check(lib.pa_decode(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache),
                          _ptr(block_tables), _ptr(seq_lens), ctypes.c_float(scale),
                          ctypes.byref(p), _stream(stream)), "pa_decode")
+
+
+def pa_decode_fixed_scratch(out, q, key_cache, value_cache, block_tables, seq_lens, scale,
+                            max_seq_len, k_scales=None, v_scales=None, partition_size=-1,
+                            algo=PA_ALGO_AUTO, stream=None):
+    """pa_decode for callers that cannot allocate a workspace: the split-K
+    scratch is the fixed area compiled into the library (FIXED_SCRATCH_BYTES per
+    device).  Calls on one device must not overlap; the first call on a device
+    synchronises its stream once and should come before any stream capture."""
+    _dev(out, q, key_cache, value_cache, block_tables, seq_lens, k_scales, v_scales)
+    for t, n in ((out, "out"), (q, "q"), (key_cache, "key_cache"), (value_cache, "value_cache"),
+                 (block_tables, "block_tables"), (seq_lens, "seq_lens")):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    if out.dtype != q.dtype or out.shape != q.shape:
+        raise ValueError("out must match q in shape and dtype")
+    p = make_params(q, key_cache, block_tables, max_seq_len, k_scales, v_scales, partition_size,
+                    None, algo)
+    _check(lib.pa_decode_fixed_scratch(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache),
+                                       _ptr(block_tables), _ptr(seq_lens), ctypes.c_float(scale),
+                                       ctypes.byref(p), _stream(stream)), "pa_decode_fixed_scratch")
 
 
 def pa_block_copy(key_cache, value_cache, pairs, k_scales=None, v_scales=None, stream=None):
