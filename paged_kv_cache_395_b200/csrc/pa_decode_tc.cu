@@ -63,6 +63,11 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
 }
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
 __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
     uint32_t y;
     asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -111,6 +116,8 @@ template <> struct Mma<__nv_bfloat16> {
 #ifndef PA_TC_WARPS
 #define PA_TC_WARPS 4
 #endif
+// ring stages per warp (two measured faster than three on the ragged trace:
+// more bytes in flight per warp only lengthen the DRAM queues)
 #ifndef PA_TC_STAGES
 #define PA_TC_STAGES 2
 #endif
@@ -121,7 +128,7 @@ template <> struct Mma<__nv_bfloat16> {
 #define PA_TC_MIN_CTAS 1
 #endif
 
-template <int D>
+template <int D, int G>
 struct TcCfg {
     static constexpr int NW = PA_TC_WARPS;        // warps (independent workers) per CTA
     static constexpr int THREADS = NW * 32;
@@ -133,8 +140,10 @@ struct TcCfg {
     static constexpr int KSTEPS = D / 16;         // QK k-steps
     static constexpr int MTILES = D / 16;         // PV m-tiles
     static constexpr int DPL = D / 32;            // dims per lane in the merge
+    static constexpr int QSLOT = G * D * 2;       // q rows of a segment's G heads
     static constexpr int RING = NW * S * STAGE;
-    static constexpr int BAR_OFF = RING;
+    static constexpr int QRING_OFF = RING;        // [NW][S] q slots, one per stage
+    static constexpr int BAR_OFF = QRING_OFF + NW * S * QSLOT;
     static constexpr int OK_OFF = BAR_OFF + NW * S * 8;
     static constexpr int CUM_OFF = OK_OFF + NW * S * 4;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (2 * B + 2) * 4; }
@@ -173,22 +182,16 @@ struct Chunks {
     __device__ int64_t of(int64_t f) const { return f / c; }
 };
 
-// Physical address of the 16-byte chunk `chunk` (0 .. D/8-1) of row `row`
-// (0..15) of a swizzled tile: box = chunk / 8, and inside the 1024-byte
-// aligned box the chunk index is XORed with row % 8 (128-byte swizzle).
-__device__ __forceinline__ uint32_t tile_chunk(uint32_t tile, int row, int chunk) {
-    return tile + (chunk >> 3) * 2048 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
-}
-
-// Ticket increment with acquire-release semantics at GPU scope: the warp's
+// Ticket increment with release semantics at GPU scope: the warp's
 // partial-result stores (ordered before lane 0 by __syncwarp) are released
-// with it, and the warp that draws the last ticket acquires every other
-// segment's partial.
-__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v) {
+// with it.  The warp that draws a row's last ticket runs fence_acq_rel_gpu
+// before it reads the other segments' partials.
+__device__ __forceinline__ int atom_add_release_gpu(int *p, int v) {
     int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
 }
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -217,7 +220,7 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
                                                                      const DecodeArgs a) {
-    using C = TcCfg<D>;
+    using C = TcCfg<D, G>;
     constexpr int NW = C::NW, S = C::S;
     constexpr bool SPLIT_P = sizeof(T) == 2 && !std::is_same<T, __half>::value;  // bf16: P = hi + lo
     extern __shared__ unsigned char smem_raw[];
@@ -348,6 +351,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     };
 
     uint64_t *my_bars = bars + warp * S;
+    constexpr uint32_t kQBytes = G * D * sizeof(T);  // multiple of 16; q rows are 16-byte aligned
+    const uint32_t qring = smem_addr(smem) + C::QRING_OFF + warp * S * C::QSLOT;
     int *my_ok = stage_ok + warp * S;
     const uint32_t ring = smem_addr(smem) + warp * S * C::STAGE;
     if (lane == 0) {
@@ -400,19 +405,29 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         if (lane == 0) {
             const int s = p_k % S;
             uint64_t *bar = &my_bars[s];
-            if (y < 0) {
-                my_ok[s] = 0;
-                raise_flag(PA_EFLAG_BAD_BLOCK);
+            // a segment's first block also brings the segment's q rows into the
+            // stage's q slot (even when the block itself is skipped)
+            const bool seg_first = pc.o == 0 && p_i == 0;
+            const uint32_t tx = (y < 0 ? 0u : (uint32_t)C::STAGE) + (seg_first ? kQBytes : 0u);
+            my_ok[s] = y >= 0;
+            if (y < 0) raise_flag(PA_EFLAG_BAD_BLOCK);
+            if (tx == 0) {
                 mbar_arrive(bar);
             } else {
-                my_ok[s] = 1;
-                mbar_arrive_expect_tx(bar, C::STAGE);
+                mbar_arrive_expect_tx(bar, tx);
+            }
+            if (y >= 0) {
                 const uint32_t dst = ring + s * C::STAGE;
 #pragma unroll
                 for (int bx = 0; bx < C::BOXES; ++bx) {
                     tma_load_2d(dst + bx * C::BOX_BYTES, &tmK, bx * 64, y, smem_addr(bar));
                     tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * 64, y, smem_addr(bar));
                 }
+            }
+            if (seg_first) {
+                const T *qsrc = reinterpret_cast<const T *>(a.q) +
+                                ((size_t)pc.sg.b * a.Hq + (size_t)pc.sg.kvh * G) * D;
+                bulk_g2s_u32(qring + s * C::QSLOT, qsrc, kQBytes, smem_addr(bar));
             }
         }
         ++p_k;
@@ -431,25 +446,37 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     // ---- consumer ------------------------------------------------------------------------
     const int g = lane >> 2, c = lane & 3;  // mma fragment coordinates
     const int h0 = 2 * c, h1 = 2 * c + 1;  // heads of this thread's S^T / O^T columns
-    auto load_q = [&](const Seg &sg, uint32_t (&bq)[C::KSTEPS][2]) {
-        const T *qp = reinterpret_cast<const T *>(a.q) + ((size_t)sg.b * a.Hq + (size_t)sg.kvh * G) * D;
+    // B fragments of q (n = heads, k = dims) from the q slot of stage s
+    auto load_q = [&](int s, uint32_t (&bq)[C::KSTEPS][2]) {
+        const uint32_t qs = qring + s * C::QSLOT + (g * D + 2 * c) * 2;
 #pragma unroll
-        for (int s = 0; s < C::KSTEPS; ++s) {
+        for (int ks = 0; ks < C::KSTEPS; ++ks) {
             if (g < G) {
-                bq[s][0] = *reinterpret_cast<const uint32_t *>(qp + g * D + 16 * s + 2 * c);
-                bq[s][1] = *reinterpret_cast<const uint32_t *>(qp + g * D + 16 * s + 2 * c + 8);
+                bq[ks][0] = lds_u32(qs + ks * 32);
+                bq[ks][1] = lds_u32(qs + ks * 32 + 16);
             } else {
-                bq[s][0] = bq[s][1] = 0u;
+                bq[ks][0] = bq[ks][1] = 0u;
             }
         }
     };
+    // per-lane ldmatrix offsets inside a stage (128-byte swizzle): K as the A
+    // operand of S^T (chunk 2i + hi of row r), V^T as the A operand of O^T; the
+    // box of k-step ks is ks / 4
+    const int mi = lane >> 3, r8 = lane & 7;
+    uint32_t koff[4], voff[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int kr = r8 + ((mi & 1) << 3), kc = 2 * i + (mi >> 1);
+        koff[i] = kr * 128 + (((kc & 7) ^ (kr & 7)) << 4);
+        const int vr = r8 + ((mi >> 1) << 3), vc = 2 * i + (mi & 1);
+        voff[i] = C::TILE + vr * 128 + (((vc & 7) ^ (vr & 7)) << 4);
+    }
 
     SegIter cit{0, 0, 0, -1, false};
     cit.done = !range(cit);
     Seg cs;
     bool have = next_seg(cit, cs);
     uint32_t bq[C::KSTEPS][2];
-    if (have) load_q(cs, bq);
     int c_k = 0;
     bool alive = true;
     // Pending ticket: the last partial's ticket is read one segment later, so the
@@ -458,93 +485,112 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     bool pend = false;
     int pend_b = 0, pend_kvh = 0, pend_nb = 0;
     int64_t pend_fr = 0;
+    bool due = false;  // a partial is written but its ticket is not taken yet
+    int due_b = 0, due_kvh = 0, due_nb = 0;
+    int64_t due_fr = 0;
     auto merge_row = [&](int b, int kvh, int64_t fr, int nb) {
         // Last segment of the row to finish: merge all of them,
-        //   out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M),
-        // loading the lse values and partial outputs of up to NB segments at once.
+        //   out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M).
+        // Pass 1: lane (i, h) reads lse of segment i, head h (32 / G segments
+        // per round) and keeps a running (max, sum); the lanes of a head then
+        // combine theirs.  Pass 2: the partial outputs, NB segments x G heads
+        // per round, all loads issued before they are used.
         const int64_t ch_first = ck.of(fr), ch_last = ck.of(fr + nb - 1);
         const int nseg = (int)(ch_last - ch_first + 1);
-        auto slot_of = [&](int64_t ch) -> int {
-            return (int)(2 * ch + ((ch == ch_first && fr > ck.start(ch)) ? 1 : 0));
+        auto slot_of = [&](int i) -> int {  // slot of the row's i-th segment
+            const int64_t ch = ch_first + i;
+            return (int)(2 * ch + ((i == 0 && fr > ck.start(ch)) ? 1 : 0));
         };
-        T *out = reinterpret_cast<T *>(a.out) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
-        constexpr int NB = 4;  // segments per batch (NB * G <= 32 lanes hold their lse)
-        using V = FVec<C::DPL>;
-        float Mh[G], Sh[G], acc[G][C::DPL];
+        constexpr int SPP = 32 / G;                 // segments per round of pass 1
+        constexpr int NB = 16 / G > 0 ? 16 / G : 1;  // segments per round of pass 2
+        const int li = lane / G, lh = lane % G;
+        float x0 = -INFINITY;  // lse of (segment li, head lh), first round
+        if (li < nseg) x0 = __ldcg(a.ws_lse + (size_t)slot_of(li) * G + lh);
+        float mx = x0, sm = x0 == -INFINITY ? 0.f : 1.f;
+        for (int i0 = SPP; i0 < nseg; i0 += SPP) {
+            if (i0 + li < nseg) {
+                const float x = __ldcg(a.ws_lse + (size_t)slot_of(i0 + li) * G + lh);
+                const float mn = fmaxf(mx, x);
+                sm = sm * fast_exp2(mx - mn) + fast_exp2(x - mn);
+                mx = mn;
+            }
+        }
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            Mh[h] = -INFINITY;
-            Sh[h] = 0.f;
+        for (int o = G; o < 32; o <<= 1) {
+            const float mo = __shfl_xor_sync(0xffffffffu, mx, o);
+            const float so = __shfl_xor_sync(0xffffffffu, sm, o);
+            const float mn = fmaxf(mx, mo);
+            sm = (mx == -INFINITY ? 0.f : sm * fast_exp2(mx - mn)) + (mo == -INFINITY ? 0.f : so * fast_exp2(mo - mn));
+            mx = mn;
+        }
+        const float inv_sum = 1.f / sm;  // lane (., h) now holds head h's max and sum
+        using V = FVec<C::DPL>;
+        float acc[G][C::DPL];
+#pragma unroll
+        for (int h = 0; h < G; ++h)
 #pragma unroll
             for (int e = 0; e < C::DPL; ++e) acc[h][e] = 0.f;
-        }
-        for (int i0 = 0; i0 < nseg; i0 += NB) {
-            const int nbat = min(NB, nseg - i0);
-            const int li = lane / G, lh = lane % G;  // lane holds lse of (segment li, head lh)
-            int sl_l = 0;
-            float lse_l = -INFINITY;
-            if (li < nbat) {
-                sl_l = slot_of(ch_first + i0 + li);
-                lse_l = __ldcg(a.ws_lse + (size_t)sl_l * G + lh);
-            }
-            int sls[NB];
+        for (int i0 = 0; i0 < nseg; i0 += SPP) {
+            float x = x0;
+            if (i0 > 0) x = i0 + li < nseg ? __ldcg(a.ws_lse + (size_t)slot_of(i0 + li) * G + lh) : -INFINITY;
+            const float wl = x == -INFINITY ? 0.f : fast_exp2(x - mx) * inv_sum;  // weight of (i0 + li, lh)
+            for (int j0 = 0; j0 < SPP && i0 + j0 < nseg; j0 += NB) {
+                typename V::type v[NB][G];
 #pragma unroll
-            for (int i = 0; i < NB; ++i) sls[i] = __shfl_sync(0xffffffffu, sl_l, i * G);
+                for (int jj = 0; jj < NB; ++jj) {
+                    if (i0 + j0 + jj < nseg) {
+                        const int sl = slot_of(i0 + j0 + jj);
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                typename V::type v[NB];
-#pragma unroll
-                for (int i = 0; i < NB; ++i)
-                    if (i < nbat) v[i] = V::ld(a.ws_o + ((size_t)sls[i] * G + h) * D + lane * C::DPL);
-                float bm = -INFINITY;
-#pragma unroll
-                for (int i = 0; i < NB; ++i) {
-                    const float x = __shfl_sync(0xffffffffu, lse_l, i * G + h);
-                    if (i < nbat) bm = fmaxf(bm, x);
-                }
-                const float mn = fmaxf(Mh[h], bm);
-                const float f = Mh[h] == -INFINITY ? 0.f : fast_exp2(Mh[h] - mn);
-                Sh[h] *= f;
-#pragma unroll
-                for (int e = 0; e < C::DPL; ++e) acc[h][e] *= f;
-#pragma unroll
-                for (int i = 0; i < NB; ++i) {
-                    const float x = __shfl_sync(0xffffffffu, lse_l, i * G + h);
-                    if (i < nbat) {
-                        const float w = fast_exp2(x - mn);
-                        Sh[h] += w;
-#pragma unroll
-                        for (int e = 0; e < C::DPL; ++e) acc[h][e] = fmaf(w, V::get(v[i], e), acc[h][e]);
+                        for (int h = 0; h < G; ++h) v[jj][h] = V::ld(a.ws_o + ((size_t)sl * G + h) * D + lane * C::DPL);
                     }
                 }
-                Mh[h] = mn;
+#pragma unroll
+                for (int jj = 0; jj < NB; ++jj) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float w = __shfl_sync(0xffffffffu, wl, (j0 + jj) * G + h);
+                        if (i0 + j0 + jj < nseg) {
+#pragma unroll
+                            for (int e = 0; e < C::DPL; ++e) acc[h][e] = fmaf(w, V::get(v[jj][h], e), acc[h][e]);
+                        }
+                    }
+                }
             }
         }
+        T *out = reinterpret_cast<T *>(a.out) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float inv = 1.f / Sh[h];
+        for (int h = 0; h < G; ++h)
 #pragma unroll
-            for (int e = 0; e < C::DPL; ++e) out[h * D + lane * C::DPL + e] = Cvt<T>::from_f(acc[h][e] * inv);
-        }
+            for (int e = 0; e < C::DPL; ++e) out[h * D + lane * C::DPL + e] = Cvt<T>::from_f(acc[h][e]);
         if (lane == 0) a.counters[(size_t)b * Hkv + kvh] = 0;  // the workspace is left as it was found
     };
     auto resolve = [&]() {
         if (!pend) return;
         pend = false;
         const int old = __shfl_sync(0xffffffffu, pend_old, 0);
-        __syncwarp();
         const int nseg = (int)(ck.of(pend_fr + pend_nb - 1) - ck.of(pend_fr) + 1);
-        if (old == nseg - 1) merge_row(pend_b, pend_kvh, pend_fr, pend_nb);
+        if (old == nseg - 1) {
+            if (lane == 0) fence_acq_rel_gpu();  // acquire the other segments' partials
+            __syncwarp();
+            merge_row(pend_b, pend_kvh, pend_fr, pend_nb);
+        }
+    };
+    // The ticket of a partial is taken one block into the next segment (or at
+    // the end), when the partial's stores have drained, so the release costs
+    // the warp nothing; its result is read at the next segment end.
+    auto take_ticket = [&]() {
+        if (!due) return;
+        due = false;
+        __syncwarp();
+        if (lane == 0) pend_old = atom_add_release_gpu(a.counters + (size_t)due_b * Hkv + due_kvh, 1);
+        pend = true;
+        pend_b = due_b;
+        pend_kvh = due_kvh;
+        pend_fr = due_fr;
+        pend_nb = due_nb;
     };
 
     while (have && alive) {
-        // the next segment's q is fetched now and lands while this one runs
-        SegIter nit = cit;
-        Seg ns;
-        uint32_t bqn[C::KSTEPS][2];
-        const bool have_next = next_seg(nit, ns);
-        if (have_next) load_q(ns, bqn);
-
         const int len = cs.j1 - cs.j0;
         const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;  // tokens in the row's last block
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -562,6 +608,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 break;
             }
             if (lane != 0) mbar_wait(&my_bars[s], parity);
+            if (j == 0) load_q(s, bq);  // the segment's q came with its first block
             const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
             const uint32_t tK = ring + s * C::STAGE;
             const uint32_t tV = tK + C::TILE;
@@ -581,15 +628,12 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                     __syncwarp();
                 }
                 // ---- fragments: K (A of S^T), then V^T (A of O^T), all issued up front
-                const int mi = lane >> 3, r8 = lane & 7;
                 uint32_t kf[C::KSTEPS][4], vf[PA_TC_HOIST_V ? C::MTILES : 1][4];
 #pragma unroll
-                for (int ks = 0; ks < C::KSTEPS; ++ks)
-                    ldsm_x4(kf[ks], tile_chunk(tK, r8 + ((mi & 1) << 3), 2 * ks + (mi >> 1)));
+                for (int ks = 0; ks < C::KSTEPS; ++ks) ldsm_x4(kf[ks], tK + koff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
                 if constexpr (PA_TC_HOIST_V) {
 #pragma unroll
-                    for (int i = 0; i < C::MTILES; ++i)
-                        ldsm_x4_t(vf[i], tile_chunk(tV, r8 + ((mi >> 1) << 3), 2 * i + (mi & 1)));
+                    for (int i = 0; i < C::MTILES; ++i) ldsm_x4_t(vf[i], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
                 }
                 // ---- S^T = K . Q^T, four independent accumulator chains
                 float sa[4][4];
@@ -646,8 +690,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 #pragma unroll
                 for (int i = 0; i < C::MTILES; ++i) {
                     const int vi = PA_TC_HOIST_V ? i : 0;
-                    if constexpr (!PA_TC_HOIST_V)
-                        ldsm_x4_t(vf[vi], tile_chunk(tV, r8 + ((mi >> 1) << 3), 2 * i + (mi & 1)));
+                    if constexpr (!PA_TC_HOIST_V) ldsm_x4_t(vf[vi], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
                     Mma<T>::mma(o[i], vf[vi], pb0, pb1);
                     if constexpr (SPLIT_P) Mma<T>::mma(o[i], vf[vi], pl0, pl1);
                 }
@@ -655,6 +698,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             __syncwarp();
             refill();
             ++c_k;
+            if (j == 0) take_ticket();  // the previous segment's partial has drained by now
         }
         if (!alive) break;
 
@@ -664,7 +708,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             l0 += __shfl_xor_sync(0xffffffffu, l0, msk);
             l1 += __shfl_xor_sync(0xffffffffu, l1, msk);
         }
-        const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+        // l == 0 only when every block of the segment was skipped (bad table entries)
+        const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
         T *out = reinterpret_cast<T *>(a.out) + ((size_t)cs.b * a.Hq + (size_t)cs.kvh * G) * D;
         if (cs.j0 == 0 && cs.j1 == cs.nb) {  // the whole row: final output
 #pragma unroll
@@ -705,24 +750,17 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 if (h0 < G) a.ws_lse[(size_t)sl * G + h0] = m0 + log2f(l0);
                 if (h1 < G) a.ws_lse[(size_t)sl * G + h1] = m1 + log2f(l1);
             }
-            __syncwarp();
             resolve();
-            if (lane == 0) pend_old = atom_add_acq_rel_gpu(a.counters + (size_t)cs.b * Hkv + cs.kvh, 1);
-            pend = true;
-            pend_b = cs.b;
-            pend_kvh = cs.kvh;
-            pend_fr = cs.fr;
-            pend_nb = cs.nb;
+            take_ticket();  // a one-block segment's ticket may still be due
+            due = true;
+            due_b = cs.b;
+            due_kvh = cs.kvh;
+            due_fr = cs.fr;
+            due_nb = cs.nb;
         }
-        cit = nit;
-        cs = ns;
-        have = have_next;
-#pragma unroll
-        for (int s = 0; s < C::KSTEPS; ++s) {
-            bq[s][0] = bqn[s][0];
-            bq[s][1] = bqn[s][1];
-        }
+        have = next_seg(cit, cs);
     }
+    take_ticket();
     resolve();
 }
 
@@ -822,7 +860,7 @@ bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
 
 template <typename T, int D, int G>
 static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
-    using C = TcCfg<D>;
+    using C = TcCfg<D, G>;
     auto kern = decode_tc_kernel<T, D, G>;
     const int smem = C::smem_bytes(a.B);
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
