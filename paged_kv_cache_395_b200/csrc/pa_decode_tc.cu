@@ -611,22 +611,14 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             if (j == 0) load_q(s, bq);  // the segment's q came with its first block
             const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
             const uint32_t tK = ring + s * C::STAGE;
-            const uint32_t tV = tK + C::TILE;
             if (my_ok[s]) {
-                if (ntok < kBlockSize) {
-                    // rows past the sequence end hold stale data (possibly NaN/Inf):
-                    // zero those V rows so that 0-probability tokens add exactly 0
-                    unsigned char *vt = smem + (tV - smem_addr(smem));
-                    const int nrow = kBlockSize - ntok;
-                    for (int i = lane; i < nrow * C::BOXES * 8; i += 32) {
-                        const int r = ntok + i / (C::BOXES * 8);
-                        const int rem = i % (C::BOXES * 8);
-                        *reinterpret_cast<uint4 *>(vt + (rem >> 3) * C::BOX_BYTES + r * 128 + (rem & 7) * 16) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();  // before the stage is refilled by TMA
-                    __syncwarp();
-                }
+                // Slots past the sequence end hold stale data (possibly NaN/Inf); their
+                // probabilities are 0, and their V values are masked to 0 in the
+                // fragments so that they add exactly 0.  V^T fragment registers 0, 1
+                // hold tokens 2c, 2c+1 and registers 2, 3 tokens 2c+8, 2c+9 (low half
+                // = even token).
+                const uint32_t vm_lo = (2 * c < ntok ? 0x0000ffffu : 0u) | (2 * c + 1 < ntok ? 0xffff0000u : 0u);
+                const uint32_t vm_hi = (2 * c + 8 < ntok ? 0x0000ffffu : 0u) | (2 * c + 9 < ntok ? 0xffff0000u : 0u);
                 // ---- fragments: K (A of S^T), then V^T (A of O^T), all issued up front
                 uint32_t kf[C::KSTEPS][4], vf[PA_TC_HOIST_V ? C::MTILES : 1][4];
 #pragma unroll
@@ -634,6 +626,13 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 if constexpr (PA_TC_HOIST_V) {
 #pragma unroll
                     for (int i = 0; i < C::MTILES; ++i) ldsm_x4_t(vf[i], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
+#pragma unroll
+                    for (int i = 0; i < C::MTILES; ++i) {
+                        vf[i][0] &= vm_lo;
+                        vf[i][1] &= vm_lo;
+                        vf[i][2] &= vm_hi;
+                        vf[i][3] &= vm_hi;
+                    }
                 }
                 // ---- S^T = K . Q^T, four independent accumulator chains
                 float sa[4][4];
@@ -690,7 +689,13 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 #pragma unroll
                 for (int i = 0; i < C::MTILES; ++i) {
                     const int vi = PA_TC_HOIST_V ? i : 0;
-                    if constexpr (!PA_TC_HOIST_V) ldsm_x4_t(vf[vi], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
+                    if constexpr (!PA_TC_HOIST_V) {
+                        ldsm_x4_t(vf[vi], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
+                        vf[vi][0] &= vm_lo;
+                        vf[vi][1] &= vm_lo;
+                        vf[vi][2] &= vm_hi;
+                        vf[vi][3] &= vm_hi;
+                    }
                     Mma<T>::mma(o[i], vf[vi], pb0, pb1);
                     if constexpr (SPLIT_P) Mma<T>::mma(o[i], vf[vi], pl0, pl1);
                 }
