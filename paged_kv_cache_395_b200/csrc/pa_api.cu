@@ -97,8 +97,13 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
     const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
                             ? p->max_seq_len
                             : p->max_blocks_per_seq * PA_BLOCK_SIZE;
+    // the tensor-core family indexes cache rows and the concatenated block stream
+    // of all (sequence, KV head) rows with 32-bit integers
+    const int64_t stream_blocks =
+        (int64_t)p->num_seqs * p->num_kv_heads * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
     const bool tc_ok = decode_tc_supported(p->q_dtype, p->kv_dtype, p->head_dim, G, p->num_seqs) &&
-                       p->num_blocks * p->num_kv_heads * PA_BLOCK_SIZE <= 2147483647LL;
+                       p->num_blocks * p->num_kv_heads * PA_BLOCK_SIZE <= 2147483647LL &&
+                       stream_blocks <= (1LL << 30);
     if (p->algo == PA_ALGO_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
     *pl = Plan{};
     pl->max_len = max_len;

@@ -153,14 +153,14 @@ struct TcCfg {
 struct Seg {
     int b, kvh, L, nb;  // row: sequence, KV head, tokens, blocks
     int j0, j1;         // this segment: blocks [j0, j1) of the row
-    int64_t fr;         // index of the row's first block in the concatenated stream
+    int fr;             // index of the row's first block in the concatenated stream
     int ch;             // chunk that holds the segment (-1: whole-row mode)
 };
 
 // Walks the ranges of one warp and cuts them into segments at row boundaries.
 struct SegIter {
     int k;              // range counter
-    int64_t f, fend;    // position and end in the concatenated stream
+    int f, fend;        // position and end in the concatenated stream
     int ch;
     bool done;
 };
@@ -176,10 +176,10 @@ struct Win {
 // Chunks of the concatenated block stream: n chunks of c blocks (the last one
 // shorter); warp w takes chunks w, w + W, w + 2W, ...
 struct Chunks {
-    int64_t total, c, n;
-    __device__ int64_t start(int64_t ch) const { return ch * c; }
-    __device__ int64_t end(int64_t ch) const { return (ch + 1) * c < total ? (ch + 1) * c : total; }
-    __device__ int64_t of(int64_t f) const { return f / c; }
+    int total, c, n;
+    __device__ int start(int ch) const { return ch * c; }
+    __device__ int end(int ch) const { return (ch + 1) * c < total ? (ch + 1) * c : total; }
+    __device__ int of(int f) const { return f / c; }
 };
 
 // Ticket increment with release semantics at GPU scope: the warp's
@@ -263,7 +263,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         if (tid == C::THREADS - 1) cum[B] = run;
         __syncthreads();
     }
-    const int64_t total = (int64_t)cum[B] * Hkv;  // blocks of all rows
+    // blocks of all rows: the host sends this family only streams below 2^31 blocks
+    const int total = cum[B] * Hkv;
     const int gw = blockIdx.x * NW + warp;
     const int W = gridDim.x * NW;
     const bool rows_mode = a.tc_chunk < 0;
@@ -276,8 +277,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         if (a.tc_chunk > 0) {
             ck.c = a.tc_chunk;
         } else {
-            const int64_t wc = min(W, kTcMaxChunks);
-            const int64_t c = (total + wc - 1) / wc;
+            const int wc = min(W, kTcMaxChunks);
+            const int c = (total + wc - 1) / wc;
             ck.c = c > kTcMinChunk ? c : kTcMinChunk;
         }
         ck.n = (total + ck.c - 1) / ck.c;
@@ -292,23 +293,23 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         }
     }
 
-    auto locate = [&](int64_t f, Seg &sg) {
+    auto locate = [&](int f, Seg &sg) {
         int lo = 0, hi = B;  // largest b with cum[b] * Hkv <= f
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if ((int64_t)cum[mid] * Hkv <= f) lo = mid; else hi = mid;
+            if (cum[mid] * Hkv <= f) lo = mid; else hi = mid;
         }
         sg.b = lo;
         sg.nb = cum[lo + 1] - cum[lo];
-        const int64_t off = f - (int64_t)cum[lo] * Hkv;
+        const int off = f - cum[lo] * Hkv;
         sg.kvh = (int)(off / sg.nb);
-        sg.j0 = (int)(off - (int64_t)sg.kvh * sg.nb);
-        sg.fr = (int64_t)cum[lo] * Hkv + (int64_t)sg.kvh * sg.nb;
+        sg.j0 = off - sg.kvh * sg.nb;
+        sg.fr = cum[lo] * Hkv + sg.kvh * sg.nb;
         sg.L = lens[lo];
     };
 
     // ---- range schedule: rows w, w+W, ... (one pass) or chunks w, w+W, ...
-    auto set_range = [&](SegIter &it, int64_t ch) {
+    auto set_range = [&](SegIter &it, int ch) {
         it.f = ck.start(ch);
         it.fend = ck.end(ch);
         it.ch = (int)ch;
@@ -316,19 +317,19 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     auto range = [&](SegIter &it) -> bool {
         if (rows_mode) {
             for (;; ++it.k) {
-                const int64_t r = (int64_t)gw + (int64_t)it.k * W;
-                if (r >= (int64_t)B * Hkv) return false;
+                const int r = gw + it.k * W;
+                if (r >= B * Hkv) return false;
                 const int b = (int)(r / Hkv), kvh = (int)(r % Hkv);
                 const int nb = cum[b + 1] - cum[b];
                 if (nb > 0) {
-                    it.f = (int64_t)cum[b] * Hkv + (int64_t)kvh * nb;
+                    it.f = cum[b] * Hkv + kvh * nb;
                     it.fend = it.f + nb;
                     it.ch = -1;
                     return true;
                 }
             }
         }
-        const int64_t ch = (int64_t)gw + (int64_t)it.k * W;
+        const int ch = gw + it.k * W;
         if (ch >= ck.n) return false;
         set_range(it, ch);
         return true;
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             }
         }
         locate(it.f, sg);
-        const int64_t end = min(it.fend, sg.fr + sg.nb);
+        const int end = min(it.fend, sg.fr + sg.nb);
         sg.j1 = sg.j0 + (int)(end - it.f);
         sg.ch = it.ch;
         it.f = end;
@@ -484,21 +485,21 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     int pend_old = 0;
     bool pend = false;
     int pend_b = 0, pend_kvh = 0, pend_nb = 0;
-    int64_t pend_fr = 0;
+    int pend_fr = 0;
     bool due = false;  // a partial is written but its ticket is not taken yet
     int due_b = 0, due_kvh = 0, due_nb = 0;
-    int64_t due_fr = 0;
-    auto merge_row = [&](int b, int kvh, int64_t fr, int nb) {
+    int due_fr = 0, due_ck = 0;
+    auto merge_row = [&](int b, int kvh, int fr, int nb) {
         // Last segment of the row to finish: merge all of them,
         //   out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M).
         // Pass 1: lane (i, h) reads lse of segment i, head h (32 / G segments
         // per round) and keeps a running (max, sum); the lanes of a head then
         // combine theirs.  Pass 2: the partial outputs, NB segments x G heads
         // per round, all loads issued before they are used.
-        const int64_t ch_first = ck.of(fr), ch_last = ck.of(fr + nb - 1);
+        const int ch_first = ck.of(fr), ch_last = ck.of(fr + nb - 1);
         const int nseg = (int)(ch_last - ch_first + 1);
         auto slot_of = [&](int i) -> int {  // slot of the row's i-th segment
-            const int64_t ch = ch_first + i;
+            const int ch = ch_first + i;
             return (int)(2 * ch + ((i == 0 && fr > ck.start(ch)) ? 1 : 0));
         };
         constexpr int SPP = 32 / G;                 // segments per round of pass 1
@@ -575,9 +576,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             merge_row(pend_b, pend_kvh, pend_fr, pend_nb);
         }
     };
-    // The ticket of a partial is taken one block into the next segment (or at
-    // the end), when the partial's stores have drained, so the release costs
-    // the warp nothing; its result is read at the next segment end.
+    // The ticket of a partial is taken kTicketLag blocks after the partial was
+    // written (or at the next partial's end, or at the end), when its stores have
+    // drained, so that the release does not hold the warp; the ticket's result
+    // is read at the next partial's end.
+    constexpr int kTicketLag = 3;
     auto take_ticket = [&]() {
         if (!due) return;
         due = false;
@@ -703,7 +706,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             __syncwarp();
             refill();
             ++c_k;
-            if (j == 0) take_ticket();  // the previous segment's partial has drained by now
+            if (due && !pend && c_k >= due_ck + kTicketLag) take_ticket();
         }
         if (!alive) break;
 
@@ -732,8 +735,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         } else {
             // Partial of a row cut by chunk boundaries: chunk ch holds at most two
             // partial segments, its first (slot 2ch) and its last (slot 2ch+1).
-            const int64_t ch_first = ck.of(cs.fr), ch_last = ck.of(cs.fr + cs.nb - 1);
-            auto slot_of = [&](int64_t ch) -> int {
+            const int ch_first = ck.of(cs.fr), ch_last = ck.of(cs.fr + cs.nb - 1);
+            auto slot_of = [&](int ch) -> int {
                 return (int)(2 * ch + ((ch == ch_first && cs.fr > ck.start(ch)) ? 1 : 0));
             };
             const int sl = slot_of(cs.ch);
@@ -756,8 +759,9 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 if (h1 < G) a.ws_lse[(size_t)sl * G + h1] = m1 + log2f(l1);
             }
             resolve();
-            take_ticket();  // a one-block segment's ticket may still be due
+            take_ticket();
             due = true;
+            due_ck = c_k;
             due_b = cs.b;
             due_kvh = cs.kvh;
             due_fr = cs.fr;
@@ -765,6 +769,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         }
         have = next_seg(cit, cs);
     }
+    resolve();
     take_ticket();
     resolve();
 }
