@@ -309,7 +309,9 @@ def main(argv=None):
     if int8:
         dw.quantize_int8()
     stream = torch.cuda.Stream()
-    calls = runner.StepCalls(dw, part, int8, algo, stream)
+    # each decode follows this library's own reshape (or decode), which writes none of
+    # q, the tables or the lengths: the decode may read those before it finishes
+    calls = runner.StepCalls(dw, part, int8, algo, stream, flags=pa.PA_DECODE_INPUTS_READY)
     T = len(w.steps)
     sbytes = step_bytes(w, int8)
     stoks = step_tokens(w)
@@ -373,6 +375,7 @@ def main(argv=None):
                    "partition_size": "library picks (-1)" if part == -1 else part, "algo": args.algo,
                    "l2": "inputs larger than L2: KV pool and per-step reads exceed 126 MB, no flush",
                    "timing": "CUDA events around the K steps issued back to back",
+                   "decode_flags": "PA_DECODE_INPUTS_READY",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "decode_tokens_per_s": toks_rank * world / (ms_max * 1e-3),
         "hbm_frac_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
@@ -404,7 +407,7 @@ def time_e2e(dw, w, int8, part, algo, args, T, sbytes, stream, dist):
     slots, copy pairs, q, block tables, seq_lens, packed in one buffer), the
     library calls, and one device -> host copy of the decode output."""
     import torch
-    from paged_kv_cache_395_b200 import runner
+    from paged_kv_cache_395_b200 import pa, runner
 
     packs, h2d, d2h = [], [], []
     for i in range(T):
@@ -437,7 +440,7 @@ def time_e2e(dw, w, int8, part, algo, args, T, sbytes, stream, dist):
         views = packs[i][2]
         staged.steps[i] = [tuple(views.get(id(x), x) if isinstance(x, torch.Tensor) else x
                                  for x in op) for op in dw.steps[i]]
-    calls = runner.StepCalls(staged, part, int8, algo, stream)
+    calls = runner.StepCalls(staged, part, int8, algo, stream, flags=pa.PA_DECODE_INPUTS_READY)
     K = args.steps
     ctx = torch.cuda.stream(stream)  # copies and library calls on one stream, in order
     ctx.__enter__()

@@ -119,7 +119,24 @@ typedef struct pa_decode_params {
                                 ready for the next (its merge counters back at zero).  Calls
                                 that share a workspace must not overlap on the device. */
     size_t workspace_bytes;
+    int flags;               /* 0, or PA_DECODE_INPUTS_READY */
 } pa_decode_params;
+
+/*
+ * Every kernel of the library is launched with programmatic dependent launch
+ * allowed: it may become resident while the kernel before it on the stream
+ * finishes, and waits for that kernel to complete (with its writes visible)
+ * before it touches any memory.  PA_DECODE_INPUTS_READY lets pa_decode start
+ * earlier: it reads seq_lens, block_tables and q while the kernel just before
+ * it on the stream may still be running, and waits only before its first read
+ * of the caches (writes to out and the workspace also come after the wait).
+ * Set it only when that kernel does not write q, block_tables or seq_lens --
+ * for example when it is a pa_reshape_and_cache, pa_block_copy or pa_decode
+ * call of this library (each of which lets its successor start only after the
+ * kernels before it have completed).  The tensor-core family uses it; the
+ * CUDA-core family ignores it.
+ */
+#define PA_DECODE_INPUTS_READY 1
 
 /*
  * Bytes of device workspace pa_decode needs for these parameters (0 for

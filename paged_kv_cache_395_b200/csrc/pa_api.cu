@@ -64,6 +64,7 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
     }
     if (p->num_seqs > 65535 || p->num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
     if (p->algo < PA_ALGO_AUTO || p->algo > PA_ALGO_TENSOR) return PA_ERR_UNSUPPORTED;
+    if (p->flags & ~PA_DECODE_INPUTS_READY) return PA_ERR_UNSUPPORTED;
     int ps = p->partition_size;
     if (ps < -1 || (ps > 0 && ps % PA_BLOCK_SIZE)) return PA_ERR_SHAPE;
     const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
@@ -258,6 +259,7 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
         a.part = 0;
         a.max_parts = 1;
         a.tc_chunk = pl.tc_chunk;
+        a.early = (p->flags & PA_DECODE_INPUTS_READY) ? 1 : 0;
         if (pl.bytes > 0) {
             const size_t o_bytes = up256((size_t)pl.tc_slots * a.G * a.D * sizeof(float));
             const size_t l_bytes = up256((size_t)pl.tc_slots * a.G * sizeof(float));

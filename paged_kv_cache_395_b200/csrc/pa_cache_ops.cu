@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     char *__restrict__ vc, const int64_t *__restrict__ slots, int num_kv_heads, int row_bytes,
     int64_t k_stride_bytes, int64_t v_stride_bytes, int64_t num_slots) {
     using V = typename VecT<VEC>::type;
+    pdl_wait();  // the previous kernel may still read the slots this one overwrites
+    pdl_release_dependents();
     const int64_t i = blockIdx.x;
     const int64_t s = slots[i];
     if (s < 0) return;
@@ -59,14 +61,15 @@ int launch_reshape_and_cache(const void *k, const void *v, void *kc, void *vc,
     const char *kp = (const char *)k, *vp = (const char *)v;
     char *kcp = (char *)kc, *vcp = (char *)vc;
     const int64_t ns = N * kBlockSize;
+    cudaError_t e;
     switch (vec) {
-    case 16: reshape_and_cache_kernel<16><<<grid, threads, 0, st>>>(kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
-    case 8: reshape_and_cache_kernel<8><<<grid, threads, 0, st>>>(kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
-    case 4: reshape_and_cache_kernel<4><<<grid, threads, 0, st>>>(kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
-    case 2: reshape_and_cache_kernel<2><<<grid, threads, 0, st>>>(kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
-    default: reshape_and_cache_kernel<1><<<grid, threads, 0, st>>>(kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
+    case 16: e = launch_pdl(reshape_and_cache_kernel<16>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
+    case 8: e = launch_pdl(reshape_and_cache_kernel<8>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
+    case 4: e = launch_pdl(reshape_and_cache_kernel<4>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
+    case 2: e = launch_pdl(reshape_and_cache_kernel<2>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
+    default: e = launch_pdl(reshape_and_cache_kernel<1>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
     }
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -79,6 +82,8 @@ __global__ void __launch_bounds__(256) block_copy_kernel(
     char *__restrict__ kc, char *__restrict__ vc, float *__restrict__ ks, float *__restrict__ vs,
     const int64_t *__restrict__ pairs, int64_t num_blocks, int64_t blk_vecs, int64_t chunk,
     int num_kv_heads) {
+    pdl_wait();
+    pdl_release_dependents();
     const int64_t src = pairs[2 * (int64_t)blockIdx.x], dst = pairs[2 * (int64_t)blockIdx.x + 1];
     if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) {
         if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) raise_flag(PA_EFLAG_BAD_PAIR);
@@ -106,9 +111,9 @@ int launch_block_copy(void *kc, void *vc, float *ks, float *vs, const int64_t *p
     const int64_t chunk = 2048;  // 32 KB per CTA
     const int64_t chunks = (blk_vecs + chunk - 1) / chunk;
     dim3 grid((unsigned)n, (unsigned)chunks, 2);
-    block_copy_kernel<<<grid, 256, 0, st>>>((char *)kc, (char *)vc, ks, vs, pairs, N, blk_vecs,
-                                            chunk, H);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e = launch_pdl(block_copy_kernel, grid, dim3(256), 0, st, (char *)kc, (char *)vc, ks, vs,
+                                     pairs, N, blk_vecs, chunk, H);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -121,6 +126,8 @@ __global__ void __launch_bounds__(128) quantize_int8_kernel(const T *__restrict_
                                                             int8_t *__restrict__ dst,
                                                             float *__restrict__ scales, int tile) {
     __shared__ float red[4];
+    pdl_wait();
+    pdl_release_dependents();
     const int64_t t = blockIdx.x;
     const T *x = src + t * tile;
     float a = 0.f;
@@ -148,13 +155,15 @@ int launch_quantize_int8(const void *src, int src_dtype, int8_t *dst, float *sca
     const int64_t tiles = N * H;
     if (tiles == 0) return PA_OK;
     const int tile = kBlockSize * D;
+    cudaError_t e;
+    const dim3 grid((unsigned)tiles);
     switch (src_dtype) {
-    case PA_F32: quantize_int8_kernel<float><<<(unsigned)tiles, 128, 0, st>>>((const float *)src, dst, scales, tile); break;
-    case PA_F16: quantize_int8_kernel<__half><<<(unsigned)tiles, 128, 0, st>>>((const __half *)src, dst, scales, tile); break;
-    case PA_BF16: quantize_int8_kernel<__nv_bfloat16><<<(unsigned)tiles, 128, 0, st>>>((const __nv_bfloat16 *)src, dst, scales, tile); break;
+    case PA_F32: e = launch_pdl(quantize_int8_kernel<float>, grid, dim3(128), 0, st, (const float *)src, dst, scales, tile); break;
+    case PA_F16: e = launch_pdl(quantize_int8_kernel<__half>, grid, dim3(128), 0, st, (const __half *)src, dst, scales, tile); break;
+    case PA_BF16: e = launch_pdl(quantize_int8_kernel<__nv_bfloat16>, grid, dim3(128), 0, st, (const __nv_bfloat16 *)src, dst, scales, tile); break;
     default: return PA_ERR_DTYPE;
     }
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace pa

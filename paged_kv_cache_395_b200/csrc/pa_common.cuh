@@ -21,6 +21,37 @@ static __device__ unsigned int g_error_flags = 0;
 
 __device__ __forceinline__ void raise_flag(unsigned int bit) { atomicOr(&g_error_flags, bit); }
 
+// Programmatic dependent launch.  Every kernel of the library is launched with
+// programmatic stream serialisation allowed, so it may become resident while
+// the kernel before it on the stream is still finishing.  pdl_wait() returns
+// once every grid this one depends on has completed and its writes are
+// visible; nothing that a previous kernel may write (or read) is touched
+// before it.  pdl_release_dependents() lets the next grid start launching; the
+// kernels call it only after pdl_wait(), so a grid that starts early always
+// finds the grids before its own predecessor complete.  Both are no-ops for a
+// plain launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kern` on `st` with programmatic stream serialisation allowed.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 #define PA_ERROR_WORD_ACCESSOR(name)                                                        \
     int name(unsigned int *flags, bool reset) {                                             \
         if (cudaMemcpyFromSymbol(flags, g_error_flags, sizeof(unsigned int)) != cudaSuccess) \

@@ -112,6 +112,8 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
 
     const int part = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_release_dependents();
     const int L = effective_len(a, b);
     const int P = a.part > 0 ? a.part : max(L, 1);
     const int t0 = part * P;
@@ -311,6 +313,8 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
 template <typename TQ>
 __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
     const int qh = blockIdx.x, b = blockIdx.y;
+    pdl_wait();  // the partials of the decode kernel before it
+    pdl_release_dependents();
     const int L = effective_len(a, b);
     if (L <= a.part) return;  // one partition (or none): written by the decode kernel
     const int np = ceil_div(L, a.part);
@@ -347,11 +351,10 @@ static int launch_one(const DecodeArgs &a, cudaStream_t st) {
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::SMEM)) return PA_ERR_CUDA;
     const int parts = a.part > 0 ? a.max_parts : 1;
     dim3 grid((unsigned)parts, (unsigned)a.Hkv, (unsigned)a.B);
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    if (launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, st, a) != cudaSuccess) return PA_ERR_CUDA;
     if (a.part > 0 && a.max_parts > 1) {
-        merge_kernel<TQ><<<dim3((unsigned)a.Hq, (unsigned)a.B), 128, 0, st>>>(a);
-        if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+        if (launch_pdl(merge_kernel<TQ>, dim3((unsigned)a.Hq, (unsigned)a.B), dim3(128), 0, st, a) != cudaSuccess)
+            return PA_ERR_CUDA;
     }
     return PA_OK;
 }

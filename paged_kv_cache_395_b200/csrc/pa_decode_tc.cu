@@ -233,6 +233,14 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = a.B, Hkv = a.Hkv;
+    // Without PA_DECODE_INPUTS_READY nothing is read before the previous kernel
+    // on the stream has finished; with it, the lengths, the block tables and q
+    // are read first (the caller guarantees that kernel does not write them) and
+    // the wait comes just before the first cache tile is requested.
+    if (!a.early) {
+        pdl_wait();
+        pdl_release_dependents();
+    }
 
     // ---- effective lengths and blocks per sequence -> exclusive prefix sum cum[0..B] ----
     {
@@ -284,14 +292,6 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         ck.n = (total + ck.c - 1) / ck.c;
     }
 
-    // rows of sequences with no token produce zeros
-    for (int r = gw; r < B * Hkv; r += W) {
-        const int b = r / Hkv;
-        if (cum[b + 1] == cum[b]) {
-            T *o = reinterpret_cast<T *>(a.out) + ((size_t)b * a.Hq + (size_t)(r % Hkv) * G) * D;
-            for (int i = lane; i < G * D; i += 32) o[i] = Cvt<T>::from_f(0.f);
-        }
-    }
 
     auto locate = [&](int f, Seg &sg) {
         int lo = 0, hi = B;  // largest b with cum[b] * Hkv <= f
@@ -440,6 +440,18 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             p_y_next = win_load(pn);
         }
     };
+    if (a.early) {
+        pdl_wait();
+        pdl_release_dependents();
+    }
+    // rows of sequences with no token produce zeros
+    for (int r = gw; r < B * Hkv; r += W) {
+        const int b = r / Hkv;
+        if (cum[b + 1] == cum[b]) {
+            T *o = reinterpret_cast<T *>(a.out) + ((size_t)b * a.Hq + (size_t)(r % Hkv) * G) * D;
+            for (int i = lane; i < G * D; i += 32) o[i] = Cvt<T>::from_f(0.f);
+        }
+    }
 #pragma unroll
     for (int i = 0; i < S; ++i) refill();
     __syncwarp();
@@ -888,8 +900,8 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     const int64_t need = (blocks + C::NW - 1) / C::NW;
     if (need < ctas) ctas = need;
     if (ctas < 1) ctas = 1;
-    kern<<<(unsigned)ctas, C::THREADS, smem, st>>>(tk, tv, a);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), smem, st, tk, tv, a) == cudaSuccess ? PA_OK
+                                                                                             : PA_ERR_CUDA;
 }
 
 template <typename T, int D>

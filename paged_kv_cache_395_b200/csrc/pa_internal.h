@@ -46,6 +46,8 @@ struct DecodeArgs {
     int *counters;           // [B][Hkv] merge tickets, zero between calls
     int tc_chunk;            // tensor-core schedule: blocks per chunk, 0 = balanced auto,
                              // -1 = whole rows (one pass)
+    int early;               // PA_DECODE_INPUTS_READY: read lengths, tables and q before
+                             // the previous kernel on the stream has finished
 };
 
 // Tensor-core schedule limits: the auto schedule cuts the block stream into at

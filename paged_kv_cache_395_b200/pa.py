@@ -27,6 +27,7 @@ PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_ALIGN = -4, -5, -6, -7
 PA_F32, PA_F16, PA_BF16, PA_I8 = 0, 1, 2, 3
 PA_ALGO_AUTO, PA_ALGO_SIMT, PA_ALGO_TENSOR = 0, 1, 2
 PA_EFLAG_BAD_BLOCK, PA_EFLAG_BAD_SLOT, PA_EFLAG_BAD_PAIR, PA_EFLAG_WAIT_TIMEOUT = 1, 2, 4, 8
+PA_DECODE_INPUTS_READY = 1
 BLOCK_SIZE = 16
 
 _TORCH_DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16,
@@ -56,6 +57,7 @@ class PaDecodeParams(ctypes.Structure):
         ("algo", ctypes.c_int),
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
+        ("flags", ctypes.c_int),
     ]
 
 
@@ -136,7 +138,7 @@ def pa_reshape_and_cache(k, v, key_cache, value_cache, slot_mapping, stream=None
 
 
 def make_params(q, key_cache, block_tables, max_seq_len, k_scales=None, v_scales=None,
-                partition_size=0, workspace=None, algo=PA_ALGO_AUTO) -> PaDecodeParams:
+                partition_size=0, workspace=None, algo=PA_ALGO_AUTO, flags=0) -> PaDecodeParams:
     B, Hq, d = q.shape
     N, Hkv, bs, _ = key_cache.shape
     p = PaDecodeParams()
@@ -152,7 +154,20 @@ def make_params(q, key_cache, block_tables, max_seq_len, k_scales=None, v_scales
     p.algo = int(algo)
     p.workspace = None if workspace is None else workspace.data_ptr()
     p.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    p.flags = int(flags)
     return p
+
+
+def uses_tensor_cores(q, key_cache, algo=PA_ALGO_AUTO) -> bool:
+    """Whether pa_decode runs the tensor-core family for these operands (the
+    library's rule: fp16/bf16 q with a cache of the same dtype, head_dim 64 or
+    128, group size 1, 2, 4 or 8, at most 4096 sequences)."""
+    B, Hq, d = q.shape
+    Hkv = key_cache.shape[1]
+    G = Hq // Hkv
+    ok = (q.dtype in (torch.float16, torch.bfloat16) and key_cache.dtype == q.dtype
+          and d in (64, 128) and G in (1, 2, 4, 8) and B <= 4096)
+    return algo == PA_ALGO_TENSOR or (algo == PA_ALGO_AUTO and ok)
 
 
 def pa_decode_workspace_size(q, key_cache, block_tables, max_seq_len, partition_size=0,
@@ -171,9 +186,10 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor | None:
 
 def pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max_seq_len,
               k_scales=None, v_scales=None, partition_size=0, workspace=None,
-              algo=PA_ALGO_AUTO, stream=None, params=None):
+              algo=PA_ALGO_AUTO, stream=None, params=None, flags=0):
     """out, q [B][H_q][d]; caches [N][H_kv][16][d]; block_tables int32 [B][M];
-    seq_lens int32 [B] (including the decoded token)."""
+    seq_lens int32 [B] (including the decoded token).  flags: 0 or
+    PA_DECODE_INPUTS_READY (see include/pa.h)."""
     _dev(out, q, key_cache, value_cache, block_tables, seq_lens, k_scales, v_scales, workspace)
     for t, n in ((out, "out"), (q, "q"), (key_cache, "key_cache"), (value_cache, "value_cache"),
                  (block_tables, "block_tables"), (seq_lens, "seq_lens")):
@@ -184,7 +200,8 @@ def pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max
     if out.dtype != q.dtype or out.shape != q.shape:
         raise ValueError("out must match q in shape and dtype")
     p = params if params is not None else make_params(
-        q, key_cache, block_tables, max_seq_len, k_scales, v_scales, partition_size, workspace, algo)
+        q, key_cache, block_tables, max_seq_len, k_scales, v_scales, partition_size, workspace, algo,
+        flags)
     _check(lib.pa_decode(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache),
                          _ptr(block_tables), _ptr(seq_lens), ctypes.c_float(scale),
                          ctypes.byref(p), _stream(stream)), "pa_decode")

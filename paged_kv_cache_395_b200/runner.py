@@ -118,7 +118,7 @@ class StepCalls:
     ctypes call per library entry point and nothing else on the host."""
 
     def __init__(self, dw: DeviceWorkload, partition_size=-1, int8=False, algo=pa.PA_ALGO_AUTO,
-                 stream=None):
+                 stream=None, flags=0):
         import ctypes
         self.dw = dw
         self.stream = stream if stream is not None else torch.cuda.current_stream()
@@ -160,13 +160,17 @@ class StepCalls:
                         launches += 1
                 else:
                     _, q, bt, sl, mx, out = op
-                    p = pa.make_params(q, kc, bt, mx, ks, vs, partition_size, self.workspace, algo)
+                    p = pa.make_params(q, kc, bt, mx, ks, vs, partition_size, self.workspace, algo,
+                                       flags)
                     self.keep.append(p)
                     split = pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+                    # the tensor-core family merges inside its decode kernel; the
+                    # CUDA-core family launches a merge kernel after a split decode
+                    tc = pa.uses_tensor_cores(q, kc, algo)
                     args = (ptr(out), ptr(q), ptr(kc), ptr(vc), ptr(bt), ptr(sl),
                             ctypes.c_float(w.scale), ctypes.byref(p), sp)
                     calls.append(("decode", pa.lib.pa_decode, args))
-                    launches += 2 if split else 1
+                    launches += 2 if (split and not tc) else 1
             self.calls[i] = calls
             self.launches[i] = launches
 

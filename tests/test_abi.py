@@ -64,6 +64,7 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails val
     (dict(q_dtype=9), pa.PA_ERR_DTYPE),
     (dict(partition_size=24), pa.PA_ERR_SHAPE),
     (dict(partition_size=-2), pa.PA_ERR_SHAPE),
+    (dict(flags=2), pa.PA_ERR_UNSUPPORTED),          # unknown flag bit
     (dict(num_seqs=-1), pa.PA_ERR_SHAPE),
     (dict(algo=7), pa.PA_ERR_UNSUPPORTED),
 ])

@@ -251,3 +251,49 @@ def test_ragged_full_trace():
     torch.cuda.synchronize()
     assert np.array_equal(bits(dw.kc), kc.view(np.uint8))
     assert np.array_equal(bits(dw.vc), vc.view(np.uint8))
+
+
+@pytest.mark.slow
+def test_ragged_trace_back_to_back_inputs_ready():
+    """The benchmark's exact issue pattern: all 128 steps (append, then decode)
+    through the pre-marshalled C-ABI calls on one stream with no synchronisation
+    in between, decodes flagged PA_DECODE_INPUTS_READY, so each kernel may start
+    while the one before it finishes.  Sampled steps against the oracle, caches
+    bit-exact at the end."""
+    w = W.ragged()
+    sample = {0, 5, 47, 90, 127}
+    ref, kc, vc = replay(w, want=lambda s: s in sample)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    calls = runner.StepCalls(dw, -1, False, pa.PA_ALGO_AUTO, stream, flags=pa.PA_DECODE_INPUTS_READY)
+    with torch.cuda.stream(stream):
+        for i in range(len(w.steps)):
+            calls.run(i)
+    torch.cuda.synchronize()
+    for i in sorted(sample):
+        out = dw.steps[i][-1][-1]
+        assert_close(out, ref[i], "float16", f"ragged step {i}")
+    assert np.array_equal(bits(dw.kc), kc.view(np.uint8))
+    assert np.array_equal(bits(dw.vc), vc.view(np.uint8))
+
+
+@pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_TENSOR])
+def test_inputs_ready_flag_same_result(algo):
+    """The early-start flag changes when the kernel waits, not what it computes."""
+    w = W.random_case([1, 16, 33, 700, 1500], num_q_heads=32, num_kv_heads=8, head_dim=128, seed=12)
+    ref, _, _ = replay(w)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    _, q, bt, sl, mx, _ = dw.steps[0][-1]
+    outs = []
+    for flags in (0, pa.PA_DECODE_INPUTS_READY):
+        out = torch.empty_like(q)
+        ws = dw.workspace_for(dw.steps[0][-1], -1, algo=algo)
+        pa.pa_decode(out, q, dw.kc, dw.vc, bt, sl, w.scale, mx, partition_size=-1, workspace=ws,
+                     algo=algo, flags=flags)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(outs[0]), bits(outs[1]))
+    assert_close(outs[1], ref[0], "float16", "inputs-ready")
