@@ -15,11 +15,14 @@ kernels, same byte counts).
 
 value = algorithmic KV-read bytes of the timed decode steps / device time of
 those steps (CUDA events around the whole step: append + decode + merge),
-inputs resident in HBM.  The KV pool (1.1 GB) and the bytes read per step
-(218-498 MB) are larger than the 126 MB L2, so no flush is needed between
-steps.  e2e = the same metric through the C ABI with the per-step inputs in
+inputs resident in HBM.  On the ragged trace the KV pool (1.1 GB) and the
+bytes read per step (140-566 MB) are larger than the 126 MB L2, so the steps
+run back to back with no flush; a workload whose steps read less than twice
+the L2 size is timed step by step with the L2 flushed in between (outside the
+events).  e2e = the same metric through the C ABI with the per-step inputs in
 pinned host memory copied in and the outputs copied out inside the timed
-region.  For N > 1 (torchrun) every rank runs an independent replica on its
+region, the copies on their own streams overlapping other steps' kernels as a
+serving loop would.  For N > 1 (torchrun) every rank runs an independent replica on its
 own GPU (the decode path has no exchange step); value = bytes of all ranks /
 max over ranks of the device time.
 
@@ -51,8 +54,8 @@ FALLBACK_HBM_GBS = 6650.0
 # It holds only for the kernel code it was taken on (hash of the source without
 # comments); after any code change the bench reports null until it is taken again.
 NCU_TRAFFIC = {
-    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "7151f0ec1a012d51",
-               "per_alg_byte": (475345920 + 4564480 + 462447872 + 5231616) / (472969728 + 459894508)},
+    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "e22851808f126c40",
+               "per_alg_byte": (475626240 + 5227008 + 462720512 + 4452864) / (472969728 + 459894508)},
 }
 
 
@@ -318,37 +321,55 @@ def main(argv=None):
     torch.cuda.synchronize()
 
     # ---- device-resident timing ----------------------------------------------------------
-    # One event pair around the K timed steps issued back to back (the host enqueues
-    # a step in well under the step's device time, so the device never waits); a
-    # second loop of only the decode calls of the same steps times the dominant kernel.
+    # Steps that read more than twice the L2 size: one event pair around the K timed
+    # steps issued back to back (the host enqueues a step in well under the step's
+    # device time, so the device never waits), then a second loop of only the decode
+    # calls of the same steps for the dominant kernel.  Smaller steps: each step
+    # timed by its own event pair, with the L2 flushed (a write of twice its size)
+    # before it, outside the events.
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    per_step = max(sbytes) < 2 * l2
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device="cuda") if per_step else None
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             calls.run(i % T)
     torch.cuda.synchronize()
     K = args.steps
     idx = [(args.warmup + j) % T for j in range(K)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(run_one):
+        """(device ms, host enqueue ms) of run_one(i) over idx; the device time
+        is the sum of per-step event pairs when the L2 is flushed between steps."""
+        if not per_step:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            h0 = time.perf_counter()
+            a.record(stream)
+            for i in idx:
+                run_one(i)
+            b.record(stream)
+            host = (time.perf_counter() - h0) * 1e3
+            torch.cuda.synchronize()
+            return a.elapsed_time(b), host
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in idx]
+        h0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            for n, i in enumerate(idx):
+                flush.fill_(n & 0xff)
+                evs[n][0].record(stream)
+                run_one(i)
+                evs[n][1].record(stream)
+        host = (time.perf_counter() - h0) * 1e3
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs), host
+
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        h0 = time.perf_counter()
-        start.record(stream)
-        for i in idx:
-            calls.run(i)
-        end.record(stream)
-        host_ms = (time.perf_counter() - h0) * 1e3
-        torch.cuda.synchronize()
+        ms, host_ms = timed(calls.run)
     if dist is not None:
         dist.barrier()
-    ms = start.elapsed_time(end)
-    d0.record(stream)
-    for i in idx:
-        calls.run_decode_only(i)
-    d1.record(stream)
-    torch.cuda.synchronize()
-    dec_ms = d0.elapsed_time(d1)
+    dec_ms, _ = timed(calls.run_decode_only)
     bytes_rank = sum(sbytes[i] for i in idx)
     toks_rank = sum(stoks[i] for i in idx)
     launches = sum(calls.launches[i] for i in idx)
@@ -373,8 +394,11 @@ def main(argv=None):
         "scaling": "weak", "vs_baseline": None, "dtype": "i8" if int8 else "f16", "data": "synthetic",
         "config": {"workload": WORKLOADS[args.workload], "name": args.workload,
                    "partition_size": "library picks (-1)" if part == -1 else part, "algo": args.algo,
-                   "l2": "inputs larger than L2: KV pool and per-step reads exceed 126 MB, no flush",
-                   "timing": "CUDA events around the K steps issued back to back",
+                   "l2": ("L2 flushed before every timed step (write of twice the L2 size, "
+                          "outside the events)" if per_step else
+                          "inputs larger than L2: every step reads more than twice the L2 size, no flush"),
+                   "timing": ("one CUDA event pair per step, summed" if per_step else
+                              "CUDA events around the K steps issued back to back"),
                    "decode_flags": "PA_DECODE_INPUTS_READY",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "decode_tokens_per_s": toks_rank * world / (ms_max * 1e-3),
@@ -405,7 +429,8 @@ def main(argv=None):
 def time_e2e(dw, w, int8, part, algo, args, T, sbytes, stream, dist):
     """Per step: one pinned host -> device copy of the step's inputs (new k/v,
     slots, copy pairs, q, block tables, seq_lens, packed in one buffer), the
-    library calls, and one device -> host copy of the decode output."""
+    library calls, and one device -> host copy of the decode output; the copies
+    of one step overlap the computation of others."""
     import torch
     from paged_kv_cache_395_b200 import pa, runner
 
@@ -442,31 +467,55 @@ def time_e2e(dw, w, int8, part, algo, args, T, sbytes, stream, dist):
                                  for x in op) for op in dw.steps[i]]
     calls = runner.StepCalls(staged, part, int8, algo, stream, flags=pa.PA_DECODE_INPUTS_READY)
     K = args.steps
-    ctx = torch.cuda.stream(stream)  # copies and library calls on one stream, in order
-    ctx.__enter__()
-    for i in range(args.warmup):
-        host, dev, _, out, host_out = packs[i % T]
-        dev.copy_(host, non_blocking=True)
-        calls.run(i % T)
-        host_out.copy_(out.view(torch.uint8).view(-1), non_blocking=True)
+    # Pipelined like a serving loop: step j's inputs are copied in on one copy
+    # stream while earlier steps compute on `stream`, and each step's output is
+    # copied out on another; events order copy -> compute -> copy per step, and
+    # a staging buffer is refilled only after the step that used it T steps
+    # earlier has finished with it.
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ring = 2 * T
+    ev_h2d = [torch.cuda.Event() for _ in range(ring)]
+    ev_comp = [torch.cuda.Event() for _ in range(ring)]
+    ev_d2h = [torch.cuda.Event() for _ in range(ring)]
+
+    def issue(j):
+        i = j % T
+        host, dev, _, out, host_out = packs[i]
+        if j >= T:
+            h2d_s.wait_event(ev_comp[(j - T) % ring])
+        with torch.cuda.stream(h2d_s):
+            dev.copy_(host, non_blocking=True)
+        ev_h2d[j % ring].record(h2d_s)
+        stream.wait_event(ev_h2d[j % ring])
+        if j >= T:
+            stream.wait_event(ev_d2h[(j - T) % ring])
+        calls.run(i)
+        ev_comp[j % ring].record(stream)
+        d2h_s.wait_event(ev_comp[j % ring])
+        with torch.cuda.stream(d2h_s):
+            host_out.copy_(out.view(torch.uint8).view(-1), non_blocking=True)
+        ev_d2h[j % ring].record(d2h_s)
+        return i
+
+    for j in range(args.warmup):
+        issue(j)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
+    start.record(h2d_s)
+    stream.wait_event(start)
+    d2h_s.wait_event(start)
     nbytes, hb, db = 0, 0, 0
-    for j in range(K):
-        i = (args.warmup + j) % T
-        host, dev, _, out, host_out = packs[i]
-        dev.copy_(host, non_blocking=True)
-        calls.run(i)
-        host_out.copy_(out.view(torch.uint8).view(-1), non_blocking=True)
+    for j in range(args.warmup, args.warmup + K):
+        i = issue(j)
         nbytes += sbytes[i]
         hb += h2d[i]
         db += d2h[i]
-    end.record(stream)
+    d2h_s.wait_stream(stream)
+    d2h_s.wait_stream(h2d_s)
+    end.record(d2h_s)
     torch.cuda.synchronize()
-    ctx.__exit__(None, None, None)
     ms = start.elapsed_time(end)
     world = 1
     if dist is not None:
