@@ -128,12 +128,15 @@ template <> struct Mma<__nv_bfloat16> {
 #define PA_TC_MIN_CTAS 1
 #endif
 
-template <int D, int G>
+// TKV: the cache element, the q/out type T or int8_t.  A tile row is D * sizeof(TKV)
+// bytes, brought in as 128-byte boxes (64 fp16/bf16 or 128 int8 elements).
+template <typename TKV, int D, int G>
 struct TcCfg {
     static constexpr int NW = PA_TC_WARPS;        // warps (independent workers) per CTA
     static constexpr int THREADS = NW * 32;
     static constexpr int S = PA_TC_STAGES;        // ring stages per warp
-    static constexpr int BOXES = D / 64;          // 64-element (128-byte) boxes per row
+    static constexpr int BOXW = 128 / (int)sizeof(TKV);  // elements per box row
+    static constexpr int BOXES = D / BOXW;        // boxes per tile row
     static constexpr int BOX_BYTES = 16 * 128;    // one box of a tile
     static constexpr int TILE = BOXES * BOX_BYTES;
     static constexpr int STAGE = 2 * TILE;        // K tile, then V tile
@@ -145,7 +148,8 @@ struct TcCfg {
     static constexpr int QRING_OFF = RING;        // [NW][S] q slots, one per stage
     static constexpr int BAR_OFF = QRING_OFF + NW * S * QSLOT;
     static constexpr int OK_OFF = BAR_OFF + NW * S * 8;
-    static constexpr int CUM_OFF = OK_OFF + NW * S * 4;
+    static constexpr int SC_OFF = OK_OFF + NW * S * 4;    // float [NW][S][2]: int8 K, V scales
+    static constexpr int CUM_OFF = SC_OFF + NW * S * 8;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (2 * B + 2) * 4; }
 };
 
@@ -216,18 +220,97 @@ template <> struct FVec<2> {
     static __device__ __forceinline__ float get(const float2 &v, int e) { return e == 0 ? v.x : v.y; }
 };
 
-template <typename T, int D, int G>
+// ---------------------------------------------------------------------------
+// int8 tiles -> fp16 MMA fragments
+// ---------------------------------------------------------------------------
+// Two int8 values -> two fp16 values, exactly.  u holds the bytes biased by 128
+// (word ^ 0x80808080); the byte permute builds the fp16 bit patterns 0x64xx =
+// 1024 + (x + 128) for the two bytes picked by `sel`, and subtracting 1152
+// (0x6480) leaves x.  Every value involved is an integer below 2048, so fp16
+// holds all of them exactly.
+__device__ __forceinline__ uint32_t i8x2_to_h2(uint32_t u, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(u), "r"(0x64646464u), "r"(sel));
+    asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(r) : "r"(0x64806480u));
+    return r;
+}
+constexpr uint32_t kLoPair = 0x5140u;  // bytes 0, 1 -> low, high half
+constexpr uint32_t kHiPair = 0x5342u;  // bytes 2, 3 -> low, high half
+
+__device__ __forceinline__ void lds_v4(uint32_t (&w)[4], uint32_t addr) {
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr)
+                 : "memory");
+}
+// 16-byte chunk `ch` of row `r` of a 128-byte-row tile written by TMA with
+// 128-byte swizzle
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int r, int ch) { return tile + r * 128 + ((ch ^ (r & 7)) << 4); }
+
+// K (A operand of S^T = K . Q^T; m = tokens, k = dims) from an int8 tile of 16
+// tokens x 128 dims.  The contraction runs over the dims in the order that lets
+// a thread read its own 32 contiguous bytes: in k-step ks, thread column c holds
+// the dims 32c + 4ks .. 32c + 4ks + 3 (k slots 2c, 2c+1 <- dims +0, +1; k slots
+// 2c+8, 2c+9 <- dims +2, +3), and q is read in the same order.  kload_i8 reads
+// the raw words (biased by 128), kfrag_i8 converts the fragment of one k-step.
+__device__ __forceinline__ void kload_i8(uint32_t (&w)[2][8], uint32_t tile, int g, int c) {
+    lds_v4(*reinterpret_cast<uint32_t(*)[4]>(&w[0][0]), swz(tile, g, 2 * c));
+    lds_v4(*reinterpret_cast<uint32_t(*)[4]>(&w[0][4]), swz(tile, g, 2 * c + 1));
+    lds_v4(*reinterpret_cast<uint32_t(*)[4]>(&w[1][0]), swz(tile, g + 8, 2 * c));
+    lds_v4(*reinterpret_cast<uint32_t(*)[4]>(&w[1][4]), swz(tile, g + 8, 2 * c + 1));
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[r][j] ^= 0x80808080u;
+}
+__device__ __forceinline__ void kfrag_i8(const uint32_t (&w)[2][8], int ks, uint32_t (&a)[4]) {
+    a[0] = i8x2_to_h2(w[0][ks], kLoPair);  // token g, k slots 2c, 2c+1
+    a[1] = i8x2_to_h2(w[1][ks], kLoPair);  // token g + 8
+    a[2] = i8x2_to_h2(w[0][ks], kHiPair);  // token g, k slots 2c+8, 2c+9
+    a[3] = i8x2_to_h2(w[1][ks], kHiPair);
+}
+
+// V^T (A operand of O^T += V^T . P^T; m = dims, k = tokens) from an int8 tile.
+// Thread row g owns the 16 dims 16g .. 16g + 15: m-tile i, row g is dim
+// 16g + i and row g + 8 is dim 16g + 8 + i.  The k slots are the tokens
+// themselves (2c, 2c+1 and 2c+8, 2c+9), as the P^T fragments expect.  vload_i8
+// reads the four token rows' 16 bytes (biased by 128), vfrag_i8 converts the
+// fragment of m-tile i: byte i % 4 of word i / 4 (row g) or 2 + i / 4 (row
+// g + 8) of each token, paired by token.
+__device__ __forceinline__ void vload_i8(uint32_t (&r)[4][4], uint32_t tile, int g, int c) {
+    lds_v4(r[0], swz(tile, 2 * c, g));
+    lds_v4(r[1], swz(tile, 2 * c + 1, g));
+    lds_v4(r[2], swz(tile, 2 * c + 8, g));
+    lds_v4(r[3], swz(tile, 2 * c + 9, g));
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r[t][j] ^= 0x80808080u;
+}
+__device__ __forceinline__ void vfrag_i8(const uint32_t (&r)[4][4], int i, uint32_t (&a)[4]) {
+    const uint32_t sel = (uint32_t)(i & 3) | ((uint32_t)(4 + (i & 3)) << 4);  // byte i%4 of both tokens
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // register q: token pair q / 2, dims row (q & 1 ? g + 8 : g)
+        const int p = q >> 1, w = ((q & 1) << 1) + (i >> 2);
+        uint32_t t;
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(r[2 * p][w]), "r"(r[2 * p + 1][w]), "r"(sel));
+        a[q] = i8x2_to_h2(t, kLoPair);
+    }
+}
+
+template <typename T, typename TKV, int D, int G>
 __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
                                                                      const DecodeArgs a) {
-    using C = TcCfg<D, G>;
+    using C = TcCfg<TKV, D, G>;
     constexpr int NW = C::NW, S = C::S;
     constexpr bool SPLIT_P = sizeof(T) == 2 && !std::is_same<T, __half>::value;  // bf16: P = hi + lo
+    constexpr bool kI8 = std::is_same<TKV, int8_t>::value;
+    static_assert(!kI8 || (std::is_same<T, __half>::value && D == 128), "int8 caches: fp16 q, head_dim 128");
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     int *stage_ok = reinterpret_cast<int *>(smem + C::OK_OFF);
+    float *stage_sc = reinterpret_cast<float *>(smem + C::SC_OFF);
     int *cum = reinterpret_cast<int *>(smem + C::CUM_OFF);  // [B + 1] blocks before sequence b
     int *lens = cum + a.B + 1;                                // [B] effective lengths
 
@@ -389,20 +472,33 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             win_first(w);
         }
     };
-    auto win_load = [&](const Win &w) -> int {
+    // lane l: TMA row of the window's entry l (-1: none, -2: block id outside
+    // the pool); for int8 caches also that block's K and V scales
+    float p_ks = 0.f, p_vs = 0.f, p_ks_next = 0.f, p_vs_next = 0.f;
+    auto win_load = [&](const Win &w, float &ks, float &vs) -> int {
         if (!w.valid || lane >= w.n) return -1;
         const int pb = a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
         if (pb < 0 || (int64_t)pb >= a.N) return -2;
+        if constexpr (kI8) {
+            ks = a.ks[(size_t)pb * Hkv + w.sg.kvh];
+            vs = a.vs[(size_t)pb * Hkv + w.sg.kvh];
+        }
         return (pb * Hkv + w.sg.kvh) * kBlockSize;
     };
     Win pc, pn;
     win_first(pc);
     win_after(pc, pn);
-    int p_y = win_load(pc), p_y_next = win_load(pn);
+    int p_y = win_load(pc, p_ks, p_vs), p_y_next = win_load(pn, p_ks_next, p_vs_next);
     int p_i = 0, p_k = 0;
+    float *my_sc = stage_sc + warp * S * 2;
     auto refill = [&]() {
         if (!pc.valid) return;
         const int y = __shfl_sync(0xffffffffu, p_y, p_i);
+        float ksv = 0.f, vsv = 0.f;
+        if constexpr (kI8) {
+            ksv = __shfl_sync(0xffffffffu, p_ks, p_i);
+            vsv = __shfl_sync(0xffffffffu, p_vs, p_i);
+        }
         if (lane == 0) {
             const int s = p_k % S;
             uint64_t *bar = &my_bars[s];
@@ -411,6 +507,10 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             const bool seg_first = pc.o == 0 && p_i == 0;
             const uint32_t tx = (y < 0 ? 0u : (uint32_t)C::STAGE) + (seg_first ? kQBytes : 0u);
             my_ok[s] = y >= 0;
+            if constexpr (kI8) {
+                my_sc[2 * s] = ksv;  // released to the consumer by the arrive below
+                my_sc[2 * s + 1] = vsv;
+            }
             if (y < 0) raise_flag(PA_EFLAG_BAD_BLOCK);
             if (tx == 0) {
                 mbar_arrive(bar);
@@ -421,8 +521,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 const uint32_t dst = ring + s * C::STAGE;
 #pragma unroll
                 for (int bx = 0; bx < C::BOXES; ++bx) {
-                    tma_load_2d(dst + bx * C::BOX_BYTES, &tmK, bx * 64, y, smem_addr(bar));
-                    tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * 64, y, smem_addr(bar));
+                    tma_load_2d(dst + bx * C::BOX_BYTES, &tmK, bx * C::BOXW, y, smem_addr(bar));
+                    tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * C::BOXW, y, smem_addr(bar));
                 }
             }
             if (seg_first) {
@@ -436,8 +536,10 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             p_i = 0;
             pc = pn;
             p_y = p_y_next;
+            p_ks = p_ks_next;
+            p_vs = p_vs_next;
             win_after(pc, pn);
-            p_y_next = win_load(pn);
+            p_y_next = win_load(pn, p_ks_next, p_vs_next);
         }
     };
     if (a.early) {
@@ -458,15 +560,21 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 
     // ---- consumer ------------------------------------------------------------------------
     const int g = lane >> 2, c = lane & 3;  // mma fragment coordinates
+    // O^T row (m-tile i, row g; row g + 8 is dim + 8) -> head dim: m-tile i holds
+    // dims 16i .. 16i + 15 for fp16/bf16 tiles; the int8 path gives thread row g
+    // the 16 dims 16g .. 16g + 15 instead (see vfrag_i8)
+    auto dmap = [&](int i, int gg) -> int { return kI8 ? 16 * gg + i : 16 * i + gg; };
     const int h0 = 2 * c, h1 = 2 * c + 1;  // heads of this thread's S^T / O^T columns
-    // B fragments of q (n = heads, k = dims) from the q slot of stage s
+    // B fragments of q (n = heads, k = dims) from the q slot of stage s.  The
+    // int8 path orders the contraction's dims differently (see kfrag_i8): k-step
+    // ks, thread column c covers dims 32c + 4ks .. 32c + 4ks + 3.
     auto load_q = [&](int s, uint32_t (&bq)[C::KSTEPS][2]) {
-        const uint32_t qs = qring + s * C::QSLOT + (g * D + 2 * c) * 2;
+        const uint32_t qs = qring + s * C::QSLOT + (kI8 ? (g * D + 32 * c) * 2 : (g * D + 2 * c) * 2);
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS; ++ks) {
             if (g < G) {
-                bq[ks][0] = lds_u32(qs + ks * 32);
-                bq[ks][1] = lds_u32(qs + ks * 32 + 16);
+                bq[ks][0] = lds_u32(qs + (kI8 ? ks * 8 : ks * 32));
+                bq[ks][1] = lds_u32(qs + (kI8 ? ks * 8 + 4 : ks * 32 + 16));
             } else {
                 bq[ks][0] = bq[ks][1] = 0u;
             }
@@ -635,7 +743,20 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 const uint32_t vm_lo = (2 * c < ntok ? 0x0000ffffu : 0u) | (2 * c + 1 < ntok ? 0xffff0000u : 0u);
                 const uint32_t vm_hi = (2 * c + 8 < ntok ? 0x0000ffffu : 0u) | (2 * c + 9 < ntok ? 0xffff0000u : 0u);
                 // ---- fragments: K (A of S^T), then V^T (A of O^T), all issued up front
-                uint32_t kf[C::KSTEPS][4], vf[PA_TC_HOIST_V ? C::MTILES : 1][4];
+                constexpr bool kHoist = PA_TC_HOIST_V && !kI8;
+                uint32_t kf[kI8 ? 1 : C::KSTEPS][4], vf[kHoist ? C::MTILES : 1][4];
+                uint32_t kw[kI8 ? 2 : 1][8], vw[kI8 ? 4 : 1][4];  // raw int8 words
+                float slog = a.scale_log2, vsc = 1.f;
+                if constexpr (kI8) {
+                    // int8 tiles (128-byte rows, 128-byte swizzle), converted exactly to fp16 in
+                    // registers fragment by fragment; the block's K scale goes into the score
+                    // scale, its V scale into the probabilities fed to P.V (the softmax sum
+                    // keeps the unscaled ones)
+                    slog *= my_sc[2 * s];
+                    vsc = my_sc[2 * s + 1];
+                    kload_i8(kw, tK, g, c);
+                    vload_i8(vw, tK + C::TILE, g, c);
+                } else {
 #pragma unroll
                 for (int ks = 0; ks < C::KSTEPS; ++ks) ldsm_x4(kf[ks], tK + koff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
                 if constexpr (PA_TC_HOIST_V) {
@@ -649,21 +770,29 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                         vf[i][3] &= vm_hi;
                     }
                 }
+                }
                 // ---- S^T = K . Q^T, four independent accumulator chains
                 float sa[4][4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) sa[u][0] = sa[u][1] = sa[u][2] = sa[u][3] = 0.f;
 #pragma unroll
-                for (int ks = 0; ks < C::KSTEPS; ++ks) Mma<T>::mma(sa[ks & 3], kf[ks], bq[ks][0], bq[ks][1]);
+                for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                    if constexpr (kI8) {
+                        kfrag_i8(kw, ks, kf[0]);
+                        Mma<T>::mma(sa[ks & 3], kf[0], bq[ks][0], bq[ks][1]);
+                    } else {
+                        Mma<T>::mma(sa[ks & 3], kf[ks], bq[ks][0], bq[ks][1]);
+                    }
+                }
                 float sc[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sc[e] = (sa[0][e] + sa[1][e]) + (sa[2][e] + sa[3][e]);
                 // ---- online softmax (log2 domain): rows g, g+8 are tokens, columns heads
                 const bool v0 = g < ntok, v1 = g + 8 < ntok;
-                const float s0 = v0 ? sc[0] * a.scale_log2 : -INFINITY;
-                const float s1 = v0 ? sc[1] * a.scale_log2 : -INFINITY;
-                const float s2 = v1 ? sc[2] * a.scale_log2 : -INFINITY;
-                const float s3 = v1 ? sc[3] * a.scale_log2 : -INFINITY;
+                const float s0 = v0 ? sc[0] * slog : -INFINITY;
+                const float s1 = v0 ? sc[1] * slog : -INFINITY;
+                const float s2 = v1 ? sc[2] * slog : -INFINITY;
+                const float s3 = v1 ? sc[3] * slog : -INFINITY;
                 float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
                 for (int msk = 4; msk < 32; msk <<= 1) {
@@ -688,7 +817,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                     }
                 }
                 // ---- P^T fragments (k = tokens, n = heads): transpose the S^T layout
-                const uint32_t ph01 = Mma<T>::pack(p0, p1), ph23 = Mma<T>::pack(p2, p3);
+                const uint32_t ph01 = Mma<T>::pack(p0 * vsc, p1 * vsc), ph23 = Mma<T>::pack(p2 * vsc, p3 * vsc);
                 const uint32_t pb0 = movm_t(ph01);  // tokens 0-7
                 const uint32_t pb1 = movm_t(ph23);  // tokens 8-15
                 uint32_t pl0 = 0, pl1 = 0;
@@ -697,14 +826,20 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                     // bf16 operand so that P enters the product to ~16 bits
                     const float r0 = __uint_as_float(ph01 << 16), r1 = __uint_as_float(ph01 & 0xffff0000u);
                     const float r2 = __uint_as_float(ph23 << 16), r3 = __uint_as_float(ph23 & 0xffff0000u);
-                    pl0 = movm_t(Mma<T>::pack(p0 - r0, p1 - r1));
-                    pl1 = movm_t(Mma<T>::pack(p2 - r2, p3 - r3));
+                    pl0 = movm_t(Mma<T>::pack(p0 * vsc - r0, p1 * vsc - r1));
+                    pl1 = movm_t(Mma<T>::pack(p2 * vsc - r2, p3 * vsc - r3));
                 }
                 // ---- O^T += V^T . P^T
 #pragma unroll
                 for (int i = 0; i < C::MTILES; ++i) {
-                    const int vi = PA_TC_HOIST_V ? i : 0;
-                    if constexpr (!PA_TC_HOIST_V) {
+                    const int vi = kHoist ? i : 0;
+                    if constexpr (kI8) {
+                        vfrag_i8(vw, i, vf[0]);
+                        vf[0][0] &= vm_lo;
+                        vf[0][1] &= vm_lo;
+                        vf[0][2] &= vm_hi;
+                        vf[0][3] &= vm_hi;
+                    } else if constexpr (!PA_TC_HOIST_V) {
                         ldsm_x4_t(vf[vi], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
                         vf[vi][0] &= vm_lo;
                         vf[vi][1] &= vm_lo;
@@ -734,7 +869,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         if (cs.j0 == 0 && cs.j1 == cs.nb) {  // the whole row: final output
 #pragma unroll
             for (int i = 0; i < C::MTILES; ++i) {
-                const int d0 = 16 * i + g, d1 = d0 + 8;
+                const int d0 = dmap(i, g), d1 = d0 + 8;
                 if (h0 < G) {
                     out[h0 * D + d0] = Cvt<T>::from_f(o[i][0] * inv0);
                     out[h0 * D + d1] = Cvt<T>::from_f(o[i][2] * inv0);
@@ -754,7 +889,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             const int sl = slot_of(cs.ch);
 #pragma unroll
             for (int i = 0; i < C::MTILES; ++i) {
-                const int d0 = 16 * i + g, d1 = d0 + 8;
+                const int d0 = dmap(i, g), d1 = d0 + 8;
                 if (h0 < G) {
                     float *w = a.ws_o + ((size_t)sl * G + h0) * D;
                     w[d0] = o[i][0] * inv0;
@@ -802,8 +937,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D map over a cache viewed as [rows = N*H_kv*16][D] with 64-element boxes
-// of 16 rows and 128-byte swizzle.  Encoded maps are cached by (address,
+// 2-D map over a cache viewed as [rows = N*H_kv*16][D] with boxes of 16 rows
+// of 128 bytes (64 fp16/bf16 or 128 int8 elements) and 128-byte swizzle.  Encoded maps are cached by (address,
 // rows, D, dtype): the encode is a host call of a few microseconds.
 static bool cache_tensor_map(CUtensorMap *m, const void *base, int64_t rows, int D, int dtype) {
     struct Key {
@@ -830,12 +965,14 @@ static bool cache_tensor_map(CUtensorMap *m, const void *base, int64_t rows, int
     }
     auto fn = encode_fn();
     if (!fn) return false;
+    const int esize = dtype == PA_I8 ? 1 : 2;
     cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64, 16};
+    cuuint64_t strides[1] = {(cuuint64_t)D * esize};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 16};  // 128-byte box rows
     cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapDataType dt =
-        dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapDataType dt = dtype == PA_BF16  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : dtype == PA_I8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -876,14 +1013,15 @@ static bool launch_shape(const void *kernel, int threads, int smem, int *sms, in
 }
 
 bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
-    return (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype && (D == 64 || D == 128) &&
-           (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
+    const bool same = (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype && (D == 64 || D == 128);
+    const bool i8 = q_dtype == PA_F16 && kv_dtype == PA_I8 && D == 128;
+    return (same || i8) && (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
 }
 
-template <typename T, int D, int G>
+template <typename T, typename TKV, int D, int G>
 static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
-    using C = TcCfg<D, G>;
-    auto kern = decode_tc_kernel<T, D, G>;
+    using C = TcCfg<TKV, D, G>;
+    auto kern = decode_tc_kernel<T, TKV, D, G>;
     const int smem = C::smem_bytes(a.B);
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
     if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are read as aligned 32-bit pairs
@@ -904,21 +1042,27 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
                                                                                              : PA_ERR_CUDA;
 }
 
-template <typename T, int D>
+template <typename T, typename TKV, int D>
 static int launch_tc_g(const DecodeArgs &a, cudaStream_t st) {
     switch (a.G) {
-    case 1: return launch_tc<T, D, 1>(a, st);
-    case 2: return launch_tc<T, D, 2>(a, st);
-    case 4: return launch_tc<T, D, 4>(a, st);
-    case 8: return launch_tc<T, D, 8>(a, st);
+    case 1: return launch_tc<T, TKV, D, 1>(a, st);
+    case 2: return launch_tc<T, TKV, D, 2>(a, st);
+    case 4: return launch_tc<T, TKV, D, 4>(a, st);
+    case 8: return launch_tc<T, TKV, D, 8>(a, st);
     default: return PA_ERR_UNSUPPORTED;
     }
 }
 
 int launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
-    if (a.q_dtype == PA_F16) return a.D == 64 ? launch_tc_g<__half, 64>(a, st) : launch_tc_g<__half, 128>(a, st);
+    if (a.q_dtype == PA_F16 && a.kv_dtype == PA_I8) {
+        if (a.D != 128) return PA_ERR_UNSUPPORTED;
+        return launch_tc_g<__half, int8_t, 128>(a, st);
+    }
+    if (a.q_dtype == PA_F16)
+        return a.D == 64 ? launch_tc_g<__half, __half, 64>(a, st) : launch_tc_g<__half, __half, 128>(a, st);
     if (a.q_dtype == PA_BF16)
-        return a.D == 64 ? launch_tc_g<__nv_bfloat16, 64>(a, st) : launch_tc_g<__nv_bfloat16, 128>(a, st);
+        return a.D == 64 ? launch_tc_g<__nv_bfloat16, __nv_bfloat16, 64>(a, st)
+                         : launch_tc_g<__nv_bfloat16, __nv_bfloat16, 128>(a, st);
     return PA_ERR_DTYPE;
 }
 

@@ -85,10 +85,12 @@ def test_random_cases(case, part, algo):
     assert_close(got[0], ref[0], w.dtype, case)
 
 
-@pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_AUTO])
+@pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("part", [0, 32, -1])
 @pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
 def test_int8_random(qdt, part, algo):
+    if algo == pa.PA_ALGO_TENSOR and qdt != "float16":
+        pytest.skip("the tensor-core family reads int8 caches with fp16 q")
     w = W.random_case([1, 17, 96, 400], num_q_heads=16, num_kv_heads=4, head_dim=128, dtype=qdt,
                       seed=4)
     dw = runner.DeviceWorkload(w)
@@ -99,6 +101,23 @@ def test_int8_random(qdt, part, algo):
     op = w.steps[0][0]
     ref = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
     assert_close(got[0], ref, qdt, "int8")
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 4), (32, 8)])
+@pytest.mark.parametrize("part", [0, 16, -1])
+def test_int8_tensor_group_sizes(hq, hkv, part):
+    """int8 caches on the tensor-core family for every group size, ragged tails,
+    one-pass, one-block and library-picked partitions, against the oracle
+    dequantising the same int8 values."""
+    w = W.random_case([1, 15, 16, 33, 250, 777], num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
+                      dtype="float16", seed=hq + hkv)
+    dw = runner.DeviceWorkload(w)
+    got, dw = run_gpu(w, part, pa.PA_ALGO_TENSOR, int8=True, dw=dw)
+    kc8, vc8 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
+    ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
+    op = w.steps[0][0]
+    ref = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
+    assert_close(got[0], ref, "float16", f"int8 tensor G={hq // hkv} part={part}")
 
 
 def test_tensor_path_rejects_unsupported():
