@@ -192,6 +192,26 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
 
 
+def max_over_ranks(ms, dist, device="cuda"):
+    """Device time of the slowest rank: every rank times its own replica, and
+    the job's time is the largest of them (one all-reduce; identity without a
+    process group)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([float(ms)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(bytes_rank, ms, dist, device="cuda"):
+    """(GB/s of the whole job, max-over-ranks ms): the ranks run identical
+    replicas, so the job moves bytes_rank x world bytes in the slowest rank's time."""
+    world = 1 if dist is None else dist.get_world_size()
+    ms_max = max_over_ranks(ms, dist, device)
+    return bytes_rank * world / (ms_max * 1e-3) / 1e9, ms_max
+
+
 def dist_setup(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -373,13 +393,7 @@ def main(argv=None):
     bytes_rank = sum(sbytes[i] for i in idx)
     toks_rank = sum(stoks[i] for i in idx)
     launches = sum(calls.launches[i] for i in idx)
-    ms_max = ms
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    total_bytes = bytes_rank * world
-    value = total_bytes / (ms_max * 1e-3) / 1e9
+    value, ms_max = replica_throughput(bytes_rank, ms, dist)
     peak, peak_kind = load_peak()
     achieved = bytes_rank / (dec_ms * 1e-3) / 1e9
 
@@ -517,13 +531,8 @@ def time_e2e(dw, w, int8, part, algo, args, T, sbytes, stream, dist):
     end.record(d2h_s)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
-    world = 1
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-        world = dist.get_world_size()
-    return {"value": nbytes * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
+    value, ms = replica_throughput(nbytes, ms, dist)
+    return {"value": value, "unit": "GB/s",
             "h2d_bytes_per_step": hb // K, "d2h_bytes_per_step": db // K, "ms_per_step": ms / K}
 
 
