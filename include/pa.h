@@ -94,8 +94,10 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
 typedef struct pa_decode_params {
     int num_seqs;            /* B >= 0 */
     int num_q_heads;         /* H_q, a multiple of num_kv_heads */
-    int num_kv_heads;        /* H_kv; group size G = H_q / H_kv must be 1, 2, 4 or 8 */
-    int head_dim;            /* 64 or 128 */
+    int num_kv_heads;        /* H_kv; group size G = H_q / H_kv: 1, 2, 4, 8, 16, 32 or 64
+                                (groups above 8, e.g. MQA with H_kv = 1, run as 8-head
+                                groups that each read the KV head's tiles) */
+    int head_dim;            /* 64 or 128; 256 on the CUDA-core family (not with PA_F32) */
     int block_size;          /* must be PA_BLOCK_SIZE */
     int max_blocks_per_seq;  /* row stride of block_tables */
     int64_t num_blocks;      /* physical blocks in the pool */

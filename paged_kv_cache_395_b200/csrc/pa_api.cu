@@ -46,6 +46,27 @@ static int auto_partition(int B, int Hkv, int max_len) {
     return 64;
 }
 
+// The heads as the kernels see them.  A group of more than 8 query heads per KV
+// head (16, 32 or 64: MQA-style) is split into 8-head groups, and each group is
+// a virtual KV head that reads the same cache tiles; the virtual heads of one
+// cache head are adjacent rows, so their repeated tile reads meet in L2.
+struct KernelHeads {
+    int G, Hkv, shift;  // group size <= 8, virtual KV heads, log2(groups per cache head)
+};
+static bool kernel_heads(const pa_decode_params *p, KernelHeads *kh) {
+    const int G = p->num_q_heads / p->num_kv_heads;
+    int shift = 0;
+    if (G > 8) {
+        const int groups = G / 8;
+        if (G % 8 || groups > 8 || (groups & (groups - 1))) return false;
+        while ((1 << shift) < groups) ++shift;
+    }
+    kh->G = G > 8 ? 8 : G;
+    kh->Hkv = p->num_kv_heads << shift;
+    kh->shift = shift;
+    return true;
+}
+
 // Checks shared by pa_decode and pa_decode_workspace_size.  Fills the partition
 // size actually used (auto resolved) and the partition count.
 static int check_decode_params(const pa_decode_params *p, int *part, int *max_parts) {
@@ -56,13 +77,14 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
     if (p->num_q_heads % p->num_kv_heads) return PA_ERR_SHAPE;
     if (p->block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
     if (!elem_size(p->q_dtype) || !elem_size(p->kv_dtype) || p->q_dtype == PA_I8) return PA_ERR_DTYPE;
-    const int G = p->num_q_heads / p->num_kv_heads;
-    if (!decode_simt_supported(p->q_dtype, p->kv_dtype, p->head_dim, G)) {
+    KernelHeads kh;
+    const bool heads_ok = kernel_heads(p, &kh);
+    if (!heads_ok || !decode_simt_supported(p->q_dtype, p->kv_dtype, p->head_dim, kh.G)) {
         const bool pair_ok = (p->q_dtype == p->kv_dtype) || p->kv_dtype == PA_I8;
         if (!pair_ok || (p->kv_dtype == PA_I8 && p->q_dtype == PA_F32)) return PA_ERR_DTYPE;
         return PA_ERR_UNSUPPORTED;
     }
-    if (p->num_seqs > 65535 || p->num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (p->num_seqs > 65535 || kh.Hkv > 65535) return PA_ERR_UNSUPPORTED;
     if (p->algo < PA_ALGO_AUTO || p->algo > PA_ALGO_TENSOR) return PA_ERR_UNSUPPORTED;
     if (p->flags & ~PA_DECODE_INPUTS_READY) return PA_ERR_UNSUPPORTED;
     int ps = p->partition_size;
@@ -70,7 +92,7 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
     const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
                             ? p->max_seq_len
                             : p->max_blocks_per_seq * PA_BLOCK_SIZE;
-    if (ps == -1) ps = auto_partition(p->num_seqs, p->num_kv_heads, max_len);
+    if (ps == -1) ps = auto_partition(p->num_seqs, kh.Hkv, max_len);
     if (ps > 0 && max_len <= ps) ps = 0;  // one partition: no split needed
     *part = ps;
     *max_parts = ps > 0 ? (max_len + ps - 1) / ps : 1;
@@ -94,14 +116,16 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
     int part = 0, mp = 0;
     const int rc = check_decode_params(p, &part, &mp);
     if (rc != PA_OK) return rc;
-    const int G = p->num_q_heads / p->num_kv_heads;
+    KernelHeads kh;
+    kernel_heads(p, &kh);
+    const int G = kh.G;
     const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
                             ? p->max_seq_len
                             : p->max_blocks_per_seq * PA_BLOCK_SIZE;
     // the tensor-core family indexes cache rows and the concatenated block stream
     // of all (sequence, KV head) rows with 32-bit integers
     const int64_t stream_blocks =
-        (int64_t)p->num_seqs * p->num_kv_heads * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
+        (int64_t)p->num_seqs * kh.Hkv * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
     const bool tc_ok = decode_tc_supported(p->q_dtype, p->kv_dtype, p->head_dim, G, p->num_seqs) &&
                        p->num_blocks * p->num_kv_heads * PA_BLOCK_SIZE <= 2147483647LL &&
                        stream_blocks <= (1LL << 30);
@@ -112,14 +136,14 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
     if (!pl->tc) {
         pl->part = part;
         pl->max_parts = mp;
-        pl->bytes = decode_workspace_bytes(p->num_seqs, p->num_q_heads, p->num_kv_heads, p->head_dim, max_len, part);
+        pl->bytes = decode_workspace_bytes(p->num_seqs, p->num_q_heads, kh.Hkv, p->head_dim, max_len, part);
         return PA_OK;
     }
     if (p->partition_size == 0 || max_len == 0) {
         pl->tc_chunk = -1;  // one warp per (sequence, KV head) row, no workspace
         return PA_OK;
     }
-    const int64_t tmax = (int64_t)p->num_seqs * p->num_kv_heads * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
+    const int64_t tmax = (int64_t)p->num_seqs * kh.Hkv * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
     int64_t nchunks;
     if (p->partition_size > 0) {
         pl->tc_chunk = p->partition_size / PA_BLOCK_SIZE;
@@ -134,7 +158,7 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
     // per (sequence, KV head) row
     pl->bytes = up256((size_t)pl->tc_slots * G * p->head_dim * sizeof(float)) +
                 up256((size_t)pl->tc_slots * G * sizeof(float)) +
-                up256((size_t)p->num_seqs * p->num_kv_heads * sizeof(int));
+                up256((size_t)p->num_seqs * kh.Hkv * sizeof(int));
     return PA_OK;
 }
 
@@ -238,9 +262,12 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     a.scale_log2 = scale * kLog2e;
     a.B = p->num_seqs;
     a.Hq = p->num_q_heads;
-    a.Hkv = p->num_kv_heads;
+    KernelHeads kh;
+    kernel_heads(p, &kh);
+    a.Hkv = kh.Hkv;
+    a.hg_shift = kh.shift;
     a.D = p->head_dim;
-    a.G = p->num_q_heads / p->num_kv_heads;
+    a.G = kh.G;
     a.mbps = p->max_blocks_per_seq;
     a.N = p->num_blocks;
     a.max_len = pl.max_len;

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
         my_blk[s] = pb;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&my_bars[s], 2 * TILE);
-        const size_t off = ((size_t)pb * a.Hkv + kvh) * TILE;
+        const size_t off = ((size_t)pb * (a.Hkv >> a.hg_shift) + (kvh >> a.hg_shift)) * TILE;
         bulk_g2s(my_ring + s * C::STAGE_BYTES, reinterpret_cast<const char *>(a.kc) + off, TILE, &my_bars[s]);
         bulk_g2s(my_ring + s * C::STAGE_BYTES + TILE, reinterpret_cast<const char *>(a.vc) + off, TILE,
                  &my_bars[s]);
@@ -199,8 +199,9 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
         if (pb >= 0) {
             float ksc = 1.f, vsc = 1.f;
             if constexpr (sizeof(TKV) == 1) {
-                ksc = a.ks[(size_t)pb * a.Hkv + kvh];
-                vsc = a.vs[(size_t)pb * a.Hkv + kvh];
+                const size_t si = (size_t)pb * (a.Hkv >> a.hg_shift) + (kvh >> a.hg_shift);
+                ksc = a.ks[si];
+                vsc = a.vs[si];
             }
             // ---- scores of the 16 tokens, lane holds (token pass*TPP+grp, head hj)
             float sc[PASSES];
@@ -375,6 +376,9 @@ static int launch_d(const DecodeArgs &a, cudaStream_t st) {
     switch (a.D) {
     case 64: return launch_g<TQ, TKV, 64>(a, st);
     case 128: return launch_g<TQ, TKV, 128>(a, st);
+    case 256:
+        if constexpr (sizeof(TKV) <= 2) return launch_g<TQ, TKV, 256>(a, st);
+        return PA_ERR_UNSUPPORTED;  // a 4-byte 256-dim ring does not fit shared memory
     default: return PA_ERR_UNSUPPORTED;
     }
 }
@@ -383,7 +387,8 @@ bool decode_simt_supported(int q_dtype, int kv_dtype, int D, int G) {
     const bool pair_ok = (q_dtype == PA_F32 && kv_dtype == PA_F32) ||
                          (q_dtype == PA_F16 && (kv_dtype == PA_F16 || kv_dtype == PA_I8)) ||
                          (q_dtype == PA_BF16 && (kv_dtype == PA_BF16 || kv_dtype == PA_I8));
-    return pair_ok && (D == 64 || D == 128) && (G == 1 || G == 2 || G == 4 || G == 8);
+    const bool d_ok = D == 64 || D == 128 || (D == 256 && kv_dtype != PA_F32);
+    return pair_ok && d_ok && (G == 1 || G == 2 || G == 4 || G == 8);
 }
 
 int launch_decode_simt(const DecodeArgs &a, cudaStream_t st) {

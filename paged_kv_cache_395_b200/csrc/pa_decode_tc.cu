@@ -479,11 +479,12 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         if (!w.valid || lane >= w.n) return -1;
         const int pb = a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
         if (pb < 0 || (int64_t)pb >= a.N) return -2;
+        const int hc = Hkv >> a.hg_shift, kc = w.sg.kvh >> a.hg_shift;  // the cache's KV head
         if constexpr (kI8) {
-            ks = a.ks[(size_t)pb * Hkv + w.sg.kvh];
-            vs = a.vs[(size_t)pb * Hkv + w.sg.kvh];
+            ks = a.ks[(size_t)pb * hc + kc];
+            vs = a.vs[(size_t)pb * hc + kc];
         }
-        return (pb * Hkv + w.sg.kvh) * kBlockSize;
+        return (pb * hc + kc) * kBlockSize;
     };
     Win pc, pn;
     win_first(pc);
@@ -1026,7 +1027,7 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
     if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are read as aligned 32-bit pairs
     CUtensorMap tk, tv;
-    const int64_t rows = a.N * a.Hkv * kBlockSize;
+    const int64_t rows = a.N * (a.Hkv >> a.hg_shift) * kBlockSize;  // the cache's rows
     if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
         return PA_ERR_CUDA;
     int sms = 0, per_sm = 0;

@@ -34,7 +34,10 @@ struct DecodeArgs {
     const int32_t *tables;
     const int32_t *lens;
     float scale_log2;        // scale * log2(e): scores are kept in the log2 domain
-    int B, Hq, Hkv, D, G;
+    int B, Hq, Hkv, D, G;    // Hkv, G: the kernel's KV heads and group size.  A group of
+                             // more than 8 query heads is split into 8-head groups, each a
+                             // virtual KV head: Hkv = real KV heads << hg_shift, G = 8.
+    int hg_shift;            // log2(virtual KV heads per cache KV head)
     int mbps;                // max_blocks_per_seq
     int64_t N;               // num_blocks
     int max_len;             // effective bound on seq_lens

@@ -161,14 +161,14 @@ def make_params(q, key_cache, block_tables, max_seq_len, k_scales=None, v_scales
 def uses_tensor_cores(q, key_cache, algo=PA_ALGO_AUTO) -> bool:
     """Whether pa_decode runs the tensor-core family for these operands (the
     library's rule: fp16/bf16 q with a cache of the same dtype and head_dim 64 or
-    128, or fp16 q with an int8 cache and head_dim 128; group size 1, 2, 4 or 8;
-    at most 4096 sequences)."""
+    128, or fp16 q with an int8 cache and head_dim 128; group size 1 to 64 (groups
+    above 8 run as 8-head groups); at most 4096 sequences)."""
     B, Hq, d = q.shape
     Hkv = key_cache.shape[1]
     G = Hq // Hkv
     same = q.dtype in (torch.float16, torch.bfloat16) and key_cache.dtype == q.dtype and d in (64, 128)
     i8 = q.dtype == torch.float16 and key_cache.dtype == torch.int8 and d == 128
-    ok = (same or i8) and G in (1, 2, 4, 8) and B <= 4096
+    ok = (same or i8) and G in (1, 2, 4, 8, 16, 32, 64) and B <= 4096
     return algo == PA_ALGO_TENSOR or (algo == PA_ALGO_AUTO and ok)
 
 

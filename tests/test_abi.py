@@ -65,6 +65,9 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails val
     (dict(partition_size=24), pa.PA_ERR_SHAPE),
     (dict(partition_size=-2), pa.PA_ERR_SHAPE),
     (dict(flags=2), pa.PA_ERR_UNSUPPORTED),          # unknown flag bit
+    (dict(num_q_heads=48, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),  # G = 24: not 8 x a power of 2
+    (dict(num_q_heads=256, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),  # G = 128
+    (dict(head_dim=256, q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32), pa.PA_ERR_UNSUPPORTED),
     (dict(num_seqs=-1), pa.PA_ERR_SHAPE),
     (dict(algo=7), pa.PA_ERR_UNSUPPORTED),
 ])
@@ -151,3 +154,22 @@ def test_product_path_does_not_touch_oracle():
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", src, flags=re.M), f
                 assert not re.search(r"#include\s*[<\"][^>\"]*oracle", src), f
                 assert "liboracle" not in src and "pa_oracle" not in src, f
+
+
+def test_large_groups_and_head_dim_256_are_planned():
+    """G = 16, 32, 64 run as 8-head groups: the workspace of a G = 32, H_kv = 1
+    decode equals that of G = 8, H_kv = 4 (same query heads, same rows); head_dim
+    256 is accepted on the CUDA-core family."""
+    big = params(num_q_heads=32, num_kv_heads=1, partition_size=16, algo=pa.PA_ALGO_TENSOR)
+    same = params(num_q_heads=32, num_kv_heads=4, partition_size=16, algo=pa.PA_ALGO_TENSOR)
+    n = pa.lib.pa_decode_workspace_size(ctypes.byref(big))
+    assert n > 0 and n == pa.lib.pa_decode_workspace_size(ctypes.byref(same))
+    for g in (16, 64):
+        p = params(num_q_heads=g, num_kv_heads=1, partition_size=16)
+        assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+    p = params(head_dim=256, partition_size=16, algo=pa.PA_ALGO_SIMT)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+    # the tensor-core family stops at head_dim 128
+    p = params(head_dim=256, algo=pa.PA_ALGO_TENSOR)
+    assert pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p),
+                            None) == pa.PA_ERR_UNSUPPORTED

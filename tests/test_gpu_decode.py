@@ -316,3 +316,54 @@ def test_inputs_ready_flag_same_result(algo):
     torch.cuda.synchronize()
     assert np.array_equal(bits(outs[0]), bits(outs[1]))
     assert_close(outs[1], ref[0], "float16", "inputs-ready")
+
+
+# -- wider shapes: MQA-style large groups, head_dim 256 ------------------------------------
+@pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_TENSOR])
+@pytest.mark.parametrize("hq,hkv", [(16, 1), (32, 1), (64, 1), (32, 2)])
+@pytest.mark.parametrize("part", [0, 16, -1])
+def test_large_groups(hq, hkv, part, algo):
+    """G = 16 .. 64 (H_kv = 1 is MQA) run as 8-head groups over the same KV
+    tiles; both families against the oracle, ragged tails included."""
+    w = W.random_case([1, 16, 40, 300, 901], num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
+                      dtype="float16", seed=hq * 7 + hkv)
+    ref, _, _ = replay(w)
+    got, _ = run_gpu(w, part, algo)
+    assert_close(got[0], ref[0], "float16", f"G={hq // hkv} part={part}")
+
+
+@pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
+def test_large_group_bf16_and_int8(qdt):
+    w = W.random_case([7, 129, 640], num_q_heads=64, num_kv_heads=1, head_dim=128, dtype=qdt, seed=77)
+    ref, _, _ = replay(w)
+    got, dw = run_gpu(w, -1)
+    assert_close(got[0], ref[0], qdt, "MQA G=64")
+    got8, dw = run_gpu(w, -1, int8=True, dw=runner.DeviceWorkload(w))
+    kc8, vc8 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
+    ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
+    op = w.steps[0][0]
+    ref8 = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
+    assert_close(got8[0], ref8, qdt, "MQA G=64 int8")
+
+
+@pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 4), (32, 4), (32, 1)])
+@pytest.mark.parametrize("part", [0, 32, -1])
+def test_head_dim_256(qdt, hq, hkv, part):
+    """head_dim 256 on the CUDA-core family (the library picks it)."""
+    w = W.random_case([1, 17, 200, 513], num_q_heads=hq, num_kv_heads=hkv, head_dim=256, dtype=qdt,
+                      seed=hq + hkv + 256)
+    ref, _, _ = replay(w)
+    got, _ = run_gpu(w, part)
+    assert_close(got[0], ref[0], qdt, f"d=256 G={hq // hkv} part={part}")
+
+
+def test_head_dim_256_int8():
+    w = W.random_case([3, 100, 700], num_q_heads=16, num_kv_heads=4, head_dim=256, dtype="float16",
+                      seed=256)
+    got, dw = run_gpu(w, -1, int8=True, dw=runner.DeviceWorkload(w))
+    kc8, vc8 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
+    ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
+    op = w.steps[0][0]
+    ref = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
+    assert_close(got[0], ref, "float16", "d=256 int8")
