@@ -83,6 +83,8 @@ WORKLOADS = {
                  "batch 16, all lengths 8192, split-K 512",
     "mha_prefix": "MHA 32/32 heads, head_dim 128, fp16, batch 16, shared 1000-token prefix with "
                   "copy-on-write + private suffix U[64,1048]",
+    "mqa": "MQA: 32 q heads / 1 KV head, head_dim 128, fp16, batch 128, all lengths 4096",
+    "d256": "head_dim 256: 16 q / 8 KV heads, fp16, batch 16, all lengths 4096",
 }
 
 
@@ -123,6 +125,10 @@ def make_workload(name):
         return W.long(), True, 512
     if name == "mha_prefix":
         return W.mha_prefix(), False, 256
+    if name == "mqa":
+        return W.mqa(), False, -1
+    if name == "d256":
+        return W.d256(), False, -1
     raise ValueError(name)
 
 

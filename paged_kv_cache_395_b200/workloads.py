@@ -238,6 +238,41 @@ def long(dtype: str = "float16", batch: int = 16, seq_len: int = 8192) -> Worklo
     return Workload("long", Hq, Hkv, d, N, dtype, 1.0 / np.sqrt(d), mb, 512, setup, [step])
 
 
+def uniform(name: str, seed: int, batch: int, seq_len: int, num_q_heads: int, num_kv_heads: int,
+            head_dim: int, dtype: str = "float16") -> Workload:
+    """A batch of equal-length sequences in a shuffled pool, the cache written by
+    one append of all tokens.  Draws: ``permutation(N)`` (free-list order), then
+    for each sequence K [L][H_kv][d] then V, then q [B][H_q][d]."""
+    B, L = batch, seq_len
+    mb = -(-L // BLOCK_SIZE)
+    N = B * mb
+    rng = np.random.default_rng(seed)
+    bm = BlockManager(N, BLOCK_SIZE, free_order=rng.permutation(N))
+    ks, vs, slots = [], [], []
+    for b in range(B):
+        k, v = _normal_tokens(rng, L, num_kv_heads, head_dim, dtype)
+        ks.append(k)
+        vs.append(v)
+        slots.append(bm.add_sequence(b, L))
+    q = normal(rng, (B, num_q_heads, head_dim), dtype)
+    setup = [Reshape(np.concatenate(ks), np.concatenate(vs), np.concatenate(slots))]
+    step = [Decode(q, bm.block_table(range(B), mb), np.full(B, L, np.int32), L)]
+    return Workload(name, num_q_heads, num_kv_heads, head_dim, N, dtype, 1.0 / np.sqrt(head_dim), mb, -1,
+                    setup, [step])
+
+
+def mqa() -> Workload:
+    """MQA decode: 32 query heads sharing one KV head, head_dim 128, fp16,
+    batch 128, every sequence 4096 tokens (seed 6)."""
+    return uniform("mqa", 6, 128, 4096, 32, 1, 128)
+
+
+def d256() -> Workload:
+    """head_dim 256 decode: 16 query / 8 KV heads, fp16, batch 16, every
+    sequence 4096 tokens (seed 7)."""
+    return uniform("d256", 7, 16, 4096, 16, 8, 256)
+
+
 def mha_prefix(dtype: str = "float16") -> Workload:
     """MHA with prefix sharing: 32 query / 32 KV heads, head_dim 128, batch 16.
 
@@ -317,7 +352,7 @@ def random_case(lens, num_q_heads=4, num_kv_heads=2, head_dim=64, dtype="float16
 
 
 NAMED = {"tiny": tiny, "gqa_b8": gqa_b8, "ragged": ragged, "long": long,
-         "mha_prefix": mha_prefix}
+         "mha_prefix": mha_prefix, "mqa": mqa, "d256": d256}
 
 
 def decode_kv_bytes(op: Decode, w: Workload, kv_elem: float | None = None) -> int:

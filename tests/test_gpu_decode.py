@@ -367,3 +367,24 @@ def test_head_dim_256_int8():
     op = w.steps[0][0]
     ref = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
     assert_close(got[0], ref, "float16", "d=256 int8")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["mqa", "d256"])
+def test_wide_workloads_full_size_sampled(name):
+    """The benchmark's MQA and head_dim-256 workloads at full size, in the bench's
+    launch configuration (library-picked partition, inputs-ready flag), against
+    the oracle on sampled (sequence, head) rows."""
+    w = W.NAMED[name]()
+    B, Hq = w.steps[0][0].q.shape[:2]
+    rng = np.random.default_rng(0)
+    rows = np.array([[b, h] for b in rng.choice(B, 3, replace=False) for h in (0, Hq // 2, Hq - 1)],
+                    dtype=np.int32)
+    ref, _, _ = replay(w, fill_nan=False, bh=rows)
+    dw = runner.DeviceWorkload(w, fill_nan=False)
+    dw.run_setup()
+    calls = runner.StepCalls(dw, -1, False, pa.PA_ALGO_AUTO, flags=pa.PA_DECODE_INPUTS_READY)
+    calls.run(0)
+    torch.cuda.synchronize()
+    out = dw.steps[0][-1][-1]
+    assert_close(out, ref[0], "float16", name, rows=rows)
