@@ -53,11 +53,13 @@ def load(path):
                                 i64, dbl, P, i64, i32]
     L.oracle_decode_partials.argtypes = [P, P, P, P, P, i32, P, P, P, P, i32, i32, i32, i32,
                                          i32, i32, i64, dbl, i32, i32, i32]
+    L.oracle_decode_multi.argtypes = [P, P, P, P, i32, P, P, P, P, i32, i32, i32, i32, i32, i32,
+                                      i32, i64, dbl, i32]
     L.oracle_merge.argtypes = [P, P, P, i64, i32, i32]
     L.oracle_kv_bytes_per_token.argtypes = [i32, i32, i32, i32]
     L.oracle_kv_bytes_per_token.restype = i64
     for name in ("oracle_reshape_and_cache", "oracle_block_copy", "oracle_quantize_int8",
-                 "oracle_decode", "oracle_decode_partials", "oracle_merge"):
+                 "oracle_decode", "oracle_decode_multi", "oracle_decode_partials", "oracle_merge"):
         getattr(L, name).restype = i32
     return L
 
@@ -158,6 +160,26 @@ def decode(q, key_cache, value_cache, block_tables, seq_lens, scale, k_scales=No
                                bs, bt.shape[1] if bt.ndim == 2 else 0, N, float(scale), _ptr(bhl),
                                0 if bhl is None else bhl.shape[0], nt),
            "oracle_decode")
+    return out
+
+
+def decode_multi(q, key_cache, value_cache, block_tables, seq_lens, scale, k_scales=None,
+                 v_scales=None, kv_code=None, nthreads=None):
+    """fp64 multi-query decode output [B][Q][H_q][d] for q [B][Q][H_q][d]: query
+    token i of sequence b attends to its first seq_lens[b] - Q + i + 1 tokens."""
+    q64 = _q64(q)
+    B, Q, Hq, d = q64.shape
+    N, Hkv, bs, d2 = key_cache.shape
+    assert d == d2
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    code = dtype_code(key_cache.dtype) if kv_code is None else kv_code
+    out = np.full((B, Q, Hq, d), np.nan, dtype=np.float64)
+    nt = nthreads_default() if nthreads is None else nthreads
+    _check(lib().oracle_decode_multi(_ptr(out), _ptr(q64), _ptr(key_cache), _ptr(value_cache), code,
+                                     _ptr(k_scales), _ptr(v_scales), _ptr(bt), _ptr(sl), B, Q, Hq, Hkv,
+                                     d, bs, bt.shape[1] if bt.ndim == 2 else 0, N, float(scale), nt),
+           "oracle_decode_multi")
     return out
 
 

@@ -242,13 +242,13 @@ static int gather(const dec_args *a, int b, int g, int t0, int t1, double *Kc, d
  * two-pass in fp64: m = max s, p = exp(s - m), l = sum p, o = sum p V / l.
  * Returns lse = m + log(l) through *lse.
  */
-static int attend_range(const dec_args *a, int b, int h, int t0, int t1, double *o, double *lse)
+static int attend_q(const dec_args *a, const double *qv, int b, int h, int t0, int t1, double *o,
+                    double *lse)
 {
     int d = a->head_dim;
     int G = a->num_q_heads / a->num_kv_heads;
     int g = MUT(1) ? h % a->num_kv_heads : h / G;
     int n = t1 - t0;
-    const double *qv = a->q + ((size_t)b * a->num_q_heads + h) * d;
     double *Kc = (double *)malloc(sizeof(double) * (size_t)n * d);
     double *Vc = (double *)malloc(sizeof(double) * (size_t)n * d);
     double *s = (double *)malloc(sizeof(double) * (size_t)n);
@@ -278,6 +278,12 @@ static int attend_range(const dec_args *a, int b, int h, int t0, int t1, double 
     free(Vc);
     free(s);
     return rc;
+}
+
+/* Attention of query row (b, h) of a [B][H_q][d] q over the tokens [t0, t1). */
+static int attend_range(const dec_args *a, int b, int h, int t0, int t1, double *o, double *lse)
+{
+    return attend_q(a, a->q + ((size_t)b * a->num_q_heads + h) * a->head_dim, b, h, t0, t1, o, lse);
 }
 
 static int check_dims(const dec_args *a)
@@ -324,6 +330,50 @@ int oracle_decode(double *out, const double *q, const void *key_cache, const voi
         }
         double lse;
         int e = attend_range(&a, b, h, 0, L, o, &lse);
+        if (e) {
+#pragma omp atomic write
+            err = e;
+        }
+    }
+    return err;
+}
+
+/*
+ * Decode of query_len > 1 new tokens per sequence (the verification step of
+ * speculative decoding, or a chunk of prefill, over the same paged cache):
+ * q and out are [B][Q][H_q][d].  seq_lens[b] = L counts every new token, so
+ * query token i sits at position L - Q + i and attends causally to the tokens
+ * 0 .. L - Q + i:
+ *   out[b][i][h][:] = sum_{t <= L-Q+i} softmax_t(scale * q[b][i][h] . K[b][t]) V[b][t].
+ * Rows whose range is empty (L - Q + i < 0) are zero.  Q = 1 is oracle_decode.
+ */
+int oracle_decode_multi(double *out, const double *q, const void *key_cache, const void *value_cache,
+                        int kv_dtype, const float *k_scales, const float *v_scales,
+                        const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                        int query_len, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                        int max_blocks_per_seq, int64_t num_blocks, double scale, int nthreads)
+{
+    dec_args a = {q, key_cache, value_cache, kv_dtype, k_scales, v_scales, block_tables,
+                  seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                  max_blocks_per_seq, num_blocks, scale};
+    int rc = check_dims(&a);
+    if (rc) return rc;
+    if (query_len <= 0) return -2;
+    int64_t rows = (int64_t)num_seqs * query_len * num_q_heads;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        int h = (int)(r % num_q_heads);
+        int i = (int)((r / num_q_heads) % query_len);
+        int b = (int)(r / ((int64_t)num_q_heads * query_len));
+        double *o = out + (size_t)r * head_dim;
+        int end = seq_lens[b] - query_len + i + (MUT(11) ? 0 : 1);  /* tokens 0 .. end-1 */
+        if (end <= 0) {
+            for (int j = 0; j < head_dim; ++j) o[j] = 0.0;
+            continue;
+        }
+        double lse;
+        int e = attend_q(&a, q + (size_t)r * head_dim, b, h, 0, end, o, &lse);
         if (e) {
 #pragma omp atomic write
             err = e;

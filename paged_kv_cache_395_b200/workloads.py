@@ -46,7 +46,7 @@ class Copy:
 
 @dataclass
 class Decode:
-    q: np.ndarray             # [B][H_q][d] storage dtype
+    q: np.ndarray             # [B][H_q][d] storage dtype, or [B][Q][H_q][d] for Q new tokens
     block_tables: np.ndarray  # int32 [B][max_blocks_per_seq]
     seq_lens: np.ndarray      # int32 [B]
     max_seq_len: int
@@ -349,6 +349,20 @@ def random_case(lens, num_q_heads=4, num_kv_heads=2, head_dim=64, dtype="float16
                    max(lens, default=0))]
     return Workload(f"random{B}", num_q_heads, num_kv_heads, head_dim, N, dtype,
                     1.0 / np.sqrt(head_dim), mb, partition_size, setup, [step], logical=logical)
+
+
+def random_multi_case(lens, query_len, num_q_heads=4, num_kv_heads=2, head_dim=64, dtype="float16",
+                      seed=0, extra_blocks=3) -> Workload:
+    """random_case with query_len new tokens per sequence: the cache holds all
+    ``lens[b]`` tokens (the last query_len of them are the new ones) and q is
+    [B][query_len][H_q][d].  Draws: as random_case, then q [B][Q][H_q][d]."""
+    w = random_case(lens, num_q_heads, num_kv_heads, head_dim, dtype, seed, extra_blocks=extra_blocks)
+    rng = np.random.default_rng(seed + 1000)
+    q = normal(rng, (len(lens), query_len, num_q_heads, head_dim), dtype)
+    op = w.steps[0][0]
+    w.steps = [[Decode(q, op.block_tables, op.seq_lens, op.max_seq_len)]]
+    w.name = f"multi{len(lens)}x{query_len}"
+    return w
 
 
 NAMED = {"tiny": tiny, "gqa_b8": gqa_b8, "ragged": ragged, "long": long,

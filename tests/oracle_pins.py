@@ -310,6 +310,62 @@ def pin_quantize():
         q.reshape(-1)[: len(vals)].tolist()
 
 
+# -- multi-query decode (query_len new tokens, causal among them) ---------------------
+MULTI_CASES = [
+    dict(lens=[2, 17, 40], query_len=2, num_q_heads=8, num_kv_heads=2, head_dim=64, dtype="float16"),
+    dict(lens=[5, 33, 16], query_len=5, num_q_heads=4, num_kv_heads=4, head_dim=64, dtype="bfloat16"),
+    dict(lens=[3, 70], query_len=3, num_q_heads=16, num_kv_heads=1, head_dim=128, dtype="float32"),
+]
+
+
+def pin_multi_dense():
+    """Query token i of a sequence of L tokens equals dense attention over the
+    unpaged first L - Q + i + 1 tokens (NumPy brute force, no paging)."""
+    for case in MULTI_CASES:
+        w = W.random_multi_case(seed=3, **case)
+        outs, _, _ = replay(w)
+        op = w.steps[0][0]
+        q = to_f64(op.q, w.dtype)
+        B, Q = q.shape[:2]
+        for b in range(B):
+            K, V = (to_f64(x, w.dtype) for x in w.logical[b])
+            L = int(op.seq_lens[b])
+            for i in range(Q):
+                n = L - Q + i + 1
+                ref = dense_attention(q[b, i], K[:n], V[:n], w.scale, w.group)
+                _close(outs[0][b, i], ref, 1e-12, f"multi {case} b={b} i={i}")
+
+
+def pin_multi_sdpa_causal_mask():
+    """torch's scaled_dot_product_attention (fp64) with an explicit mask letting
+    query i see keys 0 .. L - Q + i."""
+    case = MULTI_CASES[0]
+    w = W.random_multi_case(seed=4, **case)
+    outs, _, _ = replay(w)
+    op = w.steps[0][0]
+    q = to_f64(op.q, w.dtype)
+    B, Q, Hq, _ = q.shape
+    for b in range(B):
+        K, V = (torch.from_numpy(to_f64(x, w.dtype)) for x in w.logical[b])
+        L = K.shape[0]
+        K = K.permute(1, 0, 2).repeat_interleave(w.group, dim=0)  # [H_q][L][d]
+        V = V.permute(1, 0, 2).repeat_interleave(w.group, dim=0)
+        qq = torch.from_numpy(q[b]).permute(1, 0, 2)  # [H_q][Q][d]
+        mask = torch.arange(L)[None, :] <= (L - Q + torch.arange(Q))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, K, V, attn_mask=mask, scale=w.scale)
+        _close(outs[0][b], ref.permute(1, 0, 2).numpy(), 1e-12, "multi sdpa")
+
+
+def pin_multi_single_token_is_decode():
+    """Q = 1 gives the single-token decode, bit for bit."""
+    w = W.random_multi_case([9, 40], 1, seed=5)
+    outs, kc, vc = replay(w)
+    op = w.steps[0][0]
+    single = oracle.decode(op.q[:, 0], kc, vc, op.block_tables, op.seq_lens, w.scale)
+    assert np.array_equal(outs[0][:, 0], single)
+
+
 ALL_PINS = [pin_half_exhaustive, pin_bf16_exhaustive, pin_tiny_dense, pin_random_dense,
             pin_sdpa_library, pin_permutation_invariance, pin_gqa_expand, pin_closed_forms,
-            pin_split_merge, pin_kv_size_golden, pin_reshape, pin_block_copy, pin_quantize]
+            pin_split_merge, pin_kv_size_golden, pin_reshape, pin_block_copy, pin_quantize,
+            pin_multi_dense, pin_multi_sdpa_causal_mask, pin_multi_single_token_is_decode]

@@ -46,8 +46,12 @@ def replay(w, want=None, fill_nan=True, bh=None):
         for op in ops:
             if isinstance(op, W.Decode):
                 if want is None or want(si):
-                    outs[si] = oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale,
-                                             kv_code=code_of(w), bh=bh)
+                    if op.q.ndim == 4:  # query_len new tokens per sequence
+                        outs[si] = oracle.decode_multi(op.q, kc, vc, op.block_tables, op.seq_lens,
+                                                       w.scale, kv_code=code_of(w))
+                    else:
+                        outs[si] = oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale,
+                                                 kv_code=code_of(w), bh=bh)
             else:
                 apply(op, w, kc, vc)
     return outs, kc, vc

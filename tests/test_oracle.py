@@ -27,6 +27,7 @@ MUTATIONS = {
     8: "K used in place of V (transposed operand)",
     9: "partition lse without log l",
     10: "block copy skips V",
+    11: "multi-query causal range one token short",
 }
 
 # pins cheap enough to run once per mutant
