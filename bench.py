@@ -85,6 +85,8 @@ WORKLOADS = {
                   "copy-on-write + private suffix U[64,1048]",
     "mqa": "MQA: 32 q heads / 1 KV head, head_dim 128, fp16, batch 128, all lengths 4096",
     "d256": "head_dim 256: 16 q / 8 KV heads, fp16, batch 16, all lengths 4096",
+    "specdec": "speculative verification: 7B-GQA 32 q / 8 KV heads, head_dim 128, fp16, batch 64, "
+               "lengths U[512,4096], 2 new tokens per sequence per step (causal), 16 steps",
 }
 
 
@@ -129,6 +131,8 @@ def make_workload(name):
         return W.mqa(), False, -1
     if name == "d256":
         return W.d256(), False, -1
+    if name == "specdec":
+        return W.specdec(), False, -1
     raise ValueError(name)
 
 
@@ -143,7 +147,11 @@ def step_bytes(w, int8):
 
 def step_tokens(w):
     from paged_kv_cache_395_b200 import workloads as W
-    return [int([o for o in ops if isinstance(o, W.Decode)][0].q.shape[0]) for ops in w.steps]
+    out = []
+    for ops in w.steps:
+        q = [o for o in ops if isinstance(o, W.Decode)][0].q
+        out.append(int(q.shape[0] * (q.shape[1] if q.ndim == 4 else 1)))  # query tokens decoded
+    return out
 
 
 class ClockSampler:
@@ -249,11 +257,15 @@ def cpu_baseline(w, int8, seconds, host_caches=None):
                 oracle.block_copy(kc, vc, op.pairs)
             elif isinstance(op, W.Decode):
                 t0 = time.perf_counter()
-                oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs,
-                              nthreads=threads)
+                if op.q.ndim == 4:
+                    oracle.decode_multi(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs,
+                                        nthreads=threads)
+                else:
+                    oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs,
+                                  nthreads=threads)
                 t_work += time.perf_counter() - t0
                 done_bytes += W.decode_kv_bytes(op, w, 1 if int8 else None)
-                ntok += op.q.shape[0]
+                ntok += op.q.shape[0] * (op.q.shape[1] if op.q.ndim == 4 else 1)
                 nsteps += 1
         if t_work >= seconds:
             break
@@ -286,9 +298,13 @@ def reference_arm(args, rank, world):
     def one(i):
         op = decs[i % T]
         b = i % op.q.shape[0]
-        bh = np.array([[b, h] for h in range(w.num_q_heads)], dtype=np.int32)
-        oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs, bh=bh,
-                      nthreads=threads)
+        if op.q.ndim == 4:
+            oracle.decode_multi(op.q[b:b + 1], kc, vc, op.block_tables[b:b + 1], op.seq_lens[b:b + 1],
+                                w.scale, ks, vs, nthreads=threads)
+        else:
+            bh = np.array([[b, h] for h in range(w.num_q_heads)], dtype=np.int32)
+            oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs, bh=bh,
+                          nthreads=threads)
         L = int(max(op.seq_lens[b], 0))
         E = 1 if int8 else w.elem_size
         return L * w.num_kv_heads * w.head_dim * 2 * E

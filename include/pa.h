@@ -122,6 +122,11 @@ typedef struct pa_decode_params {
                                 that share a workspace must not overlap on the device. */
     size_t workspace_bytes;
     int flags;               /* 0, or PA_DECODE_INPUTS_READY */
+    int query_len;           /* new tokens per sequence, Q (0 or 1: single-token decode).
+                                q and out are [num_seqs][Q][num_q_heads][head_dim]; seq_lens
+                                count all Q new tokens (already appended), and query token i
+                                attends causally to tokens 0 .. seq_lens[b] - Q + i.  Q > 1
+                                runs on the tensor-core family only. */
 } pa_decode_params;
 
 /*

@@ -46,24 +46,31 @@ static int auto_partition(int B, int Hkv, int max_len) {
     return 64;
 }
 
-// The heads as the kernels see them.  A group of more than 8 query heads per KV
-// head (16, 32 or 64: MQA-style) is split into 8-head groups, and each group is
-// a virtual KV head that reads the same cache tiles; the virtual heads of one
-// cache head are adjacent rows, so their repeated tile reads meet in L2.
+// The heads as the kernels see them.  The Q x (query heads per KV head) pairs
+// of (query token, head) that share one cache KV head become the columns of
+// the kernels' rows: at most 8 per row (the MMA's n), padded up to a power of
+// two when fewer, split over ceil(pairs / 8) rows (virtual KV heads) when more.
+// The virtual heads of one cache head are adjacent rows, so their repeated
+// tile reads meet in L2.
 struct KernelHeads {
-    int G, Hkv, shift;  // group size <= 8, virtual KV heads, log2(groups per cache head)
+    int G, Hkv, ngroups, Greal, gcols, qlen;
+    bool padded;  // some columns are padding (only the tensor-core family handles that)
 };
 static bool kernel_heads(const pa_decode_params *p, KernelHeads *kh) {
-    const int G = p->num_q_heads / p->num_kv_heads;
-    int shift = 0;
-    if (G > 8) {
-        const int groups = G / 8;
-        if (G % 8 || groups > 8 || (groups & (groups - 1))) return false;
-        while ((1 << shift) < groups) ++shift;
+    const int Greal = p->num_q_heads / p->num_kv_heads;
+    const int Q = p->query_len > 1 ? p->query_len : 1;
+    const int64_t gcols = (int64_t)Q * Greal;
+    if (gcols > 512) return false;  // at most 64 virtual KV heads per cache head
+    int G, ng;
+    if (gcols <= 8) {
+        G = 1;
+        while (G < gcols) G <<= 1;
+        ng = 1;
+    } else {
+        G = 8;
+        ng = (int)((gcols + 7) / 8);
     }
-    kh->G = G > 8 ? 8 : G;
-    kh->Hkv = p->num_kv_heads << shift;
-    kh->shift = shift;
+    *kh = KernelHeads{G, p->num_kv_heads * ng, ng, Greal, (int)gcols, Q, (int64_t)G * ng != gcols};
     return true;
 }
 
@@ -77,13 +84,17 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
     if (p->num_q_heads % p->num_kv_heads) return PA_ERR_SHAPE;
     if (p->block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
     if (!elem_size(p->q_dtype) || !elem_size(p->kv_dtype) || p->q_dtype == PA_I8) return PA_ERR_DTYPE;
+    if (p->query_len < 0) return PA_ERR_SHAPE;
     KernelHeads kh;
     const bool heads_ok = kernel_heads(p, &kh);
-    if (!heads_ok || !decode_simt_supported(p->q_dtype, p->kv_dtype, p->head_dim, kh.G)) {
-        const bool pair_ok = (p->q_dtype == p->kv_dtype) || p->kv_dtype == PA_I8;
-        if (!pair_ok || (p->kv_dtype == PA_I8 && p->q_dtype == PA_F32)) return PA_ERR_DTYPE;
-        return PA_ERR_UNSUPPORTED;
-    }
+    const bool pair_ok = (p->q_dtype == p->kv_dtype) || p->kv_dtype == PA_I8;
+    if (!pair_ok || (p->kv_dtype == PA_I8 && p->q_dtype == PA_F32)) return PA_ERR_DTYPE;
+    if (!heads_ok) return PA_ERR_UNSUPPORTED;
+    const bool simt_ok = kh.qlen == 1 && !kh.padded &&
+                         decode_simt_supported(p->q_dtype, p->kv_dtype, p->head_dim, kh.G);
+    const bool tc_ok = decode_tc_supported(p->q_dtype, p->kv_dtype, p->head_dim, kh.G, p->num_seqs);
+    if (!simt_ok && !tc_ok) return PA_ERR_UNSUPPORTED;
+    if (p->algo == PA_ALGO_SIMT && !simt_ok) return PA_ERR_UNSUPPORTED;
     if (p->num_seqs > 65535 || kh.Hkv > 65535) return PA_ERR_UNSUPPORTED;
     if (p->algo < PA_ALGO_AUTO || p->algo > PA_ALGO_TENSOR) return PA_ERR_UNSUPPORTED;
     if (p->flags & ~PA_DECODE_INPUTS_READY) return PA_ERR_UNSUPPORTED;
@@ -130,6 +141,8 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
                        p->num_blocks * p->num_kv_heads * PA_BLOCK_SIZE <= 2147483647LL &&
                        stream_blocks <= (1LL << 30);
     if (p->algo == PA_ALGO_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
+    // several new tokens per sequence, or padded columns: the tensor-core family only
+    if ((kh.qlen > 1 || kh.padded) && !tc_ok) return PA_ERR_UNSUPPORTED;
     *pl = Plan{};
     pl->max_len = max_len;
     pl->tc = p->algo == PA_ALGO_TENSOR || (p->algo == PA_ALGO_AUTO && tc_ok);
@@ -265,7 +278,10 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     KernelHeads kh;
     kernel_heads(p, &kh);
     a.Hkv = kh.Hkv;
-    a.hg_shift = kh.shift;
+    a.ngroups = kh.ngroups;
+    a.qlen = kh.qlen;
+    a.Greal = kh.Greal;
+    a.gcols = kh.gcols;
     a.D = p->head_dim;
     a.G = kh.G;
     a.mbps = p->max_blocks_per_seq;

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
         my_blk[s] = pb;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&my_bars[s], 2 * TILE);
-        const size_t off = ((size_t)pb * (a.Hkv >> a.hg_shift) + (kvh >> a.hg_shift)) * TILE;
+        const size_t off = ((size_t)pb * (a.Hkv / a.ngroups) + (kvh / a.ngroups)) * TILE;
         bulk_g2s(my_ring + s * C::STAGE_BYTES, reinterpret_cast<const char *>(a.kc) + off, TILE, &my_bars[s]);
         bulk_g2s(my_ring + s * C::STAGE_BYTES + TILE, reinterpret_cast<const char *>(a.vc) + off, TILE,
                  &my_bars[s]);
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
         if (pb >= 0) {
             float ksc = 1.f, vsc = 1.f;
             if constexpr (sizeof(TKV) == 1) {
-                const size_t si = (size_t)pb * (a.Hkv >> a.hg_shift) + (kvh >> a.hg_shift);
+                const size_t si = (size_t)pb * (a.Hkv / a.ngroups) + (kvh / a.ngroups);
                 ksc = a.ks[si];
                 vsc = a.vs[si];
             }

@@ -159,6 +159,7 @@ struct Seg {
     int j0, j1;         // this segment: blocks [j0, j1) of the row
     int fr;             // index of the row's first block in the concatenated stream
     int ch;             // chunk that holds the segment (-1: whole-row mode)
+    int ncol;           // the row's real (not padding) columns
 };
 
 // Walks the ranges of one warp and cuts them into segments at row boundaries.
@@ -316,6 +317,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = a.B, Hkv = a.Hkv;
+    const int Hc = Hkv / a.ngroups;  // the cache's KV heads
     // Without PA_DECODE_INPUTS_READY nothing is read before the previous kernel
     // on the stream has finished; with it, the lengths, the block tables and q
     // are read first (the caller guarantees that kernel does not write them) and
@@ -359,6 +361,15 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     const int gw = blockIdx.x * NW + warp;
     const int W = gridDim.x * NW;
     const bool rows_mode = a.tc_chunk < 0;
+    // Columns: column j of row kvh is the (query token, head) pair jg = (kvh % ngroups) * G
+    // + j of cache KV head kvh / ngroups; pairs from gcols on are padding.
+    auto col_jg = [&](int kvh, int j) { return (kvh % a.ngroups) * G + j; };
+    auto ncol_of = [&](int kvh) { return min(G, a.gcols - (kvh % a.ngroups) * G); };
+    auto col_row = [&](int b, int kvh, int j) -> size_t {  // row of q / out [B][qlen][Hq]
+        const int jg = col_jg(kvh, j);
+        const int i = jg / a.Greal, h = jg - i * a.Greal;
+        return ((size_t)b * a.qlen + i) * a.Hq + (size_t)(kvh / a.ngroups) * a.Greal + h;
+    };
 
     // Static schedule: by default one chunk of ceil(total / W) blocks (at least
     // kTcMinChunk) per warp, so every warp reads the same number of blocks;
@@ -430,12 +441,12 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         const int end = min(it.fend, sg.fr + sg.nb);
         sg.j1 = sg.j0 + (int)(end - it.f);
         sg.ch = it.ch;
+        sg.ncol = ncol_of(sg.kvh);
         it.f = end;
         return true;
     };
 
     uint64_t *my_bars = bars + warp * S;
-    constexpr uint32_t kQBytes = G * D * sizeof(T);  // multiple of 16; q rows are 16-byte aligned
     const uint32_t qring = smem_addr(smem) + C::QRING_OFF + warp * S * C::QSLOT;
     int *my_ok = stage_ok + warp * S;
     const uint32_t ring = smem_addr(smem) + warp * S * C::STAGE;
@@ -479,12 +490,12 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         if (!w.valid || lane >= w.n) return -1;
         const int pb = a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
         if (pb < 0 || (int64_t)pb >= a.N) return -2;
-        const int hc = Hkv >> a.hg_shift, kc = w.sg.kvh >> a.hg_shift;  // the cache's KV head
+        const int kc = w.sg.kvh / a.ngroups;  // the cache's KV head
         if constexpr (kI8) {
-            ks = a.ks[(size_t)pb * hc + kc];
-            vs = a.vs[(size_t)pb * hc + kc];
+            ks = a.ks[(size_t)pb * Hc + kc];
+            vs = a.vs[(size_t)pb * Hc + kc];
         }
-        return (pb * hc + kc) * kBlockSize;
+        return (pb * Hc + kc) * kBlockSize;
     };
     Win pc, pn;
     win_first(pc);
@@ -506,7 +517,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             // a segment's first block also brings the segment's q rows into the
             // stage's q slot (even when the block itself is skipped)
             const bool seg_first = pc.o == 0 && p_i == 0;
-            const uint32_t tx = (y < 0 ? 0u : (uint32_t)C::STAGE) + (seg_first ? kQBytes : 0u);
+            const int ncol = seg_first ? pc.sg.ncol : 0;
+            const uint32_t tx = (y < 0 ? 0u : (uint32_t)C::STAGE) + (uint32_t)(ncol * D * (int)sizeof(T));
             my_ok[s] = y >= 0;
             if constexpr (kI8) {
                 my_sc[2 * s] = ksv;  // released to the consumer by the arrive below
@@ -527,9 +539,16 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 }
             }
             if (seg_first) {
-                const T *qsrc = reinterpret_cast<const T *>(a.q) +
-                                ((size_t)pc.sg.b * a.Hq + (size_t)pc.sg.kvh * G) * D;
-                bulk_g2s_u32(qring + s * C::QSLOT, qsrc, kQBytes, smem_addr(bar));
+                // the segment's q rows: runs of columns that are consecutive heads of one
+                // query token, each one bulk copy
+                for (int j = 0; j < ncol;) {
+                    const int h = col_jg(pc.sg.kvh, j) % a.Greal;
+                    const int run = min(ncol - j, a.Greal - h);
+                    const T *qsrc = reinterpret_cast<const T *>(a.q) + col_row(pc.sg.b, pc.sg.kvh, j) * D;
+                    bulk_g2s_u32(qring + s * C::QSLOT + j * D * (int)sizeof(T), qsrc,
+                                 run * D * (int)sizeof(T), smem_addr(bar));
+                    j += run;
+                }
             }
         }
         ++p_k;
@@ -551,8 +570,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     for (int r = gw; r < B * Hkv; r += W) {
         const int b = r / Hkv;
         if (cum[b + 1] == cum[b]) {
-            T *o = reinterpret_cast<T *>(a.out) + ((size_t)b * a.Hq + (size_t)(r % Hkv) * G) * D;
-            for (int i = lane; i < G * D; i += 32) o[i] = Cvt<T>::from_f(0.f);
+            const int kvh = r % Hkv, ncol = ncol_of(kvh);
+            for (int j = 0; j < ncol; ++j) {
+                T *o = reinterpret_cast<T *>(a.out) + col_row(b, kvh, j) * D;
+                for (int i = lane; i < D; i += 32) o[i] = Cvt<T>::from_f(0.f);
+            }
         }
     }
 #pragma unroll
@@ -569,11 +591,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     // B fragments of q (n = heads, k = dims) from the q slot of stage s.  The
     // int8 path orders the contraction's dims differently (see kfrag_i8): k-step
     // ks, thread column c covers dims 32c + 4ks .. 32c + 4ks + 3.
-    auto load_q = [&](int s, uint32_t (&bq)[C::KSTEPS][2]) {
+    auto load_q = [&](int s, uint32_t (&bq)[C::KSTEPS][2], int ncol) {
         const uint32_t qs = qring + s * C::QSLOT + (kI8 ? (g * D + 32 * c) * 2 : (g * D + 2 * c) * 2);
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS; ++ks) {
-            if (g < G) {
+            if (g < ncol) {
                 bq[ks][0] = lds_u32(qs + (kI8 ? ks * 8 : ks * 32));
                 bq[ks][1] = lds_u32(qs + (kI8 ? ks * 8 + 4 : ks * 32 + 16));
             } else {
@@ -679,11 +701,15 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 }
             }
         }
-        T *out = reinterpret_cast<T *>(a.out) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
+        const int ncol = ncol_of(kvh);
 #pragma unroll
-        for (int h = 0; h < G; ++h)
+        for (int h = 0; h < G; ++h) {
+            if (h < ncol) {
+                T *out = reinterpret_cast<T *>(a.out) + col_row(b, kvh, h) * D;
 #pragma unroll
-            for (int e = 0; e < C::DPL; ++e) out[h * D + lane * C::DPL + e] = Cvt<T>::from_f(acc[h][e]);
+                for (int e = 0; e < C::DPL; ++e) out[lane * C::DPL + e] = Cvt<T>::from_f(acc[h][e]);
+            }
+        }
         if (lane == 0) a.counters[(size_t)b * Hkv + kvh] = 0;  // the workspace is left as it was found
     };
     auto resolve = [&]() {
@@ -717,6 +743,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     while (have && alive) {
         const int len = cs.j1 - cs.j0;
         const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;  // tokens in the row's last block
+        // causal limits: column (query token i) sees positions < L - qlen + 1 + i;
+        // padding columns see none
+        const int ncol = cs.ncol;
+        const int lim0 = h0 < ncol ? cs.L - a.qlen + 1 + col_jg(cs.kvh, h0) / a.Greal : -1;
+        const int lim1 = h1 < ncol ? cs.L - a.qlen + 1 + col_jg(cs.kvh, h1) / a.Greal : -1;
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         float o[C::MTILES][4];
 #pragma unroll
@@ -732,7 +763,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 break;
             }
             if (lane != 0) mbar_wait(&my_bars[s], parity);
-            if (j == 0) load_q(s, bq);  // the segment's q came with its first block
+            if (j == 0) load_q(s, bq, ncol);  // the segment's q came with its first block
             const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
             const uint32_t tK = ring + s * C::STAGE;
             if (my_ok[s]) {
@@ -789,11 +820,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sc[e] = (sa[0][e] + sa[1][e]) + (sa[2][e] + sa[3][e]);
                 // ---- online softmax (log2 domain): rows g, g+8 are tokens, columns heads
-                const bool v0 = g < ntok, v1 = g + 8 < ntok;
-                const float s0 = v0 ? sc[0] * slog : -INFINITY;
-                const float s1 = v0 ? sc[1] * slog : -INFINITY;
-                const float s2 = v1 ? sc[2] * slog : -INFINITY;
-                const float s3 = v1 ? sc[3] * slog : -INFINITY;
+                const int pos = (cs.j0 + j) * kBlockSize + g;  // token of rows g; g + 8 is pos + 8
+                const float s0 = pos < lim0 ? sc[0] * slog : -INFINITY;
+                const float s1 = pos < lim1 ? sc[1] * slog : -INFINITY;
+                const float s2 = pos + 8 < lim0 ? sc[2] * slog : -INFINITY;
+                const float s3 = pos + 8 < lim1 ? sc[3] * slog : -INFINITY;
                 float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
                 for (int msk = 4; msk < 32; msk <<= 1) {
@@ -801,9 +832,14 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
                 }
                 const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
-                const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
-                const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
+                // A column with no visible token so far keeps m = -inf: its l and o are 0, so
+                // it needs no rescale (al = 1, which also keeps padding columns from forcing
+                // the rescale below), and its p are measured from 0 (exp2(-inf) = 0).
+                const float mc0 = mn0 == -INFINITY ? 0.f : mn0, mc1 = mn1 == -INFINITY ? 0.f : mn1;
+                const float al0 = m0 == -INFINITY ? 1.f : fast_exp2(m0 - mc0);
+                const float al1 = m1 == -INFINITY ? 1.f : fast_exp2(m1 - mc1);
+                const float p0 = fast_exp2(s0 - mc0), p1 = fast_exp2(s1 - mc1);
+                const float p2 = fast_exp2(s2 - mc0), p3 = fast_exp2(s3 - mc1);
                 l0 = l0 * al0 + (p0 + p2);
                 l1 = l1 * al1 + (p1 + p3);
                 m0 = mn0;
@@ -866,18 +902,19 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         }
         // l == 0 only when every block of the segment was skipped (bad table entries)
         const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
-        T *out = reinterpret_cast<T *>(a.out) + ((size_t)cs.b * a.Hq + (size_t)cs.kvh * G) * D;
         if (cs.j0 == 0 && cs.j1 == cs.nb) {  // the whole row: final output
+            T *out0 = reinterpret_cast<T *>(a.out) + col_row(cs.b, cs.kvh, h0) * D;
+            T *out1 = reinterpret_cast<T *>(a.out) + col_row(cs.b, cs.kvh, h1) * D;
 #pragma unroll
             for (int i = 0; i < C::MTILES; ++i) {
                 const int d0 = dmap(i, g), d1 = d0 + 8;
-                if (h0 < G) {
-                    out[h0 * D + d0] = Cvt<T>::from_f(o[i][0] * inv0);
-                    out[h0 * D + d1] = Cvt<T>::from_f(o[i][2] * inv0);
+                if (h0 < ncol) {
+                    out0[d0] = Cvt<T>::from_f(o[i][0] * inv0);
+                    out0[d1] = Cvt<T>::from_f(o[i][2] * inv0);
                 }
-                if (h1 < G) {
-                    out[h1 * D + d0] = Cvt<T>::from_f(o[i][1] * inv1);
-                    out[h1 * D + d1] = Cvt<T>::from_f(o[i][3] * inv1);
+                if (h1 < ncol) {
+                    out1[d0] = Cvt<T>::from_f(o[i][1] * inv1);
+                    out1[d1] = Cvt<T>::from_f(o[i][3] * inv1);
                 }
             }
         } else {
@@ -1027,7 +1064,7 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
     if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are read as aligned 32-bit pairs
     CUtensorMap tk, tv;
-    const int64_t rows = a.N * (a.Hkv >> a.hg_shift) * kBlockSize;  // the cache's rows
+    const int64_t rows = a.N * (a.Hkv / a.ngroups) * kBlockSize;  // the cache's rows
     if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
         return PA_ERR_CUDA;
     int sms = 0, per_sm = 0;

@@ -34,10 +34,16 @@ struct DecodeArgs {
     const int32_t *tables;
     const int32_t *lens;
     float scale_log2;        // scale * log2(e): scores are kept in the log2 domain
-    int B, Hq, Hkv, D, G;    // Hkv, G: the kernel's KV heads and group size.  A group of
-                             // more than 8 query heads is split into 8-head groups, each a
-                             // virtual KV head: Hkv = real KV heads << hg_shift, G = 8.
-    int hg_shift;            // log2(virtual KV heads per cache KV head)
+    int B, Hq, Hkv, D, G;    // Hkv, G: the kernel's rows per sequence and columns per row.
+                             // The gcols = qlen * Greal (query token, head) pairs of one
+                             // cache KV head fill the G <= 8 columns of `ngroups` rows
+                             // (virtual KV heads; Hkv = cache KV heads * ngroups); column j
+                             // of row kvh is pair (kvh % ngroups) * G + j, and pairs past
+                             // gcols are padding.
+    int ngroups;             // virtual KV heads per cache KV head
+    int qlen;                // new tokens per sequence (q, out: [B][qlen][Hq][D])
+    int Greal;               // query heads per cache KV head
+    int gcols;               // qlen * Greal
     int mbps;                // max_blocks_per_seq
     int64_t N;               // num_blocks
     int max_len;             // effective bound on seq_lens

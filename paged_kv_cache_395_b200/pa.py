@@ -58,6 +58,7 @@ class PaDecodeParams(ctypes.Structure):
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
         ("flags", ctypes.c_int),
+        ("query_len", ctypes.c_int),
     ]
 
 
@@ -139,7 +140,11 @@ def pa_reshape_and_cache(k, v, key_cache, value_cache, slot_mapping, stream=None
 
 def make_params(q, key_cache, block_tables, max_seq_len, k_scales=None, v_scales=None,
                 partition_size=0, workspace=None, algo=PA_ALGO_AUTO, flags=0) -> PaDecodeParams:
-    B, Hq, d = q.shape
+    """q is [B][H_q][d], or [B][Q][H_q][d] for Q new tokens per sequence."""
+    if q.dim() == 4:
+        B, Q, Hq, d = q.shape
+    else:
+        (B, Hq, d), Q = q.shape, 1
     N, Hkv, bs, _ = key_cache.shape
     p = PaDecodeParams()
     p.num_seqs, p.num_q_heads, p.num_kv_heads, p.head_dim, p.block_size = B, Hq, Hkv, d, bs
@@ -155,20 +160,23 @@ def make_params(q, key_cache, block_tables, max_seq_len, k_scales=None, v_scales
     p.workspace = None if workspace is None else workspace.data_ptr()
     p.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     p.flags = int(flags)
+    p.query_len = int(Q)
     return p
 
 
 def uses_tensor_cores(q, key_cache, algo=PA_ALGO_AUTO) -> bool:
     """Whether pa_decode runs the tensor-core family for these operands (the
     library's rule: fp16/bf16 q with a cache of the same dtype and head_dim 64 or
-    128, or fp16 q with an int8 cache and head_dim 128; group size 1 to 64 (groups
-    above 8 run as 8-head groups); at most 4096 sequences)."""
-    B, Hq, d = q.shape
+    128, or fp16 q with an int8 cache and head_dim 128; at most 512 (query token,
+    head) pairs per KV head; at most 4096 sequences)."""
+    B, d = q.shape[0], q.shape[-1]
+    Hq = q.shape[-2]
+    Q = q.shape[1] if q.dim() == 4 else 1
     Hkv = key_cache.shape[1]
     G = Hq // Hkv
     same = q.dtype in (torch.float16, torch.bfloat16) and key_cache.dtype == q.dtype and d in (64, 128)
     i8 = q.dtype == torch.float16 and key_cache.dtype == torch.int8 and d == 128
-    ok = (same or i8) and G in (1, 2, 4, 8, 16, 32, 64) and B <= 4096
+    ok = (same or i8) and Q * G <= 512 and B <= 4096
     return algo == PA_ALGO_TENSOR or (algo == PA_ALGO_AUTO and ok)
 
 
@@ -189,9 +197,10 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor | None:
 def pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max_seq_len,
               k_scales=None, v_scales=None, partition_size=0, workspace=None,
               algo=PA_ALGO_AUTO, stream=None, params=None, flags=0):
-    """out, q [B][H_q][d]; caches [N][H_kv][16][d]; block_tables int32 [B][M];
-    seq_lens int32 [B] (including the decoded token).  flags: 0 or
-    PA_DECODE_INPUTS_READY (see include/pa.h)."""
+    """out, q [B][H_q][d] (or [B][Q][H_q][d]: Q new tokens per sequence, causal
+    among them); caches [N][H_kv][16][d]; block_tables int32 [B][M]; seq_lens int32
+    [B] (including the new tokens).  flags: 0 or PA_DECODE_INPUTS_READY (see
+    include/pa.h)."""
     _dev(out, q, key_cache, value_cache, block_tables, seq_lens, k_scales, v_scales, workspace)
     for t, n in ((out, "out"), (q, "q"), (key_cache, "key_cache"), (value_cache, "value_cache"),
                  (block_tables, "block_tables"), (seq_lens, "seq_lens")):

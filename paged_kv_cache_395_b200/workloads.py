@@ -273,6 +273,40 @@ def d256() -> Workload:
     return uniform("d256", 7, 16, 4096, 16, 8, 256)
 
 
+def specdec(num_steps: int = 16, query_len: int = 2, dtype: str = "float16", batch: int = 64) -> Workload:
+    """Speculative-decoding verification: 7B-GQA heads (32 q / 8 KV, head_dim
+    128), batch 64, initial lengths U[512, 4096], and per step every sequence
+    appends query_len tokens and decodes them together (causal among them).
+
+    Draws, seed 8: ``permutation(N)`` (free-list order); initial lengths
+    ``integers(512, 4097, size=64)``; for each sequence its K then V; then per
+    step k, v [64 * Q][8][128] and q [64][Q][32][128]."""
+    B, Hq, Hkv, d, Q = batch, 32, 8, 128, query_len
+    max_len = 4096 + num_steps * Q
+    mb = -(-max_len // BLOCK_SIZE)
+    N = B * mb
+    rng = np.random.default_rng(8)
+    bm = BlockManager(N, BLOCK_SIZE, free_order=rng.permutation(N))
+    init = rng.integers(512, 4097, size=B)
+    ks, vs, slots = [], [], []
+    for b in range(B):
+        k, v = _normal_tokens(rng, int(init[b]), Hkv, d, dtype)
+        ks.append(k)
+        vs.append(v)
+        slots.append(bm.add_sequence(b, int(init[b])))
+    setup = [Reshape(np.concatenate(ks), np.concatenate(vs), np.concatenate(slots))]
+    steps = []
+    for _ in range(num_steps):
+        k_new = normal(rng, (B * Q, Hkv, d), dtype)
+        v_new = normal(rng, (B * Q, Hkv, d), dtype)
+        q = normal(rng, (B, Q, Hq, d), dtype)
+        new_slots = np.array([bm.append_slot(b)[0] for b in range(B) for _ in range(Q)], dtype=np.int64)
+        lens = np.array([bm.lens[b] for b in range(B)], dtype=np.int32)
+        steps.append([Reshape(k_new, v_new, new_slots),
+                      Decode(q, bm.block_table(range(B), mb), lens, int(lens.max()))])
+    return Workload("specdec", Hq, Hkv, d, N, dtype, 1.0 / np.sqrt(d), mb, -1, setup, steps)
+
+
 def mha_prefix(dtype: str = "float16") -> Workload:
     """MHA with prefix sharing: 32 query / 32 KV heads, head_dim 128, batch 16.
 
@@ -366,7 +400,7 @@ def random_multi_case(lens, query_len, num_q_heads=4, num_kv_heads=2, head_dim=6
 
 
 NAMED = {"tiny": tiny, "gqa_b8": gqa_b8, "ragged": ragged, "long": long,
-         "mha_prefix": mha_prefix, "mqa": mqa, "d256": d256}
+         "mha_prefix": mha_prefix, "mqa": mqa, "d256": d256, "specdec": specdec}
 
 
 def decode_kv_bytes(op: Decode, w: Workload, kv_elem: float | None = None) -> int:
@@ -380,5 +414,5 @@ def decode_kv_bytes(op: Decode, w: Workload, kv_elem: float | None = None) -> in
     B = op.seq_lens.shape[0]
     kv = int(L.sum()) * w.num_kv_heads * w.head_dim * 2 * E
     scales = int(nblk.sum()) * w.num_kv_heads * 2 * 4 if kv_elem == 1 else 0
-    qo = B * w.num_q_heads * w.head_dim * 2 * w.elem_size
+    qo = int(op.q.size) * 2 * w.elem_size  # q in, out out (Q query tokens each)
     return int(kv + scales + qo + int(nblk.sum()) * 4 + B * 4)

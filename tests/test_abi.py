@@ -58,15 +58,18 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails val
     (dict(head_dim=0), pa.PA_ERR_SHAPE),
     (dict(block_size=32), pa.PA_ERR_UNSUPPORTED),
     (dict(num_q_heads=6, num_kv_heads=4), pa.PA_ERR_SHAPE),
-    (dict(num_q_heads=6, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),   # G = 3
+    (dict(num_q_heads=6, num_kv_heads=2, algo=pa.PA_ALGO_SIMT), pa.PA_ERR_UNSUPPORTED),  # G = 3
+    (dict(num_q_heads=6, num_kv_heads=2, q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32), pa.PA_ERR_UNSUPPORTED),
+    (dict(query_len=2, algo=pa.PA_ALGO_SIMT), pa.PA_ERR_UNSUPPORTED),  # several new tokens: TC only
+    (dict(query_len=-1), pa.PA_ERR_SHAPE),
+    (dict(query_len=129, num_q_heads=8, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),  # 516 pairs per KV head
     (dict(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F16), pa.PA_ERR_DTYPE),
     (dict(q_dtype=pa.PA_I8, kv_dtype=pa.PA_I8), pa.PA_ERR_DTYPE),
     (dict(q_dtype=9), pa.PA_ERR_DTYPE),
     (dict(partition_size=24), pa.PA_ERR_SHAPE),
     (dict(partition_size=-2), pa.PA_ERR_SHAPE),
     (dict(flags=2), pa.PA_ERR_UNSUPPORTED),          # unknown flag bit
-    (dict(num_q_heads=48, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),  # G = 24: not 8 x a power of 2
-    (dict(num_q_heads=256, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),  # G = 128
+    (dict(num_q_heads=1024, num_kv_heads=1), pa.PA_ERR_UNSUPPORTED),  # G = 1024
     (dict(head_dim=256, q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32), pa.PA_ERR_UNSUPPORTED),
     (dict(num_seqs=-1), pa.PA_ERR_SHAPE),
     (dict(algo=7), pa.PA_ERR_UNSUPPORTED),
@@ -173,3 +176,22 @@ def test_large_groups_and_head_dim_256_are_planned():
     p = params(head_dim=256, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p),
                             None) == pa.PA_ERR_UNSUPPORTED
+
+
+def test_multi_query_and_padded_groups_are_planned():
+    """Q new tokens per sequence and group sizes that are not powers of two run
+    on the tensor-core family: Q x G (query token, head) pairs per KV head fill
+    rows of 8 columns (padded up to a power of two below 8)."""
+    for kw in (dict(query_len=2), dict(query_len=3, num_q_heads=8, num_kv_heads=8),
+               dict(num_q_heads=6, num_kv_heads=2), dict(num_q_heads=48, num_kv_heads=2),
+               dict(query_len=4, num_q_heads=32, num_kv_heads=8)):
+        p = params(partition_size=16, algo=pa.PA_ALGO_TENSOR, **kw)
+        assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0, kw
+    # G = 24 is three full 8-head groups: the CUDA-core family takes it too
+    p = params(num_q_heads=48, num_kv_heads=2, partition_size=16, algo=pa.PA_ALGO_SIMT)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+    # Q = 2 at G = 4 fills exactly the 8 columns of one row per KV head: same
+    # workspace as a G = 8 single-token decode over the same KV heads
+    a = params(query_len=2, num_q_heads=8, num_kv_heads=2, partition_size=16, algo=pa.PA_ALGO_TENSOR)
+    b = params(num_q_heads=16, num_kv_heads=2, partition_size=16, algo=pa.PA_ALGO_TENSOR)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(a)) == pa.lib.pa_decode_workspace_size(ctypes.byref(b))

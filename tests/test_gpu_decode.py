@@ -388,3 +388,68 @@ def test_wide_workloads_full_size_sampled(name):
     torch.cuda.synchronize()
     out = dw.steps[0][-1][-1]
     assert_close(out, ref[0], "float16", name, rows=rows)
+
+
+# -- several new tokens per sequence (causal among them) -----------------------------------
+MULTI = [
+    # (H_q, H_kv, Q): columns per KV head = Q * G
+    (8, 2, 2),    # 8 columns, one row
+    (32, 8, 3),   # 12 columns: a full row and a half-padded one
+    (8, 8, 5),    # G = 1: 5 columns padded to 8
+    (32, 1, 2),   # MQA: 64 columns, 8 rows per KV head
+    (16, 8, 1),   # single token, G = 2
+    (6, 2, 1),    # G = 3 padded to 4
+]
+
+
+@pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
+@pytest.mark.parametrize("hq,hkv,Q", MULTI)
+@pytest.mark.parametrize("part", [0, 16, -1])
+def test_multi_query(qdt, hq, hkv, Q, part):
+    """Q new tokens per sequence against the oracle; lengths below 16, equal to
+    Q, and ragged tails."""
+    lens = [Q, Q + 3, 16, 100, 513]
+    w = W.random_multi_case(lens, Q, num_q_heads=hq, num_kv_heads=hkv, head_dim=128, dtype=qdt,
+                            seed=hq * 10 + hkv + Q)
+    ref, _, _ = replay(w)
+    got, _ = run_gpu(w, part, pa.PA_ALGO_TENSOR)
+    assert got[0].shape == (len(lens), Q, hq, 128)
+    assert_close(got[0], ref[0], qdt, f"Q={Q} G={hq // hkv} part={part}")
+
+
+def test_multi_query_int8_and_d64():
+    w = W.random_multi_case([4, 90, 300], 4, num_q_heads=8, num_kv_heads=4, head_dim=128,
+                            dtype="float16", seed=31)
+    got, dw = run_gpu(w, -1, int8=True, dw=runner.DeviceWorkload(w))
+    kc8, vc8 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
+    ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
+    op = w.steps[0][0]
+    ref = oracle.decode_multi(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
+    assert_close(got[0], ref, "float16", "multi int8")
+    w = W.random_multi_case([7, 64, 129], 3, num_q_heads=4, num_kv_heads=2, head_dim=64,
+                            dtype="bfloat16", seed=32)
+    ref, _, _ = replay(w)
+    got, _ = run_gpu(w, 16)
+    assert_close(got[0], ref[0], "bfloat16", "multi d=64")
+
+
+@pytest.mark.slow
+def test_specdec_trace_back_to_back():
+    """The speculative-verification workload in the bench's issue pattern: 16
+    steps of (append 2 tokens per sequence, decode both) back to back with the
+    inputs-ready flag; sampled steps against the oracle."""
+    w = W.specdec()
+    sample = {0, 7, 15}
+    ref, kc, vc = replay(w, want=lambda s: s in sample, fill_nan=False)
+    dw = runner.DeviceWorkload(w, fill_nan=False)
+    dw.run_setup()
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    calls = runner.StepCalls(dw, -1, False, pa.PA_ALGO_AUTO, stream, flags=pa.PA_DECODE_INPUTS_READY)
+    with torch.cuda.stream(stream):
+        for i in range(len(w.steps)):
+            calls.run(i)
+    torch.cuda.synchronize()
+    for i in sorted(sample):
+        assert_close(dw.steps[i][-1][-1], ref[i], "float16", f"specdec step {i}")
+    assert np.array_equal(bits(dw.kc), kc.view(np.uint8))
