@@ -297,7 +297,10 @@ __device__ __forceinline__ void vfrag_i8(const uint32_t (&r)[4][4], int i, uint3
     }
 }
 
-template <typename T, typename TKV, int D, int G>
+// MQ: the general column mapping (several new tokens per sequence, causal among
+// them, or padding columns); without it every row's G columns are the G query
+// heads of one single-token decode, and the kernel keeps the plain addressing.
+template <typename T, typename TKV, int D, int G, bool MQ>
 __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
                                                                      const DecodeArgs a) {
@@ -363,9 +366,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     const bool rows_mode = a.tc_chunk < 0;
     // Columns: column j of row kvh is the (query token, head) pair jg = (kvh % ngroups) * G
     // + j of cache KV head kvh / ngroups; pairs from gcols on are padding.
+    // Without MQ, column j of row kvh is query head kvh * G + j of a [B][Hq] q.
     auto col_jg = [&](int kvh, int j) { return (kvh % a.ngroups) * G + j; };
-    auto ncol_of = [&](int kvh) { return min(G, a.gcols - (kvh % a.ngroups) * G); };
+    auto ncol_of = [&](int kvh) { return MQ ? min(G, a.gcols - (kvh % a.ngroups) * G) : G; };
     auto col_row = [&](int b, int kvh, int j) -> size_t {  // row of q / out [B][qlen][Hq]
+        if constexpr (!MQ) return (size_t)b * a.Hq + (size_t)kvh * G + j;
         const int jg = col_jg(kvh, j);
         const int i = jg / a.Greal, h = jg - i * a.Greal;
         return ((size_t)b * a.qlen + i) * a.Hq + (size_t)(kvh / a.ngroups) * a.Greal + h;
@@ -538,7 +543,10 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                     tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * C::BOXW, y, smem_addr(bar));
                 }
             }
-            if (seg_first) {
+            if (!MQ && seg_first) {
+                bulk_g2s_u32(qring + s * C::QSLOT, reinterpret_cast<const T *>(a.q) + col_row(pc.sg.b, pc.sg.kvh, 0) * D,
+                             G * D * (int)sizeof(T), smem_addr(bar));
+            } else if (seg_first) {
                 // the segment's q rows: runs of columns that are consecutive heads of one
                 // query token, each one bulk copy
                 for (int j = 0; j < ncol;) {
@@ -820,11 +828,22 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sc[e] = (sa[0][e] + sa[1][e]) + (sa[2][e] + sa[3][e]);
                 // ---- online softmax (log2 domain): rows g, g+8 are tokens, columns heads
-                const int pos = (cs.j0 + j) * kBlockSize + g;  // token of rows g; g + 8 is pos + 8
-                const float s0 = pos < lim0 ? sc[0] * slog : -INFINITY;
-                const float s1 = pos < lim1 ? sc[1] * slog : -INFINITY;
-                const float s2 = pos + 8 < lim0 ? sc[2] * slog : -INFINITY;
-                const float s3 = pos + 8 < lim1 ? sc[3] * slog : -INFINITY;
+                float s0, s1, s2, s3;
+                if constexpr (MQ) {
+                    const int pos = (cs.j0 + j) * kBlockSize + g;  // token of rows g; g + 8 is pos + 8
+                    s0 = pos < lim0 ? sc[0] * slog : -INFINITY;
+                    s1 = pos < lim1 ? sc[1] * slog : -INFINITY;
+                    s2 = pos + 8 < lim0 ? sc[2] * slog : -INFINITY;
+                    s3 = pos + 8 < lim1 ? sc[3] * slog : -INFINITY;
+                } else {
+                    // every column sees the same tokens; padding columns (h >= G) hold
+                    // zero q rows and score 0, which keeps them finite
+                    const bool v0 = g < ntok, v1 = g + 8 < ntok;
+                    s0 = v0 ? sc[0] * slog : -INFINITY;
+                    s1 = v0 ? sc[1] * slog : -INFINITY;
+                    s2 = v1 ? sc[2] * slog : -INFINITY;
+                    s3 = v1 ? sc[3] * slog : -INFINITY;
+                }
                 float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
                 for (int msk = 4; msk < 32; msk <<= 1) {
@@ -835,9 +854,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 // A column with no visible token so far keeps m = -inf: its l and o are 0, so
                 // it needs no rescale (al = 1, which also keeps padding columns from forcing
                 // the rescale below), and its p are measured from 0 (exp2(-inf) = 0).
-                const float mc0 = mn0 == -INFINITY ? 0.f : mn0, mc1 = mn1 == -INFINITY ? 0.f : mn1;
-                const float al0 = m0 == -INFINITY ? 1.f : fast_exp2(m0 - mc0);
-                const float al1 = m1 == -INFINITY ? 1.f : fast_exp2(m1 - mc1);
+                // (Without MQ every column sees a token in every block, so m is finite.)
+                const float mc0 = (MQ && mn0 == -INFINITY) ? 0.f : mn0;
+                const float mc1 = (MQ && mn1 == -INFINITY) ? 0.f : mn1;
+                const float al0 = (MQ && m0 == -INFINITY) ? 1.f : fast_exp2(m0 - mc0);
+                const float al1 = (MQ && m1 == -INFINITY) ? 1.f : fast_exp2(m1 - mc1);
                 const float p0 = fast_exp2(s0 - mc0), p1 = fast_exp2(s1 - mc1);
                 const float p2 = fast_exp2(s2 - mc0), p3 = fast_exp2(s3 - mc1);
                 l0 = l0 * al0 + (p0 + p2);
@@ -1056,10 +1077,10 @@ bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
     return (same || i8) && (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
 }
 
-template <typename T, typename TKV, int D, int G>
+template <typename T, typename TKV, int D, int G, bool MQ>
 static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     using C = TcCfg<TKV, D, G>;
-    auto kern = decode_tc_kernel<T, TKV, D, G>;
+    auto kern = decode_tc_kernel<T, TKV, D, G, MQ>;
     const int smem = C::smem_bytes(a.B);
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
     if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are read as aligned 32-bit pairs
@@ -1080,15 +1101,22 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
                                                                                              : PA_ERR_CUDA;
 }
 
-template <typename T, typename TKV, int D>
-static int launch_tc_g(const DecodeArgs &a, cudaStream_t st) {
+template <typename T, typename TKV, int D, bool MQ>
+static int launch_tc_mq(const DecodeArgs &a, cudaStream_t st) {
     switch (a.G) {
-    case 1: return launch_tc<T, TKV, D, 1>(a, st);
-    case 2: return launch_tc<T, TKV, D, 2>(a, st);
-    case 4: return launch_tc<T, TKV, D, 4>(a, st);
-    case 8: return launch_tc<T, TKV, D, 8>(a, st);
+    case 1: return launch_tc<T, TKV, D, 1, MQ>(a, st);
+    case 2: return launch_tc<T, TKV, D, 2, MQ>(a, st);
+    case 4: return launch_tc<T, TKV, D, 4, MQ>(a, st);
+    case 8: return launch_tc<T, TKV, D, 8, MQ>(a, st);
     default: return PA_ERR_UNSUPPORTED;
     }
+}
+
+template <typename T, typename TKV, int D>
+static int launch_tc_g(const DecodeArgs &a, cudaStream_t st) {
+    // several new tokens, or padding columns: the general column mapping
+    const bool mq = a.qlen > 1 || (int64_t)a.G * a.ngroups != a.gcols;
+    return mq ? launch_tc_mq<T, TKV, D, true>(a, st) : launch_tc_mq<T, TKV, D, false>(a, st);
 }
 
 int launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
