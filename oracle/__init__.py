@@ -32,7 +32,7 @@ import numpy as np
 
 from . import build as _build
 
-F32, F16, BF16, I8 = 0, 1, 2, 3
+F32, F16, BF16, I8, I4 = 0, 1, 2, 3, 4
 
 _lib = None
 
@@ -49,6 +49,7 @@ def load(path):
     L.oracle_reshape_and_cache.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, i64, i64]
     L.oracle_block_copy.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32]
     L.oracle_quantize_int8.argtypes = [P, i32, P, P, i64, i32, i32, i32]
+    L.oracle_quantize_int4.argtypes = [P, i32, P, P, i64, i32, i32, i32]
     L.oracle_decode.argtypes = [P, P, P, P, i32, P, P, P, P, i32, i32, i32, i32, i32, i32,
                                 i64, dbl, P, i64, i32]
     L.oracle_decode_partials.argtypes = [P, P, P, P, P, i32, P, P, P, P, i32, i32, i32, i32,
@@ -58,7 +59,7 @@ def load(path):
     L.oracle_merge.argtypes = [P, P, P, i64, i32, i32]
     L.oracle_kv_bytes_per_token.argtypes = [i32, i32, i32, i32]
     L.oracle_kv_bytes_per_token.restype = i64
-    for name in ("oracle_reshape_and_cache", "oracle_block_copy", "oracle_quantize_int8",
+    for name in ("oracle_reshape_and_cache", "oracle_block_copy", "oracle_quantize_int8", "oracle_quantize_int4",
                  "oracle_decode", "oracle_decode_multi", "oracle_decode_partials", "oracle_merge"):
         getattr(L, name).restype = i32
     return L
@@ -76,7 +77,9 @@ def dtype_code(dt) -> int:
     dt = np.dtype(dt) if not isinstance(dt, str) else dt
     if dt == "bfloat16":
         return BF16
-    return {np.dtype(np.float32): F32, np.dtype(np.float16): F16, np.dtype(np.int8): I8}[dt]
+    # uint8 caches hold packed 4-bit values (two per byte)
+    return {np.dtype(np.float32): F32, np.dtype(np.float16): F16, np.dtype(np.int8): I8,
+            np.dtype(np.uint8): I4}[dt]
 
 
 def _ptr(a):
@@ -135,6 +138,19 @@ def quantize_int8(src_cache, code=None):
     return dst, scales
 
 
+def quantize_int4(src_cache, code=None):
+    """Return (packed 4-bit cache uint8 [N][H_kv][bs][d/2], fp32 scales [N][H_kv])
+    for a [N][H_kv][bs][d] cache."""
+    N, H, bs, d = src_cache.shape
+    src = np.ascontiguousarray(src_cache)
+    code = dtype_code(src.dtype) if code is None else code
+    dst = np.zeros((N, H, bs, d // 2), dtype=np.uint8)
+    scales = np.empty((N, H), dtype=np.float32)
+    _check(lib().oracle_quantize_int4(_ptr(src), code, _ptr(dst), _ptr(scales), N, H, d, bs),
+           "oracle_quantize_int4")
+    return dst, scales
+
+
 def _q64(q):
     if q.dtype == np.uint16:  # bf16 bit patterns
         return (q.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
@@ -148,10 +164,10 @@ def decode(q, key_cache, value_cache, block_tables, seq_lens, scale, k_scales=No
     q64 = _q64(q)
     B, Hq, d = q64.shape
     N, Hkv, bs, d2 = key_cache.shape
-    assert d == d2
+    code = dtype_code(key_cache.dtype) if kv_code is None else kv_code
+    assert d == (2 * d2 if code == I4 else d2)
     bt = np.ascontiguousarray(block_tables, dtype=np.int32)
     sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
-    code = dtype_code(key_cache.dtype) if kv_code is None else kv_code
     out = np.full((B, Hq, d), np.nan, dtype=np.float64)
     bhl = None if bh is None else np.ascontiguousarray(bh, dtype=np.int32).reshape(-1, 2)
     nt = nthreads_default() if nthreads is None else nthreads
@@ -170,10 +186,10 @@ def decode_multi(q, key_cache, value_cache, block_tables, seq_lens, scale, k_sca
     q64 = _q64(q)
     B, Q, Hq, d = q64.shape
     N, Hkv, bs, d2 = key_cache.shape
-    assert d == d2
+    code = dtype_code(key_cache.dtype) if kv_code is None else kv_code
+    assert d == (2 * d2 if code == I4 else d2)
     bt = np.ascontiguousarray(block_tables, dtype=np.int32)
     sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
-    code = dtype_code(key_cache.dtype) if kv_code is None else kv_code
     out = np.full((B, Q, Hq, d), np.nan, dtype=np.float64)
     nt = nthreads_default() if nthreads is None else nthreads
     _check(lib().oracle_decode_multi(_ptr(out), _ptr(q64), _ptr(key_cache), _ptr(value_cache), code,

@@ -38,7 +38,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2, OR_I8 = 3 };
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2, OR_I8 = 3, OR_I4 = 4 };
 
 /* Planted-mistake switch for the pin tests: a build with -DORACLE_MUTATION=n
  * (n > 0) carries one deliberate error, and the tests check that some pin
@@ -86,7 +86,15 @@ static size_t elem_bytes(int dt)
     }
 }
 
-/* Element idx of a buffer of dtype dt, as a double.  For int8 the raw integer. */
+/* Bytes of a row of d elements of dtype dt (4-bit values pack two per byte). */
+static size_t row_bytes(int dt, int d)
+{
+    return dt == OR_I4 ? (size_t)d / 2 : (size_t)d * elem_bytes(dt);
+}
+
+/* Element idx of a buffer of dtype dt, as a double.  For int8 the raw integer;
+ * for int4 the integer n - 8 of the 4-bit value n, element 2k being the low
+ * half of byte k and element 2k+1 its high half. */
 static double load_elem(const void *base, size_t idx, int dt)
 {
     switch (dt) {
@@ -94,6 +102,11 @@ static double load_elem(const void *base, size_t idx, int dt)
     case OR_F16: return oracle_half_to_double(((const uint16_t *)base)[idx]);
     case OR_BF16: return oracle_bf16_to_double(((const uint16_t *)base)[idx]);
     case OR_I8: return (double)((const int8_t *)base)[idx];
+    case OR_I4: {
+        const uint8_t byte = ((const uint8_t *)base)[idx / 2];
+        const int hi = MUT(12) ? !(idx & 1) : (int)(idx & 1);
+        return (double)((hi ? byte >> 4 : byte & 15) - 8);
+    }
     default: return NAN;
     }
 }
@@ -137,9 +150,8 @@ int oracle_block_copy(void *key_cache, void *value_cache, float *k_scales, float
                       const int64_t *pairs, int64_t num_pairs, int num_kv_heads, int head_dim,
                       int block_size, int64_t num_blocks, int dtype)
 {
-    size_t E = elem_bytes(dtype);
-    if (!E) return -2;
-    size_t blk_bytes = (size_t)num_kv_heads * block_size * head_dim * E;
+    if (!elem_bytes(dtype) && dtype != OR_I4) return -2;
+    size_t blk_bytes = (size_t)num_kv_heads * block_size * row_bytes(dtype, head_dim);
     for (int64_t p = 0; p < num_pairs; ++p) {
         int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
         if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) return -3;
@@ -194,6 +206,46 @@ int oracle_quantize_int8(const void *src, int src_dtype, int8_t *dst, float *sca
     return 0;
 }
 
+/*
+ * 4-bit KV with one scale per group (the pages' second grouped-scale width), the
+ * group again one (block, KV head) tile.  Symmetric absmax in IEEE fp32:
+ *   a = max |x|,  s = a / 7,  q = clamp(rint(x / s), -7, 7)
+ * stored as n = q + 8 in [1, 15]: element 2k in the low four bits of byte k of
+ * the tile, element 2k+1 in the high four.  a = 0 gives s = 0 and q = 0.  dst
+ * holds num_blocks * num_kv_heads * block_size * head_dim / 2 bytes.
+ */
+int oracle_quantize_int4(const void *src, int src_dtype, uint8_t *dst, float *scales,
+                         int64_t num_blocks, int num_kv_heads, int head_dim, int block_size)
+{
+    if (src_dtype != OR_F32 && src_dtype != OR_F16 && src_dtype != OR_BF16) return -4;
+    if (head_dim % 2) return -2;
+    size_t tile = (size_t)block_size * head_dim;
+    for (int64_t t = 0; t < num_blocks * num_kv_heads; ++t) {
+        float a = 0.0f;
+        for (size_t i = 0; i < tile; ++i) {
+            float ax = fabsf((float)load_elem(src, t * tile + i, src_dtype));
+            if (ax > a) a = ax;
+        }
+        float s = MUT(13) ? a / 8.0f : a / 7.0f;
+        scales[t] = s;
+        uint8_t *out = dst + t * (tile / 2);
+        for (size_t i = 0; i < tile; ++i) {
+            float r = 0.0f;
+            if (a != 0.0f) {
+                r = rintf((float)load_elem(src, t * tile + i, src_dtype) / s);
+                if (r > 7.0f) r = 7.0f;
+                if (r < -7.0f) r = -7.0f;
+            }
+            uint8_t n = (uint8_t)((int)r + 8);
+            if (i % 2 == 0)
+                out[i / 2] = n;
+            else
+                out[i / 2] = (uint8_t)(out[i / 2] | (n << 4));
+        }
+    }
+    return 0;
+}
+
 /* Common argument block for the decode functions. */
 typedef struct {
     const double *q;          /* [B][H_q][d], already upcast to fp64 */
@@ -225,7 +277,7 @@ static int gather(const dec_args *a, int b, int g, int t0, int t1, double *Kc, d
         int off = MUT(2) ? (t + 1) % bs : t % bs;
         size_t base = (size_t)(((blk * a->num_kv_heads + g) * bs + off)) * d;
         double ks = 1.0, vs = 1.0;
-        if (a->kv_dtype == OR_I8) {
+        if (a->kv_dtype == OR_I8 || a->kv_dtype == OR_I4) {
             ks = (double)a->k_scales[blk * a->num_kv_heads + g];
             vs = (double)a->v_scales[blk * a->num_kv_heads + g];
         }
@@ -292,8 +344,9 @@ static int check_dims(const dec_args *a)
         a->block_size <= 0)
         return -2;
     if (a->num_q_heads % a->num_kv_heads) return -2;
-    if (a->kv_dtype == OR_I8 && (!a->k_scales || !a->v_scales)) return -1;
-    if (!elem_bytes(a->kv_dtype)) return -4;
+    if ((a->kv_dtype == OR_I8 || a->kv_dtype == OR_I4) && (!a->k_scales || !a->v_scales)) return -1;
+    if (!elem_bytes(a->kv_dtype) && a->kv_dtype != OR_I4) return -4;
+    if (a->kv_dtype == OR_I4 && a->head_dim % 2) return -2;
     return 0;
 }
 

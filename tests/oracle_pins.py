@@ -310,6 +310,68 @@ def pin_quantize():
         q.reshape(-1)[: len(vals)].tolist()
 
 
+# -- 4-bit KV -------------------------------------------------------------------------
+def unpack_int4(packed):
+    """Independent statement of the 4-bit layout: element 2k is the low four bits
+    of byte k, element 2k+1 the high four, each holding q + 8."""
+    lo = (packed & 15).astype(np.int64) - 8
+    hi = (packed >> 4).astype(np.int64) - 8
+    out = np.empty(packed.shape[:-1] + (2 * packed.shape[-1],), dtype=np.int64)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def pin_quantize_int4():
+    rng = np.random.default_rng(52)
+    N, H, d = 5, 2, 64
+    src = (rng.standard_normal((N, H, 16, d)) * 2).astype(np.float16)
+    src[3, 0] = 0  # all-zero tile
+    packed, s = oracle.quantize_int4(src)
+    assert packed.shape == (N, H, 16, d // 2) and packed.dtype == np.uint8
+    q = unpack_int4(packed)
+    assert q.min() >= -7 and q.max() <= 7
+    x = src.astype(np.float64)
+    deq = q * s.astype(np.float64)[:, :, None, None]
+    bound = s.astype(np.float64)[:, :, None, None] * (0.5 + 1e-6)
+    assert np.all(np.abs(deq - x) <= bound), "int4 dequantisation error above s/2"
+    assert s[3, 0] == 0 and np.all(packed[3, 0] == 0x88), "zero tile: q = 0 stored as 8"
+    amax = np.abs(x).reshape(N, H, -1).max(-1)
+    for n in range(N):
+        for h in range(H):
+            if amax[n, h] == 0:
+                continue
+            i = int(np.argmax(np.abs(x[n, h]).reshape(-1)))
+            assert abs(int(q[n, h].reshape(-1)[i])) == 7, "absmax maps to +-7"
+            assert s[n, h] == np.float32(np.float32(amax[n, h]) / np.float32(7)), "scale"
+    # crafted tile: absmax 7 gives s = 1, so q = round-half-even(x), clamped to +-7
+    t = np.zeros((1, 1, 16, d), dtype=np.float32)
+    vals = [7.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.49, -6.5, 6.5, -7.0]
+    t.reshape(-1)[: len(vals)] = vals
+    packed, s = oracle.quantize_int4(t)
+    assert s[0, 0] == 1.0
+    assert unpack_int4(packed).reshape(-1)[: len(vals)].tolist() == [7, 0, 2, 2, 0, -2, -2, 3, -6, 6, -7]
+
+
+def pin_int4_decode_dense():
+    """Decode over packed 4-bit caches equals dense attention on the values the
+    NumPy unpacker gives, scaled, in logical order."""
+    w = W.random_case([1, 17, 40, 64], num_q_heads=8, num_kv_heads=2, head_dim=64, dtype="float16", seed=8)
+    _, kc, vc = replay(w, fill_nan=False)
+    k4, ks = oracle.quantize_int4(kc)
+    v4, vs = oracle.quantize_int4(vc)
+    op = w.steps[0][0]
+    out = oracle.decode(op.q, k4, v4, op.block_tables, op.seq_lens, w.scale, ks, vs)
+    kd = unpack_int4(k4) * ks.astype(np.float64)[:, :, None, None]
+    vd = unpack_int4(v4) * vs.astype(np.float64)[:, :, None, None]
+    q = to_f64(op.q, w.dtype)
+    for b, L in enumerate(op.seq_lens):
+        blocks = op.block_tables[b, : -(-int(L) // 16)]
+        K = np.concatenate([kd[blk].transpose(1, 0, 2) for blk in blocks])[:L]  # [L][H_kv][d]
+        V = np.concatenate([vd[blk].transpose(1, 0, 2) for blk in blocks])[:L]
+        _close(out[b], dense_attention(q[b], K, V, w.scale, w.group), 1e-12, f"int4 b={b}")
+
+
 # -- multi-query decode (query_len new tokens, causal among them) ---------------------
 MULTI_CASES = [
     dict(lens=[2, 17, 40], query_len=2, num_q_heads=8, num_kv_heads=2, head_dim=64, dtype="float16"),
@@ -368,4 +430,5 @@ def pin_multi_single_token_is_decode():
 ALL_PINS = [pin_half_exhaustive, pin_bf16_exhaustive, pin_tiny_dense, pin_random_dense,
             pin_sdpa_library, pin_permutation_invariance, pin_gqa_expand, pin_closed_forms,
             pin_split_merge, pin_kv_size_golden, pin_reshape, pin_block_copy, pin_quantize,
-            pin_multi_dense, pin_multi_sdpa_causal_mask, pin_multi_single_token_is_decode]
+            pin_multi_dense, pin_multi_sdpa_causal_mask, pin_multi_single_token_is_decode,
+            pin_quantize_int4, pin_int4_decode_dense]

@@ -28,6 +28,8 @@ MUTATIONS = {
     9: "partition lse without log l",
     10: "block copy skips V",
     11: "multi-query causal range one token short",
+    12: "int4 nibbles read in swapped order",
+    13: "int4 scale absmax / 8",
 }
 
 # pins cheap enough to run once per mutant
