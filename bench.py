@@ -79,6 +79,8 @@ WORKLOADS = {
               "new sequences U[16,512]",
     "gqa_b8": "7B-GQA decode: 32 q / 8 KV heads, head_dim 128, fp16, batch 8, all lengths 1024",
     "long": "long context: 7B-GQA heads, fp16, batch 16, all lengths 8192, split-K 512",
+    "long_int4": "long context: 7B-GQA heads, 4-bit KV (per-(block, KV head) scales), fp16 q/out, "
+                 "batch 16, all lengths 8192, split-K 512",
     "long_int8": "long context: 7B-GQA heads, int8 KV (per-(block, KV head) scales), fp16 q/out, "
                  "batch 16, all lengths 8192, split-K 512",
     "mha_prefix": "MHA 32/32 heads, head_dim 128, fp16, batch 16, shared 1000-token prefix with "
@@ -124,7 +126,9 @@ def make_workload(name):
     if name == "long":
         return W.long(), False, 512
     if name == "long_int8":
-        return W.long(), True, 512
+        return W.long(), "i8", 512
+    if name == "long_int4":
+        return W.long(), "i4", 512
     if name == "mha_prefix":
         return W.mha_prefix(), False, 256
     if name == "mqa":
@@ -136,12 +140,23 @@ def make_workload(name):
     raise ValueError(name)
 
 
+def kv_elem_bytes(int8):
+    """Bytes per cached value of a quantised pool ("i8": 1, "i4": 0.5), None if not."""
+    return {"i8": 1, "i4": 0.5}.get(int8) if int8 else None
+
+
+def quantize_host(kc, int8):
+    """The oracle's quantiser for the pool kind ("i8" or "i4")."""
+    import oracle
+    return oracle.quantize_int4(kc) if int8 == "i4" else oracle.quantize_int8(kc)
+
+
 def step_bytes(w, int8):
     from paged_kv_cache_395_b200 import workloads as W
     out = []
     for ops in w.steps:
         dec = [o for o in ops if isinstance(o, W.Decode)][0]
-        out.append(W.decode_kv_bytes(dec, w, 1 if int8 else None))
+        out.append(W.decode_kv_bytes(dec, w, kv_elem_bytes(int8)))
     return out
 
 
@@ -245,8 +260,8 @@ def cpu_baseline(w, int8, seconds, host_caches=None):
         oracle.reshape_and_cache(op.k, op.v, kc, vc, op.slot_mapping)
     ks = vs = None
     if int8:
-        kc, ks = oracle.quantize_int8(kc)
-        vc, vs = oracle.quantize_int8(vc)
+        kc, ks = quantize_host(kc, int8)
+        vc, vs = quantize_host(vc, int8)
     threads = oracle.nthreads_default()
     done_bytes, t_work, nsteps, ntok = 0, 0.0, 0, 0
     for si, ops in enumerate(w.steps):
@@ -264,7 +279,7 @@ def cpu_baseline(w, int8, seconds, host_caches=None):
                     oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs,
                                   nthreads=threads)
                 t_work += time.perf_counter() - t0
-                done_bytes += W.decode_kv_bytes(op, w, 1 if int8 else None)
+                done_bytes += W.decode_kv_bytes(op, w, kv_elem_bytes(int8))
                 ntok += op.q.shape[0] * (op.q.shape[1] if op.q.ndim == 4 else 1)
                 nsteps += 1
         if t_work >= seconds:
@@ -288,8 +303,8 @@ def reference_arm(args, rank, world):
         oracle.reshape_and_cache(op.k, op.v, kc, vc, op.slot_mapping)
     ks = vs = None
     if int8:
-        kc, ks = oracle.quantize_int8(kc)
-        vc, vs = oracle.quantize_int8(vc)
+        kc, ks = quantize_host(kc, int8)
+        vc, vs = quantize_host(vc, int8)
     threads = oracle.nthreads_default()
     # each step: the trace's step i % T, a bounded sample of one sequence (all heads)
     decs = [[o for o in ops if isinstance(o, W.Decode)][0] for ops in w.steps]
@@ -306,7 +321,7 @@ def reference_arm(args, rank, world):
             oracle.decode(op.q, kc, vc, op.block_tables, op.seq_lens, w.scale, ks, vs, bh=bh,
                           nthreads=threads)
         L = int(max(op.seq_lens[b], 0))
-        E = 1 if int8 else w.elem_size
+        E = kv_elem_bytes(int8) if int8 else w.elem_size
         return L * w.num_kv_heads * w.head_dim * 2 * E
 
     for i in range(args.warmup):
@@ -351,7 +366,9 @@ def main(argv=None):
     part = args.partition
     dw = runner.DeviceWorkload(w, fill_nan=False)
     dw.run_setup()
-    if int8:
+    if int8 == "i4":
+        dw.quantize_int4()
+    elif int8:
         dw.quantize_int8()
     stream = torch.cuda.Stream()
     # each decode follows this library's own reshape (or decode), which writes none of
@@ -427,7 +444,7 @@ def main(argv=None):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "i8" if int8 else "f16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": int8 if int8 else "f16", "data": "synthetic",
         "config": {"workload": WORKLOADS[args.workload], "name": args.workload,
                    "partition_size": "library picks (-1)" if part == -1 else part, "algo": args.algo,
                    "l2": ("L2 flushed before every timed step (write of twice the L2 size, "

@@ -57,7 +57,9 @@ enum pa_status {
     PA_ERR_ALIGN = -7        /* a buffer is not aligned as documented */
 };
 
-enum pa_dtype { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_I8 = 3 };
+/* PA_I4: 4-bit values, two per byte (see pa_quantize_int4); a PA_I4 cache row of
+ * head_dim values is head_dim / 2 bytes. */
+enum pa_dtype { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_I8 = 3, PA_I4 = 4 };
 
 /* Kernel family for pa_decode.  AUTO picks the fastest built one. */
 enum pa_algo { PA_ALGO_AUTO = 0, PA_ALGO_SIMT = 1, PA_ALGO_TENSOR = 2 };
@@ -105,8 +107,9 @@ typedef struct pa_decode_params {
                                 Tokens beyond max_seq_len or max_blocks_per_seq * 16 are ignored. */
     int q_dtype;             /* dtype of q and out: PA_F32, PA_F16 or PA_BF16 */
     int kv_dtype;            /* PA_F32 (q PA_F32), PA_F16 (q PA_F16), PA_BF16 (q PA_BF16),
-                                or PA_I8 (q PA_F16 or PA_BF16) */
-    const float *k_scales;   /* PA_I8 only: [num_blocks][num_kv_heads], else NULL */
+                                PA_I8 (q PA_F16 or PA_BF16), or PA_I4 (q PA_F16, head_dim
+                                128, tensor-core family) */
+    const float *k_scales;   /* PA_I8 / PA_I4 only: [num_blocks][num_kv_heads], else NULL */
     const float *v_scales;
     int partition_size;      /* 0: one pass, one CTA per (sequence, KV head), no workspace.
                                 > 0: split-K, partitions of this many tokens (a multiple of
@@ -223,6 +226,23 @@ int pa_block_copy(void *key_cache, void *value_cache, float *k_scales, float *v_
  * scales [num_blocks][H_kv].  Call once for K and once for V.
  */
 int pa_quantize_int8(const void *src_cache, int src_dtype, int8_t *dst_cache, float *scales,
+                     int64_t num_blocks, int num_kv_heads, int head_dim, int block_size,
+                     pa_stream_t stream);
+
+
+/*
+ * 4-bit KV with one scale per group (lqnn.cn/news/235768 section 4.1 names
+ * 4-bit storage with grouped scales next to 8-bit), the group being one (block,
+ * KV head) tile of 16 * head_dim values.  For each of the first num_blocks
+ * blocks and each KV head, in IEEE fp32:
+ *   a = max |x|,  s = a / 7,  q = clamp(round_half_even(x / s), -7, 7)
+ * stored as n = q + 8: element 2k of a tile in the low four bits of its byte k,
+ * element 2k+1 in the high four.  a == 0 gives s = 0 and q = 0 (bytes 0x88).
+ * src_cache: [num_blocks][H_kv][16][head_dim] of src_dtype (PA_F32, PA_F16 or
+ * PA_BF16); dst_cache: [num_blocks][H_kv][16][head_dim / 2] bytes; scales
+ * [num_blocks][H_kv].  head_dim must be even.  Call once for K and once for V.
+ */
+int pa_quantize_int4(const void *src_cache, int src_dtype, uint8_t *dst_cache, float *scales,
                      int64_t num_blocks, int num_kv_heads, int head_dim, int block_size,
                      pa_stream_t stream);
 

@@ -121,8 +121,9 @@ def block_copy(key_cache, value_cache, pairs, k_scales=None, v_scales=None, code
     N, H, bs, d = key_cache.shape
     pr = np.ascontiguousarray(pairs, dtype=np.int64).reshape(-1, 2)
     code = dtype_code(key_cache.dtype) if code is None else code
+    head_dim = 2 * d if code == I4 else d  # a packed 4-bit row holds two values per byte
     _check(lib().oracle_block_copy(_ptr(key_cache), _ptr(value_cache), _ptr(k_scales),
-                                   _ptr(v_scales), _ptr(pr), pr.shape[0], H, d, bs, N, code),
+                                   _ptr(v_scales), _ptr(pr), pr.shape[0], H, head_dim, bs, N, code),
            "oracle_block_copy")
 
 

@@ -83,12 +83,15 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
         return PA_ERR_SHAPE;
     if (p->num_q_heads % p->num_kv_heads) return PA_ERR_SHAPE;
     if (p->block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
-    if (!elem_size(p->q_dtype) || !elem_size(p->kv_dtype) || p->q_dtype == PA_I8) return PA_ERR_DTYPE;
+    if (!elem_size(p->q_dtype) || (!elem_size(p->kv_dtype) && p->kv_dtype != PA_I4) || p->q_dtype == PA_I8)
+        return PA_ERR_DTYPE;
     if (p->query_len < 0) return PA_ERR_SHAPE;
     KernelHeads kh;
     const bool heads_ok = kernel_heads(p, &kh);
-    const bool pair_ok = (p->q_dtype == p->kv_dtype) || p->kv_dtype == PA_I8;
-    if (!pair_ok || (p->kv_dtype == PA_I8 && p->q_dtype == PA_F32)) return PA_ERR_DTYPE;
+    const bool quant = p->kv_dtype == PA_I8 || p->kv_dtype == PA_I4;
+    const bool pair_ok = (p->q_dtype == p->kv_dtype) || quant;
+    if (!pair_ok || (quant && p->q_dtype == PA_F32) || (p->kv_dtype == PA_I4 && p->q_dtype != PA_F16))
+        return PA_ERR_DTYPE;
     if (!heads_ok) return PA_ERR_UNSUPPORTED;
     const bool simt_ok = kh.qlen == 1 && !kh.padded &&
                          decode_simt_supported(p->q_dtype, p->kv_dtype, p->head_dim, kh.G);
@@ -221,14 +224,30 @@ int pa_block_copy(void *key_cache, void *value_cache, float *k_scales, float *v_
                   int block_size, int64_t num_blocks, int dtype, pa_stream_t stream) {
     if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0) return PA_ERR_SHAPE;
     if (block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
-    const int E = elem_size(dtype);
+    // a 4-bit cache row is head_dim / 2 bytes: copy it as bytes
+    const int E = dtype == PA_I4 ? 1 : elem_size(dtype);
     if (!E) return PA_ERR_DTYPE;
+    if (dtype == PA_I4 && head_dim % 2) return PA_ERR_SHAPE;
+    const int row_elems = dtype == PA_I4 ? head_dim / 2 : head_dim;
     if (num_pairs == 0) return PA_OK;
     if (!key_cache || !value_cache || !src_dst_pairs) return PA_ERR_NULL;
     if ((k_scales == nullptr) != (v_scales == nullptr)) return PA_ERR_NULL;
     if (num_pairs > 2147483647LL) return PA_ERR_UNSUPPORTED;
     return launch_block_copy(key_cache, value_cache, k_scales, v_scales, src_dst_pairs, num_pairs,
-                             num_kv_heads, head_dim, num_blocks, E, (cudaStream_t)stream);
+                             num_kv_heads, row_elems, num_blocks, E, (cudaStream_t)stream);
+}
+
+int pa_quantize_int4(const void *src_cache, int src_dtype, uint8_t *dst_cache, float *scales,
+                     int64_t num_blocks, int num_kv_heads, int head_dim, int block_size,
+                     pa_stream_t stream) {
+    if (num_blocks < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 2) return PA_ERR_SHAPE;
+    if (block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
+    if (src_dtype != PA_F32 && src_dtype != PA_F16 && src_dtype != PA_BF16) return PA_ERR_DTYPE;
+    if (num_blocks == 0) return PA_OK;
+    if (!src_cache || !dst_cache || !scales) return PA_ERR_NULL;
+    if (num_blocks * num_kv_heads > 2147483647LL) return PA_ERR_UNSUPPORTED;
+    return launch_quantize_int4(src_cache, src_dtype, dst_cache, scales, num_blocks, num_kv_heads, head_dim,
+                                (cudaStream_t)stream);
 }
 
 int pa_quantize_int8(const void *src_cache, int src_dtype, int8_t *dst_cache, float *scales,
@@ -258,7 +277,7 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     if (rc != PA_OK) return rc;
     if (p->num_seqs == 0) return PA_OK;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !seq_lens) return PA_ERR_NULL;
-    if (p->kv_dtype == PA_I8 && (!p->k_scales || !p->v_scales)) return PA_ERR_NULL;
+    if ((p->kv_dtype == PA_I8 || p->kv_dtype == PA_I4) && (!p->k_scales || !p->v_scales)) return PA_ERR_NULL;
     if (((uintptr_t)key_cache | (uintptr_t)value_cache) % 16) return PA_ERR_ALIGN;
     if (pl.bytes > 0 && (!p->workspace || p->workspace_bytes < pl.bytes)) return PA_ERR_WORKSPACE;
     if (pl.bytes > 0 && (uintptr_t)p->workspace % 16) return PA_ERR_ALIGN;

@@ -166,4 +166,54 @@ int launch_quantize_int8(const void *src, int src_dtype, int8_t *dst, float *sca
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// quantize_int4 (lqnn.cn/news/235768 section 4.1: 4-bit KV with a grouped
+// scale; the group is one (block, KV head) tile).  One CTA of 128 threads per
+// tile; IEEE fp32 divide and round-half-even; each thread writes whole bytes
+// (two elements).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) quantize_int4_kernel(const T *__restrict__ src,
+                                                            uint8_t *__restrict__ dst,
+                                                            float *__restrict__ scales, int tile) {
+    __shared__ float red[4];
+    pdl_wait();
+    pdl_release_dependents();
+    const int64_t t = blockIdx.x;
+    const T *x = src + t * tile;
+    float a = 0.f;
+    for (int i = threadIdx.x; i < tile; i += blockDim.x) a = fmaxf(a, fabsf(Cvt<T>::to_f(x[i])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    a = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float s = __fdiv_rn(a, 7.0f);
+    if (threadIdx.x == 0) scales[t] = s;
+    uint8_t *y = dst + t * (tile / 2);
+    auto q4 = [&](float v) -> int {
+        if (a == 0.f) return 8;
+        const int r = __float2int_rn(__fdiv_rn(v, s));
+        return max(-7, min(7, r)) + 8;
+    };
+    for (int k = threadIdx.x; k < tile / 2; k += blockDim.x)
+        y[k] = (uint8_t)(q4(Cvt<T>::to_f(x[2 * k])) | (q4(Cvt<T>::to_f(x[2 * k + 1])) << 4));
+}
+
+int launch_quantize_int4(const void *src, int src_dtype, uint8_t *dst, float *scales,
+                         int64_t N, int H, int D, cudaStream_t st) {
+    const int64_t tiles = N * H;
+    if (tiles == 0) return PA_OK;
+    const int tile = kBlockSize * D;
+    cudaError_t e;
+    const dim3 grid((unsigned)tiles);
+    switch (src_dtype) {
+    case PA_F32: e = launch_pdl(quantize_int4_kernel<float>, grid, dim3(128), 0, st, (const float *)src, dst, scales, tile); break;
+    case PA_F16: e = launch_pdl(quantize_int4_kernel<__half>, grid, dim3(128), 0, st, (const __half *)src, dst, scales, tile); break;
+    case PA_BF16: e = launch_pdl(quantize_int4_kernel<__nv_bfloat16>, grid, dim3(128), 0, st, (const __nv_bfloat16 *)src, dst, scales, tile); break;
+    default: return PA_ERR_DTYPE;
+    }
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 }  // namespace pa

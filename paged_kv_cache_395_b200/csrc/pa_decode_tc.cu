@@ -63,6 +63,11 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
 }
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+    return v;
+}
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
@@ -128,16 +133,23 @@ template <> struct Mma<__nv_bfloat16> {
 #define PA_TC_MIN_CTAS 1
 #endif
 
-// TKV: the cache element, the q/out type T or int8_t.  A tile row is D * sizeof(TKV)
-// bytes, brought in as 128-byte boxes (64 fp16/bf16 or 128 int8 elements).
+// TKV: the cache element: the q/out type T, int8_t, or U4x2 (two 4-bit values
+// per byte).  fp16/bf16 and int8 tile rows come as 128-byte boxes (64 or 128
+// elements) with 128-byte swizzle; a 4-bit tile row is D / 2 bytes, one box, no
+// swizzle.
+struct U4x2 {
+    uint8_t v;
+};
 template <typename TKV, int D, int G>
 struct TcCfg {
+    static constexpr bool I4 = std::is_same<TKV, U4x2>::value;
     static constexpr int NW = PA_TC_WARPS;        // warps (independent workers) per CTA
     static constexpr int THREADS = NW * 32;
     static constexpr int S = PA_TC_STAGES;        // ring stages per warp
-    static constexpr int BOXW = 128 / (int)sizeof(TKV);  // elements per box row
-    static constexpr int BOXES = D / BOXW;        // boxes per tile row
-    static constexpr int BOX_BYTES = 16 * 128;    // one box of a tile
+    static constexpr int ROW_BYTES = I4 ? D / 2 : 128;              // bytes per box row
+    static constexpr int BOXW = I4 ? D / 2 : 128 / (int)sizeof(TKV);  // TMA elements per box row
+    static constexpr int BOXES = I4 ? 1 : D / BOXW;                  // boxes per tile row
+    static constexpr int BOX_BYTES = 16 * ROW_BYTES;                 // one box of a tile
     static constexpr int TILE = BOXES * BOX_BYTES;
     static constexpr int STAGE = 2 * TILE;        // K tile, then V tile
     static constexpr int KSTEPS = D / 16;         // QK k-steps
@@ -297,6 +309,61 @@ __device__ __forceinline__ void vfrag_i8(const uint32_t (&r)[4][4], int i, uint3
     }
 }
 
+// ---------------------------------------------------------------------------
+// 4-bit tiles -> fp16 MMA fragments
+// ---------------------------------------------------------------------------
+// A 4-bit tile row is D / 2 bytes (64 at D = 128), unswizzled; byte k holds
+// element 2k in its low four bits and 2k+1 in its high four, each as q + 8, so
+// nibble t of a 32-bit word (bits 4t .. 4t+3) is element 8w + t of that word w.
+// Two nibbles in bits 0-3 and 16-19 become an fp16 pair exactly: OR-ing
+// 0x6400 gives 1024 + n, and subtracting 1032 (0x6408) leaves n - 8 = q.
+__device__ __forceinline__ uint32_t u4pair_to_h2(uint32_t x) {  // x: nibbles in bits 0-3, 16-19
+    uint32_t r = (x & 0x000f000fu) | 0x64006400u;
+    asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(r) : "r"(0x64086408u));
+    return r;
+}
+__device__ __forceinline__ void lds_v2(uint32_t (&w)[2], uint32_t addr) {
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr) : "memory");
+}
+
+// K from a 4-bit tile (D = 128): thread column c reads the 16 bytes (32 dims
+// 32c .. 32c + 31) of tokens g and g + 8.  The contraction runs over the dims in
+// the order the nibble pairs give: in k-step ks (word w = ks / 2, t0 = 2 (ks % 2),
+// t1 = t0 + 1) k slots 2c, 2c+1 are dims 32c + 8w + t0 and + t0 + 4, k slots 2c+8,
+// 2c+9 dims 32c + 8w + t1 and + t1 + 4; q is read in the same order.
+__device__ __forceinline__ void kload_i4(uint32_t (&w)[2][4], uint32_t tile, int g, int c) {
+    lds_v4(w[0], tile + g * 64 + c * 16);
+    lds_v4(w[1], tile + (g + 8) * 64 + c * 16);
+}
+__device__ __forceinline__ void kfrag_i4(const uint32_t (&w)[2][4], int ks, uint32_t (&a)[4]) {
+    const int wi = ks >> 1, t0 = 2 * (ks & 1);
+    a[0] = u4pair_to_h2(w[0][wi] >> (4 * t0));        // token g
+    a[1] = u4pair_to_h2(w[1][wi] >> (4 * t0));        // token g + 8
+    a[2] = u4pair_to_h2(w[0][wi] >> (4 * t0 + 4));
+    a[3] = u4pair_to_h2(w[1][wi] >> (4 * t0 + 4));
+}
+
+// V^T from a 4-bit tile: thread row g owns dims 16g .. 16g + 15 (8 bytes of each
+// token row), as in the int8 path; the tokens are 2c, 2c+1 and 2c+8, 2c+9.
+__device__ __forceinline__ void vload_i4(uint32_t (&r)[4][2], uint32_t tile, int g, int c) {
+    lds_v2(r[0], tile + (2 * c) * 64 + g * 8);
+    lds_v2(r[1], tile + (2 * c + 1) * 64 + g * 8);
+    lds_v2(r[2], tile + (2 * c + 8) * 64 + g * 8);
+    lds_v2(r[3], tile + (2 * c + 9) * 64 + g * 8);
+}
+__device__ __forceinline__ void vfrag_i4(const uint32_t (&r)[4][2], int i, uint32_t (&a)[4]) {
+    // byte i / 2 of both tokens' words into bytes 0 and 2, then nibble i % 2 of each
+    const uint32_t sel = (uint32_t)(i >> 1) | ((uint32_t)(4 + (i >> 1)) << 8);
+    const int sh = 4 * (i & 1);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // register q: token pair q / 2, word q % 2 (dim 16g + 8 (q % 2) + i)
+        const int p = q >> 1, wi = q & 1;
+        uint32_t y;
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(y) : "r"(r[2 * p][wi]), "r"(r[2 * p + 1][wi]), "r"(sel));
+        a[q] = u4pair_to_h2(y >> sh);
+    }
+}
+
 // MQ: the general column mapping (several new tokens per sequence, causal among
 // them, or padding columns); without it every row's G columns are the G query
 // heads of one single-token decode, and the kernel keeps the plain addressing.
@@ -308,7 +375,10 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     constexpr int NW = C::NW, S = C::S;
     constexpr bool SPLIT_P = sizeof(T) == 2 && !std::is_same<T, __half>::value;  // bf16: P = hi + lo
     constexpr bool kI8 = std::is_same<TKV, int8_t>::value;
-    static_assert(!kI8 || (std::is_same<T, __half>::value && D == 128), "int8 caches: fp16 q, head_dim 128");
+    constexpr bool kI4 = C::I4;
+    constexpr bool kQz = kI8 || kI4;  // quantised cache: per-(block, KV head) scales
+    static_assert(!kQz || (std::is_same<T, __half>::value && D == 128),
+                  "int8 and 4-bit caches: fp16 q, head_dim 128");
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -496,7 +566,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         const int pb = a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
         if (pb < 0 || (int64_t)pb >= a.N) return -2;
         const int kc = w.sg.kvh / a.ngroups;  // the cache's KV head
-        if constexpr (kI8) {
+        if constexpr (kQz) {
             ks = a.ks[(size_t)pb * Hc + kc];
             vs = a.vs[(size_t)pb * Hc + kc];
         }
@@ -512,7 +582,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         if (!pc.valid) return;
         const int y = __shfl_sync(0xffffffffu, p_y, p_i);
         float ksv = 0.f, vsv = 0.f;
-        if constexpr (kI8) {
+        if constexpr (kQz) {
             ksv = __shfl_sync(0xffffffffu, p_ks, p_i);
             vsv = __shfl_sync(0xffffffffu, p_vs, p_i);
         }
@@ -525,7 +595,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             const int ncol = seg_first ? pc.sg.ncol : 0;
             const uint32_t tx = (y < 0 ? 0u : (uint32_t)C::STAGE) + (uint32_t)(ncol * D * (int)sizeof(T));
             my_ok[s] = y >= 0;
-            if constexpr (kI8) {
+            if constexpr (kQz) {
                 my_sc[2 * s] = ksv;  // released to the consumer by the arrive below
                 my_sc[2 * s + 1] = vsv;
             }
@@ -594,13 +664,27 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     // O^T row (m-tile i, row g; row g + 8 is dim + 8) -> head dim: m-tile i holds
     // dims 16i .. 16i + 15 for fp16/bf16 tiles; the int8 path gives thread row g
     // the 16 dims 16g .. 16g + 15 instead (see vfrag_i8)
-    auto dmap = [&](int i, int gg) -> int { return kI8 ? 16 * gg + i : 16 * i + gg; };
+    auto dmap = [&](int i, int gg) -> int { return kQz ? 16 * gg + i : 16 * i + gg; };
     const int h0 = 2 * c, h1 = 2 * c + 1;  // heads of this thread's S^T / O^T columns
     // B fragments of q (n = heads, k = dims) from the q slot of stage s.  The
     // int8 path orders the contraction's dims differently (see kfrag_i8): k-step
     // ks, thread column c covers dims 32c + 4ks .. 32c + 4ks + 3.
     auto load_q = [&](int s, uint32_t (&bq)[C::KSTEPS][2], int ncol) {
-        const uint32_t qs = qring + s * C::QSLOT + (kI8 ? (g * D + 32 * c) * 2 : (g * D + 2 * c) * 2);
+        const uint32_t qs = qring + s * C::QSLOT + (kQz ? (g * D + 32 * c) * 2 : (g * D + 2 * c) * 2);
+        if constexpr (kI4) {
+            // the 4-bit order (see kfrag_i4): k-step ks pairs dims 8w + t and 8w + t + 4
+#pragma unroll
+            for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                const int w8 = 8 * (ks >> 1), t0 = 2 * (ks & 1);
+                if (g < ncol) {
+                    bq[ks][0] = lds_u16(qs + (w8 + t0) * 2) | (lds_u16(qs + (w8 + t0 + 4) * 2) << 16);
+                    bq[ks][1] = lds_u16(qs + (w8 + t0 + 1) * 2) | (lds_u16(qs + (w8 + t0 + 5) * 2) << 16);
+                } else {
+                    bq[ks][0] = bq[ks][1] = 0u;
+                }
+            }
+            return;
+        }
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS; ++ks) {
             if (g < ncol) {
@@ -783,11 +867,17 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 const uint32_t vm_lo = (2 * c < ntok ? 0x0000ffffu : 0u) | (2 * c + 1 < ntok ? 0xffff0000u : 0u);
                 const uint32_t vm_hi = (2 * c + 8 < ntok ? 0x0000ffffu : 0u) | (2 * c + 9 < ntok ? 0xffff0000u : 0u);
                 // ---- fragments: K (A of S^T), then V^T (A of O^T), all issued up front
-                constexpr bool kHoist = PA_TC_HOIST_V && !kI8;
-                uint32_t kf[kI8 ? 1 : C::KSTEPS][4], vf[kHoist ? C::MTILES : 1][4];
+                constexpr bool kHoist = PA_TC_HOIST_V && !kQz;
+                uint32_t kf[kQz ? 1 : C::KSTEPS][4], vf[kHoist ? C::MTILES : 1][4];
                 uint32_t kw[kI8 ? 2 : 1][8], vw[kI8 ? 4 : 1][4];  // raw int8 words
+                uint32_t kw4[kI4 ? 2 : 1][4], vw4[kI4 ? 4 : 1][2];  // raw 4-bit words
                 float slog = a.scale_log2, vsc = 1.f;
-                if constexpr (kI8) {
+                if constexpr (kI4) {
+                    slog *= my_sc[2 * s];
+                    vsc = my_sc[2 * s + 1];
+                    kload_i4(kw4, tK, g, c);
+                    vload_i4(vw4, tK + C::TILE, g, c);
+                } else if constexpr (kI8) {
                     // int8 tiles (128-byte rows, 128-byte swizzle), converted exactly to fp16 in
                     // registers fragment by fragment; the block's K scale goes into the score
                     // scale, its V scale into the probabilities fed to P.V (the softmax sum
@@ -817,7 +907,10 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 for (int u = 0; u < 4; ++u) sa[u][0] = sa[u][1] = sa[u][2] = sa[u][3] = 0.f;
 #pragma unroll
                 for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                    if constexpr (kI8) {
+                    if constexpr (kI4) {
+                        kfrag_i4(kw4, ks, kf[0]);
+                        Mma<T>::mma(sa[ks & 3], kf[0], bq[ks][0], bq[ks][1]);
+                    } else if constexpr (kI8) {
                         kfrag_i8(kw, ks, kf[0]);
                         Mma<T>::mma(sa[ks & 3], kf[0], bq[ks][0], bq[ks][1]);
                     } else {
@@ -891,8 +984,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 #pragma unroll
                 for (int i = 0; i < C::MTILES; ++i) {
                     const int vi = kHoist ? i : 0;
-                    if constexpr (kI8) {
-                        vfrag_i8(vw, i, vf[0]);
+                    if constexpr (kQz) {
+                        if constexpr (kI4)
+                            vfrag_i4(vw4, i, vf[0]);
+                        else
+                            vfrag_i8(vw, i, vf[0]);
                         vf[0][0] &= vm_lo;
                         vf[0][1] &= vm_lo;
                         vf[0][2] &= vm_hi;
@@ -1024,16 +1120,19 @@ static bool cache_tensor_map(CUtensorMap *m, const void *base, int64_t rows, int
     }
     auto fn = encode_fn();
     if (!fn) return false;
-    const int esize = dtype == PA_I8 ? 1 : 2;
-    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)D * esize};
-    cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 16};  // 128-byte box rows
+    // 4-bit caches: rows of D / 2 bytes, one unswizzled box per tile row
+    const bool i4 = dtype == PA_I4;
+    const int esize = (dtype == PA_I8 || i4) ? 1 : 2;
+    const int width = i4 ? D / 2 : D;  // TMA elements per cache row
+    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)width * esize};
+    cuuint32_t box[2] = {(cuuint32_t)(i4 ? width : 128 / esize), 16};  // 128-byte (4-bit: D/2-byte) box rows
     cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapDataType dt = dtype == PA_BF16  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                   : dtype == PA_I8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
-                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapDataType dt = dtype == PA_BF16                  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : (dtype == PA_I8 || i4)          ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    i4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
     std::lock_guard<std::mutex> lock(mu);
@@ -1073,8 +1172,8 @@ static bool launch_shape(const void *kernel, int threads, int smem, int *sms, in
 
 bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
     const bool same = (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype && (D == 64 || D == 128);
-    const bool i8 = q_dtype == PA_F16 && kv_dtype == PA_I8 && D == 128;
-    return (same || i8) && (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
+    const bool quant = q_dtype == PA_F16 && (kv_dtype == PA_I8 || kv_dtype == PA_I4) && D == 128;
+    return (same || quant) && (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
 }
 
 template <typename T, typename TKV, int D, int G, bool MQ>
@@ -1123,6 +1222,10 @@ int launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
     if (a.q_dtype == PA_F16 && a.kv_dtype == PA_I8) {
         if (a.D != 128) return PA_ERR_UNSUPPORTED;
         return launch_tc_g<__half, int8_t, 128>(a, st);
+    }
+    if (a.q_dtype == PA_F16 && a.kv_dtype == PA_I4) {
+        if (a.D != 128) return PA_ERR_UNSUPPORTED;
+        return launch_tc_g<__half, U4x2, 128>(a, st);
     }
     if (a.q_dtype == PA_F16)
         return a.D == 64 ? launch_tc_g<__half, __half, 64>(a, st) : launch_tc_g<__half, __half, 128>(a, st);

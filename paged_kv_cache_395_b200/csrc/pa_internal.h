@@ -22,6 +22,8 @@ int launch_block_copy(void *kc, void *vc, float *ks, float *vs, const int64_t *p
                       int H, int D, int64_t N, int E, cudaStream_t st);
 int launch_quantize_int8(const void *src, int src_dtype, int8_t *dst, float *scales, int64_t N,
                          int H, int D, cudaStream_t st);
+int launch_quantize_int4(const void *src, int src_dtype, uint8_t *dst, float *scales, int64_t N,
+                         int H, int D, cudaStream_t st);
 
 // Everything pa_decode needs after validation.
 struct DecodeArgs {

@@ -24,14 +24,15 @@ LIB_PATH = os.path.join(_HERE, "libpa.so")
 
 PA_OK, PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_DTYPE = 0, -1, -2, -3
 PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_ALIGN = -4, -5, -6, -7
-PA_F32, PA_F16, PA_BF16, PA_I8 = 0, 1, 2, 3
+PA_F32, PA_F16, PA_BF16, PA_I8, PA_I4 = 0, 1, 2, 3, 4
 PA_ALGO_AUTO, PA_ALGO_SIMT, PA_ALGO_TENSOR = 0, 1, 2
 PA_EFLAG_BAD_BLOCK, PA_EFLAG_BAD_SLOT, PA_EFLAG_BAD_PAIR, PA_EFLAG_WAIT_TIMEOUT = 1, 2, 4, 8
 PA_DECODE_INPUTS_READY = 1
 BLOCK_SIZE = 16
 
+# a uint8 cache tensor [N][H_kv][16][d/2] holds 4-bit values, two per byte
 _TORCH_DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16,
-                torch.int8: PA_I8}
+                torch.int8: PA_I8, torch.uint8: PA_I4}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -72,12 +73,13 @@ def _load():
     L.pa_decode_workspace_size.restype = ctypes.c_size_t
     L.pa_block_copy.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, P]
     L.pa_quantize_int8.argtypes = [P, i32, P, P, i64, i32, i32, i32, P]
+    L.pa_quantize_int4.argtypes = [P, i32, P, P, i64, i32, i32, i32, P]
     L.pa_get_error_flags.argtypes = [ctypes.POINTER(ctypes.c_uint), i32, P]
     L.pa_status_string.argtypes = [i32]
     L.pa_status_string.restype = ctypes.c_char_p
     L.pa_version.argtypes = []
     for n in ("pa_reshape_and_cache", "pa_decode", "pa_decode_fixed_scratch", "pa_block_copy",
-              "pa_quantize_int8", "pa_get_error_flags", "pa_version"):
+              "pa_quantize_int8", "pa_quantize_int4", "pa_get_error_flags", "pa_version"):
         getattr(L, n).restype = i32
     return L
 
@@ -86,7 +88,8 @@ lib = _load()
 
 # the C-ABI symbols include/pa.h declares
 EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_fixed_scratch",
-            "pa_block_copy", "pa_quantize_int8", "pa_get_error_flags", "pa_status_string", "pa_version")
+            "pa_block_copy", "pa_quantize_int8", "pa_quantize_int4", "pa_get_error_flags",
+            "pa_status_string", "pa_version")
 FIXED_SCRATCH_BYTES = 32 << 20  # PA_FIXED_SCRATCH_BYTES
 
 
@@ -175,7 +178,7 @@ def uses_tensor_cores(q, key_cache, algo=PA_ALGO_AUTO) -> bool:
     Hkv = key_cache.shape[1]
     G = Hq // Hkv
     same = q.dtype in (torch.float16, torch.bfloat16) and key_cache.dtype == q.dtype and d in (64, 128)
-    i8 = q.dtype == torch.float16 and key_cache.dtype == torch.int8 and d == 128
+    i8 = q.dtype == torch.float16 and key_cache.dtype in (torch.int8, torch.uint8) and d == 128
     ok = (same or i8) and Q * G <= 512 and B <= 4096
     return algo == PA_ALGO_TENSOR or (algo == PA_ALGO_AUTO and ok)
 
@@ -242,9 +245,12 @@ def pa_decode_fixed_scratch(out, q, key_cache, value_cache, block_tables, seq_le
 
 
 def pa_block_copy(key_cache, value_cache, pairs, k_scales=None, v_scales=None, stream=None):
-    """pairs int64 [n][2] (src, dst) on the device."""
+    """pairs int64 [n][2] (src, dst) on the device.  A uint8 (4-bit) cache
+    [N][H_kv][16][d/2] is copied as such."""
     _dev(key_cache, value_cache, pairs, k_scales, v_scales)
     N, H, bs, d = key_cache.shape
+    if key_cache.dtype == torch.uint8:
+        d *= 2  # head_dim of a 4-bit cache
     if pairs.dtype != torch.int64 or not pairs.is_contiguous():
         raise ValueError("pairs must be contiguous int64")
     n = pairs.numel() // 2
@@ -261,6 +267,19 @@ def pa_quantize_int8(src_cache, dst_cache, scales, stream=None):
         raise ValueError("dst must be int8 and scales float32")
     _check(lib.pa_quantize_int8(_ptr(src_cache), dtype_code(src_cache.dtype), _ptr(dst_cache),
                                 _ptr(scales), N, H, d, bs, _stream(stream)), "pa_quantize_int8")
+
+
+def pa_quantize_int4(src_cache, dst_cache, scales, stream=None):
+    """src [N][H_kv][16][d] fp32/fp16/bf16 -> dst uint8 [N][H_kv][16][d/2] (4-bit
+    values q + 8, element 2k in the low half of byte k), scales fp32 [N][H_kv]."""
+    _dev(src_cache, dst_cache, scales)
+    N, H, bs, d = src_cache.shape
+    if dst_cache.dtype != torch.uint8 or tuple(dst_cache.shape) != (N, H, bs, d // 2):
+        raise ValueError("dst must be uint8 [N][H_kv][16][d/2]")
+    if scales.dtype != torch.float32:
+        raise ValueError("scales must be float32")
+    _check(lib.pa_quantize_int4(_ptr(src_cache), dtype_code(src_cache.dtype), _ptr(dst_cache),
+                                _ptr(scales), N, H, d, bs, _stream(stream)), "pa_quantize_int4")
 
 
 def pa_get_error_flags(reset: bool = True, stream=None) -> int:

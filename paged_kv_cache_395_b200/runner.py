@@ -71,7 +71,19 @@ class DeviceWorkload:
         pa.pa_quantize_int8(self.kc, self.kc8, self.k_scales)
         pa.pa_quantize_int8(self.vc, self.vc8, self.v_scales)
 
+    def quantize_int4(self):
+        """Replace the pool by its 4-bit form (two values per byte, one scale per
+        (block, KV head)); the caches become uint8 [N][H_kv][16][d/2]."""
+        N, H, bs, d = self.kc.shape
+        self.kc8 = torch.empty((N, H, bs, d // 2), dtype=torch.uint8, device=self.device)
+        self.vc8 = torch.empty_like(self.kc8)
+        self.k_scales = torch.empty((N, H), dtype=torch.float32, device=self.device)
+        self.v_scales = torch.empty_like(self.k_scales)
+        pa.pa_quantize_int4(self.kc, self.kc8, self.k_scales)
+        pa.pa_quantize_int4(self.vc, self.vc8, self.v_scales)
+
     def workspace_for(self, op, partition_size, int8=False, algo=pa.PA_ALGO_AUTO):
+        """int8: the quantised pool (int8, or 4-bit after quantize_int4) is decoded."""
         _, q, bt, _, mx, _ = op
         kc = self.kc8 if int8 else self.kc
         n = pa.pa_decode_workspace_size(q, kc, bt, mx, partition_size,

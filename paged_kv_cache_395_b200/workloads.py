@@ -407,12 +407,12 @@ def decode_kv_bytes(op: Decode, w: Workload, kv_elem: float | None = None) -> in
     """Algorithmic bytes of one decode: every K and V element of every logical
     token once, int8 scales once per (block, KV head) read, q in, out out,
     table entries read and seq_lens."""
-    E = w.elem_size if kv_elem is None else kv_elem
+    E = w.elem_size if kv_elem is None else kv_elem  # int8 1, 4-bit 0.5
     L = op.seq_lens.astype(np.int64)
     L = L[L > 0]
     nblk = -(-L // w.block_size)
     B = op.seq_lens.shape[0]
-    kv = int(L.sum()) * w.num_kv_heads * w.head_dim * 2 * E
-    scales = int(nblk.sum()) * w.num_kv_heads * 2 * 4 if kv_elem == 1 else 0
+    kv = int(int(L.sum()) * w.num_kv_heads * w.head_dim * 2 * E)
+    scales = int(nblk.sum()) * w.num_kv_heads * 2 * 4 if kv_elem is not None and kv_elem <= 1 else 0
     qo = int(op.q.size) * 2 * w.elem_size  # q in, out out (Q query tokens each)
     return int(kv + scales + qo + int(nblk.sum()) * 4 + B * 4)

@@ -65,6 +65,9 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails val
     (dict(query_len=129, num_q_heads=8, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),  # 516 pairs per KV head
     (dict(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F16), pa.PA_ERR_DTYPE),
     (dict(q_dtype=pa.PA_I8, kv_dtype=pa.PA_I8), pa.PA_ERR_DTYPE),
+    (dict(q_dtype=pa.PA_BF16, kv_dtype=pa.PA_I4), pa.PA_ERR_DTYPE),   # 4-bit caches take fp16 q
+    (dict(kv_dtype=pa.PA_I4, algo=pa.PA_ALGO_SIMT), pa.PA_ERR_UNSUPPORTED),
+    (dict(kv_dtype=pa.PA_I4, head_dim=64, algo=pa.PA_ALGO_TENSOR), pa.PA_ERR_UNSUPPORTED),
     (dict(q_dtype=9), pa.PA_ERR_DTYPE),
     (dict(partition_size=24), pa.PA_ERR_SHAPE),
     (dict(partition_size=-2), pa.PA_ERR_SHAPE),

@@ -141,3 +141,49 @@ def test_quantize_long_config_bit_exact():
         q_ref, s_ref = oracle.quantize_int8(host)
         assert np.array_equal(bits(dev_q), np_bits(q_ref))
         assert np.array_equal(bits(dev_s), np_bits(s_ref))
+
+
+@pytest.mark.parametrize("dtype", ["float16", "bfloat16", "float32"])
+def test_quantize_int4_bit_exact(dtype):
+    """The 4-bit quantiser byte for byte (and its scales bit for bit) against the
+    oracle: random tiles of very different ranges, an all-zero tile, and a tile
+    with absmax 7 (s = 1) holding round-half-even cases."""
+    dev = "cuda"
+    rng = np.random.default_rng(14)
+    N, H, d = 64, 4, 128
+    x = rng.standard_normal((N, H, 16, d)) * rng.uniform(0.01, 30, size=(N, H, 1, 1))
+    x[3, 1] = 0.0
+    x[5, 2] = 0.0
+    x[5, 2].reshape(-1)[:10] = [7, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 6.5, -6.5, -7]
+    if dtype == "bfloat16":
+        t = torch.from_numpy(x).to(torch.bfloat16)
+        host = t.view(torch.int16).numpy().view(np.uint16)
+        dsrc = t.to(dev)
+        code = oracle.BF16
+    else:
+        host = x.astype(dtype)
+        dsrc = torch.from_numpy(host).to(dev)
+        code = None
+    q_ref, s_ref = oracle.quantize_int4(host, code=code)
+    q = torch.empty((N, H, 16, d // 2), dtype=torch.uint8, device=dev)
+    s = torch.empty((N, H), dtype=torch.float32, device=dev)
+    pa.pa_quantize_int4(dsrc, q, s)
+    assert np.array_equal(bits(q), np_bits(q_ref))
+    assert np.array_equal(bits(s), np_bits(s_ref))
+
+
+def test_block_copy_int4():
+    """Copy-on-write of packed 4-bit blocks (rows of d / 2 bytes) with their scales."""
+    dev = "cuda"
+    rng = np.random.default_rng(9)
+    N, H, d = 9, 2, 128
+    kc = rng.integers(0, 256, size=(N, H, 16, d // 2)).astype(np.uint8)
+    vc = rng.integers(0, 256, size=(N, H, 16, d // 2)).astype(np.uint8)
+    ks = rng.random((N, H)).astype(np.float32)
+    vs = rng.random((N, H)).astype(np.float32)
+    pairs = np.array([[1, 6], [3, 0]], dtype=np.int64)
+    g = [torch.from_numpy(x.copy()).to(dev) for x in (kc, vc, ks, vs)]
+    pa.pa_block_copy(g[0], g[1], torch.from_numpy(pairs).to(dev), g[2], g[3])
+    oracle.block_copy(kc, vc, pairs, ks, vs)
+    for t, e in zip(g, (kc, vc, ks, vs)):
+        assert np.array_equal(bits(t), np_bits(e))

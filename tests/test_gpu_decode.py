@@ -453,3 +453,52 @@ def test_specdec_trace_back_to_back():
     for i in sorted(sample):
         assert_close(dw.steps[i][-1][-1], ref[i], "float16", f"specdec step {i}")
     assert np.array_equal(bits(dw.kc), kc.view(np.uint8))
+
+
+# -- 4-bit caches ---------------------------------------------------------------------------
+def _int4_ref(w, dw, multi=False):
+    kc4, vc4 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
+    ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
+    op = w.steps[0][0]
+    fn = oracle.decode_multi if multi else oracle.decode
+    return fn(op.q, kc4, vc4, op.block_tables, op.seq_lens, w.scale, ks, vs)
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 8), (64, 8), (32, 1)])
+@pytest.mark.parametrize("part", [0, 16, -1])
+def test_int4_decode(hq, hkv, part):
+    """4-bit caches on the tensor-core family against the oracle decoding the very
+    same packed bytes and scales (device-quantised, bit-exact with the oracle's
+    quantiser per test_gpu_cache_ops)."""
+    w = W.random_case([1, 15, 16, 33, 250, 777], num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
+                      dtype="float16", seed=hq + 2 * hkv)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    dw.quantize_int4()
+    got = dw.run_step(0, part, int8=True, algo=pa.PA_ALGO_TENSOR)
+    torch.cuda.synchronize()
+    assert_close(got, _int4_ref(w, dw), "float16", f"int4 G={hq // hkv} part={part}")
+
+
+def test_int4_multi_query_and_auto():
+    w = W.random_multi_case([3, 64, 500], 2, num_q_heads=16, num_kv_heads=4, head_dim=128,
+                            dtype="float16", seed=44)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    dw.quantize_int4()
+    got = dw.run_step(0, -1, int8=True, algo=pa.PA_ALGO_AUTO)
+    torch.cuda.synchronize()
+    assert_close(got, _int4_ref(w, dw, multi=True), "float16", "int4 multi-query")
+
+
+def test_int4_rejected_off_its_path():
+    """4-bit caches need fp16 q and head_dim 128 on the tensor-core family."""
+    w = W.random_case([40], num_q_heads=8, num_kv_heads=2, head_dim=128, dtype="float16", seed=45)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    dw.quantize_int4()
+    _, q, bt, sl, mx, out = dw.steps[0][-1]
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode(out, q, dw.kc8, dw.vc8, bt, sl, w.scale, mx, dw.k_scales, dw.v_scales,
+                     algo=pa.PA_ALGO_SIMT)
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
