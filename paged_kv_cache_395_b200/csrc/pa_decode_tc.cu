@@ -78,6 +78,9 @@ __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
     asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
     return y;
 }
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint32_t bar) {
     asm volatile(
@@ -121,10 +124,23 @@ template <> struct Mma<__nv_bfloat16> {
 #ifndef PA_TC_WARPS
 #define PA_TC_WARPS 4
 #endif
-// ring stages per warp (two measured faster than three on the ragged trace:
-// more bytes in flight per warp only lengthen the DRAM queues)
-#ifndef PA_TC_STAGES
-#define PA_TC_STAGES 2
+// Cache bytes each warp keeps in flight.  A warp's ring stage holds one block's
+// K and V tiles, so the stage count is this over the stage size: two stages of
+// fp16 at d = 128 (three measured slower on the ragged trace: more bytes in
+// flight per warp only lengthen the DRAM queues), and proportionally more for
+// the smaller int8, 4-bit and d = 64 tiles, which otherwise leave the warps
+// latency-bound at a fraction of the bandwidth.
+#ifndef PA_TC_INFLIGHT
+#define PA_TC_INFLIGHT (16 * 1024)
+#endif
+// shared memory for the rings and q slots of one CTA; two CTAs fit on an SM
+#ifndef PA_TC_RING_BUDGET
+#define PA_TC_RING_BUDGET (96 * 1024)
+#endif
+// int8 and 4-bit caches: consume the blocks of a segment two at a time (their
+// conversion-heavy fragment work interleaves), with the ring twice as deep
+#ifndef PA_TC_PAIRS
+#define PA_TC_PAIRS 1
 #endif
 #ifndef PA_TC_HOIST_V
 #define PA_TC_HOIST_V 1
@@ -145,17 +161,23 @@ struct TcCfg {
     static constexpr bool I4 = std::is_same<TKV, U4x2>::value;
     static constexpr int NW = PA_TC_WARPS;        // warps (independent workers) per CTA
     static constexpr int THREADS = NW * 32;
-    static constexpr int S = PA_TC_STAGES;        // ring stages per warp
     static constexpr int ROW_BYTES = I4 ? D / 2 : 128;              // bytes per box row
     static constexpr int BOXW = I4 ? D / 2 : 128 / (int)sizeof(TKV);  // TMA elements per box row
     static constexpr int BOXES = I4 ? 1 : D / BOXW;                  // boxes per tile row
     static constexpr int BOX_BYTES = 16 * ROW_BYTES;                 // one box of a tile
     static constexpr int TILE = BOXES * BOX_BYTES;
     static constexpr int STAGE = 2 * TILE;        // K tile, then V tile
+    static constexpr int QSLOT = G * D * 2;       // q rows of a segment's G heads
+    static constexpr int stages() {
+        int s = PA_TC_INFLIGHT / STAGE;
+        s = s < 2 ? 2 : (s > 8 ? 8 : s);
+        while (s > 2 && NW * s * (STAGE + QSLOT) > PA_TC_RING_BUDGET) --s;
+        return s;
+    }
+    static constexpr int S = stages();            // ring stages per warp
     static constexpr int KSTEPS = D / 16;         // QK k-steps
     static constexpr int MTILES = D / 16;         // PV m-tiles
     static constexpr int DPL = D / 32;            // dims per lane in the merge
-    static constexpr int QSLOT = G * D * 2;       // q rows of a segment's G heads
     static constexpr int RING = NW * S * STAGE;
     static constexpr int QRING_OFF = RING;        // [NW][S] q slots, one per stage
     static constexpr int BAR_OFF = QRING_OFF + NW * S * QSLOT;
@@ -187,6 +209,7 @@ struct SegIter {
 struct Win {
     Seg sg;
     int o, n;
+    int kc;  // the cache's KV head of the window's row
     bool valid;
 };
 
@@ -391,6 +414,10 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = a.B, Hkv = a.Hkv;
     const int Hc = Hkv / a.ngroups;  // the cache's KV heads
+    if (tid == 0) {  // bring the two tensor maps into the SM's descriptor cache before the first copy
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
     // Without PA_DECODE_INPUTS_READY nothing is read before the previous kernel
     // on the stream has finished; with it, the lengths, the block tables and q
     // are read first (the caller guarantees that kernel does not write them) and
@@ -542,6 +569,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             w.sg = sg;
             w.o = 0;
             w.n = min(32, sg.j1 - sg.j0);
+            w.kc = sg.kvh / a.ngroups;
         }
     };
     auto win_after = [&](const Win &cur, Win &w) {
@@ -558,19 +586,21 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             win_first(w);
         }
     };
-    // lane l: TMA row of the window's entry l (-1: none, -2: block id outside
-    // the pool); for int8 caches also that block's K and V scales
+    // lane l: the physical block of the window's entry l, loaded a window ahead
+    // of its use and checked against the pool only when its copy is issued, so
+    // that the table load never holds the warp (-1: no entry).  Quantised caches
+    // also load the block's K and V scales, which need the block id at once: an
+    // id outside the pool is marked -2 there.
     float p_ks = 0.f, p_vs = 0.f, p_ks_next = 0.f, p_vs_next = 0.f;
     auto win_load = [&](const Win &w, float &ks, float &vs) -> int {
         if (!w.valid || lane >= w.n) return -1;
         const int pb = a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
-        if (pb < 0 || (int64_t)pb >= a.N) return -2;
-        const int kc = w.sg.kvh / a.ngroups;  // the cache's KV head
         if constexpr (kQz) {
-            ks = a.ks[(size_t)pb * Hc + kc];
-            vs = a.vs[(size_t)pb * Hc + kc];
+            if (pb < 0 || (int64_t)pb >= a.N) return -2;
+            ks = a.ks[(size_t)pb * Hc + w.kc];
+            vs = a.vs[(size_t)pb * Hc + w.kc];
         }
-        return (pb * Hc + kc) * kBlockSize;
+        return pb;
     };
     Win pc, pn;
     win_first(pc);
@@ -580,7 +610,9 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     float *my_sc = stage_sc + warp * S * 2;
     auto refill = [&]() {
         if (!pc.valid) return;
-        const int y = __shfl_sync(0xffffffffu, p_y, p_i);
+        const int pb = __shfl_sync(0xffffffffu, p_y, p_i);
+        // TMA row of the block's tile for the cache's KV head, -1 for an id outside the pool
+        const int y = (pb < 0 || (int64_t)pb >= a.N) ? -1 : (pb * Hc + pc.kc) * kBlockSize;
         float ksv = 0.f, vsv = 0.f;
         if constexpr (kQz) {
             ksv = __shfl_sync(0xffffffffu, p_ks, p_i);
@@ -600,10 +632,15 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 my_sc[2 * s + 1] = vsv;
             }
             if (y < 0) raise_flag(PA_EFLAG_BAD_BLOCK);
+            // Relaxed arrival: a releasing one would first wait for this lane's
+            // outstanding loads (the next window's table entries).  The stage's tiles
+            // and q rows are published by the transaction count; the flag and scales
+            // stored above reach the other lanes through the __syncwarp that every
+            // consumer iteration runs before this stage is read again.
             if (tx == 0) {
-                mbar_arrive(bar);
+                mbar_arrive_relaxed(bar);
             } else {
-                mbar_arrive_expect_tx(bar, tx);
+                mbar_arrive_expect_tx_relaxed(bar, tx);
             }
             if (y >= 0) {
                 const uint32_t dst = ring + s * C::STAGE;
@@ -846,6 +883,152 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
         for (int j = 0; j < len; ++j) {
+            if constexpr (kQz && PA_TC_PAIRS) {
+                if (j + 1 < len) {
+                    // ---- two blocks (stages sA, sB) at once: one max/sum reduction and
+                    // one rescale for both, two independent MMA streams
+                    const int sA = c_k % S, sB = (c_k + 1) % S;
+                    const bool okw = __all_sync(0xffffffffu, mbar_wait(&my_bars[sA], (c_k / S) & 1) &&
+                                                                 mbar_wait(&my_bars[sB], ((c_k + 1) / S) & 1));
+                    if (!okw) {
+                        alive = false;
+                        break;
+                    }
+                    if (j == 0) load_q(sA, bq, ncol);
+                    // block j is not the row's last block (block j + 1 follows it)
+                    const int ntokB = (cs.j0 + j + 1 == cs.nb - 1) ? ntok_last : kBlockSize;
+                    const bool okA = my_ok[sA] != 0, okB = my_ok[sB] != 0;
+                    if (okA || okB) {
+                        const uint32_t tA = ring + sA * C::STAGE, tB = ring + sB * C::STAGE;
+                        const float slA = a.scale_log2 * my_sc[2 * sA], slB = a.scale_log2 * my_sc[2 * sB];
+                        const float vsA = my_sc[2 * sA + 1], vsB = my_sc[2 * sB + 1];
+                        uint32_t kwA[kI8 ? 2 : 1][8], kwB[kI8 ? 2 : 1][8], vwA[kI8 ? 4 : 1][4], vwB[kI8 ? 4 : 1][4];
+                        uint32_t k4A[kI4 ? 2 : 1][4], k4B[kI4 ? 2 : 1][4], v4A[kI4 ? 4 : 1][2], v4B[kI4 ? 4 : 1][2];
+                        if constexpr (kI4) {
+                            kload_i4(k4A, tA, g, c);
+                            kload_i4(k4B, tB, g, c);
+                            vload_i4(v4A, tA + C::TILE, g, c);
+                            vload_i4(v4B, tB + C::TILE, g, c);
+                        } else {
+                            kload_i8(kwA, tA, g, c);
+                            kload_i8(kwB, tB, g, c);
+                            vload_i8(vwA, tA + C::TILE, g, c);
+                            vload_i8(vwB, tB + C::TILE, g, c);
+                        }
+                        // ---- S^T of both blocks, NCH accumulator chains each (two where the
+                        // general column mapping leaves too few registers for four)
+                        constexpr int NCH = (MQ && kI8) ? 2 : 4;
+                        float sa[2][NCH][4];
+#pragma unroll
+                        for (int u = 0; u < NCH; ++u)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) sa[0][u][e] = sa[1][u][e] = 0.f;
+#pragma unroll
+                        for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                            uint32_t fa[4], fb[4];
+                            if constexpr (kI4) {
+                                kfrag_i4(k4A, ks, fa);
+                                kfrag_i4(k4B, ks, fb);
+                            } else {
+                                kfrag_i8(kwA, ks, fa);
+                                kfrag_i8(kwB, ks, fb);
+                            }
+                            Mma<T>::mma(sa[0][ks % NCH], fa, bq[ks][0], bq[ks][1]);
+                            Mma<T>::mma(sa[1][ks % NCH], fb, bq[ks][0], bq[ks][1]);
+                        }
+                        // ---- scores: block A is full, block B may end the row; a skipped
+                        // block (id outside the pool) sees no token
+                        float sp[2][4];
+#pragma unroll
+                        for (int bb = 0; bb < 2; ++bb) {
+                            float sc[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                sc[e] = sa[bb][0][e] + sa[bb][1][e];
+                                if constexpr (NCH == 4) sc[e] += sa[bb][2][e] + sa[bb][3][e];
+                            }
+                            const bool okb = bb ? okB : okA;
+                            const float sl = bb ? slB : slA;
+                            if constexpr (MQ) {
+                                const int pos = (cs.j0 + j + bb) * kBlockSize + g;
+                                sp[bb][0] = okb && pos < lim0 ? sc[0] * sl : -INFINITY;
+                                sp[bb][1] = okb && pos < lim1 ? sc[1] * sl : -INFINITY;
+                                sp[bb][2] = okb && pos + 8 < lim0 ? sc[2] * sl : -INFINITY;
+                                sp[bb][3] = okb && pos + 8 < lim1 ? sc[3] * sl : -INFINITY;
+                            } else {
+                                const int nt = okb ? (bb ? ntokB : kBlockSize) : 0;
+                                const bool v0 = g < nt, v1 = g + 8 < nt;
+                                sp[bb][0] = v0 ? sc[0] * sl : -INFINITY;
+                                sp[bb][1] = v0 ? sc[1] * sl : -INFINITY;
+                                sp[bb][2] = v1 ? sc[2] * sl : -INFINITY;
+                                sp[bb][3] = v1 ? sc[3] * sl : -INFINITY;
+                            }
+                        }
+                        float mx0 = fmaxf(fmaxf(sp[0][0], sp[0][2]), fmaxf(sp[1][0], sp[1][2]));
+                        float mx1 = fmaxf(fmaxf(sp[0][1], sp[0][3]), fmaxf(sp[1][1], sp[1][3]));
+#pragma unroll
+                        for (int msk = 4; msk < 32; msk <<= 1) {
+                            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
+                            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
+                        }
+                        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                        // as for one block: without MQ one of the two blocks holds a token of
+                        // every column, so m is finite
+                        const float mc0 = (MQ && mn0 == -INFINITY) ? 0.f : mn0;
+                        const float mc1 = (MQ && mn1 == -INFINITY) ? 0.f : mn1;
+                        const float al0 = (MQ && m0 == -INFINITY) ? 1.f : fast_exp2(m0 - mc0);
+                        const float al1 = (MQ && m1 == -INFINITY) ? 1.f : fast_exp2(m1 - mc1);
+                        float pp[2][4];
+#pragma unroll
+                        for (int bb = 0; bb < 2; ++bb) {
+                            pp[bb][0] = fast_exp2(sp[bb][0] - mc0);
+                            pp[bb][1] = fast_exp2(sp[bb][1] - mc1);
+                            pp[bb][2] = fast_exp2(sp[bb][2] - mc0);
+                            pp[bb][3] = fast_exp2(sp[bb][3] - mc1);
+                        }
+                        l0 = l0 * al0 + ((pp[0][0] + pp[0][2]) + (pp[1][0] + pp[1][2]));
+                        l1 = l1 * al1 + ((pp[0][1] + pp[0][3]) + (pp[1][1] + pp[1][3]));
+                        m0 = mn0;
+                        m1 = mn1;
+                        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+                            for (int i = 0; i < C::MTILES; ++i) {
+                                o[i][0] *= al0;
+                                o[i][1] *= al1;
+                                o[i][2] *= al0;
+                                o[i][3] *= al1;
+                            }
+                        }
+                        // ---- P^T fragments of both blocks, each carrying its block's V scale
+                        const uint32_t pa0 = movm_t(Mma<T>::pack(pp[0][0] * vsA, pp[0][1] * vsA));
+                        const uint32_t pa1 = movm_t(Mma<T>::pack(pp[0][2] * vsA, pp[0][3] * vsA));
+                        const uint32_t pb0 = movm_t(Mma<T>::pack(pp[1][0] * vsB, pp[1][1] * vsB));
+                        const uint32_t pb1 = movm_t(Mma<T>::pack(pp[1][2] * vsB, pp[1][3] * vsB));
+                        // ---- O^T += V_A^T . P_A^T + V_B^T . P_B^T (no V mask: quantised slots
+                        // past the end are finite and weighted 0)
+#pragma unroll
+                        for (int i = 0; i < C::MTILES; ++i) {
+                            uint32_t fa[4], fb[4];
+                            if constexpr (kI4) {
+                                vfrag_i4(v4A, i, fa);
+                                vfrag_i4(v4B, i, fb);
+                            } else {
+                                vfrag_i8(vwA, i, fa);
+                                vfrag_i8(vwB, i, fb);
+                            }
+                            Mma<T>::mma(o[i], fa, pa0, pa1);
+                            Mma<T>::mma(o[i], fb, pb0, pb1);
+                        }
+                    }
+                    __syncwarp();
+                    refill();
+                    refill();
+                    c_k += 2;
+                    if (due && !pend && c_k >= due_ck + kTicketLag) take_ticket();
+                    ++j;  // with the loop's own increment: two blocks
+                    continue;
+                }
+            }
             const int s = c_k % S;
             const uint32_t parity = (c_k / S) & 1;
             int ok = lane == 0 ? (int)mbar_wait(&my_bars[s], parity) : 0;
@@ -859,9 +1042,9 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
             const uint32_t tK = ring + s * C::STAGE;
             if (my_ok[s]) {
-                // Slots past the sequence end hold stale data (possibly NaN/Inf); their
-                // probabilities are 0, and their V values are masked to 0 in the
-                // fragments so that they add exactly 0.  V^T fragment registers 0, 1
+                // Slots past the sequence end hold stale data (in fp16/bf16 caches possibly
+                // NaN/Inf); their probabilities are 0, and fp16/bf16 V values are masked
+                // to 0 in the fragments so that they add exactly 0.  V^T fragment registers 0, 1
                 // hold tokens 2c, 2c+1 and registers 2, 3 tokens 2c+8, 2c+9 (low half
                 // = even token).
                 const uint32_t vm_lo = (2 * c < ntok ? 0x0000ffffu : 0u) | (2 * c + 1 < ntok ? 0xffff0000u : 0u);
@@ -989,10 +1172,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                             vfrag_i4(vw4, i, vf[0]);
                         else
                             vfrag_i8(vw, i, vf[0]);
-                        vf[0][0] &= vm_lo;
-                        vf[0][1] &= vm_lo;
-                        vf[0][2] &= vm_hi;
-                        vf[0][3] &= vm_hi;
+                        // no mask: an int8 or 4-bit slot past the sequence end holds a finite
+                        // value, and its probability is exactly 0
                     } else if constexpr (!PA_TC_HOIST_V) {
                         ldsm_x4_t(vf[vi], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
                         vf[vi][0] &= vm_lo;

@@ -221,6 +221,48 @@ def test_bad_block_id_flagged():
     assert pa.pa_get_error_flags(reset=True) == pa.PA_EFLAG_BAD_BLOCK
 
 
+@pytest.mark.parametrize("kind", ["float16", "int8", "int4"])
+@pytest.mark.parametrize("part", [0, -1])
+def test_skipped_block_leaves_the_rest_exact(kind, part):
+    """A block id outside the pool inside a sequence: the kernel skips that block's
+    16 tokens and attends over the others.  Attention has no token order, so the
+    expected output is the oracle's on the table row without that block and the
+    length 16 shorter; the other sequences are untouched.  Covers the blocks the
+    quantised kernels consume two at a time (a skipped block beside a good one)."""
+    w = W.random_case([100, 200, 37], num_q_heads=16, num_kv_heads=4, head_dim=128, dtype="float16",
+                      seed=71)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    quant = kind != "float16"
+    if kind == "int8":
+        dw.quantize_int8()
+    elif kind == "int4":
+        dw.quantize_int4()
+    _, q, bt, sl, mx, out = dw.steps[0][-1]
+    op = w.steps[0][0]
+    for skip in (2, 5):  # the first or the second block of a pair
+        bt_bad = bt.clone()
+        bt_bad[1, skip] = w.num_blocks + 5
+        kc, vc = (dw.kc8, dw.vc8) if quant else (dw.kc, dw.vc)
+        ks, vs = (dw.k_scales, dw.v_scales) if quant else (None, None)
+        ws = torch.zeros(pa.pa_decode_workspace_size(q, kc, bt_bad, mx, part, ks, vs, pa.PA_ALGO_TENSOR),
+                         dtype=torch.uint8, device=q.device)  # zero-filled before first use
+        pa.pa_decode(out, q, kc, vc, bt_bad, sl, w.scale, mx, ks, vs, part, ws, pa.PA_ALGO_TENSOR)
+        torch.cuda.synchronize()
+        assert pa.pa_get_error_flags(reset=True) == pa.PA_EFLAG_BAD_BLOCK
+        tables = op.block_tables.copy()
+        row = [b for j, b in enumerate(tables[1]) if j != skip] + [tables[1][-1]]
+        tables[1] = np.array(row, dtype=tables.dtype)
+        lens = op.seq_lens.copy()
+        lens[1] -= 16
+        if quant:
+            ref = oracle.decode(op.q, dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy(), tables, lens, w.scale,
+                                dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy())
+        else:
+            ref = oracle.decode(op.q, dw.kc.cpu().numpy(), dw.vc.cpu().numpy(), tables, lens, w.scale)
+        assert_close(out, ref, "float16", f"{kind} part={part} skip={skip}")
+
+
 # -- the study's workloads at full size ---------------------------------------------------
 def test_gqa_b8_full():
     w = W.gqa_b8()
