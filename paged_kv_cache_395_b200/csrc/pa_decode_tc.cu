@@ -777,6 +777,18 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         constexpr int SPP = 32 / G;                 // segments per round of pass 1
         constexpr int NB = 16 / G > 0 ? 16 / G : 1;  // segments per round of pass 2
         const int li = lane / G, lh = lane % G;
+        using V = FVec<C::DPL>;
+        // the first round's partial outputs do not depend on the weights: their loads
+        // go out with the lse loads, so the merge waits for one round trip, not two
+        typename V::type v[NB][G];
+#pragma unroll
+        for (int jj = 0; jj < NB; ++jj) {
+            if (jj < nseg) {
+                const int sl = slot_of(jj);
+#pragma unroll
+                for (int h = 0; h < G; ++h) v[jj][h] = V::ld(a.ws_o + ((size_t)sl * G + h) * D + lane * C::DPL);
+            }
+        }
         float x0 = -INFINITY;  // lse of (segment li, head lh), first round
         if (li < nseg) x0 = __ldcg(a.ws_lse + (size_t)slot_of(li) * G + lh);
         float mx = x0, sm = x0 == -INFINITY ? 0.f : 1.f;
@@ -797,7 +809,6 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             mx = mn;
         }
         const float inv_sum = 1.f / sm;  // lane (., h) now holds head h's max and sum
-        using V = FVec<C::DPL>;
         float acc[G][C::DPL];
 #pragma unroll
         for (int h = 0; h < G; ++h)
@@ -808,13 +819,15 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             if (i0 > 0) x = i0 + li < nseg ? __ldcg(a.ws_lse + (size_t)slot_of(i0 + li) * G + lh) : -INFINITY;
             const float wl = x == -INFINITY ? 0.f : fast_exp2(x - mx) * inv_sum;  // weight of (i0 + li, lh)
             for (int j0 = 0; j0 < SPP && i0 + j0 < nseg; j0 += NB) {
-                typename V::type v[NB][G];
+                if (i0 + j0 > 0) {  // the first round's outputs are already loaded
 #pragma unroll
-                for (int jj = 0; jj < NB; ++jj) {
-                    if (i0 + j0 + jj < nseg) {
-                        const int sl = slot_of(i0 + j0 + jj);
+                    for (int jj = 0; jj < NB; ++jj) {
+                        if (i0 + j0 + jj < nseg) {
+                            const int sl = slot_of(i0 + j0 + jj);
 #pragma unroll
-                        for (int h = 0; h < G; ++h) v[jj][h] = V::ld(a.ws_o + ((size_t)sl * G + h) * D + lane * C::DPL);
+                            for (int h = 0; h < G; ++h)
+                                v[jj][h] = V::ld(a.ws_o + ((size_t)sl * G + h) * D + lane * C::DPL);
+                        }
                     }
                 }
 #pragma unroll
