@@ -25,23 +25,30 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     pdl_wait();  // the previous kernel may still read the slots this one overwrites
     pdl_release_dependents();
     const int64_t i = blockIdx.x;
+    const bool is_v = blockIdx.y != 0;
+    const char *src = (is_v ? v : k) + i * (is_v ? v_stride_bytes : k_stride_bytes);
+    const int vecs_per_row = row_bytes / VEC;
+    const int total = num_kv_heads * vecs_per_row;
+    auto src_vec = [&](int idx) {
+        const int h = idx / vecs_per_row, c = idx % vecs_per_row;
+        return reinterpret_cast<const V *>(src + (int64_t)h * row_bytes)[c];
+    };
+    // The token's row does not depend on its slot: its first vector is requested
+    // together with the slot, so the two loads overlap.
+    V first{};
+    if ((int)threadIdx.x < total) first = src_vec(threadIdx.x);
     const int64_t s = slots[i];
     if (s < 0) return;
     if (s >= num_slots) {
         if (threadIdx.x == 0 && blockIdx.y == 0) raise_flag(PA_EFLAG_BAD_SLOT);
         return;
     }
-    const bool is_v = blockIdx.y != 0;
-    const char *src = (is_v ? v : k) + i * (is_v ? v_stride_bytes : k_stride_bytes);
     char *dst = is_v ? vc : kc;
     const int64_t blk = s / kBlockSize, off = s % kBlockSize;
-    const int vecs_per_row = row_bytes / VEC;
-    const int total = num_kv_heads * vecs_per_row;
     for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
         const int h = idx / vecs_per_row, c = idx % vecs_per_row;
         const int64_t drow = ((blk * num_kv_heads + h) * kBlockSize + off) * (int64_t)row_bytes;
-        reinterpret_cast<V *>(dst + drow)[c] =
-            reinterpret_cast<const V *>(src + (int64_t)h * row_bytes)[c];
+        reinterpret_cast<V *>(dst + drow)[c] = idx == (int)threadIdx.x ? first : src_vec(idx);
     }
 }
 
