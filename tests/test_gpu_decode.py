@@ -340,6 +340,32 @@ def test_ragged_trace_back_to_back_inputs_ready():
     assert np.array_equal(bits(dw.vc), vc.view(np.uint8))
 
 
+@pytest.mark.parametrize("hq,hkv", [(32, 1), (64, 2), (16, 1)])
+@pytest.mark.parametrize("kind", ["float16", "int8"])
+def test_virtual_heads_uniform_and_near_uniform_lengths(hq, hkv, kind):
+    """Groups above 8 heads (virtual KV heads sharing one cache head's tiles)
+    with every sequence the same length, and with one sequence a token shorter,
+    on the tensor-core family's balanced schedule, fp16 and int8 caches, against
+    the oracle."""
+    for lens in ([1024] * 4, [1024] * 3 + [1023]):
+        w = W.random_case(lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=128, dtype="float16",
+                          seed=hq + hkv)
+        dw = runner.DeviceWorkload(w)
+        dw.run_setup()
+        if kind == "int8":
+            dw.quantize_int8()
+        got = dw.run_step(0, -1, int8=kind == "int8", algo=pa.PA_ALGO_TENSOR)
+        torch.cuda.synchronize()
+        op = w.steps[0][0]
+        if kind == "int8":
+            ref = oracle.decode(op.q, dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy(), op.block_tables, op.seq_lens,
+                                w.scale, dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy())
+        else:
+            ref = oracle.decode(op.q, dw.kc.cpu().numpy(), dw.vc.cpu().numpy(), op.block_tables, op.seq_lens,
+                                w.scale)
+        assert_close(got, ref, "float16", f"{kind} G={hq // hkv} lens={lens[-1]}")
+
+
 @pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_TENSOR])
 def test_inputs_ready_flag_same_result(algo):
     """The early-start flag changes when the kernel waits, not what it computes."""
