@@ -1,4 +1,5 @@
-// Paged decode attention, tensor-core kernel family (fp16 / bf16 KV, G <= 8).
+// Paged decode attention, tensor-core kernel family (fp16 / bf16, int8 and 4-bit
+// KV; up to 8 (query token, head) columns per row, larger groups as several rows).
 //
 // Same computation as the CUDA-core kernel (lqnn.cn/news/235768 sections 1.2,
 // 2.2, 3.2, 4.2; chanyi.net.cn/article/49 section 四):
@@ -18,7 +19,8 @@
 // 16 bytes hit 8 different bank groups.
 //
 // Scheduling: a persistent grid; every warp is an independent worker with its
-// own 2-stage ring of (K tile, V tile) stages and its own mbarriers.  The
+// own ring of (K tile, V tile) stages (a fixed byte depth: two stages of fp16 at
+// d = 128, more for smaller tiles) and its own mbarriers.  The
 // (sequence, KV head) rows are laid end to end as one stream of blocks (row
 // order: sequence, then KV head; total = sum_b ceil(L_b / 16) * H_kv blocks).
 // With partition_size == 0 warp w takes whole rows w, w + W, ... (W = warps in
