@@ -19,7 +19,9 @@ What it computes, and the passages it follows (page, section):
   algebra of the softmax, checked against the unsplit form);
 * cache append (byte scatter), copy-on-write block copy (byte copy) and the
   symmetric absmax int8 quantiser with one scale per (block, KV head)
-  (lqnn.cn/news/235768 section 4.1).
+  (lqnn.cn/news/235768 section 4.1), its 4-bit form, and the append of single
+  tokens into an int8 cache that raises a tile's scale when needed (this
+  library's reading of the same section).
 
 The arithmetic lives in ``pa_oracle.c`` (plain C, fp64 loops).  This module
 only marshals numpy arrays.  ``dense.py`` is an independent NumPy brute force
@@ -50,6 +52,7 @@ def load(path):
     L.oracle_block_copy.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32]
     L.oracle_quantize_int8.argtypes = [P, i32, P, P, i64, i32, i32, i32]
     L.oracle_quantize_int4.argtypes = [P, i32, P, P, i64, i32, i32, i32]
+    L.oracle_append_int8.argtypes = [P, P, i32, P, P, P, P, P, i64, i32, i32, i32, i64]
     L.oracle_decode.argtypes = [P, P, P, P, i32, P, P, P, P, i32, i32, i32, i32, i32, i32,
                                 i64, dbl, P, i64, i32]
     L.oracle_decode_partials.argtypes = [P, P, P, P, P, i32, P, P, P, P, i32, i32, i32, i32,
@@ -137,6 +140,24 @@ def quantize_int8(src_cache, code=None):
     _check(lib().oracle_quantize_int8(_ptr(src), code, _ptr(dst), _ptr(scales), N, H, d, bs),
            "oracle_quantize_int8")
     return dst, scales
+
+
+def append_int8(k, v, key_cache8, value_cache8, k_scales, v_scales, slot_mapping, code=None):
+    """Append tokens k, v ([T][H_kv][d], fp32/fp16/bf16) into int8 caches
+    [N][H_kv][bs][d] with fp32 scales [N][H_kv], in place, raising a tile's scale
+    and re-rounding its other codes when the token needs it (see pa_oracle.c)."""
+    T, H, d = k.shape
+    N, Hc, bs, dc = key_cache8.shape
+    assert (H, d) == (Hc, dc) and v.shape == k.shape
+    for a in (key_cache8, value_cache8, k_scales, v_scales):
+        assert a.flags["C_CONTIGUOUS"]
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    code = dtype_code(k.dtype) if code is None else code
+    _check(lib().oracle_append_int8(_ptr(k), _ptr(v), code, _ptr(key_cache8), _ptr(value_cache8),
+                                    _ptr(k_scales), _ptr(v_scales), _ptr(sm), T, H, d, bs, N),
+           "oracle_append_int8")
 
 
 def quantize_int4(src_cache, code=None):

@@ -207,6 +207,79 @@ int oracle_quantize_int8(const void *src, int src_dtype, int8_t *dst, float *sca
 }
 
 /*
+ * Appending single tokens into an int8 cache (the rescaling the 8-bit grouped-scale
+ * KV of lqnn.cn/news/235768 section 4.1 needs once blocks are quantised: the pages
+ * do not spell it out; this is the library's reading).  For each token i with
+ * slot s = slot_mapping[i] >= 0 (s >= num_blocks * block_size is skipped), block
+ * b = s / block_size, slot o = s % block_size, and every KV head h, separately for
+ * K (k, key_cache, k_scales) and V:
+ *   a = max_j |x_j| over the token's head_dim values,  c = a / 127,
+ *   s_old = scales[b][h];  s_new = c > s_old ? c : s_old;
+ *   if s_new > s_old: every code of the tile in the other slots is re-rounded,
+ *       q <- clamp(rint((q * s_old) / s_new), -127, 127);
+ *   the token's codes are clamp(rint(x_j / s_new), -127, 127) (0 when s_new = 0);
+ *   scales[b][h] = s_new.
+ * All arithmetic in IEEE fp32 (products and quotients rounded to nearest, rint
+ * half to even).  So the scale never shrinks, every stored value moves by at
+ * most s_new / 2 when re-rounded, and an append that does not raise the scale
+ * leaves the other codes untouched.  Tokens are applied in order; the library
+ * requires the tokens of one call to fall in distinct blocks.
+ */
+int oracle_append_int8(const void *k, const void *v, int src_dtype, int8_t *key_cache, int8_t *value_cache,
+                       float *k_scales, float *v_scales, const int64_t *slot_mapping, int64_t num_tokens,
+                       int num_kv_heads, int head_dim, int block_size, int64_t num_blocks)
+{
+    if (src_dtype != OR_F32 && src_dtype != OR_F16 && src_dtype != OR_BF16) return -4;
+    const size_t tile = (size_t)block_size * head_dim;
+    for (int64_t i = 0; i < num_tokens; ++i) {
+        const int64_t s = slot_mapping[i];
+        if (s < 0 || s >= num_blocks * block_size) continue;
+        const int64_t b = s / block_size;
+        const int o = (int)(s % block_size);
+        for (int kv = 0; kv < 2; ++kv) {
+            const void *src = kv ? v : k;
+            int8_t *cache = kv ? value_cache : key_cache;
+            float *scales = kv ? v_scales : k_scales;
+            for (int h = 0; h < num_kv_heads; ++h) {
+                const size_t x0 = ((size_t)i * num_kv_heads + h) * head_dim;
+                float a = 0.0f;
+                for (int j = 0; j < head_dim; ++j) {
+                    float ax = fabsf((float)load_elem(src, x0 + j, src_dtype));
+                    if (ax > a) a = ax;
+                }
+                const float c = a / 127.0f;
+                const float s_old = scales[b * num_kv_heads + h];
+                const float s_new = c > s_old ? c : s_old;
+                int8_t *t = cache + ((size_t)b * num_kv_heads + h) * tile;
+                if (s_new > s_old) {
+                    for (int r = 0; r < block_size; ++r) {
+                        if (r == o) continue;
+                        for (int j = 0; j < head_dim; ++j) {
+                            const float prod = (float)t[(size_t)r * head_dim + j] * s_old;
+                            float q = rintf(MUT(14) ? (prod / s_old) : (prod / s_new));
+                            if (q > 127.0f) q = 127.0f;
+                            if (q < -127.0f) q = -127.0f;
+                            t[(size_t)r * head_dim + j] = (int8_t)q;
+                        }
+                    }
+                }
+                for (int j = 0; j < head_dim; ++j) {
+                    float q = 0.0f;
+                    if (s_new != 0.0f) {
+                        q = rintf((float)load_elem(src, x0 + j, src_dtype) / s_new);
+                        if (q > 127.0f) q = 127.0f;
+                        if (q < -127.0f) q = -127.0f;
+                    }
+                    t[(size_t)o * head_dim + j] = (int8_t)q;
+                }
+                scales[b * num_kv_heads + h] = s_new;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
  * 4-bit KV with one scale per group (the pages' second grouped-scale width), the
  * group again one (block, KV head) tile.  Symmetric absmax in IEEE fp32:
  *   a = max |x|,  s = a / 7,  q = clamp(rint(x / s), -7, 7)

@@ -310,6 +310,82 @@ def pin_quantize():
         q.reshape(-1)[: len(vals)].tolist()
 
 
+# -- appending into an int8 cache -----------------------------------------------------
+def pin_append_int8():
+    """Appending single tokens into int8 tiles: (1) into an empty tile it equals
+    quantising a tile that holds only that token (the pinned quantiser); (2) a
+    token that fits the tile's scale leaves every other code and the scale as they
+    were; (3) a token that raises the scale re-rounds the other codes within half
+    the new scale of their old values, and its own values within half the new
+    scale of the inputs; (4) after any sequence of appends every stored value is
+    within the sum of the half-scales it went through of the original input."""
+    rng = np.random.default_rng(61)
+    N, H, d, bs = 6, 2, 64, 16
+    # (1) empty tiles: scale 0, codes 0
+    kc = np.zeros((N, H, bs, d), dtype=np.int8)
+    vc = np.zeros_like(kc)
+    ks = np.zeros((N, H), dtype=np.float32)
+    vs = np.zeros_like(ks)
+    k = (rng.standard_normal((2, H, d)) * 3).astype(np.float16)
+    v = (rng.standard_normal((2, H, d)) * 3).astype(np.float16)
+    slots = np.array([1 * bs + 5, 4 * bs + 0], dtype=np.int64)
+    oracle.append_int8(k, v, kc, vc, ks, vs, slots)
+    for i, s in enumerate(slots):
+        b, o = divmod(int(s), bs)
+        for src, cache, sc in ((k, kc, ks), (v, vc, vs)):
+            tile = np.zeros((1, H, bs, d), dtype=np.float16)
+            tile[0, :, o] = src[i]
+            q, qs = oracle.quantize_int8(tile)
+            assert np.array_equal(cache[b], q[0]) and np.array_equal(sc[b], qs[0]), "empty tile"
+    # a quantised pool to append into
+    src = (rng.standard_normal((N, H, bs, d)) * 2).astype(np.float16)
+    kc, ks = oracle.quantize_int8(src)
+    vc, vs = oracle.quantize_int8(src[::-1].copy())
+    # (2) a small token: nothing else changes
+    kc0, ks0 = kc.copy(), ks.copy()
+    small = (rng.standard_normal((1, H, d)) * 0.1).astype(np.float16)
+    oracle.append_int8(small, small, kc, vc, ks, vs, np.array([2 * bs + 7], dtype=np.int64))
+    assert np.array_equal(ks, ks0), "scale changed without need"
+    keep = np.ones((N, H, bs), dtype=bool)
+    keep[2, :, 7] = False
+    assert np.array_equal(kc[keep], kc0[keep]), "codes changed without need"
+    x = small.astype(np.float64)[0]
+    got = kc[2, :, 7].astype(np.float64) * ks[2].astype(np.float64)[:, None]
+    assert np.all(np.abs(got - x) <= ks[2].astype(np.float64)[:, None] * (0.5 + 1e-6)), "small token"
+    # (3) a large token raises the scale and re-rounds the rest
+    kc0, ks0 = kc.copy(), ks.copy()
+    big = (rng.standard_normal((1, H, d)) * 20).astype(np.float16)
+    oracle.append_int8(big, big, kc, vc, ks, vs, np.array([3 * bs + 2], dtype=np.int64))
+    s_new = ks[3].astype(np.float64)
+    amax = np.abs(big.astype(np.float64)[0]).max(-1)
+    assert np.all(ks[3] == (amax.astype(np.float32) / np.float32(127))), "raised scale = absmax / 127"
+    assert np.all(ks[3] > ks0[3])
+    old = kc0[3].astype(np.float64) * ks0[3].astype(np.float64)[:, None, None]
+    new = kc[3].astype(np.float64) * s_new[:, None, None]
+    others = np.ones((H, bs), dtype=bool)
+    others[:, 2] = False
+    bound = s_new[:, None, None] * (0.5 + 1e-6)
+    assert np.all((np.abs(new - old) <= bound)[others]), "re-rounding moved a value by more than s/2"
+    tok = kc[3, :, 2].astype(np.float64) * s_new[:, None]
+    assert np.all(np.abs(tok - big.astype(np.float64)[0]) <= s_new[:, None] * (0.5 + 1e-6)), "large token"
+    unchanged = np.ones(N, dtype=bool)
+    unchanged[[2, 3]] = False
+    assert np.array_equal(kc[unchanged], kc0[unchanged]) and np.array_equal(ks[unchanged], ks0[unchanged])
+    # (4) a sequence of appends into one tile: error stays within the accumulated half-scales
+    kc = np.zeros((1, 1, bs, d), dtype=np.int8)
+    ks = np.zeros((1, 1), dtype=np.float32)
+    vc, vs = kc.copy(), ks.copy()
+    x = np.zeros((bs, d))
+    budget = np.zeros(bs)
+    for o in range(bs):
+        t = (rng.standard_normal((1, 1, d)) * (1 + o)).astype(np.float32)
+        oracle.append_int8(t, t, kc, vc, ks, vs, np.array([o], dtype=np.int64))
+        x[o] = t[0, 0]
+        budget[: o + 1] += float(ks[0, 0]) * 0.5 * (1 + 1e-6)
+        err = np.abs(kc[0, 0, : o + 1].astype(np.float64) * float(ks[0, 0]) - x[: o + 1]).max(-1)
+        assert np.all(err <= budget[: o + 1]), "accumulated re-rounding error"
+
+
 # -- 4-bit KV -------------------------------------------------------------------------
 def unpack_int4(packed):
     """Independent statement of the 4-bit layout: element 2k is the low four bits
@@ -431,4 +507,4 @@ ALL_PINS = [pin_half_exhaustive, pin_bf16_exhaustive, pin_tiny_dense, pin_random
             pin_sdpa_library, pin_permutation_invariance, pin_gqa_expand, pin_closed_forms,
             pin_split_merge, pin_kv_size_golden, pin_reshape, pin_block_copy, pin_quantize,
             pin_multi_dense, pin_multi_sdpa_causal_mask, pin_multi_single_token_is_decode,
-            pin_quantize_int4, pin_int4_decode_dense]
+            pin_quantize_int4, pin_int4_decode_dense, pin_append_int8]

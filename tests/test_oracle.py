@@ -30,6 +30,7 @@ MUTATIONS = {
     11: "multi-query causal range one token short",
     12: "int4 nibbles read in swapped order",
     13: "int4 scale absmax / 8",
+    14: "int8 append re-rounds with the old scale",
 }
 
 # pins cheap enough to run once per mutant
