@@ -85,7 +85,7 @@ enum pa_error_flag {
  * sets PA_EFLAG_BAD_SLOT and is skipped.  Strides are in elements.  Slots
  * must be distinct (two tokens writing one slot race).
  * dtype: PA_F32, PA_F16 or PA_BF16 (PA_I8 caches are written by
- * pa_quantize_int8, so PA_I8 returns PA_ERR_UNSUPPORTED).
+ * pa_quantize_int8 and pa_append_int8, so PA_I8 returns PA_ERR_UNSUPPORTED).
  * Any alignment works; 16-byte aligned rows are copied with 16-byte vectors.
  */
 int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *value_cache,
@@ -228,6 +228,31 @@ int pa_block_copy(void *key_cache, void *value_cache, float *k_scales, float *v_
 int pa_quantize_int8(const void *src_cache, int src_dtype, int8_t *dst_cache, float *scales,
                      int64_t num_blocks, int num_kv_heads, int head_dim, int block_size,
                      pa_stream_t stream);
+
+/*
+ * Append single tokens into an int8 cache (the 8-bit grouped-scale KV of
+ * lqnn.cn/news/235768 section 4.1 after its blocks were quantised; the pages do
+ * not spell out the update, this is the library's reading).  For every token i
+ * with s = slot_mapping[i] >= 0, block b = s / 16, slot o = s % 16, every KV
+ * head h, separately for K (k, key_cache, k_scales) and V:
+ *   a = max_j |x_j| over the token's head_dim values, c = a / 127,
+ *   s_old = scales[b][h], s_new = max(c, s_old);
+ *   if s_new > s_old, every other code of the tile becomes
+ *     clamp(rint((q * s_old) / s_new), -127, 127);
+ *   the token's codes are clamp(rint(x_j / s_new), -127, 127) (0 when s_new = 0);
+ *   scales[b][h] = s_new.
+ * IEEE fp32, round half to even: bit-exact with the library's oracle.  The
+ * scale never shrinks; a re-rounded value moves by at most s_new / 2.
+ * k, v: [num_tokens][num_kv_heads][head_dim] with the given token strides (in
+ * elements) of src_dtype PA_F32, PA_F16 or PA_BF16.  Caches int8
+ * [num_blocks][num_kv_heads][16][head_dim], scales fp32 [num_blocks][num_kv_heads].
+ * The tokens of one call must fall in distinct blocks (one writer per tile).
+ * s < 0 is skipped; s >= num_blocks * 16 sets PA_EFLAG_BAD_SLOT and is skipped.
+ */
+int pa_append_int8(const void *k, const void *v, int src_dtype, int8_t *key_cache, int8_t *value_cache,
+                   float *k_scales, float *v_scales, const int64_t *slot_mapping, int64_t num_tokens,
+                   int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                   int64_t k_token_stride, int64_t v_token_stride, pa_stream_t stream);
 
 
 /*

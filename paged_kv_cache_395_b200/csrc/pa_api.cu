@@ -263,6 +263,23 @@ int pa_quantize_int8(const void *src_cache, int src_dtype, int8_t *dst_cache, fl
                                 (cudaStream_t)stream);
 }
 
+int pa_append_int8(const void *k, const void *v, int src_dtype, int8_t *key_cache, int8_t *value_cache,
+                   float *k_scales, float *v_scales, const int64_t *slot_mapping, int64_t num_tokens,
+                   int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                   int64_t k_token_stride, int64_t v_token_stride, pa_stream_t stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0) return PA_ERR_SHAPE;
+    if (block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
+    if (src_dtype != PA_F32 && src_dtype != PA_F16 && src_dtype != PA_BF16) return PA_ERR_DTYPE;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !key_cache || !value_cache || !k_scales || !v_scales || !slot_mapping) return PA_ERR_NULL;
+    if (k_token_stride < (int64_t)num_kv_heads * head_dim || v_token_stride < (int64_t)num_kv_heads * head_dim)
+        return PA_ERR_SHAPE;
+    if (num_tokens > 2147483647LL) return PA_ERR_UNSUPPORTED;
+    return launch_append_int8(k, v, key_cache, value_cache, k_scales, v_scales, slot_mapping, num_tokens,
+                              num_kv_heads, head_dim, num_blocks, src_dtype, k_token_stride, v_token_stride,
+                              (cudaStream_t)stream);
+}
+
 size_t pa_decode_workspace_size(const pa_decode_params *p) {
     Plan pl;
     if (make_plan(p, &pl) != PA_OK) return 0;

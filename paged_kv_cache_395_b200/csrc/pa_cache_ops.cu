@@ -174,6 +174,87 @@ int launch_quantize_int8(const void *src, int src_dtype, int8_t *dst, float *sca
 }
 
 // ---------------------------------------------------------------------------
+// append_int8: single tokens into an int8 cache (the 8-bit grouped-scale KV of
+// lqnn.cn/news/235768 section 4.1 once its blocks are quantised).  For token i
+// at slot s, block s / 16, slot s % 16, each KV head, K and V separately: the
+// token's absmax a gives c = a / 127; when c exceeds the tile's scale the scale
+// becomes c and the tile's other codes are re-rounded, q <- rint(q * s_old /
+// s_new); the token's codes are rint(x / s_new); all in IEEE fp32 with round
+// half to even, clamped to +-127.  Grid (tokens, 2): y selects K or V; warp w
+// of the CTA takes KV heads w, w + 4, ...  The tokens of one call must fall in
+// distinct blocks (each tile has one writer).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) append_int8_kernel(const T *__restrict__ k, const T *__restrict__ v,
+                                                          int8_t *__restrict__ kc, int8_t *__restrict__ vc,
+                                                          float *__restrict__ ks, float *__restrict__ vs,
+                                                          const int64_t *__restrict__ slots, int H, int D,
+                                                          int64_t k_stride, int64_t v_stride, int64_t num_slots) {
+    pdl_wait();  // the previous kernel may still read the tiles this one rewrites
+    pdl_release_dependents();
+    const int64_t i = blockIdx.x;
+    const int64_t s = slots[i];
+    if (s < 0) return;
+    if (s >= num_slots) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) raise_flag(PA_EFLAG_BAD_SLOT);
+        return;
+    }
+    const bool is_v = blockIdx.y != 0;
+    const T *x = (is_v ? v : k) + i * (is_v ? v_stride : k_stride);
+    int8_t *cache = is_v ? vc : kc;
+    float *scales = is_v ? vs : ks;
+    const int64_t blk = s / kBlockSize;
+    const int o = (int)(s % kBlockSize);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int h = warp; h < H; h += 4) {
+        const T *xh = x + (int64_t)h * D;
+        float a = 0.f;
+        for (int j = lane; j < D; j += 32) a = fmaxf(a, fabsf(Cvt<T>::to_f(xh[j])));
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
+        const float c = __fdiv_rn(a, 127.0f);
+        float *sp = scales + blk * H + h;
+        const float s_old = *sp;
+        const float s_new = c > s_old ? c : s_old;
+        int8_t *t = cache + (blk * H + h) * (int64_t)kBlockSize * D;
+        if (s_new > s_old) {
+            for (int e = lane; e < kBlockSize * D; e += 32) {
+                if (e / D == o) continue;
+                const float prod = __fmul_rn((float)t[e], s_old);
+                int q = __float2int_rn(__fdiv_rn(prod, s_new));
+                t[e] = (int8_t)max(-127, min(127, q));
+            }
+        }
+        for (int j = lane; j < D; j += 32) {
+            int q = 0;
+            if (s_new != 0.f) {
+                q = __float2int_rn(__fdiv_rn(Cvt<T>::to_f(xh[j]), s_new));
+                q = max(-127, min(127, q));
+            }
+            t[o * D + j] = (int8_t)q;
+        }
+        __syncwarp();
+        if (lane == 0) *sp = s_new;
+    }
+}
+
+int launch_append_int8(const void *k, const void *v, int8_t *kc, int8_t *vc, float *ks, float *vs,
+                       const int64_t *slots, int64_t T, int H, int D, int64_t N, int src_dtype,
+                       int64_t k_stride, int64_t v_stride, cudaStream_t st) {
+    if (T == 0) return PA_OK;
+    const dim3 grid((unsigned)T, 2);
+    const int64_t ns = N * kBlockSize;
+    cudaError_t e;
+    switch (src_dtype) {
+    case PA_F32: e = launch_pdl(append_int8_kernel<float>, grid, dim3(128), 0, st, (const float *)k, (const float *)v, kc, vc, ks, vs, slots, H, D, k_stride, v_stride, ns); break;
+    case PA_F16: e = launch_pdl(append_int8_kernel<__half>, grid, dim3(128), 0, st, (const __half *)k, (const __half *)v, kc, vc, ks, vs, slots, H, D, k_stride, v_stride, ns); break;
+    case PA_BF16: e = launch_pdl(append_int8_kernel<__nv_bfloat16>, grid, dim3(128), 0, st, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, kc, vc, ks, vs, slots, H, D, k_stride, v_stride, ns); break;
+    default: return PA_ERR_DTYPE;
+    }
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // quantize_int4 (lqnn.cn/news/235768 section 4.1: 4-bit KV with a grouped
 // scale; the group is one (block, KV head) tile).  One CTA of 128 threads per
 // tile; IEEE fp32 divide and round-half-even; each thread writes whole bytes

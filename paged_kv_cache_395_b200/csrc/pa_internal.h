@@ -20,6 +20,9 @@ int launch_reshape_and_cache(const void *k, const void *v, void *kc, void *vc,
                              int64_t k_stride, int64_t v_stride, cudaStream_t st);
 int launch_block_copy(void *kc, void *vc, float *ks, float *vs, const int64_t *pairs, int64_t n,
                       int H, int D, int64_t N, int E, cudaStream_t st);
+int launch_append_int8(const void *k, const void *v, int8_t *kc, int8_t *vc, float *ks, float *vs,
+                       const int64_t *slots, int64_t T, int H, int D, int64_t N, int src_dtype,
+                       int64_t k_stride, int64_t v_stride, cudaStream_t st);
 int launch_quantize_int8(const void *src, int src_dtype, int8_t *dst, float *scales, int64_t N,
                          int H, int D, cudaStream_t st);
 int launch_quantize_int4(const void *src, int src_dtype, uint8_t *dst, float *scales, int64_t N,

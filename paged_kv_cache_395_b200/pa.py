@@ -73,12 +73,13 @@ def _load():
     L.pa_decode_workspace_size.restype = ctypes.c_size_t
     L.pa_block_copy.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, P]
     L.pa_quantize_int8.argtypes = [P, i32, P, P, i64, i32, i32, i32, P]
+    L.pa_append_int8.argtypes = [P, P, i32, P, P, P, P, P, i64, i32, i32, i32, i64, i64, i64, P]
     L.pa_quantize_int4.argtypes = [P, i32, P, P, i64, i32, i32, i32, P]
     L.pa_get_error_flags.argtypes = [ctypes.POINTER(ctypes.c_uint), i32, P]
     L.pa_status_string.argtypes = [i32]
     L.pa_status_string.restype = ctypes.c_char_p
     L.pa_version.argtypes = []
-    for n in ("pa_reshape_and_cache", "pa_decode", "pa_decode_fixed_scratch", "pa_block_copy",
+    for n in ("pa_reshape_and_cache", "pa_append_int8", "pa_decode", "pa_decode_fixed_scratch", "pa_block_copy",
               "pa_quantize_int8", "pa_quantize_int4", "pa_get_error_flags", "pa_version"):
         getattr(L, n).restype = i32
     return L
@@ -87,7 +88,7 @@ def _load():
 lib = _load()
 
 # the C-ABI symbols include/pa.h declares
-EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_fixed_scratch",
+EXPORTED = ("pa_reshape_and_cache", "pa_append_int8", "pa_decode_workspace_size", "pa_decode", "pa_decode_fixed_scratch",
             "pa_block_copy", "pa_quantize_int8", "pa_quantize_int4", "pa_get_error_flags",
             "pa_status_string", "pa_version")
 FIXED_SCRATCH_BYTES = 32 << 20  # PA_FIXED_SCRATCH_BYTES
@@ -267,6 +268,35 @@ def pa_quantize_int8(src_cache, dst_cache, scales, stream=None):
         raise ValueError("dst must be int8 and scales float32")
     _check(lib.pa_quantize_int8(_ptr(src_cache), dtype_code(src_cache.dtype), _ptr(dst_cache),
                                 _ptr(scales), N, H, d, bs, _stream(stream)), "pa_quantize_int8")
+
+
+def pa_append_int8(k, v, key_cache, value_cache, k_scales, v_scales, slot_mapping, stream=None):
+    """Append tokens k, v ([T][H_kv][d] fp32/fp16/bf16, rows contiguous) into int8
+    caches [N][H_kv][16][d] with fp32 scales [N][H_kv], raising a tile's scale and
+    re-rounding its other codes when a token needs it.  The tokens of one call must
+    fall in distinct blocks (see include/pa.h)."""
+    _dev(k, v, key_cache, value_cache, k_scales, v_scales, slot_mapping)
+    T, H, d = k.shape
+    N = key_cache.shape[0]
+    if k.stride(2) != 1 or k.stride(1) != d or v.stride(2) != 1 or v.stride(1) != d or v.shape != k.shape:
+        raise ValueError("k/v heads must be contiguous rows of head_dim elements")
+    if k.dtype != v.dtype:
+        raise ValueError("k and v must share a dtype")
+    if key_cache.dtype != torch.int8 or value_cache.dtype != torch.int8:
+        raise ValueError("caches must be int8")
+    if k_scales.dtype != torch.float32 or v_scales.dtype != torch.float32:
+        raise ValueError("scales must be float32")
+    if tuple(key_cache.shape) != (N, H, 16, d) or value_cache.shape != key_cache.shape or \
+            tuple(k_scales.shape) != (N, H) or v_scales.shape != k_scales.shape:
+        raise ValueError("caches must be [N][H_kv][16][d] and scales [N][H_kv]")
+    for t in (key_cache, value_cache, k_scales, v_scales):
+        if not t.is_contiguous():
+            raise ValueError("caches and scales must be contiguous")
+    if slot_mapping.dtype != torch.int64 or not slot_mapping.is_contiguous():
+        raise ValueError("slot_mapping must be contiguous int64")
+    _check(lib.pa_append_int8(_ptr(k), _ptr(v), dtype_code(k.dtype), _ptr(key_cache), _ptr(value_cache),
+                              _ptr(k_scales), _ptr(v_scales), _ptr(slot_mapping), T, H, d, 16, N,
+                              k.stride(0), v.stride(0), _stream(stream)), "pa_append_int8")
 
 
 def pa_quantize_int4(src_cache, dst_cache, scales, stream=None):

@@ -57,6 +57,82 @@ def test_reshape_strided_padding_and_unaligned():
     assert np.array_equal(bits(kc), np_bits(ek)) and np.array_equal(bits(vc), np_bits(ev))
 
 
+def _host_rows(t):
+    """Device tensor -> (numpy array, oracle dtype code); bf16 as uint16 bits."""
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16), oracle.BF16
+    return t.cpu().numpy(), None
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.float16, 128), (torch.bfloat16, 64), (torch.float32, 128)])
+def test_append_int8_bit_exact(dtype, d):
+    """Single tokens appended into a quantised int8 pool, in distinct blocks: tokens
+    that fit a tile's scale and tokens that raise it (re-rounding the tile), an
+    empty tile, padding and an out-of-pool slot.  Codes and scales bit-exact with
+    the oracle's rule."""
+    dev = "cuda"
+    N, H = 24, 4
+    rng = np.random.default_rng(21)
+    src = torch.from_numpy((rng.standard_normal((N, H, 16, d)) * 2).astype(np.float32)).to(dev).to(dtype)
+    kc = torch.empty((N, H, 16, d), dtype=torch.int8, device=dev)
+    vc = torch.empty_like(kc)
+    ks = torch.empty((N, H), dtype=torch.float32, device=dev)
+    vs = torch.empty_like(ks)
+    pa.pa_quantize_int8(src, kc, ks)
+    pa.pa_quantize_int8(src.flip(0).contiguous(), vc, vs)
+    kc[5].zero_(); ks[5].zero_()  # an empty tile
+    T = 14
+    blocks = rng.choice([b for b in range(N) if b != 5], size=T, replace=False)  # one token per block
+    slots = blocks.astype(np.int64) * 16 + rng.integers(0, 16, size=T)
+    slots[3] = -1
+    slots[8] = N * 16 + 7  # outside the pool
+    slots[0] = 5 * 16 + 9  # into the empty tile
+    mag = np.where(np.arange(T) % 2 == 0, 0.2, 12.0)[:, None, None]  # fit, raise
+    k = torch.from_numpy((rng.standard_normal((T, H, d)) * mag).astype(np.float32)).to(dev).to(dtype)
+    v = torch.from_numpy((rng.standard_normal((T, H, d)) * mag[::-1]).astype(np.float32)).to(dev).to(dtype)
+    torch.cuda.synchronize()
+    ekc, evc = kc.cpu().numpy(), vc.cpu().numpy()
+    eks, evs = ks.cpu().numpy(), vs.cpu().numpy()
+    ks0 = eks.copy()
+    kh, code = _host_rows(k)
+    vh, _ = _host_rows(v)
+    oracle.append_int8(kh, vh, ekc, evc, eks, evs, slots, code=code)
+    pa.pa_append_int8(k, v, kc, vc, ks, vs, torch.from_numpy(slots).to(dev))
+    torch.cuda.synchronize()
+    assert pa.pa_get_error_flags(reset=True) == pa.PA_EFLAG_BAD_SLOT
+    assert np.array_equal(ks.cpu().numpy().view(np.uint32), eks.view(np.uint32))
+    assert np.array_equal(vs.cpu().numpy().view(np.uint32), evs.view(np.uint32))
+    assert np.array_equal(kc.cpu().numpy(), ekc) and np.array_equal(vc.cpu().numpy(), evc)
+    # the case mix happened: some tiles' scales were raised, the others kept theirs
+    after = ks.cpu().numpy()
+    assert (after > ks0).any() and (after == ks0).any()
+
+
+def test_append_int8_token_by_token_into_one_block():
+    """Sixteen calls, each appending the next token of one block (the decode-step
+    pattern), on fp16 tokens of growing size: every call may raise the scale and
+    re-round what is there.  Bit-exact with the oracle after every call."""
+    dev = "cuda"
+    H, d, N = 2, 128, 3
+    rng = np.random.default_rng(22)
+    kc = torch.zeros((N, H, 16, d), dtype=torch.int8, device=dev)
+    vc = torch.zeros_like(kc)
+    ks = torch.zeros((N, H), dtype=torch.float32, device=dev)
+    vs = torch.zeros_like(ks)
+    ekc, evc = kc.cpu().numpy(), vc.cpu().numpy()
+    eks, evs = ks.cpu().numpy(), vs.cpu().numpy()
+    for o in range(16):
+        k = (rng.standard_normal((1, H, d)) * (0.5 + o)).astype(np.float16)
+        v = (rng.standard_normal((1, H, d)) * (16 - o)).astype(np.float16)
+        slot = np.array([1 * 16 + o], dtype=np.int64)
+        oracle.append_int8(k, v, ekc, evc, eks, evs, slot)
+        pa.pa_append_int8(torch.from_numpy(k).to(dev), torch.from_numpy(v).to(dev), kc, vc, ks, vs,
+                          torch.from_numpy(slot).to(dev))
+        torch.cuda.synchronize()
+        assert np.array_equal(kc.cpu().numpy(), ekc) and np.array_equal(vc.cpu().numpy(), evc), f"slot {o}"
+        assert np.array_equal(ks.cpu().numpy(), eks) and np.array_equal(vs.cpu().numpy(), evs), f"slot {o}"
+
+
 def test_reshape_bad_slot_sets_flag_and_skips():
     dev = "cuda"
     k = torch.ones((2, 1, 64), dtype=torch.float16, device=dev)
