@@ -380,14 +380,14 @@ def main(argv=None):
     torch.cuda.synchronize()
 
     # ---- device-resident timing ----------------------------------------------------------
-    # Steps that read more than twice the L2 size: one event pair around the K timed
-    # steps issued back to back (the host enqueues a step in well under the step's
-    # device time, so the device never waits), then a second loop of only the decode
-    # calls of the same steps for the dominant kernel.  Smaller steps: each step
-    # timed by its own event pair, with the L2 flushed (a write of twice its size)
-    # before it, outside the events.
+    # Every step reads more than the L2 holds, and the largest more than twice that:
+    # one event pair around the K timed steps issued back to back (the host enqueues
+    # a step in well under the step's device time, so the device never waits), then a
+    # second loop of only the decode calls of the same steps for the dominant kernel.
+    # Otherwise each step is timed by its own event pair, with the L2 flushed (a
+    # write of twice its size) before it, outside the events.
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
-    per_step = max(sbytes) < 2 * l2
+    per_step = min(sbytes) <= l2 or max(sbytes) < 2 * l2
     flush = torch.empty(2 * l2, dtype=torch.uint8, device="cuda") if per_step else None
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -449,7 +449,8 @@ def main(argv=None):
                    "partition_size": "library picks (-1)" if part == -1 else part, "algo": args.algo,
                    "l2": ("L2 flushed before every timed step (write of twice the L2 size, "
                           "outside the events)" if per_step else
-                          "inputs larger than L2: every step reads more than twice the L2 size, no flush"),
+                          f"inputs larger than L2: every step reads {min(sbytes) / 1e6:.0f}-"
+                          f"{max(sbytes) / 1e6:.0f} MB against {l2 / 1e6:.0f} MB of L2, no flush"),
                    "timing": ("one CUDA event pair per step, summed" if per_step else
                               "CUDA events around the K steps issued back to back"),
                    "decode_flags": "PA_DECODE_INPUTS_READY",
