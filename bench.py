@@ -456,6 +456,8 @@ def main(argv=None):
                    "decode_flags": "PA_DECODE_INPUTS_READY",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "decode_tokens_per_s": toks_rank * world / (ms_max * 1e-3),
+        # the same step repeated for 32 layers: attention-only context for a 7B-class model
+        "decode_tokens_per_s_32_layers": toks_rank * world / (ms_max * 1e-3) / 32,
         "hbm_frac_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
         "hbm_frac_of_" + peak_kind: value / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
