@@ -11,8 +11,10 @@
  *
  * Memory layouts (row-major, innermost last):
  *   key_cache, value_cache  [num_blocks][num_kv_heads][PA_BLOCK_SIZE][head_dim]
- *   k_scales, v_scales      [num_blocks][num_kv_heads]  fp32 (int8 caches only)
+ *                           (PA_I4: head_dim / 2 bytes per row, two values per byte)
+ *   k_scales, v_scales      [num_blocks][num_kv_heads]  fp32 (int8 and 4-bit caches only)
  *   q, out                  [num_seqs][num_q_heads][head_dim]
+ *                           ([num_seqs][Q][num_q_heads][head_dim] for Q = query_len > 1)
  *   block_tables            [num_seqs][max_blocks_per_seq]  int32
  *   seq_lens                [num_seqs]  int32
  *   slot_mapping            [num_tokens]  int64, slot = block * PA_BLOCK_SIZE + offset
@@ -96,9 +98,13 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
 typedef struct pa_decode_params {
     int num_seqs;            /* B >= 0 */
     int num_q_heads;         /* H_q, a multiple of num_kv_heads */
-    int num_kv_heads;        /* H_kv; group size G = H_q / H_kv: 1, 2, 4, 8, 16, 32 or 64
-                                (groups above 8, e.g. MQA with H_kv = 1, run as 8-head
-                                groups that each read the KV head's tiles) */
+    int num_kv_heads;        /* H_kv; group size G = H_q / H_kv with Q * G <= 512 (Q =
+                                query_len).  The Q * G (query token, head) pairs of a KV head
+                                run as up to 8 columns per kernel row, more as several rows
+                                that each read the KV head's tiles (MQA: H_kv = 1).  Counts
+                                other than 1, 2, 4, 8 or multiples of 8 are padded, on the
+                                tensor-core family only; the CUDA-core family takes
+                                single-token decode with G in 1, 2, 4, 8, 16, 32, 64. */
     int head_dim;            /* 64 or 128; 256 on the CUDA-core family (not with PA_F32) */
     int block_size;          /* must be PA_BLOCK_SIZE */
     int max_blocks_per_seq;  /* row stride of block_tables */
