@@ -248,6 +248,19 @@ def dist_setup(args):
     return rank, world, local
 
 
+def cpu_model():
+    """The host CPU's model name (as lscpu prints it), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def cpu_baseline(w, int8, seconds, host_caches=None):
     """The oracle as it stands, on this host's cores, over whole decode steps
     of the workload replayed in order until ``seconds`` of work are done."""
@@ -284,10 +297,23 @@ def cpu_baseline(w, int8, seconds, host_caches=None):
                 nsteps += 1
         if t_work >= seconds:
             break
+    # the same oracle on one thread, over the first four sequences of the first decode
+    first = next(op for ops in w.steps for op in ops if isinstance(op, W.Decode))
+    n1 = min(4, first.q.shape[0])
+    sub = W.Decode(first.q[:n1], first.block_tables[:n1], first.seq_lens[:n1], first.max_seq_len)
+    t0 = time.perf_counter()
+    if sub.q.ndim == 4:
+        oracle.decode_multi(sub.q, kc, vc, sub.block_tables, sub.seq_lens, w.scale, ks, vs, nthreads=1)
+    else:
+        oracle.decode(sub.q, kc, vc, sub.block_tables, sub.seq_lens, w.scale, ks, vs, nthreads=1)
+    t1 = time.perf_counter() - t0
     return {"value": done_bytes / t_work / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"{nsteps} whole decode step(s) of the workload in trace order "
                       f"({ntok} sequence decodes, all heads), fp64 C oracle, {t_work:.2f} s",
-            "tokens_per_s": ntok / t_work}
+            "tokens_per_s": ntok / t_work,
+            "value_1_thread": W.decode_kv_bytes(sub, w, kv_elem_bytes(int8)) / t1 / 1e9,
+            "sample_1_thread": f"the first {n1} sequences of the first decode step on one thread, {t1:.2f} s",
+            "cpu_model": cpu_model()}
 
 
 def reference_arm(args, rank, world):
@@ -338,7 +364,7 @@ def reference_arm(args, rank, world):
         "config": {"workload": WORKLOADS[args.workload], "name": args.workload},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": "per step: one sequence (all query heads) of trace step "
-                                   "i mod T, fp64 C oracle"},
+                                   "i mod T, fp64 C oracle", "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -78,3 +78,16 @@ def test_traffic_is_reported_only_for_the_captured_kernel(monkeypatch):
     assert bench.traffic_per_launch("ragged", "simt", -1, 2.0e8) is None
     assert bench.traffic_per_launch("ragged", "auto", 512, 2.0e8) is None
     assert bench.traffic_per_launch("long", "auto", -1, 2.0e8) is None
+
+
+@pytest.mark.parametrize("int8", [False, "i8", "i4"])
+def test_cpu_baseline_reports_its_sample(int8):
+    """The oracle leg of the bench line: GB/s over whole decode steps on all host
+    threads, a one-thread figure on a named sample, and the CPU model."""
+    w = W.random_case([40, 300, 17, 64, 5], num_q_heads=8, num_kv_heads=2, head_dim=128, dtype="float16",
+                      seed=4)
+    cb = bench.cpu_baseline(w, int8, 0.01)
+    assert cb["kind"] == "oracle" and cb["unit"] == "GB/s" and cb["cores"] >= 1
+    assert cb["value"] > 0 and cb["value_1_thread"] > 0 and cb["tokens_per_s"] > 0
+    assert "1 whole decode step" in cb["sample"] and "first 4 sequences" in cb["sample_1_thread"]
+    assert isinstance(cb["cpu_model"], str) and cb["cpu_model"]
