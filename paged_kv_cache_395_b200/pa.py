@@ -2,8 +2,9 @@
 
 The names mirror the C ABI in ``include/pa.h``:
 
-* ``pa_reshape_and_cache``, ``pa_decode``, ``pa_block_copy``,
-  ``pa_quantize_int8``, ``pa_decode_workspace_size``, ``pa_get_error_flags``
+* ``pa_reshape_and_cache``, ``pa_decode``, ``pa_decode_fixed_scratch``,
+  ``pa_block_copy``, ``pa_quantize_int8``, ``pa_quantize_int4``,
+  ``pa_append_int8``, ``pa_decode_workspace_size``, ``pa_get_error_flags``
   take torch CUDA tensors (or raw device pointers via ``lib``), check device,
   dtype and contiguity, and call the library on
   ``torch.cuda.current_stream()``.  Every step of the computation runs in the
