@@ -50,7 +50,7 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of the decode kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum of the two captured launches, trace steps 8 and 9 of the
-# ragged workload), per algorithmic byte; the summary is profiles/decode_tc_ragged.md.
+# ragged workload), per algorithmic byte.
 # It holds only for the kernel code it was taken on (hash of the source without
 # comments); after any code change the bench reports null until it is taken again.
 NCU_TRAFFIC = {
@@ -178,7 +178,7 @@ class ClockSampler:
         "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
     }
 
-    def __init__(self, device_index, period=0.002):
+    def __init__(self, device_index, period=0.001):
         self.samples, self.reasons, self.max_mhz, self.ok = [], 0, None, False
         self.period = period
         self._stop = threading.Event()
@@ -452,15 +452,31 @@ def main(argv=None):
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         ms, host_ms = timed(calls.run)
-    if dist is not None:
-        dist.barrier()
-    dec_ms, _ = timed(calls.run_decode_only)
+        if dist is not None:
+            dist.barrier()
+        dec_ms, _ = timed(calls.run_decode_only)
+        # The same K-step window repeated (at least 5 times and ~60 ms of device
+        # time, so the clock sampler sees the GPU under load), then one full lap of
+        # the trace: every step once, in order, right after the window.
+        reps = []
+        n_rep = max(5, min(200, int(np.ceil(60.0 / max(ms, 1e-3)))))
+        for _ in range(n_rep):
+            reps.append(timed(calls.run)[0])
+        idx_window = idx
+        idx = [(args.warmup + K + j) % T for j in range(T)]
+        lap_ms, _ = timed(calls.run)
+        lap_dec_ms, _ = timed(calls.run_decode_only)
+        lap_bytes = sum(sbytes[i] for i in idx)
+        idx = idx_window
     bytes_rank = sum(sbytes[i] for i in idx)
     toks_rank = sum(stoks[i] for i in idx)
     launches = sum(calls.launches[i] for i in idx)
     value, ms_max = replica_throughput(bytes_rank, ms, dist)
     peak, peak_kind = load_peak()
     achieved = bytes_rank / (dec_ms * 1e-3) / 1e9
+    rep_vals = [replica_throughput(bytes_rank, r, dist)[0] for r in reps]
+    lap_value, lap_ms_max = replica_throughput(lap_bytes, lap_ms, dist)
+    lap_dec_value, _ = replica_throughput(lap_bytes, lap_dec_ms, dist)
 
     # ---- end to end through the C ABI with host buffers ------------------------------------------
     e2e = None
@@ -494,6 +510,16 @@ def main(argv=None):
                      "peak_kind": peak_kind},
         "gpu_launches": launches,
         "host_enqueue_ms": host_ms,
+        # the K-step window timed again, n times back to back
+        "value_repeats": {"median": statistics.median(rep_vals), "min": min(rep_vals),
+                          "max": max(rep_vals), "n": len(rep_vals), "unit": "GB/s"},
+        # one full lap of the trace (all T steps once, in trace order), timed after the
+        # window: the sum of its algorithmic bytes over its device time, whole steps and
+        # the decode calls alone
+        "value_full_trace": lap_value,
+        "decode_full_trace": lap_dec_value,
+        "full_trace": {"steps": T, "ms_per_step": lap_ms_max / T, "bytes": lap_bytes * world,
+                       "decode_frac_of_" + peak_kind: lap_dec_value / world / peak},
         "clocks": clk.report(),
     }
     if e2e is not None:

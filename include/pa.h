@@ -126,11 +126,16 @@ typedef struct pa_decode_params {
     int algo;                /* enum pa_algo */
     void *workspace;         /* device scratch, >= pa_decode_workspace_size(p) bytes,
                                 16-byte aligned; NULL allowed when that size is 0.  Must be
-                                zero-filled once before its first use; every call leaves it
-                                ready for the next (its merge counters back at zero).  Calls
-                                that share a workspace must not overlap on the device. */
+                                zero-filled once before its first use.  Its first
+                                PA_WORKSPACE_COUNTER_BYTES hold merge counters, at the same
+                                place for every call, and partial results come after them;
+                                every call returns the counters to zero, also when a bounded
+                                wait gave up (PA_EFLAG_WAIT_TIMEOUT).  So one workspace serves
+                                any sequence of calls, whatever their parameters or kernel
+                                family, without clearing it again.  Calls that share a
+                                workspace must not overlap on the device. */
     size_t workspace_bytes;
-    int flags;               /* 0, or PA_DECODE_INPUTS_READY */
+    int flags;               /* 0, or PA_DECODE_INPUTS_READY and/or PA_DECODE_OUT_F32 */
     int query_len;           /* new tokens per sequence, Q (0 or 1: single-token decode).
                                 q and out are [num_seqs][Q][num_q_heads][head_dim]; seq_lens
                                 count all Q new tokens (already appended), and query token i
@@ -155,11 +160,40 @@ typedef struct pa_decode_params {
 #define PA_DECODE_INPUTS_READY 1
 
 /*
- * Bytes of device workspace pa_decode needs for these parameters (0 for
- * partition_size == 0).  Depends only on num_seqs, num_q_heads, num_kv_heads,
- * head_dim, max_seq_len and partition_size.  Returns 0 for invalid params.
+ * PA_DECODE_OUT_F32: out is fp32, of q's shape, holding the fp32 result before
+ * the one rounding to q_dtype that pa_decode otherwise applies.  With an fp16 or
+ * bf16 q the fp16/bf16 output is exactly that fp32 value rounded to nearest
+ * even, so the flag shows the arithmetic's accuracy apart from the output
+ * format's (bf16 keeps 8 significant bits: its rounding alone moves a value by
+ * up to 2^-8 of its size).
+ */
+#define PA_DECODE_OUT_F32 2
+
+/* Size of the merge-counter region at the start of every split-K workspace:
+ * one int per (sequence, KV head) row of the tensor-core family's split
+ * (num_seqs * num_kv_heads * ceil(Q * G / 8) rows at most 65536; beyond that
+ * the library runs that family in one pass, or the CUDA-core family). */
+#define PA_WORKSPACE_COUNTER_BYTES (256 * 1024)
+
+/*
+ * Bytes of device workspace pa_decode needs for these parameters (0 when the
+ * call runs in one pass; else PA_WORKSPACE_COUNTER_BYTES plus the partial
+ * results).  Depends only on num_seqs, num_q_heads, num_kv_heads, head_dim,
+ * query_len, max_seq_len, max_blocks_per_seq, the dtypes, algo and
+ * partition_size.  Returns 0 for invalid params.
  */
 size_t pa_decode_workspace_size(const pa_decode_params *p);
+
+/*
+ * The kernel family pa_decode runs for these parameters and this q:
+ * PA_ALGO_TENSOR or PA_ALGO_SIMT, or a negative pa_status for parameters
+ * pa_decode would reject.  q (a device pointer, not read) matters only through
+ * its alignment: the tensor-core family reads q rows with 16-byte copies, so an
+ * unaligned q goes to the CUDA-core family.  Together with
+ * pa_decode_workspace_size it also gives the kernel launches of a call: one,
+ * plus a merge kernel when the CUDA-core family splits (workspace size > 0).
+ */
+int pa_decode_algo(const pa_decode_params *p, const void *q);
 
 /*
  * Single-token decode attention over the paged cache
@@ -200,12 +234,34 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
  *    before any stream capture.
  *  - All calls on one device share the area: calls that overlap on the device
  *    (different streams, or host threads without ordering) race on it.  Issue
- *    them in one stream order.
+ *    them in one stream order.  Calls in order may use any parameters: the
+ *    area's merge counters sit at its start, where no partial result goes.
+ *  - The area's address is kept for the life of the process: do not use the
+ *    library after cudaDeviceReset.
  */
 #define PA_FIXED_SCRATCH_BYTES ((size_t)32 << 20)
 int pa_decode_fixed_scratch(void *out, const void *q, const void *key_cache, const void *value_cache,
                             const int32_t *block_tables, const int32_t *seq_lens, float scale,
                             const pa_decode_params *p, pa_stream_t stream);
+
+/*
+ * Self-test of the failure path of the bounded waits (no counterpart in the
+ * pages: it exists so that the library's handling of a copy that never lands
+ * can be checked on a working GPU without faulting it).  Runs pa_decode on the
+ * tensor-core family (the parameters must select it) with two changes: every
+ * bounded wait gives up after limit_ns nanoseconds instead of one second, and
+ * the first worker never issues its stall_at-th copy (counted from 0 over its
+ * (K tile, V tile) stages), so its wait for that stage runs out: no memory is
+ * read or written for it, and nothing hangs.  Expected outcome: PA_OK, the
+ * error word gains PA_EFLAG_WAIT_TIMEOUT, the rows that worker had not finished
+ * hold no valid result, and the workspace is left ready for the next call (the
+ * worker waits, again bounded, for its copies in flight, then takes the merge
+ * tickets of its remaining partial results with empty partials).
+ */
+int pa_decode_stall_selftest(void *out, const void *q, const void *key_cache, const void *value_cache,
+                             const int32_t *block_tables, const int32_t *seq_lens, float scale,
+                             const pa_decode_params *p, int stall_at, uint64_t limit_ns,
+                             pa_stream_t stream);
 
 /*
  * Copy-on-write block copy (chanyi.net.cn/article/49 section 三: shared prefix

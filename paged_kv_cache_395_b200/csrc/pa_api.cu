@@ -100,7 +100,7 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
     if (p->algo == PA_ALGO_SIMT && !simt_ok) return PA_ERR_UNSUPPORTED;
     if (p->num_seqs > 65535 || kh.Hkv > 65535) return PA_ERR_UNSUPPORTED;
     if (p->algo < PA_ALGO_AUTO || p->algo > PA_ALGO_TENSOR) return PA_ERR_UNSUPPORTED;
-    if (p->flags & ~PA_DECODE_INPUTS_READY) return PA_ERR_UNSUPPORTED;
+    if (p->flags & ~(PA_DECODE_INPUTS_READY | PA_DECODE_OUT_F32)) return PA_ERR_UNSUPPORTED;
     int ps = p->partition_size;
     if (ps < -1 || (ps > 0 && ps % PA_BLOCK_SIZE)) return PA_ERR_SHAPE;
     const int max_len = p->max_seq_len < p->max_blocks_per_seq * PA_BLOCK_SIZE
@@ -140,9 +140,12 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
     // of all (sequence, KV head) rows with 32-bit integers
     const int64_t stream_blocks =
         (int64_t)p->num_seqs * kh.Hkv * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
+    // a split on the tensor-core family keeps one merge counter per row in the
+    // workspace's fixed counter region
+    const bool rows_fit = (int64_t)p->num_seqs * kh.Hkv <= kCounterRows;
     const bool tc_ok = decode_tc_supported(p->q_dtype, p->kv_dtype, p->head_dim, G, p->num_seqs) &&
                        p->num_blocks * p->num_kv_heads * PA_BLOCK_SIZE <= 2147483647LL &&
-                       stream_blocks <= (1LL << 30);
+                       stream_blocks <= (1LL << 30) && (rows_fit || p->partition_size <= 0);
     if (p->algo == PA_ALGO_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
     // several new tokens per sequence, or padded columns: the tensor-core family only
     if ((kh.qlen > 1 || kh.padded) && !tc_ok) return PA_ERR_UNSUPPORTED;
@@ -155,8 +158,10 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
         pl->bytes = decode_workspace_bytes(p->num_seqs, p->num_q_heads, kh.Hkv, p->head_dim, max_len, part);
         return PA_OK;
     }
-    if (p->partition_size == 0 || max_len == 0) {
-        pl->tc_chunk = -1;  // one warp per (sequence, KV head) row, no workspace
+    if (p->partition_size == 0 || max_len == 0 || !rows_fit) {
+        // one warp per (sequence, KV head) row, no workspace (with more rows than
+        // counters, rows far outnumber the warps and balance without a split)
+        pl->tc_chunk = -1;
         return PA_OK;
     }
     const int64_t tmax = (int64_t)p->num_seqs * kh.Hkv * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
@@ -170,11 +175,10 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
         nchunks = tmax < kTcMaxChunks ? tmax : kTcMaxChunks;
     }
     pl->tc_slots = 2 * nchunks;
-    // partial outputs and lse of two segments per chunk, then one merge ticket
-    // per (sequence, KV head) row
-    pl->bytes = up256((size_t)pl->tc_slots * G * p->head_dim * sizeof(float)) +
-                up256((size_t)pl->tc_slots * G * sizeof(float)) +
-                up256((size_t)p->num_seqs * kh.Hkv * sizeof(int));
+    // the merge counters' fixed region, then partial outputs and lse of two
+    // segments per chunk
+    pl->bytes = kCounterBytes + up256((size_t)pl->tc_slots * G * p->head_dim * sizeof(float)) +
+                up256((size_t)pl->tc_slots * G * sizeof(float));
     return PA_OK;
 }
 
@@ -286,9 +290,15 @@ size_t pa_decode_workspace_size(const pa_decode_params *p) {
     return pl.bytes;
 }
 
-int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
-              const int32_t *block_tables, const int32_t *seq_lens, float scale,
-              const pa_decode_params *p, pa_stream_t stream) {
+}  // extern "C"
+
+namespace pa {
+
+// pa_decode with the two knobs of pa_decode_stall_selftest.
+static int decode_impl(void *out, const void *q, const void *key_cache, const void *value_cache,
+                       const int32_t *block_tables, const int32_t *seq_lens, float scale,
+                       const pa_decode_params *p, pa_stream_t stream, int stall_at,
+                       unsigned long long wait_ns) {
     Plan pl;
     const int rc = make_plan(p, &pl);
     if (rc != PA_OK) return rc;
@@ -325,15 +335,22 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     a.max_len = pl.max_len;
     a.q_dtype = p->q_dtype;
     a.kv_dtype = p->kv_dtype;
+    a.out_f32 = (p->flags & PA_DECODE_OUT_F32) ? 1 : 0;
+    a.stall_at = stall_at;
+    a.wait_ns = wait_ns;
     char *ws = reinterpret_cast<char *>(p->workspace);
     if (pl.tc && (uintptr_t)q % 16) {
-        if (p->algo == PA_ALGO_TENSOR) return PA_ERR_ALIGN;
+        if (p->algo == PA_ALGO_TENSOR || stall_at >= 0) return PA_ERR_ALIGN;
         // the tensor-core family reads q rows with 16-byte bulk copies; a q that is not
         // 16-byte aligned goes to the CUDA-core family, which needs its own plan
         pa_decode_params p2 = *p;
         p2.algo = PA_ALGO_SIMT;
-        return pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, &p2, stream);
+        return decode_impl(out, q, key_cache, value_cache, block_tables, seq_lens, scale, &p2, stream, -1,
+                           wait_ns);
     }
+    if (stall_at >= 0 && !pl.tc) return PA_ERR_UNSUPPORTED;
+    // workspace: the merge counters' fixed region, then the partial outputs, then their lse
+    if (pl.bytes > 0) a.counters = reinterpret_cast<int *>(ws);
     if (pl.tc) {
         a.part = 0;
         a.max_parts = 1;
@@ -341,10 +358,8 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
         a.early = (p->flags & PA_DECODE_INPUTS_READY) ? 1 : 0;
         if (pl.bytes > 0) {
             const size_t o_bytes = up256((size_t)pl.tc_slots * a.G * a.D * sizeof(float));
-            const size_t l_bytes = up256((size_t)pl.tc_slots * a.G * sizeof(float));
-            a.ws_o = reinterpret_cast<float *>(ws);
-            a.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
-            a.counters = reinterpret_cast<int *>(ws + o_bytes + l_bytes);
+            a.ws_o = reinterpret_cast<float *>(ws + kCounterBytes);
+            a.ws_lse = reinterpret_cast<float *>(ws + kCounterBytes + o_bytes);
         }
         return launch_decode_tc(a, (cudaStream_t)stream);
     }
@@ -352,10 +367,8 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
     a.max_parts = pl.max_parts;
     if (pl.bytes > 0) {
         const size_t o_bytes = up256((size_t)a.B * a.Hq * pl.max_parts * a.D * sizeof(float));
-        const size_t l_bytes = up256((size_t)a.B * a.Hq * pl.max_parts * sizeof(float));
-        a.ws_o = reinterpret_cast<float *>(ws);
-        a.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
-        a.counters = reinterpret_cast<int *>(ws + o_bytes + l_bytes);
+        a.ws_o = reinterpret_cast<float *>(ws + kCounterBytes);
+        a.ws_lse = reinterpret_cast<float *>(ws + kCounterBytes + o_bytes);
     }
     if (pl.max_len == 0) {
         // every row is zero: the one-pass kernel writes zeros for seq_len <= 0
@@ -363,6 +376,34 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
         a.max_parts = 1;
     }
     return launch_decode_simt(a, (cudaStream_t)stream);
+}
+
+}  // namespace pa
+
+extern "C" {
+
+int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
+              const int32_t *block_tables, const int32_t *seq_lens, float scale,
+              const pa_decode_params *p, pa_stream_t stream) {
+    return decode_impl(out, q, key_cache, value_cache, block_tables, seq_lens, scale, p, stream, -1,
+                       kWaitLimitNs);
+}
+
+int pa_decode_stall_selftest(void *out, const void *q, const void *key_cache, const void *value_cache,
+                             const int32_t *block_tables, const int32_t *seq_lens, float scale,
+                             const pa_decode_params *p, int stall_at, uint64_t limit_ns,
+                             pa_stream_t stream) {
+    if (stall_at < 0 || limit_ns == 0) return PA_ERR_SHAPE;
+    return decode_impl(out, q, key_cache, value_cache, block_tables, seq_lens, scale, p, stream, stall_at,
+                       (unsigned long long)limit_ns);
+}
+
+int pa_decode_algo(const pa_decode_params *p, const void *q) {
+    Plan pl;
+    const int rc = make_plan(p, &pl);
+    if (rc != PA_OK) return rc;
+    if (pl.tc && (uintptr_t)q % 16) return p->algo == PA_ALGO_TENSOR ? PA_ERR_ALIGN : PA_ALGO_SIMT;
+    return pl.tc ? PA_ALGO_TENSOR : PA_ALGO_SIMT;
 }
 
 int pa_get_error_flags(unsigned int *flags, int reset, pa_stream_t stream) {

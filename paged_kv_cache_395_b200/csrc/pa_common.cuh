@@ -84,6 +84,16 @@ template <> struct Cvt<int8_t> {
     static __device__ __forceinline__ float to_f(int8_t x) { return (float)x; }
 };
 
+// Element idx of a decode output: fp32 when the call asked for an fp32 output
+// (PA_DECODE_OUT_F32), else rounded once to T.
+template <typename T>
+__device__ __forceinline__ void store_out(void *out, int f32, size_t idx, float v) {
+    if (f32)
+        reinterpret_cast<float *>(out)[idx] = v;
+    else
+        reinterpret_cast<T *>(out)[idx] = Cvt<T>::from_f(v);
+}
+
 // Convert N consecutive elements held in registers (as raw 32-bit words) to float.
 template <typename T, int N>
 __device__ __forceinline__ void to_float(const uint32_t *w, float *f);
@@ -216,15 +226,16 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after about
-// one second (a copy that never lands), raises PA_EFLAG_WAIT_TIMEOUT and
-// returns false; the caller then abandons its remaining work.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete.  Gives up after
+// limit_ns nanoseconds (one second in every library call; a copy that never
+// lands), raises PA_EFLAG_WAIT_TIMEOUT and returns false; the caller then
+// abandons its remaining work.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63) == 63 && global_timer_ns() - t0 > 1000000000ull) {
+        if ((it & 63) == 63 && global_timer_ns() - t0 > limit_ns) {
             raise_flag(PA_EFLAG_WAIT_TIMEOUT);
             return false;
         }

@@ -117,10 +117,10 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
     const int L = effective_len(a, b);
     const int P = a.part > 0 ? a.part : max(L, 1);
     const int t0 = part * P;
-    TQ *out = reinterpret_cast<TQ *>(a.out) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
+    const size_t out0 = ((size_t)b * a.Hq + (size_t)kvh * G) * D;  // first element of the group's rows
     if (L <= 0) {
         if (part == 0)
-            for (int i = threadIdx.x; i < G * D; i += blockDim.x) out[i] = Cvt<TQ>::from_f(0.f);
+            for (int i = threadIdx.x; i < G * D; i += blockDim.x) store_out<TQ>(a.out, a.out_f32, out0 + i, 0.f);
         return;
     }
     if (t0 >= L) return;
@@ -154,8 +154,10 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
     __syncwarp();
 
     // lane 0: start the copy of this warp's it-th block into stage it % STAGES
+    int issued = 0;  // lane 0: blocks whose copy was started
     auto issue = [&](int it) {
         const int s = it % STAGES;
+        issued = it + 1;
         const int pb = table[warp + it * NW];
         if (pb < 0 || (int64_t)pb >= a.N) {
             my_blk[s] = -1;
@@ -187,10 +189,17 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
     for (int it = 0; it < my_nblk; ++it) {
         const int s = it % STAGES;
         const uint32_t parity = (it / STAGES) & 1;
-        int ok = lane == 0 ? (int)mbar_wait(&my_bars[s], parity) : 0;
+        int ok = lane == 0 ? (int)mbar_wait(&my_bars[s], parity, a.wait_ns) : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        if (lane != 0) mbar_wait(&my_bars[s], parity);  // completed: acquires the copied data
+        if (!ok) {
+            // a copy did not land in time: wait (bounded again) for the copies still in
+            // flight, so that none lands in shared memory reused below or after exit
+            if (lane == 0)
+                for (int k = it; k < issued; ++k) mbar_wait(&my_bars[k % STAGES], (k / STAGES) & 1, a.wait_ns);
+            __syncwarp();
+            break;
+        }
+        if (lane != 0) mbar_wait(&my_bars[s], parity, a.wait_ns);  // completed: acquires the copied data
         const int jb = warp + it * NW;
         const int pb = my_blk[s];
         const int ntok = (jb == nblk - 1) ? ntok_last : kBlockSize;
@@ -300,7 +309,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(const DecodeArgs a) {
             Os = fmaf(co[(w * G + h) * D + dim], f, Os);
         }
         if (nparts == 1) {
-            out[h * D + dim] = Cvt<TQ>::from_f(Os / Ls);
+            store_out<TQ>(a.out, a.out_f32, out0 + h * D + dim, Os / Ls);
         } else {
             const size_t row = ((size_t)b * a.Hq + (size_t)kvh * G + h) * a.max_parts + part;
             a.ws_o[row * D + dim] = Os / Ls;
@@ -323,7 +332,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
     const float *lse = a.ws_lse + row;
     float M = -INFINITY;
     for (int p = 0; p < np; ++p) M = fmaxf(M, lse[p]);
-    TQ *out = reinterpret_cast<TQ *>(a.out) + ((size_t)b * a.Hq + qh) * a.D;
+    const size_t out0 = ((size_t)b * a.Hq + qh) * a.D;
     for (int dim = threadIdx.x; dim < a.D; dim += blockDim.x) {
         float S = 0.f, acc = 0.f;
         for (int p = 0; p < np; ++p) {
@@ -331,7 +340,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
             S += w;
             acc = fmaf(w, a.ws_o[(row + p) * a.D + dim], acc);
         }
-        out[dim] = Cvt<TQ>::from_f(acc / S);
+        store_out<TQ>(a.out, a.out_f32, out0 + dim, acc / S);
     }
 }
 
@@ -340,9 +349,10 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int pa
     const size_t mp = (size_t)((max_len + part - 1) / part);
     const size_t o = (size_t)B * Hq * mp * D * sizeof(float);
     const size_t lse = (size_t)B * Hq * mp * sizeof(float);
-    const size_t cnt = (size_t)B * Hkv * sizeof(int);
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    return up(o) + up(lse) + up(cnt);
+    // the counter region is not used by this family, but kept free so that one
+    // workspace serves calls of either family
+    return kCounterBytes + up(o) + up(lse);
 }
 
 template <typename TQ, typename TKV, int D, int G>

@@ -634,6 +634,9 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 my_sc[2 * s + 1] = vsv;
             }
             if (y < 0) raise_flag(PA_EFLAG_BAD_BLOCK);
+            // the failure-path self-test leaves one stage's copies unissued, so that the
+            // consumer's bounded wait for it runs out (never set in a normal call)
+            const bool stall = gw == 0 && p_k == a.stall_at;
             // Relaxed arrival: a releasing one would first wait for this lane's
             // outstanding loads (the next window's table entries).  The stage's tiles
             // and q rows are published by the transaction count; the flag and scales
@@ -644,7 +647,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             } else {
                 mbar_arrive_expect_tx_relaxed(bar, tx);
             }
-            if (y >= 0) {
+            if (y >= 0 && !stall) {
                 const uint32_t dst = ring + s * C::STAGE;
 #pragma unroll
                 for (int bx = 0; bx < C::BOXES; ++bx) {
@@ -652,7 +655,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                     tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * C::BOXW, y, smem_addr(bar));
                 }
             }
-            if (!MQ && seg_first) {
+            if (stall) {
+            } else if (!MQ && seg_first) {
                 bulk_g2s_u32(qring + s * C::QSLOT, reinterpret_cast<const T *>(a.q) + col_row(pc.sg.b, pc.sg.kvh, 0) * D,
                              G * D * (int)sizeof(T), smem_addr(bar));
             } else if (seg_first) {
@@ -688,10 +692,8 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         const int b = r / Hkv;
         if (cum[b + 1] == cum[b]) {
             const int kvh = r % Hkv, ncol = ncol_of(kvh);
-            for (int j = 0; j < ncol; ++j) {
-                T *o = reinterpret_cast<T *>(a.out) + col_row(b, kvh, j) * D;
-                for (int i = lane; i < D; i += 32) o[i] = Cvt<T>::from_f(0.f);
-            }
+            for (int j = 0; j < ncol; ++j)
+                for (int i = lane; i < D; i += 32) store_out<T>(a.out, a.out_f32, col_row(b, kvh, j) * D + i, 0.f);
         }
     }
 #pragma unroll
@@ -753,7 +755,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
     bool have = next_seg(cit, cs);
     uint32_t bq[C::KSTEPS][2];
     int c_k = 0;
-    bool alive = true;
+    bool alive = true, drained = false;
     // Pending ticket: the last partial's ticket is read one segment later, so the
     // atomic's round trip never stalls the warp.
     int pend_old = 0;
@@ -849,9 +851,9 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             if (h < ncol) {
-                T *out = reinterpret_cast<T *>(a.out) + col_row(b, kvh, h) * D;
+                const size_t o0 = col_row(b, kvh, h) * D + lane * C::DPL;
 #pragma unroll
-                for (int e = 0; e < C::DPL; ++e) out[lane * C::DPL + e] = Cvt<T>::from_f(acc[h][e]);
+                for (int e = 0; e < C::DPL; ++e) store_out<T>(a.out, a.out_f32, o0 + e, acc[h][e]);
             }
         }
         if (lane == 0) a.counters[(size_t)b * Hkv + kvh] = 0;  // the workspace is left as it was found
@@ -884,7 +886,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         pend_nb = due_nb;
     };
 
-    while (have && alive) {
+    while (have) {
         const int len = cs.j1 - cs.j0;
         const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;  // tokens in the row's last block
         // causal limits: column (query token i) sees positions < L - qlen + 1 + i;
@@ -897,14 +899,14 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
 #pragma unroll
         for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
-        for (int j = 0; j < len; ++j) {
+        for (int j = 0; alive && j < len; ++j) {
             if constexpr (kQz && PA_TC_PAIRS) {
                 if (j + 1 < len) {
                     // ---- two blocks (stages sA, sB) at once: one max/sum reduction and
                     // one rescale for both, two independent MMA streams
                     const int sA = c_k % S, sB = (c_k + 1) % S;
-                    const bool okw = __all_sync(0xffffffffu, mbar_wait(&my_bars[sA], (c_k / S) & 1) &&
-                                                                 mbar_wait(&my_bars[sB], ((c_k + 1) / S) & 1));
+                    const bool okw = __all_sync(0xffffffffu, mbar_wait(&my_bars[sA], (c_k / S) & 1, a.wait_ns) &&
+                                                                 mbar_wait(&my_bars[sB], ((c_k + 1) / S) & 1, a.wait_ns));
                     if (!okw) {
                         alive = false;
                         break;
@@ -1046,13 +1048,13 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             }
             const int s = c_k % S;
             const uint32_t parity = (c_k / S) & 1;
-            int ok = lane == 0 ? (int)mbar_wait(&my_bars[s], parity) : 0;
+            int ok = lane == 0 ? (int)mbar_wait(&my_bars[s], parity, a.wait_ns) : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) {
                 alive = false;
                 break;
             }
-            if (lane != 0) mbar_wait(&my_bars[s], parity);
+            if (lane != 0) mbar_wait(&my_bars[s], parity, a.wait_ns);
             if (j == 0) load_q(s, bq, ncol);  // the segment's q came with its first block
             const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
             const uint32_t tK = ring + s * C::STAGE;
@@ -1205,7 +1207,25 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             ++c_k;
             if (due && !pend && c_k >= due_ck + kTicketLag) take_ticket();
         }
-        if (!alive) break;
+        if (!alive) {
+            // A copy did not land within the limit (PA_EFLAG_WAIT_TIMEOUT is raised).
+            // First wait, bounded again, for the warp's copies still in flight, so that
+            // none lands in shared memory after the warp has moved on or exited.  Then
+            // this segment and every later one of the warp finish without data: a whole
+            // row writes zeros, a partial writes an empty result (o = 0, lse = -inf,
+            // weight 0 in the merge) and takes its ticket, so every row's merge still
+            // runs and the workspace counters return to zero.
+            if (!drained) {
+                if (lane == 0)
+                    for (int k = c_k; k < p_k; ++k) mbar_wait(&my_bars[k % S], (k / S) & 1, a.wait_ns);
+                __syncwarp();
+                drained = true;
+            }
+            m0 = m1 = -INFINITY;
+            l0 = l1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        }
 
         // ---- finish the segment
 #pragma unroll
@@ -1216,18 +1236,17 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
         // l == 0 only when every block of the segment was skipped (bad table entries)
         const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
         if (cs.j0 == 0 && cs.j1 == cs.nb) {  // the whole row: final output
-            T *out0 = reinterpret_cast<T *>(a.out) + col_row(cs.b, cs.kvh, h0) * D;
-            T *out1 = reinterpret_cast<T *>(a.out) + col_row(cs.b, cs.kvh, h1) * D;
+            const size_t out0 = col_row(cs.b, cs.kvh, h0) * D, out1 = col_row(cs.b, cs.kvh, h1) * D;
 #pragma unroll
             for (int i = 0; i < C::MTILES; ++i) {
                 const int d0 = dmap(i, g), d1 = d0 + 8;
                 if (h0 < ncol) {
-                    out0[d0] = Cvt<T>::from_f(o[i][0] * inv0);
-                    out0[d1] = Cvt<T>::from_f(o[i][2] * inv0);
+                    store_out<T>(a.out, a.out_f32, out0 + d0, o[i][0] * inv0);
+                    store_out<T>(a.out, a.out_f32, out0 + d1, o[i][2] * inv0);
                 }
                 if (h1 < ncol) {
-                    out1[d0] = Cvt<T>::from_f(o[i][1] * inv1);
-                    out1[d1] = Cvt<T>::from_f(o[i][3] * inv1);
+                    store_out<T>(a.out, a.out_f32, out1 + d0, o[i][1] * inv1);
+                    store_out<T>(a.out, a.out_f32, out1 + d1, o[i][3] * inv1);
                 }
             }
         } else {

@@ -19,7 +19,14 @@
 //     device (on different streams, or from different host threads without
 //     ordering) race on it: issue them in one stream order;
 //   * parameters whose workspace is larger than PA_FIXED_SCRATCH_BYTES are
-//     rejected with PA_ERR_WORKSPACE before anything is launched.
+//     rejected with PA_ERR_WORKSPACE before anything is launched;
+//   * calls with different parameters share the area safely: like every
+//     workspace, it keeps the merge counters in a fixed region at its start that
+//     no partial result ever occupies, and every call (one whose bounded wait gave
+//     up included) returns them to zero;
+//   * the device address is looked up once per device and kept for the process:
+//     after cudaDeviceReset the library must not be used again (its kernel
+//     attributes and encoded copy descriptors are per-context state as well).
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -37,8 +44,8 @@ std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices];  // device address of g_fixed_scratch per device, once set up
 
 // Device address of the fixed area on the current device; the first call per
-// device looks it up and clears it (the merge counters in it must start at zero;
-// every decode leaves them at zero again).
+// device looks it up and clears it (the merge counters at its start must start
+// at zero; every decode leaves them at zero again).
 int fixed_scratch(cudaStream_t st, void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;

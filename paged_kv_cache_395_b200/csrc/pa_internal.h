@@ -57,12 +57,28 @@ struct DecodeArgs {
     int max_parts;           // ceil(max_len / part) when part > 0
     float *ws_o;             // [B][Hq][max_parts][D]
     float *ws_lse;           // [B][Hq][max_parts]  (log2 domain)
-    int *counters;           // [B][Hkv] merge tickets, zero between calls
+    int *counters;           // [B][Hkv] merge tickets at the start of the workspace, zero
+                             // between calls
     int tc_chunk;            // tensor-core schedule: blocks per chunk, 0 = balanced auto,
                              // -1 = whole rows (one pass)
     int early;               // PA_DECODE_INPUTS_READY: read lengths, tables and q before
                              // the previous kernel on the stream has finished
+    int out_f32;             // PA_DECODE_OUT_F32: out is fp32 of q's shape
+    int stall_at;            // -1; else the first worker of the tensor-core family leaves
+                             // its stall_at-th copy unissued (pa_decode_stall_selftest)
+    unsigned long long wait_ns;  // limit of every bounded wait on a copy
 };
+
+// The tensor-core family's merge counters occupy the first kCounterBytes of every
+// split-K workspace, one int per (sequence, kernel KV head) row, whatever the
+// parameters or the family of the call; partial results always start after them.
+// So a counter never lands on memory that an earlier call with other parameters
+// filled with partial results, and a workspace shared by calls of any shape stays
+// valid.  Split-K on the tensor-core family therefore needs B * H_kv <= kCounterRows.
+constexpr int kCounterRows = PA_WORKSPACE_COUNTER_BYTES / 4;
+constexpr size_t kCounterBytes = PA_WORKSPACE_COUNTER_BYTES;
+// Default limit of a bounded wait: one second.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 // Tensor-core schedule limits: the auto schedule cuts the block stream into at
 // most kTcMaxChunks chunks (one per warp of the grid) of at least kTcMinChunk

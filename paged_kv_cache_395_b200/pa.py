@@ -3,9 +3,9 @@
 The names mirror the C ABI in ``include/pa.h``:
 
 * ``pa_reshape_and_cache``, ``pa_decode``, ``pa_decode_fixed_scratch``,
-  ``pa_block_copy``, ``pa_quantize_int8``, ``pa_quantize_int4``,
-  ``pa_append_int8``, ``pa_decode_workspace_size``, ``pa_get_error_flags``
-  take torch CUDA tensors (or raw device pointers via ``lib``), check device,
+  ``pa_decode_stall_selftest``, ``pa_block_copy``, ``pa_quantize_int8``,
+  ``pa_quantize_int4``, ``pa_append_int8``, ``pa_decode_workspace_size``,
+  ``pa_decode_algo``, ``pa_get_error_flags`` take torch CUDA tensors (or raw device pointers via ``lib``), check device,
   dtype and contiguity, and call the library on
   ``torch.cuda.current_stream()``.  Every step of the computation runs in the
   library's kernels; there is no fallback of any kind.  If ``libpa.so`` is
@@ -28,7 +28,8 @@ PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_ALIGN = -4, -5, -6, -7
 PA_F32, PA_F16, PA_BF16, PA_I8, PA_I4 = 0, 1, 2, 3, 4
 PA_ALGO_AUTO, PA_ALGO_SIMT, PA_ALGO_TENSOR = 0, 1, 2
 PA_EFLAG_BAD_BLOCK, PA_EFLAG_BAD_SLOT, PA_EFLAG_BAD_PAIR, PA_EFLAG_WAIT_TIMEOUT = 1, 2, 4, 8
-PA_DECODE_INPUTS_READY = 1
+PA_DECODE_INPUTS_READY, PA_DECODE_OUT_F32 = 1, 2
+WORKSPACE_COUNTER_BYTES = 256 * 1024  # PA_WORKSPACE_COUNTER_BYTES
 BLOCK_SIZE = 16
 
 # a uint8 cache tensor [N][H_kv][16][d/2] holds 4-bit values, two per byte
@@ -72,6 +73,9 @@ def _load():
     L.pa_decode_fixed_scratch.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), P]
     L.pa_decode_workspace_size.argtypes = [ctypes.POINTER(PaDecodeParams)]
     L.pa_decode_workspace_size.restype = ctypes.c_size_t
+    L.pa_decode_algo.argtypes = [ctypes.POINTER(PaDecodeParams), P]
+    L.pa_decode_stall_selftest.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), i32,
+                                           ctypes.c_uint64, P]
     L.pa_block_copy.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, P]
     L.pa_quantize_int8.argtypes = [P, i32, P, P, i64, i32, i32, i32, P]
     L.pa_append_int8.argtypes = [P, P, i32, P, P, P, P, P, i64, i32, i32, i32, i64, i64, i64, P]
@@ -80,8 +84,9 @@ def _load():
     L.pa_status_string.argtypes = [i32]
     L.pa_status_string.restype = ctypes.c_char_p
     L.pa_version.argtypes = []
-    for n in ("pa_reshape_and_cache", "pa_append_int8", "pa_decode", "pa_decode_fixed_scratch", "pa_block_copy",
-              "pa_quantize_int8", "pa_quantize_int4", "pa_get_error_flags", "pa_version"):
+    for n in ("pa_reshape_and_cache", "pa_append_int8", "pa_decode", "pa_decode_fixed_scratch",
+              "pa_decode_stall_selftest", "pa_decode_algo", "pa_block_copy", "pa_quantize_int8",
+              "pa_quantize_int4", "pa_get_error_flags", "pa_version"):
         getattr(L, n).restype = i32
     return L
 
@@ -89,9 +94,9 @@ def _load():
 lib = _load()
 
 # the C-ABI symbols include/pa.h declares
-EXPORTED = ("pa_reshape_and_cache", "pa_append_int8", "pa_decode_workspace_size", "pa_decode", "pa_decode_fixed_scratch",
-            "pa_block_copy", "pa_quantize_int8", "pa_quantize_int4", "pa_get_error_flags",
-            "pa_status_string", "pa_version")
+EXPORTED = ("pa_reshape_and_cache", "pa_append_int8", "pa_decode_workspace_size", "pa_decode_algo", "pa_decode",
+            "pa_decode_fixed_scratch", "pa_decode_stall_selftest", "pa_block_copy", "pa_quantize_int8",
+            "pa_quantize_int4", "pa_get_error_flags", "pa_status_string", "pa_version")
 FIXED_SCRATCH_BYTES = 32 << 20  # PA_FIXED_SCRATCH_BYTES
 
 
@@ -169,20 +174,15 @@ def make_params(q, key_cache, block_tables, max_seq_len, k_scales=None, v_scales
     return p
 
 
-def uses_tensor_cores(q, key_cache, algo=PA_ALGO_AUTO) -> bool:
-    """Whether pa_decode runs the tensor-core family for these operands (the
-    library's rule: fp16/bf16 q with a cache of the same dtype and head_dim 64 or
-    128, or fp16 q with an int8 cache and head_dim 128; at most 512 (query token,
-    head) pairs per KV head; at most 4096 sequences)."""
-    B, d = q.shape[0], q.shape[-1]
-    Hq = q.shape[-2]
-    Q = q.shape[1] if q.dim() == 4 else 1
-    Hkv = key_cache.shape[1]
-    G = Hq // Hkv
-    same = q.dtype in (torch.float16, torch.bfloat16) and key_cache.dtype == q.dtype and d in (64, 128)
-    i8 = q.dtype == torch.float16 and key_cache.dtype in (torch.int8, torch.uint8) and d == 128
-    ok = (same or i8) and Q * G <= 512 and B <= 4096
-    return algo == PA_ALGO_TENSOR or (algo == PA_ALGO_AUTO and ok)
+def pa_decode_algo(q, key_cache, block_tables, max_seq_len, partition_size=0, k_scales=None,
+                   v_scales=None, algo=PA_ALGO_AUTO) -> int:
+    """The kernel family pa_decode runs for these operands, as the library
+    reports it: PA_ALGO_TENSOR or PA_ALGO_SIMT."""
+    p = make_params(q, key_cache, block_tables, max_seq_len, k_scales, v_scales, partition_size,
+                    None, algo)
+    r = int(lib.pa_decode_algo(ctypes.byref(p), _ptr(q)))
+    _check(min(r, 0), "pa_decode_algo")
+    return r
 
 
 def pa_decode_workspace_size(q, key_cache, block_tables, max_seq_len, partition_size=0,
@@ -199,13 +199,21 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor | None:
     return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
+def _out_flag(out, q) -> int:
+    """out matches q in shape, and in dtype or is fp32 (PA_DECODE_OUT_F32)."""
+    if out.shape != q.shape or out.dtype not in (q.dtype, torch.float32):
+        raise ValueError("out must match q in shape, and in dtype or be float32")
+    return PA_DECODE_OUT_F32 if out.dtype != q.dtype else 0
+
+
 def pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max_seq_len,
               k_scales=None, v_scales=None, partition_size=0, workspace=None,
               algo=PA_ALGO_AUTO, stream=None, params=None, flags=0):
     """out, q [B][H_q][d] (or [B][Q][H_q][d]: Q new tokens per sequence, causal
     among them); caches [N][H_kv][16][d]; block_tables int32 [B][M]; seq_lens int32
     [B] (including the new tokens).  flags: 0 or PA_DECODE_INPUTS_READY (see
-    include/pa.h)."""
+    include/pa.h).  A float32 out of an fp16/bf16 q receives the fp32 result
+    before its rounding (PA_DECODE_OUT_F32 is added)."""
     _dev(out, q, key_cache, value_cache, block_tables, seq_lens, k_scales, v_scales, workspace)
     for t, n in ((out, "out"), (q, "q"), (key_cache, "key_cache"), (value_cache, "value_cache"),
                  (block_tables, "block_tables"), (seq_lens, "seq_lens")):
@@ -213,8 +221,7 @@ def pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max
             raise ValueError(f"{n} must be contiguous")
     if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
         raise ValueError("block_tables and seq_lens must be int32")
-    if out.dtype != q.dtype or out.shape != q.shape:
-        raise ValueError("out must match q in shape and dtype")
+    flags |= _out_flag(out, q)
     p = params if params is not None else make_params(
         q, key_cache, block_tables, max_seq_len, k_scales, v_scales, partition_size, workspace, algo,
         flags)
@@ -237,13 +244,26 @@ def pa_decode_fixed_scratch(out, q, key_cache, value_cache, block_tables, seq_le
             raise ValueError(f"{n} must be contiguous")
     if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
         raise ValueError("block_tables and seq_lens must be int32")
-    if out.dtype != q.dtype or out.shape != q.shape:
-        raise ValueError("out must match q in shape and dtype")
     p = make_params(q, key_cache, block_tables, max_seq_len, k_scales, v_scales, partition_size,
-                    None, algo)
+                    None, algo, _out_flag(out, q))
     _check(lib.pa_decode_fixed_scratch(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache),
                                        _ptr(block_tables), _ptr(seq_lens), ctypes.c_float(scale),
                                        ctypes.byref(p), _stream(stream)), "pa_decode_fixed_scratch")
+
+
+def pa_decode_stall_selftest(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max_seq_len,
+                             stall_at, limit_ns, partition_size=-1, workspace=None, stream=None):
+    """pa_decode on the tensor-core family with the failure path exercised: the
+    first worker leaves its stall_at-th copy unissued, so its bounded wait runs
+    out after limit_ns (see include/pa.h).  Returns after the launch; the error
+    word then holds PA_EFLAG_WAIT_TIMEOUT."""
+    _dev(out, q, key_cache, value_cache, block_tables, seq_lens, workspace)
+    p = make_params(q, key_cache, block_tables, max_seq_len, None, None, partition_size, workspace,
+                    PA_ALGO_TENSOR, _out_flag(out, q))
+    _check(lib.pa_decode_stall_selftest(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache),
+                                        _ptr(block_tables), _ptr(seq_lens), ctypes.c_float(scale),
+                                        ctypes.byref(p), int(stall_at), int(limit_ns), _stream(stream)),
+           "pa_decode_stall_selftest")
 
 
 def pa_block_copy(key_cache, value_cache, pairs, k_scales=None, v_scales=None, stream=None):

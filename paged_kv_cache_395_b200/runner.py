@@ -92,7 +92,9 @@ class DeviceWorkload:
         return pa.alloc_workspace(n, self.device)
 
     def run(self, op, partition_size=0, workspace=None, int8=False, algo=pa.PA_ALGO_AUTO,
-            stream=None):
+            stream=None, out_f32=False):
+        """out_f32: decode into a new float32 tensor (the fp32 result before the
+        output's rounding) instead of the step's own output."""
         kind = op[0]
         if kind == "reshape":
             _, k, v, s = op
@@ -102,6 +104,8 @@ class DeviceWorkload:
                 pa.pa_block_copy(self.kc, self.vc, op[1], stream=stream)
         else:
             _, q, bt, sl, mx, out = op
+            if out_f32:
+                out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
             if workspace is None and partition_size != 0:
                 workspace = self.workspace_for(op, partition_size, int8, algo)
             kc, vc = (self.kc8, self.vc8) if int8 else (self.kc, self.vc)
@@ -114,15 +118,21 @@ class DeviceWorkload:
         for op in self.setup:
             self.run(op)
 
-    def run_step(self, i, partition_size=0, int8=False, algo=pa.PA_ALGO_AUTO, decode=True):
+    def run_step(self, i, partition_size=0, int8=False, algo=pa.PA_ALGO_AUTO, decode=True,
+                 out_f32=False):
         out = None
         for op in self.steps[i]:
             if op[0] == "decode":
                 if decode:
-                    out = self.run(op, partition_size, None, int8, algo)
+                    out = self.run(op, partition_size, None, int8, algo, out_f32=out_f32)
             else:
                 self.run(op)
         return out
+
+    def decode_again(self, i, partition_size=0, int8=False, algo=pa.PA_ALGO_AUTO, out_f32=False):
+        """Repeat step i's decode alone (its appends already ran)."""
+        op = [o for o in self.steps[i] if o[0] == "decode"][0]
+        return self.run(op, partition_size, None, int8, algo, out_f32=out_f32)
 
 
 class StepCalls:
@@ -178,7 +188,7 @@ class StepCalls:
                     split = pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
                     # the tensor-core family merges inside its decode kernel; the
                     # CUDA-core family launches a merge kernel after a split decode
-                    tc = pa.uses_tensor_cores(q, kc, algo)
+                    tc = pa.lib.pa_decode_algo(ctypes.byref(p), ptr(q)) == pa.PA_ALGO_TENSOR
                     args = (ptr(out), ptr(q), ptr(kc), ptr(vc), ptr(bt), ptr(sl),
                             ctypes.c_float(w.scale), ctypes.byref(p), sp)
                     calls.append(("decode", pa.lib.pa_decode, args))

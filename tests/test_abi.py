@@ -71,7 +71,7 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails val
     (dict(q_dtype=9), pa.PA_ERR_DTYPE),
     (dict(partition_size=24), pa.PA_ERR_SHAPE),
     (dict(partition_size=-2), pa.PA_ERR_SHAPE),
-    (dict(flags=2), pa.PA_ERR_UNSUPPORTED),          # unknown flag bit
+    (dict(flags=4), pa.PA_ERR_UNSUPPORTED),          # unknown flag bit
     (dict(num_q_heads=1024, num_kv_heads=1), pa.PA_ERR_UNSUPPORTED),  # G = 1024
     (dict(head_dim=256, q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32), pa.PA_ERR_UNSUPPORTED),
     (dict(num_seqs=-1), pa.PA_ERR_SHAPE),
@@ -95,27 +95,29 @@ def test_decode_null_and_workspace_checks():
     assert rc == pa.PA_ERR_NULL
     p = params(partition_size=16, algo=pa.PA_ALGO_SIMT)  # split-K without a workspace
     need = pa.lib.pa_decode_workspace_size(ctypes.byref(p))
-    # CUDA-core family: 2 seqs x 8 heads x 4 partitions x 128 floats, their 64 lse
-    # floats and 2 x 2 merge counters, each region rounded up to 256 B
-    assert need == 2 * 8 * 4 * 128 * 4 + 256 + 256
+    # CUDA-core family: the fixed merge-counter region (kept free in every workspace),
+    # then 2 seqs x 8 heads x 4 partitions x 128 floats and their 64 lse floats,
+    # each region rounded up to 256 B
+    C = pa.WORKSPACE_COUNTER_BYTES
+    assert need == C + 2 * 8 * 4 * 128 * 4 + 256
     rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
     assert rc == pa.PA_ERR_WORKSPACE
     p.workspace, p.workspace_bytes = 0x1000, need - 1
     rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
     assert rc == pa.PA_ERR_WORKSPACE
-    # tensor-core family: 2 x 2 rows x 4 blocks = 16 blocks in chunks of 1 block ->
-    # 32 partial slots of 4 heads x (128 + 1) floats, plus the counters
+    # tensor-core family: the counters, then 2 x 2 rows x 4 blocks = 16 blocks in
+    # chunks of 1 block -> 32 partial slots of 4 heads x (128 + 1) floats
     p = params(partition_size=16, algo=pa.PA_ALGO_TENSOR)
-    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == 32 * 4 * 128 * 4 + 512 + 256
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == C + 32 * 4 * 128 * 4 + 512
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(params(partition_size=0, algo=pa.PA_ALGO_TENSOR))) == 0
-    # auto schedule on the tensor-core family: at most 2048 chunks (one per warp),
-    # two partial slots each; then 64 x 2 row tickets
+    # auto schedule on the tensor-core family: the counters, then at most 2048 chunks
+    # (one per warp), two partial slots each
     p = params(partition_size=-1, algo=pa.PA_ALGO_TENSOR, num_seqs=64, max_blocks_per_seq=264,
                max_seq_len=4224)
     slots = 2 * 2048
     up = lambda x: (x + 255) // 256 * 256
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == \
-        up(slots * 4 * 128 * 4) + up(slots * 4 * 4) + up(64 * 2 * 4)
+        C + up(slots * 4 * 128 * 4) + up(slots * 4 * 4)
     # the tensor-core family needs fp16/bf16 q and cache
     p = params(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p),
@@ -198,3 +200,58 @@ def test_multi_query_and_padded_groups_are_planned():
     a = params(query_len=2, num_q_heads=8, num_kv_heads=2, partition_size=16, algo=pa.PA_ALGO_TENSOR)
     b = params(num_q_heads=16, num_kv_heads=2, partition_size=16, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(a)) == pa.lib.pa_decode_workspace_size(ctypes.byref(b))
+
+
+def test_decode_algo_reports_the_family():
+    """pa_decode_algo returns the family pa_decode would run (host only, q not read)."""
+    q16, q8 = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1008)
+    algo = lambda p, q=q16: pa.lib.pa_decode_algo(ctypes.byref(p), q)  # noqa: E731
+    assert algo(params()) == pa.PA_ALGO_TENSOR
+    assert algo(params(algo=pa.PA_ALGO_SIMT)) == pa.PA_ALGO_SIMT
+    assert algo(params(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32)) == pa.PA_ALGO_SIMT
+    assert algo(params(head_dim=256)) == pa.PA_ALGO_SIMT
+    assert algo(params(kv_dtype=pa.PA_I8, q_dtype=pa.PA_BF16)) == pa.PA_ALGO_SIMT
+    assert algo(params(kv_dtype=pa.PA_I8)) == pa.PA_ALGO_TENSOR
+    # a q that is not 16-byte aligned goes to the CUDA-core family, or is refused
+    assert algo(params(), q8) == pa.PA_ALGO_SIMT
+    assert algo(params(algo=pa.PA_ALGO_TENSOR), q8) == pa.PA_ERR_ALIGN
+    assert algo(params(head_dim=96)) == pa.PA_ERR_UNSUPPORTED
+    assert algo(params(flags=pa.PA_DECODE_OUT_F32 | pa.PA_DECODE_INPUTS_READY)) == pa.PA_ALGO_TENSOR
+
+
+def test_counter_region_bounds_the_tensor_core_split():
+    """The tensor-core family's split keeps one merge counter per (sequence, KV
+    head) row in the fixed counter region: beyond its 65536 rows the library-picked
+    schedule runs in one pass (no workspace), an explicit split goes to the
+    CUDA-core family, and the tensor-core family refuses it."""
+    rows = pa.WORKSPACE_COUNTER_BYTES // 4
+    assert rows == 4096 * 16
+    fit = params(num_seqs=4096, num_q_heads=64, num_kv_heads=16, partition_size=-1,
+                 max_blocks_per_seq=64, max_seq_len=1024)
+    over = params(num_seqs=4096, num_q_heads=128, num_kv_heads=32, partition_size=-1,
+                  max_blocks_per_seq=64, max_seq_len=1024)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(fit)) > 0
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(over)) == 0
+    assert pa.lib.pa_decode_algo(ctypes.byref(over), ctypes.c_void_p(0x1000)) == pa.PA_ALGO_TENSOR
+    over.partition_size = 256
+    assert pa.lib.pa_decode_algo(ctypes.byref(over), ctypes.c_void_p(0x1000)) == pa.PA_ALGO_SIMT
+    over.algo = pa.PA_ALGO_TENSOR
+    assert pa.lib.pa_decode_algo(ctypes.byref(over), ctypes.c_void_p(0x1000)) == pa.PA_ERR_UNSUPPORTED
+
+
+def test_stall_selftest_rejects_bad_args():
+    """The failure-path self-test validates like pa_decode, needs a stage index
+    and a positive limit, and runs only on the tensor-core family."""
+    L = pa.lib
+    p = params()
+    f = ctypes.c_float(0.1)
+    assert L.pa_decode_stall_selftest(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f, ctypes.byref(p), -1, 1000, None) \
+        == pa.PA_ERR_SHAPE
+    assert L.pa_decode_stall_selftest(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f, ctypes.byref(p), 0, 0, None) \
+        == pa.PA_ERR_SHAPE
+    p = params(head_dim=96)
+    assert L.pa_decode_stall_selftest(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f, ctypes.byref(p), 0, 1000, None) \
+        == pa.PA_ERR_UNSUPPORTED
+    p = params(algo=pa.PA_ALGO_SIMT)
+    assert L.pa_decode_stall_selftest(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f, ctypes.byref(p), 0, 1000, None) \
+        == pa.PA_ERR_UNSUPPORTED

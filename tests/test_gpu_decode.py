@@ -3,7 +3,10 @@
 Every case runs through the C ABI (paged_kv_cache_395_b200.pa).  Tolerance:
 |err| <= 2e-3 + 2e-3 |ref| for fp16/bf16 outputs (fp32 accumulation), and
 1e-5 + 1e-5 |ref| for the fp32 case; int8 caches are compared with the oracle
-dequantising the same int8 values and scales in fp64.
+dequantising the same int8 values and scales in fp64.  A bf16 case checks that
+bound on the fp32 result before the output's rounding (the same call with a
+float32 out) and that the bf16 output is that result rounded to nearest even
+(gpu_util.check_bf16).
 """
 import numpy as np
 import pytest
@@ -12,7 +15,7 @@ import torch
 import oracle
 from paged_kv_cache_395_b200 import pa, runner, workloads as W
 
-from .gpu_util import assert_close, bits
+from .gpu_util import assert_close, bits, check_bf16
 from .oracle_replay import replay
 
 pytestmark = pytest.mark.gpu
@@ -31,6 +34,16 @@ def _clear_flags():
     pa.pa_get_error_flags(reset=True)
     yield
     assert pa.pa_get_error_flags(reset=True) == 0
+
+
+def check(got, ref, dtype, what, dw, part, algo, int8=False, rows=None):
+    """The oracle comparison of step 0's output; a bf16 output is checked with its
+    fp32 result, which a second decode of the same step (into a float32 out) gives."""
+    if dtype != "bfloat16":
+        return assert_close(got, ref, dtype, what, rows=rows)
+    f32 = dw.decode_again(0, part, int8=int8, algo=algo, out_f32=True)
+    torch.cuda.synchronize()
+    check_bf16(got, f32, ref, what, rows=rows)
 
 
 def run_gpu(w, partition_size=0, algo=pa.PA_ALGO_AUTO, int8=False, dw=None):
@@ -81,8 +94,8 @@ def test_random_cases(case, part, algo):
         pytest.skip("fp32 has no tensor-core path")
     w = W.random_case(seed=sorted(CASES).index(case) + 100, **CASES[case])
     ref, _, _ = replay(w)
-    got, _ = run_gpu(w, part, algo)
-    assert_close(got[0], ref[0], w.dtype, case)
+    got, dw = run_gpu(w, part, algo)
+    check(got[0], ref[0], w.dtype, case, dw, part, algo)
 
 
 @pytest.mark.parametrize("algo", ALGOS)
@@ -100,7 +113,7 @@ def test_int8_random(qdt, part, algo):
     ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
     op = w.steps[0][0]
     ref = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
-    assert_close(got[0], ref, qdt, "int8")
+    check(got[0], ref, qdt, "int8", dw, part, algo, int8=True)
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 4), (32, 8)])
@@ -155,9 +168,9 @@ def test_workspace_reused_across_calls():
         pa.pa_decode(out, q, dw.kc, dw.vc, bt, sl, w.scale, mx, partition_size=32, workspace=ws,
                      algo=pa.PA_ALGO_TENSOR)
         assert_close(out, ref[0], "float16", "reuse")
-    # the last region holds the 3 x 8 merge counters (rounded up to 256 bytes)
+    # the first region holds the merge counters
     torch.cuda.synchronize()
-    assert ws[-256:].count_nonzero().item() == 0
+    assert ws[:pa.WORKSPACE_COUNTER_BYTES].count_nonzero().item() == 0
 
 
 def test_zero_length_and_empty_batch():
@@ -405,13 +418,13 @@ def test_large_group_bf16_and_int8(qdt):
     w = W.random_case([7, 129, 640], num_q_heads=64, num_kv_heads=1, head_dim=128, dtype=qdt, seed=77)
     ref, _, _ = replay(w)
     got, dw = run_gpu(w, -1)
-    assert_close(got[0], ref[0], qdt, "MQA G=64")
+    check(got[0], ref[0], qdt, "MQA G=64", dw, -1, pa.PA_ALGO_AUTO)
     got8, dw = run_gpu(w, -1, int8=True, dw=runner.DeviceWorkload(w))
     kc8, vc8 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
     ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
     op = w.steps[0][0]
     ref8 = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
-    assert_close(got8[0], ref8, qdt, "MQA G=64 int8")
+    check(got8[0], ref8, qdt, "MQA G=64 int8", dw, -1, pa.PA_ALGO_AUTO, int8=True)
 
 
 @pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
@@ -422,8 +435,8 @@ def test_head_dim_256(qdt, hq, hkv, part):
     w = W.random_case([1, 17, 200, 513], num_q_heads=hq, num_kv_heads=hkv, head_dim=256, dtype=qdt,
                       seed=hq + hkv + 256)
     ref, _, _ = replay(w)
-    got, _ = run_gpu(w, part)
-    assert_close(got[0], ref[0], qdt, f"d=256 G={hq // hkv} part={part}")
+    got, dw = run_gpu(w, part)
+    check(got[0], ref[0], qdt, f"d=256 G={hq // hkv} part={part}", dw, part, pa.PA_ALGO_AUTO)
 
 
 def test_head_dim_256_int8():
@@ -480,9 +493,9 @@ def test_multi_query(qdt, hq, hkv, Q, part):
     w = W.random_multi_case(lens, Q, num_q_heads=hq, num_kv_heads=hkv, head_dim=128, dtype=qdt,
                             seed=hq * 10 + hkv + Q)
     ref, _, _ = replay(w)
-    got, _ = run_gpu(w, part, pa.PA_ALGO_TENSOR)
+    got, dw = run_gpu(w, part, pa.PA_ALGO_TENSOR)
     assert got[0].shape == (len(lens), Q, hq, 128)
-    assert_close(got[0], ref[0], qdt, f"Q={Q} G={hq // hkv} part={part}")
+    check(got[0], ref[0], qdt, f"Q={Q} G={hq // hkv} part={part}", dw, part, pa.PA_ALGO_TENSOR)
 
 
 def test_multi_query_int8_and_d64():
@@ -497,8 +510,8 @@ def test_multi_query_int8_and_d64():
     w = W.random_multi_case([7, 64, 129], 3, num_q_heads=4, num_kv_heads=2, head_dim=64,
                             dtype="bfloat16", seed=32)
     ref, _, _ = replay(w)
-    got, _ = run_gpu(w, 16)
-    assert_close(got[0], ref[0], "bfloat16", "multi d=64")
+    got, dw = run_gpu(w, 16)
+    check(got[0], ref[0], "bfloat16", "multi d=64", dw, 16, pa.PA_ALGO_AUTO)
 
 
 @pytest.mark.slow
@@ -570,3 +583,90 @@ def test_int4_rejected_off_its_path():
         pa.pa_decode(out, q, dw.kc8, dw.vc8, bt, sl, w.scale, mx, dw.k_scales, dw.v_scales,
                      algo=pa.PA_ALGO_SIMT)
     assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
+# -- one workspace across calls of any shape; the failure path of the bounded waits ---------
+def _oracle_ref(w, dw, int8=False):
+    op = w.steps[0][0]
+    if int8:
+        return oracle.decode(op.q, dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy(), op.block_tables,
+                             op.seq_lens, w.scale, dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy())
+    return oracle.decode(op.q, dw.kc.cpu().numpy(), dw.vc.cpu().numpy(), op.block_tables, op.seq_lens,
+                         w.scale)
+
+
+def test_workspace_shared_across_parameter_sets():
+    """One workspace, zero-filled once, serves calls whose parameters differ:
+    a 6-sequence batch split into 16-token partitions, a 3-sequence batch with
+    256-token partitions, the CUDA-core family's split (whose partial results
+    land where the tensor-core family's counters would be without the fixed
+    counter region), MQA rows, and the first call again; each against the oracle."""
+    wa = W.random_case([1, 40, 300, 777, 1500, 2047], num_q_heads=32, num_kv_heads=8, head_dim=128, seed=81)
+    wb = W.random_case([900, 3000, 20], num_q_heads=16, num_kv_heads=2, head_dim=128, seed=82)
+    wc = W.random_case([64, 1000, 513, 2], num_q_heads=32, num_kv_heads=1, head_dim=128, seed=83)
+    runs = []
+    for w in (wa, wb, wc):
+        dw = runner.DeviceWorkload(w)
+        dw.run_setup()
+        runs.append((w, dw, _oracle_ref(w, dw)))
+    calls = [(0, 16, pa.PA_ALGO_TENSOR), (1, 256, pa.PA_ALGO_TENSOR), (0, 32, pa.PA_ALGO_SIMT),
+             (1, 16, pa.PA_ALGO_TENSOR), (2, -1, pa.PA_ALGO_TENSOR), (1, 64, pa.PA_ALGO_SIMT),
+             (0, 16, pa.PA_ALGO_TENSOR), (2, 16, pa.PA_ALGO_TENSOR), (0, -1, pa.PA_ALGO_AUTO)]
+    need = 0
+    for k, part, algo in calls:
+        w, dw, _ = runs[k]
+        _, q, bt, _, mx, _ = dw.steps[0][-1]
+        need = max(need, pa.pa_decode_workspace_size(q, dw.kc, bt, mx, part, algo=algo))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for n, (k, part, algo) in enumerate(calls):
+        w, dw, ref = runs[k]
+        _, q, bt, sl, mx, _ = dw.steps[0][-1]
+        out = torch.full_like(q, float("nan"))
+        pa.pa_decode(out, q, dw.kc, dw.vc, bt, sl, w.scale, mx, partition_size=part, workspace=ws, algo=algo)
+        assert_close(out, ref, "float16", f"call {n}: case {k} part={part} algo={algo}")
+    torch.cuda.synchronize()
+    assert ws[:pa.WORKSPACE_COUNTER_BYTES].count_nonzero().item() == 0
+
+
+@pytest.mark.parametrize("stall_at", [0, 3])
+def test_wait_timeout_reported_and_workspace_left_ready(stall_at):
+    """The failure path of the bounded waits on a working GPU, without a fault:
+    the first worker of the tensor-core family leaves one of its copies
+    unissued, so its wait for that stage runs out after 5 ms.  The call returns,
+    the host reads PA_EFLAG_WAIT_TIMEOUT, every row the worker did not touch still
+    matches the oracle, the merge counters are back at zero, and the next decode
+    on the same workspace matches the oracle on every row."""
+    lens = [1000, 3000, 500]
+    w = W.random_case(lens, num_q_heads=32, num_kv_heads=8, head_dim=128, seed=91)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    ref = _oracle_ref(w, dw)
+    _, q, bt, sl, mx, _ = dw.steps[0][-1]
+    ws = dw.workspace_for(dw.steps[0][-1], -1, algo=pa.PA_ALGO_TENSOR)
+    out = torch.full_like(q, float("nan"))
+    pa.pa_get_error_flags(reset=True)
+    limit_ns = 5_000_000
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    pa.pa_decode_stall_selftest(out, q, dw.kc, dw.vc, bt, sl, w.scale, mx, stall_at, limit_ns,
+                                partition_size=-1, workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    assert a.elapsed_time(b) >= limit_ns / 1e6  # the wait ran its whole limit, then gave up
+    assert pa.pa_get_error_flags(reset=True) == pa.PA_EFLAG_WAIT_TIMEOUT
+    assert ws[:pa.WORKSPACE_COUNTER_BYTES].count_nonzero().item() == 0
+    # the stream's first 8-block chunk (the first worker's) lies in sequence 0, KV head 0:
+    # query heads 0-3 of sequence 0; every other row is untouched by the failure
+    got = out.double().cpu().numpy()
+    keep = np.ones(got.shape[:2], dtype=bool)
+    keep[0, 0:4] = False
+    assert np.all(np.isfinite(got))
+    rows = np.argwhere(keep)
+    assert_close(out, ref, "float16", "rows away from the stalled worker", rows=rows)
+    # the workspace serves the next call unchanged
+    out2 = torch.full_like(q, float("nan"))
+    pa.pa_decode(out2, q, dw.kc, dw.vc, bt, sl, w.scale, mx, partition_size=-1, workspace=ws,
+                 algo=pa.PA_ALGO_TENSOR)
+    assert_close(out2, ref, "float16", "next call")
+    torch.cuda.synchronize()
+    assert ws[:pa.WORKSPACE_COUNTER_BYTES].count_nonzero().item() == 0

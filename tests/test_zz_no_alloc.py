@@ -1,10 +1,11 @@
 """pa_decode_fixed_scratch (split-K decode on the library's fixed scratch area)
-against pa_decode with a caller-allocated workspace.
+against pa_decode with a caller-allocated workspace, and against the oracle.
 
 The file name sorts last so that, in a full run, these calls come after every
 other test has used the device; the tests also pass when run alone.  Two calls
 in a row check that a call leaves the fixed area ready for the next one (its
-merge counters back at zero).
+merge counters back at zero); calls with different parameters in a row check
+that the counters' place does not move with the parameters.
 """
 import numpy as np
 import pytest
@@ -12,7 +13,8 @@ import torch
 
 from paged_kv_cache_395_b200 import pa, runner, workloads as W
 
-from .gpu_util import TOL, gpu_f64
+from .gpu_util import TOL, assert_close, gpu_f64
+from .oracle_replay import replay
 
 pytestmark = pytest.mark.gpu
 
@@ -91,3 +93,39 @@ def test_fixed_scratch_rejects_oversized_request():
     assert e.value.status == pa.PA_ERR_WORKSPACE
     torch.cuda.synchronize()
     assert torch.count_nonzero(out) == 0
+
+
+def test_fixed_scratch_alternating_parameter_sets():
+    """Calls with different parameters in a row share the fixed area: a ragged
+    7-sequence batch split into 16-token partitions, then a 3-sequence batch with
+    256-token partitions, the CUDA-core family's split (its partial results start
+    at the same offset as the tensor-core family's), and the first case again.
+    Each call against pa_decode with a fresh zeroed workspace and against the
+    oracle."""
+    cases = [
+        (W.random_case([1, 16, 17, 100, 513, 1000, 2047], num_q_heads=32, num_kv_heads=8, head_dim=128,
+                       dtype="float16", seed=60), 16, pa.PA_ALGO_TENSOR),
+        (W.random_case([900, 3000, 20], num_q_heads=16, num_kv_heads=2, head_dim=128, dtype="float16",
+                       seed=61), 256, pa.PA_ALGO_TENSOR),
+        (W.random_case([700, 64, 1500], num_q_heads=8, num_kv_heads=2, head_dim=128, dtype="float16",
+                       seed=62), 128, pa.PA_ALGO_SIMT),
+    ]
+    prepared = []
+    for w, part, algo in cases:
+        dw = runner.DeviceWorkload(w)
+        dw.run_setup()
+        ref, _, _ = replay(w)
+        prepared.append((w, dw, ref[0], part, algo))
+    torch.cuda.synchronize()
+    for n, k in enumerate([0, 1, 2, 0, 1, 0]):
+        w, dw, ref, part, algo = prepared[k]
+        _, q, bt, sl, mx, _ = dw.steps[0][-1]
+        fresh = torch.empty_like(q)
+        ws = dw.workspace_for(dw.steps[0][-1], part, algo=algo)
+        pa.pa_decode(fresh, q, dw.kc, dw.vc, bt, sl, w.scale, mx, None, None, part, ws, algo)
+        o = torch.full_like(q, float("nan"))
+        pa.pa_decode_fixed_scratch(o, q, dw.kc, dw.vc, bt, sl, w.scale, mx, None, None, part, algo)
+        torch.cuda.synchronize()
+        _close(o, fresh, "float16", f"call {n} (case {k}) vs pa_decode")
+        assert_close(o, ref, "float16", f"call {n} (case {k}) vs oracle")
+    assert pa.pa_get_error_flags(reset=True) == 0
