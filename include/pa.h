@@ -95,6 +95,27 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
                          int head_dim, int block_size, int64_t num_blocks, int dtype,
                          int64_t k_token_stride, int64_t v_token_stride, pa_stream_t stream);
 
+/*
+ * pa_reshape_and_cache with flags: 0, or PA_APPEND_OVERLAP_PREVIOUS.
+ *
+ * PA_APPEND_OVERLAP_PREVIOUS: the caller guarantees that no kernel still running
+ * before this call on `stream` reads or writes any slot this call writes -- for
+ * example a decode engine that puts the blocks of sequences finished after a
+ * decode step back on its free list only one step later, so a step's appends
+ * never land in a block the previous step's decode reads (slots past a
+ * sequence's length are never part of its result).  The copies then run while
+ * the previous kernel finishes, and the next kernel may launch at once; the call
+ * still completes only after the previous kernel has, so a kernel that waits for
+ * this one finds every earlier one complete.  Without the guarantee the result
+ * of the previous kernel is undefined.  (No counterpart in the pages: it hides
+ * the append's latency behind the decode before it.)
+ */
+#define PA_APPEND_OVERLAP_PREVIOUS 1
+int pa_reshape_and_cache_ex(const void *k, const void *v, void *key_cache, void *value_cache,
+                            const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
+                            int head_dim, int block_size, int64_t num_blocks, int dtype,
+                            int64_t k_token_stride, int64_t v_token_stride, int flags, pa_stream_t stream);
+
 typedef struct pa_decode_params {
     int num_seqs;            /* B >= 0 */
     int num_q_heads;         /* H_q, a multiple of num_kv_heads */

@@ -14,6 +14,12 @@ therefore writes in place.
 
 The free list is a LIFO stack.  ``free_order`` fixes which blocks are handed
 out first, so a seeded permutation scatters sequences across the pool.
+
+Deferred reuse (``free_sequence(..., defer=True)``, then ``release_deferred()``):
+the blocks of a sequence that ends after a decode step are held back until the
+caller releases them, one step later.  A step's appends then never write a block
+that the previous step's decode may still be reading, which lets the library
+run those appends while that decode finishes (PA_APPEND_OVERLAP_PREVIOUS).
 """
 from __future__ import annotations
 
@@ -36,6 +42,7 @@ class BlockManager:
         # pop() takes from the end, so the first block to hand out goes last.
         self._free: list[int] = [int(b) for b in order[::-1]]
         self.refcount = np.zeros(num_blocks, dtype=np.int64)
+        self._deferred: list[int] = []  # freed, not yet back on the free list
         self.tables: dict[object, list[int]] = {}
         self.lens: dict[object, int] = {}
 
@@ -109,10 +116,25 @@ class BlockManager:
         self.lens[seq_id] = n + 1
         return int(slot), cow
 
-    def free_sequence(self, seq_id) -> None:
+    def free_sequence(self, seq_id, defer: bool = False) -> None:
+        """Drop the sequence; with ``defer`` its blocks whose reference count falls
+        to zero wait for release_deferred() before they can be handed out again."""
         for b in self.tables.pop(seq_id):
-            self._release(b)
+            if defer:
+                if self.refcount[b] <= 0:
+                    raise RuntimeError(f"double free of block {b}")
+                self.refcount[b] -= 1
+                if self.refcount[b] == 0:
+                    self._deferred.append(int(b))
+            else:
+                self._release(b)
         del self.lens[seq_id]
+
+    def release_deferred(self) -> None:
+        """Put the blocks held back by free_sequence(defer=True) on the free list
+        (in the order they were freed, as an immediate free would have)."""
+        self._free.extend(self._deferred)
+        self._deferred = []
 
     def slots(self, seq_id, start: int, stop: int) -> np.ndarray:
         table = np.asarray(self.tables[seq_id], dtype=np.int64)
@@ -140,7 +162,7 @@ class BlockManager:
                 refs[b] += 1
         if not np.array_equal(refs, self.refcount):
             raise AssertionError("reference counts disagree with block tables")
-        free = np.asarray(self._free, dtype=np.int64)
+        free = np.asarray(self._free + self._deferred, dtype=np.int64)
         if len(set(free.tolist())) != len(free):
             raise AssertionError("block on the free list twice")
         if np.any(self.refcount[free] != 0):

@@ -208,6 +208,15 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
                          const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
                          int head_dim, int block_size, int64_t num_blocks, int dtype,
                          int64_t k_token_stride, int64_t v_token_stride, pa_stream_t stream) {
+    return pa_reshape_and_cache_ex(k, v, key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                   block_size, num_blocks, dtype, k_token_stride, v_token_stride, 0, stream);
+}
+
+int pa_reshape_and_cache_ex(const void *k, const void *v, void *key_cache, void *value_cache,
+                            const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
+                            int head_dim, int block_size, int64_t num_blocks, int dtype,
+                            int64_t k_token_stride, int64_t v_token_stride, int flags, pa_stream_t stream) {
+    if (flags & ~PA_APPEND_OVERLAP_PREVIOUS) return PA_ERR_UNSUPPORTED;
     if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0) return PA_ERR_SHAPE;
     if (block_size != PA_BLOCK_SIZE) return PA_ERR_UNSUPPORTED;
     const int E = elem_size(dtype);
@@ -220,7 +229,7 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
     if (num_tokens > 2147483647LL) return PA_ERR_UNSUPPORTED;
     return launch_reshape_and_cache(k, v, key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads,
                                     head_dim, num_blocks, E, k_token_stride, v_token_stride,
-                                    (cudaStream_t)stream);
+                                    (flags & PA_APPEND_OVERLAP_PREVIOUS) ? 1 : 0, (cudaStream_t)stream);
 }
 
 int pa_block_copy(void *key_cache, void *value_cache, float *k_scales, float *v_scales,

@@ -16,14 +16,19 @@ PA_ERROR_WORD_ACCESSOR(error_word_cache_ops)
 // Grid: (num_tokens, 2) -- y selects K or V.  Each CTA copies the H_kv rows of
 // one token with VEC-byte accesses.
 // ---------------------------------------------------------------------------
+//
+// overlap (PA_APPEND_OVERLAP_PREVIOUS): the caller guarantees that no kernel still
+// running before this one reads or writes the slots written here.  The next kernel
+// may then launch at once and the copies run while the previous kernel finishes;
+// CTA (0, 0) waits for the previous kernel before it exits, so this grid still
+// completes after it and a kernel that waits for this one finds every earlier one
+// complete.
 template <int VEC>
-__global__ void __launch_bounds__(256) reshape_and_cache_kernel(
+__device__ __forceinline__ void reshape_and_cache_body(
     const char *__restrict__ k, const char *__restrict__ v, char *__restrict__ kc,
     char *__restrict__ vc, const int64_t *__restrict__ slots, int num_kv_heads, int row_bytes,
     int64_t k_stride_bytes, int64_t v_stride_bytes, int64_t num_slots) {
     using V = typename VecT<VEC>::type;
-    pdl_wait();  // the previous kernel may still read the slots this one overwrites
-    pdl_release_dependents();
     const int64_t i = blockIdx.x;
     const bool is_v = blockIdx.y != 0;
     const char *src = (is_v ? v : k) + i * (is_v ? v_stride_bytes : k_stride_bytes);
@@ -52,9 +57,21 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     }
 }
 
+template <int VEC>
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(
+    const char *__restrict__ k, const char *__restrict__ v, char *__restrict__ kc,
+    char *__restrict__ vc, const int64_t *__restrict__ slots, int num_kv_heads, int row_bytes,
+    int64_t k_stride_bytes, int64_t v_stride_bytes, int64_t num_slots, int overlap) {
+    if (!overlap) pdl_wait();  // the previous kernel may still read the slots this one overwrites
+    pdl_release_dependents();
+    reshape_and_cache_body<VEC>(k, v, kc, vc, slots, num_kv_heads, row_bytes, k_stride_bytes, v_stride_bytes,
+                                num_slots);
+    if (overlap && blockIdx.x == 0 && blockIdx.y == 0) pdl_wait();
+}
+
 int launch_reshape_and_cache(const void *k, const void *v, void *kc, void *vc,
                              const int64_t *slots, int64_t T, int H, int D, int64_t N, int E,
-                             int64_t k_stride, int64_t v_stride, cudaStream_t st) {
+                             int64_t k_stride, int64_t v_stride, int overlap, cudaStream_t st) {
     if (T == 0) return PA_OK;
     const int row = D * E;
     const int64_t ksb = k_stride * E, vsb = v_stride * E;
@@ -70,11 +87,11 @@ int launch_reshape_and_cache(const void *k, const void *v, void *kc, void *vc,
     const int64_t ns = N * kBlockSize;
     cudaError_t e;
     switch (vec) {
-    case 16: e = launch_pdl(reshape_and_cache_kernel<16>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
-    case 8: e = launch_pdl(reshape_and_cache_kernel<8>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
-    case 4: e = launch_pdl(reshape_and_cache_kernel<4>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
-    case 2: e = launch_pdl(reshape_and_cache_kernel<2>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
-    default: e = launch_pdl(reshape_and_cache_kernel<1>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns); break;
+    case 16: e = launch_pdl(reshape_and_cache_kernel<16>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns, overlap); break;
+    case 8: e = launch_pdl(reshape_and_cache_kernel<8>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns, overlap); break;
+    case 4: e = launch_pdl(reshape_and_cache_kernel<4>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns, overlap); break;
+    case 2: e = launch_pdl(reshape_and_cache_kernel<2>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns, overlap); break;
+    default: e = launch_pdl(reshape_and_cache_kernel<1>, grid, dim3(threads), 0, st, kp, vp, kcp, vcp, slots, H, row, ksb, vsb, ns, overlap); break;
     }
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -161,7 +161,11 @@ struct U4x2 {
 template <typename TKV, int D, int G>
 struct TcCfg {
     static constexpr bool I4 = std::is_same<TKV, U4x2>::value;
-    static constexpr int NW = PA_TC_WARPS;        // warps (independent workers) per CTA
+    // warps (independent workers) per CTA, and CTAs per SM the registers are sized
+    // for.  A head_dim-256 stage is 16 KB (K and V tiles of 8 KB), so two stages per
+    // warp and three warps per CTA keep two CTAs (six warps, 192 KB in flight) on an SM.
+    static constexpr int NW = D == 256 ? 3 : PA_TC_WARPS;
+    static constexpr int MIN_CTAS = D == 256 ? 2 : PA_TC_MIN_CTAS;
     static constexpr int THREADS = NW * 32;
     static constexpr int ROW_BYTES = I4 ? D / 2 : 128;              // bytes per box row
     static constexpr int BOXW = I4 ? D / 2 : 128 / (int)sizeof(TKV);  // TMA elements per box row
@@ -251,6 +255,19 @@ template <> struct FVec<4> {
     using type = float4;
     static __device__ __forceinline__ float4 ld(const float *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
     static __device__ __forceinline__ float get(const float4 &v, int e) { return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w; }
+};
+template <> struct FVec<8> {
+    struct type {
+        float4 a, b;
+    };
+    static __device__ __forceinline__ type ld(const float *p) {
+        return {__ldcg(reinterpret_cast<const float4 *>(p)), __ldcg(reinterpret_cast<const float4 *>(p) + 1)};
+    }
+    static __device__ __forceinline__ float get(const type &v, int e) {
+        const float4 &h = e < 4 ? v.a : v.b;
+        const int f = e & 3;
+        return f == 0 ? h.x : f == 1 ? h.y : f == 2 ? h.z : h.w;
+    }
 };
 template <> struct FVec<2> {
     using type = float2;
@@ -393,7 +410,8 @@ __device__ __forceinline__ void vfrag_i4(const uint32_t (&r)[4][2], int i, uint3
 // them, or padding columns); without it every row's G columns are the G query
 // heads of one single-token decode, and the kernel keeps the plain addressing.
 template <typename T, typename TKV, int D, int G, bool MQ>
-__global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::MIN_CTAS)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
                                                                      const DecodeArgs a) {
     using C = TcCfg<TKV, D, G>;
@@ -779,7 +797,9 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
             return (int)(2 * ch + ((i == 0 && fr > ck.start(ch)) ? 1 : 0));
         };
         constexpr int SPP = 32 / G;                 // segments per round of pass 1
-        constexpr int NB = 16 / G > 0 ? 16 / G : 1;  // segments per round of pass 2
+        // segments per round of pass 2 (16 / G at head_dim <= 128; half that at 256,
+        // whose lanes hold twice the dims)
+        constexpr int NB = (D <= 128 ? 16 : 8) / G > 0 ? (D <= 128 ? 16 : 8) / G : 1;
         const int li = lane / G, lh = lane % G;
         using V = FVec<C::DPL>;
         // the first round's partial outputs do not depend on the weights: their loads
@@ -1067,8 +1087,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                 const uint32_t vm_lo = (2 * c < ntok ? 0x0000ffffu : 0u) | (2 * c + 1 < ntok ? 0xffff0000u : 0u);
                 const uint32_t vm_hi = (2 * c + 8 < ntok ? 0x0000ffffu : 0u) | (2 * c + 9 < ntok ? 0xffff0000u : 0u);
                 // ---- fragments: K (A of S^T), then V^T (A of O^T), all issued up front
-                constexpr bool kHoist = PA_TC_HOIST_V && !kQz;
-                uint32_t kf[kQz ? 1 : C::KSTEPS][4], vf[kHoist ? C::MTILES : 1][4];
+                // fragments of a head_dim-256 tile are loaded just before their MMAs (all
+                // of them at once would take 128 more registers)
+                constexpr bool kHoist = PA_TC_HOIST_V && !kQz && D <= 128;
+                constexpr bool kHoistK = !kQz && D <= 128;
+                uint32_t kf[kHoistK ? C::KSTEPS : 1][4], vf[kHoist ? C::MTILES : 1][4];
                 uint32_t kw[kI8 ? 2 : 1][8], vw[kI8 ? 4 : 1][4];  // raw int8 words
                 uint32_t kw4[kI4 ? 2 : 1][4], vw4[kI4 ? 4 : 1][2];  // raw 4-bit words
                 float slog = a.scale_log2, vsc = 1.f;
@@ -1086,10 +1109,10 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                     vsc = my_sc[2 * s + 1];
                     kload_i8(kw, tK, g, c);
                     vload_i8(vw, tK + C::TILE, g, c);
-                } else {
+                } else if constexpr (kHoistK) {
 #pragma unroll
                 for (int ks = 0; ks < C::KSTEPS; ++ks) ldsm_x4(kf[ks], tK + koff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
-                if constexpr (PA_TC_HOIST_V) {
+                if constexpr (kHoist) {
 #pragma unroll
                     for (int i = 0; i < C::MTILES; ++i) ldsm_x4_t(vf[i], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
 #pragma unroll
@@ -1113,8 +1136,11 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                     } else if constexpr (kI8) {
                         kfrag_i8(kw, ks, kf[0]);
                         Mma<T>::mma(sa[ks & 3], kf[0], bq[ks][0], bq[ks][1]);
-                    } else {
+                    } else if constexpr (kHoistK) {
                         Mma<T>::mma(sa[ks & 3], kf[ks], bq[ks][0], bq[ks][1]);
+                    } else {
+                        ldsm_x4(kf[0], tK + koff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
+                        Mma<T>::mma(sa[ks & 3], kf[0], bq[ks][0], bq[ks][1]);
                     }
                 }
                 float sc[4];
@@ -1191,7 +1217,7 @@ __global__ void __launch_bounds__(PA_TC_WARPS * 32, PA_TC_MIN_CTAS) decode_tc_ke
                             vfrag_i8(vw, i, vf[0]);
                         // no mask: an int8 or 4-bit slot past the sequence end holds a finite
                         // value, and its probability is exactly 0
-                    } else if constexpr (!PA_TC_HOIST_V) {
+                    } else if constexpr (!kHoist) {
                         ldsm_x4_t(vf[vi], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
                         vf[vi][0] &= vm_lo;
                         vf[vi][1] &= vm_lo;
@@ -1386,7 +1412,8 @@ static bool launch_shape(const void *kernel, int threads, int smem, int *sms, in
 }
 
 bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
-    const bool same = (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype && (D == 64 || D == 128);
+    const bool same = (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype &&
+                      (D == 64 || D == 128 || D == 256);
     const bool quant = q_dtype == PA_F16 && (kv_dtype == PA_I8 || kv_dtype == PA_I4) && D == 128;
     return (same || quant) && (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
 }
@@ -1443,10 +1470,13 @@ int launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
         return launch_tc_g<__half, U4x2, 128>(a, st);
     }
     if (a.q_dtype == PA_F16)
-        return a.D == 64 ? launch_tc_g<__half, __half, 64>(a, st) : launch_tc_g<__half, __half, 128>(a, st);
+        return a.D == 64    ? launch_tc_g<__half, __half, 64>(a, st)
+               : a.D == 128 ? launch_tc_g<__half, __half, 128>(a, st)
+                            : launch_tc_g<__half, __half, 256>(a, st);
     if (a.q_dtype == PA_BF16)
-        return a.D == 64 ? launch_tc_g<__nv_bfloat16, __nv_bfloat16, 64>(a, st)
-                         : launch_tc_g<__nv_bfloat16, __nv_bfloat16, 128>(a, st);
+        return a.D == 64    ? launch_tc_g<__nv_bfloat16, __nv_bfloat16, 64>(a, st)
+               : a.D == 128 ? launch_tc_g<__nv_bfloat16, __nv_bfloat16, 128>(a, st)
+                            : launch_tc_g<__nv_bfloat16, __nv_bfloat16, 256>(a, st);
     return PA_ERR_DTYPE;
 }
 

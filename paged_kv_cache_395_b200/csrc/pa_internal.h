@@ -17,7 +17,7 @@ template <> struct VecT<1> { using type = uint8_t; };
 
 int launch_reshape_and_cache(const void *k, const void *v, void *kc, void *vc,
                              const int64_t *slots, int64_t T, int H, int D, int64_t N, int E,
-                             int64_t k_stride, int64_t v_stride, cudaStream_t st);
+                             int64_t k_stride, int64_t v_stride, int overlap, cudaStream_t st);
 int launch_block_copy(void *kc, void *vc, float *ks, float *vs, const int64_t *pairs, int64_t n,
                       int H, int D, int64_t N, int E, cudaStream_t st);
 int launch_append_int8(const void *k, const void *v, int8_t *kc, int8_t *vc, float *ks, float *vs,

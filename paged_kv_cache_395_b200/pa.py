@@ -29,6 +29,7 @@ PA_F32, PA_F16, PA_BF16, PA_I8, PA_I4 = 0, 1, 2, 3, 4
 PA_ALGO_AUTO, PA_ALGO_SIMT, PA_ALGO_TENSOR = 0, 1, 2
 PA_EFLAG_BAD_BLOCK, PA_EFLAG_BAD_SLOT, PA_EFLAG_BAD_PAIR, PA_EFLAG_WAIT_TIMEOUT = 1, 2, 4, 8
 PA_DECODE_INPUTS_READY, PA_DECODE_OUT_F32 = 1, 2
+PA_APPEND_OVERLAP_PREVIOUS = 1
 WORKSPACE_COUNTER_BYTES = 256 * 1024  # PA_WORKSPACE_COUNTER_BYTES
 BLOCK_SIZE = 16
 
@@ -69,6 +70,7 @@ def _load():
     L = ctypes.CDLL(LIB_PATH)
     P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
     L.pa_reshape_and_cache.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, i64, i64, P]
+    L.pa_reshape_and_cache_ex.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, i64, i64, i32, P]
     L.pa_decode.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), P]
     L.pa_decode_fixed_scratch.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), P]
     L.pa_decode_workspace_size.argtypes = [ctypes.POINTER(PaDecodeParams)]
@@ -84,7 +86,7 @@ def _load():
     L.pa_status_string.argtypes = [i32]
     L.pa_status_string.restype = ctypes.c_char_p
     L.pa_version.argtypes = []
-    for n in ("pa_reshape_and_cache", "pa_append_int8", "pa_decode", "pa_decode_fixed_scratch",
+    for n in ("pa_reshape_and_cache", "pa_reshape_and_cache_ex", "pa_append_int8", "pa_decode", "pa_decode_fixed_scratch",
               "pa_decode_stall_selftest", "pa_decode_algo", "pa_block_copy", "pa_quantize_int8",
               "pa_quantize_int4", "pa_get_error_flags", "pa_version"):
         getattr(L, n).restype = i32
@@ -94,7 +96,7 @@ def _load():
 lib = _load()
 
 # the C-ABI symbols include/pa.h declares
-EXPORTED = ("pa_reshape_and_cache", "pa_append_int8", "pa_decode_workspace_size", "pa_decode_algo", "pa_decode",
+EXPORTED = ("pa_reshape_and_cache", "pa_reshape_and_cache_ex", "pa_append_int8", "pa_decode_workspace_size", "pa_decode_algo", "pa_decode",
             "pa_decode_fixed_scratch", "pa_decode_stall_selftest", "pa_block_copy", "pa_quantize_int8",
             "pa_quantize_int4", "pa_get_error_flags", "pa_status_string", "pa_version")
 FIXED_SCRATCH_BYTES = 32 << 20  # PA_FIXED_SCRATCH_BYTES
@@ -131,8 +133,9 @@ def dtype_code(dt: torch.dtype) -> int:
     return _TORCH_DTYPE[dt]
 
 
-def pa_reshape_and_cache(k, v, key_cache, value_cache, slot_mapping, stream=None):
-    """k, v [T][H_kv][d] (rows contiguous; token stride free) -> caches [N][H_kv][16][d]."""
+def pa_reshape_and_cache(k, v, key_cache, value_cache, slot_mapping, stream=None, flags=0):
+    """k, v [T][H_kv][d] (rows contiguous; token stride free) -> caches [N][H_kv][16][d].
+    flags: 0 or PA_APPEND_OVERLAP_PREVIOUS (see include/pa.h)."""
     _dev(k, v, key_cache, value_cache, slot_mapping)
     T, H, d = k.shape
     N = key_cache.shape[0]
@@ -142,9 +145,10 @@ def pa_reshape_and_cache(k, v, key_cache, value_cache, slot_mapping, stream=None
         raise ValueError("slot_mapping must be contiguous int64")
     if not (key_cache.is_contiguous() and value_cache.is_contiguous()):
         raise ValueError("caches must be contiguous")
-    _check(lib.pa_reshape_and_cache(_ptr(k), _ptr(v), _ptr(key_cache), _ptr(value_cache),
-                                    _ptr(slot_mapping), T, H, d, key_cache.shape[2], N,
-                                    dtype_code(k.dtype), k.stride(0), v.stride(0), _stream(stream)),
+    _check(lib.pa_reshape_and_cache_ex(_ptr(k), _ptr(v), _ptr(key_cache), _ptr(value_cache),
+                                       _ptr(slot_mapping), T, H, d, key_cache.shape[2], N,
+                                       dtype_code(k.dtype), k.stride(0), v.stride(0), int(flags),
+                                       _stream(stream)),
            "pa_reshape_and_cache")
 
 

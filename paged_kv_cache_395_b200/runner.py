@@ -150,6 +150,9 @@ class StepCalls:
         ks = dw.k_scales if int8 else None
         vs = dw.v_scales if int8 else None
         ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        # appends that never touch what the previous step's decode reads may run while
+        # it finishes (the recipe reuses freed blocks one step late)
+        aflags = pa.PA_APPEND_OVERLAP_PREVIOUS if getattr(w, "appends_overlap_previous", False) else 0
         # one workspace, sized for the largest step
         need = 0
         for ops in dw.steps.values():
@@ -169,8 +172,8 @@ class StepCalls:
                     _, k, v, s = op
                     N, H, bs, d = dw.kc.shape
                     args = (ptr(k), ptr(v), ptr(dw.kc), ptr(dw.vc), ptr(s), k.shape[0], H, d, bs, N,
-                            pa.dtype_code(k.dtype), k.stride(0), v.stride(0), sp)
-                    calls.append(("reshape", pa.lib.pa_reshape_and_cache, args))
+                            pa.dtype_code(k.dtype), k.stride(0), v.stride(0), aflags, sp)
+                    calls.append(("reshape", pa.lib.pa_reshape_and_cache_ex, args))
                     launches += 1 if k.shape[0] else 0
                 elif op[0] == "copy":
                     n = op[1].numel() // 2

@@ -68,6 +68,10 @@ class Workload:
     block_size: int = BLOCK_SIZE
     logical: dict | None = None  # seq -> (K [L][H_kv][d], V) for small workloads
     notes: str = ""
+    # a step's appends never write a slot that the previous step's decode reads
+    # (blocks of finished sequences are reused one step late), so the library may
+    # run them while that decode finishes (PA_APPEND_OVERLAP_PREVIOUS)
+    appends_overlap_previous: bool = False
 
     @property
     def group(self) -> int:
@@ -170,7 +174,12 @@ def ragged(num_steps: int = 128, dtype: str = "float16", batch: int = 64,
     cached + 1; then ``random(64) < 0.02`` marks finished sequences, which free
     their blocks and are replaced, in batch order, by new sequences of
     ``integers(16, 513)`` tokens whose K then V are drawn at once.
-    Pool: 64 x ceil(4224 / 16) = 16896 blocks, enough for the worst case."""
+    Pool: 64 x ceil(4224 / 16) = 16896 blocks, enough for the worst case.
+
+    Blocks freed by the sequences that finish after step i's decode go back on
+    the free list just before the admissions of step i + 1 (deferred reuse), so
+    neither step i + 1's token appends nor the prompts admitted with them (both
+    written by step i + 1's append) land in a block step i's decode reads."""
     B, Hq, Hkv, d = batch, 32, 8, 128
     max_len = 4096 + num_steps
     mb = -(-max_len // BLOCK_SIZE)
@@ -202,8 +211,9 @@ def ragged(num_steps: int = 128, dtype: str = "float16", batch: int = 64,
                       Decode(q, bm.block_table(seq_ids, mb), lens, int(lens.max()))])
         finished = rng.random(B) < finish_p
         pending = ([], [], [])
+        bm.release_deferred()  # freed after the previous step's decode
         for i in np.nonzero(finished)[0]:
-            bm.free_sequence(seq_ids[i])
+            bm.free_sequence(seq_ids[i], defer=True)
             L = int(rng.integers(16, 513))
             k, v = _normal_tokens(rng, L, Hkv, d, dtype)
             seq_ids[i] = next_id
@@ -211,7 +221,8 @@ def ragged(num_steps: int = 128, dtype: str = "float16", batch: int = 64,
             pending[1].append(v)
             pending[2].append(bm.add_sequence(next_id, L))
             next_id += 1
-    return Workload("ragged", Hq, Hkv, d, N, dtype, 1.0 / np.sqrt(d), mb, 256, setup, steps)
+    return Workload("ragged", Hq, Hkv, d, N, dtype, 1.0 / np.sqrt(d), mb, 256, setup, steps,
+                    appends_overlap_previous=True)
 
 
 def long(dtype: str = "float16", batch: int = 16, seq_len: int = 8192) -> Workload:
@@ -304,7 +315,9 @@ def specdec(num_steps: int = 16, query_len: int = 2, dtype: str = "float16", bat
         lens = np.array([bm.lens[b] for b in range(B)], dtype=np.int32)
         steps.append([Reshape(k_new, v_new, new_slots),
                       Decode(q, bm.block_table(range(B), mb), lens, int(lens.max()))])
-    return Workload("specdec", Hq, Hkv, d, N, dtype, 1.0 / np.sqrt(d), mb, -1, setup, steps)
+    # no sequence ends: every appended slot lies past the lengths of every earlier decode
+    return Workload("specdec", Hq, Hkv, d, N, dtype, 1.0 / np.sqrt(d), mb, -1, setup, steps,
+                    appends_overlap_previous=True)
 
 
 def mha_prefix(dtype: str = "float16") -> Workload:

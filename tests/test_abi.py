@@ -167,7 +167,7 @@ def test_product_path_does_not_touch_oracle():
 def test_large_groups_and_head_dim_256_are_planned():
     """G = 16, 32, 64 run as 8-head groups: the workspace of a G = 32, H_kv = 1
     decode equals that of G = 8, H_kv = 4 (same query heads, same rows); head_dim
-    256 is accepted on the CUDA-core family."""
+    256 is accepted on both families."""
     big = params(num_q_heads=32, num_kv_heads=1, partition_size=16, algo=pa.PA_ALGO_TENSOR)
     same = params(num_q_heads=32, num_kv_heads=4, partition_size=16, algo=pa.PA_ALGO_TENSOR)
     n = pa.lib.pa_decode_workspace_size(ctypes.byref(big))
@@ -177,8 +177,10 @@ def test_large_groups_and_head_dim_256_are_planned():
         assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
     p = params(head_dim=256, partition_size=16, algo=pa.PA_ALGO_SIMT)
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
-    # the tensor-core family stops at head_dim 128
-    p = params(head_dim=256, algo=pa.PA_ALGO_TENSOR)
+    # the tensor-core family takes fp16/bf16 head_dim 256 too (not int8 or 4-bit caches)
+    p = params(head_dim=256, partition_size=16, algo=pa.PA_ALGO_TENSOR)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+    p = params(head_dim=256, kv_dtype=pa.PA_I8, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p),
                             None) == pa.PA_ERR_UNSUPPORTED
 
@@ -209,7 +211,9 @@ def test_decode_algo_reports_the_family():
     assert algo(params()) == pa.PA_ALGO_TENSOR
     assert algo(params(algo=pa.PA_ALGO_SIMT)) == pa.PA_ALGO_SIMT
     assert algo(params(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32)) == pa.PA_ALGO_SIMT
-    assert algo(params(head_dim=256)) == pa.PA_ALGO_SIMT
+    assert algo(params(head_dim=256)) == pa.PA_ALGO_TENSOR
+    assert algo(params(head_dim=256, q_dtype=pa.PA_BF16, kv_dtype=pa.PA_BF16)) == pa.PA_ALGO_TENSOR
+    assert algo(params(head_dim=256, kv_dtype=pa.PA_I8)) == pa.PA_ALGO_SIMT
     assert algo(params(kv_dtype=pa.PA_I8, q_dtype=pa.PA_BF16)) == pa.PA_ALGO_SIMT
     assert algo(params(kv_dtype=pa.PA_I8)) == pa.PA_ALGO_TENSOR
     # a q that is not 16-byte aligned goes to the CUDA-core family, or is refused

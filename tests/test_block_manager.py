@@ -140,3 +140,42 @@ def test_ragged_recipe_replays_without_leak():
         # every (block, offset) written this step is distinct
         s = ops[0].slot_mapping
         assert len(np.unique(s)) == len(s)
+
+
+def test_deferred_free_holds_blocks_back_one_step():
+    """free_sequence(defer=True) keeps the blocks off the free list until
+    release_deferred(); an immediate free hands the same block out next (LIFO)."""
+    bm = BlockManager(4, 16)
+    bm.add_sequence("a", 16)
+    a_block = bm.tables["a"][0]
+    bm.free_sequence("a")
+    bm.add_sequence("b", 16)
+    assert bm.tables["b"][0] == a_block  # immediate reuse
+    bm.free_sequence("b", defer=True)
+    bm.check_invariants()
+    bm.add_sequence("c", 16)
+    assert bm.tables["c"][0] != a_block and bm.num_free == 2
+    bm.release_deferred()
+    bm.add_sequence("d", 16)
+    assert bm.tables["d"][0] == a_block
+    bm.check_invariants()
+
+
+@pytest.mark.parametrize("name", ["ragged", "specdec"])
+def test_appends_never_touch_the_previous_decode(name):
+    """The recipes that mark appends_overlap_previous (so their appends run with
+    PA_APPEND_OVERLAP_PREVIOUS): no slot that step i + 1's appends write lies
+    within a sequence's length in step i's decode, the prompts of newly admitted
+    sequences included."""
+    w = getattr(W, name)()
+    assert w.appends_overlap_previous
+    for i in range(len(w.steps) - 1):
+        dec = [op for op in w.steps[i] if isinstance(op, W.Decode)][0]
+        read = []
+        for b, L in enumerate(dec.seq_lens):
+            t = np.arange(int(L), dtype=np.int64)
+            read.append(dec.block_tables[b][t // 16].astype(np.int64) * 16 + t % 16)
+        read = np.concatenate(read)
+        written = np.concatenate([op.slot_mapping for op in w.steps[i + 1] if isinstance(op, W.Reshape)])
+        written = written[written >= 0]
+        assert not np.isin(written, read).any(), f"step {i + 1} appends into slots step {i} reads"

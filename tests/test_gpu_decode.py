@@ -427,16 +427,31 @@ def test_large_group_bf16_and_int8(qdt):
     check(got8[0], ref8, qdt, "MQA G=64 int8", dw, -1, pa.PA_ALGO_AUTO, int8=True)
 
 
+@pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_TENSOR])
 @pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
-@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 4), (32, 4), (32, 1)])
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 4), (32, 4), (32, 1), (6, 2)])
 @pytest.mark.parametrize("part", [0, 32, -1])
-def test_head_dim_256(qdt, hq, hkv, part):
-    """head_dim 256 on the CUDA-core family (the library picks it)."""
+def test_head_dim_256(qdt, hq, hkv, part, algo):
+    """head_dim 256 on both families (the tensor-core family is the library's pick
+    for fp16/bf16), ragged tails and partitions, padded groups (G = 3) on the
+    tensor-core family only."""
+    if algo == pa.PA_ALGO_SIMT and hq // hkv == 3:
+        pytest.skip("the CUDA-core family takes G in 1, 2, 4, 8 and multiples of 8")
     w = W.random_case([1, 17, 200, 513], num_q_heads=hq, num_kv_heads=hkv, head_dim=256, dtype=qdt,
                       seed=hq + hkv + 256)
     ref, _, _ = replay(w)
-    got, dw = run_gpu(w, part)
-    check(got[0], ref[0], qdt, f"d=256 G={hq // hkv} part={part}", dw, part, pa.PA_ALGO_AUTO)
+    got, dw = run_gpu(w, part, algo)
+    check(got[0], ref[0], qdt, f"d=256 G={hq // hkv} part={part} algo={algo}", dw, part, algo)
+
+
+@pytest.mark.parametrize("Q", [2, 3])
+def test_head_dim_256_multi_query(Q):
+    """Several new tokens per sequence at head_dim 256 (tensor-core family)."""
+    w = W.random_multi_case([Q, 40, 300], Q, num_q_heads=16, num_kv_heads=4, head_dim=256,
+                            dtype="float16", seed=256 + Q)
+    ref, _, _ = replay(w)
+    got, dw = run_gpu(w, -1, pa.PA_ALGO_TENSOR)
+    assert_close(got[0], ref[0], "float16", f"d=256 Q={Q}")
 
 
 def test_head_dim_256_int8():
