@@ -107,8 +107,12 @@ int pa_reshape_and_cache(const void *k, const void *v, void *key_cache, void *va
  * the previous kernel finishes, and the next kernel may launch at once; the call
  * still completes only after the previous kernel has, so a kernel that waits for
  * this one finds every earlier one complete.  Without the guarantee the result
- * of the previous kernel is undefined.  (No counterpart in the pages: it hides
- * the append's latency behind the decode before it.)
+ * of the previous kernel is undefined.  The inputs (k, v, slot_mapping) must not
+ * be produced by the previous kernel either: the flag suits appends of K/V made
+ * earlier (the prompt of a newly admitted sequence, written after an earlier
+ * prefill), not a decode loop's new token, whose K/V come from the computation
+ * just before.  (No counterpart in the pages: it hides an append's latency
+ * behind the kernel before it.)
  */
 #define PA_APPEND_OVERLAP_PREVIOUS 1
 int pa_reshape_and_cache_ex(const void *k, const void *v, void *key_cache, void *value_cache,

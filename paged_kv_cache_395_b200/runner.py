@@ -140,7 +140,10 @@ class StepCalls:
     ctypes call per library entry point and nothing else on the host."""
 
     def __init__(self, dw: DeviceWorkload, partition_size=-1, int8=False, algo=pa.PA_ALGO_AUTO,
-                 stream=None, flags=0):
+                 stream=None, flags=0, append_flags=0):
+        """flags: pa_decode flags; append_flags: pa_reshape_and_cache_ex flags
+        (PA_APPEND_OVERLAP_PREVIOUS only for recipes whose appends never touch
+        what the previous step's decode reads, ``appends_overlap_previous``)."""
         import ctypes
         self.dw = dw
         self.stream = stream if stream is not None else torch.cuda.current_stream()
@@ -150,9 +153,9 @@ class StepCalls:
         ks = dw.k_scales if int8 else None
         vs = dw.v_scales if int8 else None
         ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
-        # appends that never touch what the previous step's decode reads may run while
-        # it finishes (the recipe reuses freed blocks one step late)
-        aflags = pa.PA_APPEND_OVERLAP_PREVIOUS if getattr(w, "appends_overlap_previous", False) else 0
+        if append_flags and not getattr(w, "appends_overlap_previous", False):
+            raise ValueError("this recipe's appends may touch what the previous decode reads")
+        aflags = int(append_flags)
         # one workspace, sized for the largest step
         need = 0
         for ops in dw.steps.values():

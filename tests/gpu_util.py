@@ -60,7 +60,7 @@ def check_bf16(got_bf16: torch.Tensor, got_f32: torch.Tensor, ref: np.ndarray, w
     assert got_f32.dtype == torch.float32 and got_bf16.dtype == torch.bfloat16
     assert_close(got_f32, ref, "bfloat16", f"{what} (fp32 result)", rows=rows)
     rne = got_f32.to(torch.bfloat16)
-    assert torch.equal(bits(got_bf16), bits(rne)), f"{what}: bf16 output is not the fp32 result rounded"
+    assert np.array_equal(bits(got_bf16), bits(rne)), f"{what}: bf16 output is not the fp32 result rounded"
     assert_close(got_bf16, ref, "bfloat16", what, rows=rows)
 
 

@@ -353,6 +353,31 @@ def test_ragged_trace_back_to_back_inputs_ready():
     assert np.array_equal(bits(dw.vc), vc.view(np.uint8))
 
 
+@pytest.mark.slow
+def test_ragged_trace_appends_overlapping_the_previous_decode():
+    """The ragged trace issued back to back with every append flagged
+    PA_APPEND_OVERLAP_PREVIOUS (the recipe reuses freed blocks one step late, so
+    no append writes a slot the previous decode reads): each append runs while the
+    previous decode finishes.  Sampled steps against the oracle, caches bit-exact."""
+    w = W.ragged()
+    sample = {1, 2, 33, 77, 127}
+    ref, kc, vc = replay(w, want=lambda s: s in sample)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    calls = runner.StepCalls(dw, -1, False, pa.PA_ALGO_AUTO, stream, flags=pa.PA_DECODE_INPUTS_READY,
+                             append_flags=pa.PA_APPEND_OVERLAP_PREVIOUS)
+    with torch.cuda.stream(stream):
+        for i in range(len(w.steps)):
+            calls.run(i)
+    torch.cuda.synchronize()
+    for i in sorted(sample):
+        assert_close(dw.steps[i][-1][-1], ref[i], "float16", f"ragged step {i}")
+    assert np.array_equal(bits(dw.kc), kc.view(np.uint8))
+    assert np.array_equal(bits(dw.vc), vc.view(np.uint8))
+
+
 @pytest.mark.parametrize("hq,hkv", [(32, 1), (64, 2), (16, 1)])
 @pytest.mark.parametrize("kind", ["float16", "int8"])
 def test_virtual_heads_uniform_and_near_uniform_lengths(hq, hkv, kind):
