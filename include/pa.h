@@ -150,15 +150,13 @@ typedef struct pa_decode_params {
                                 fits one partition). */
     int algo;                /* enum pa_algo */
     void *workspace;         /* device scratch, >= pa_decode_workspace_size(p) bytes,
-                                16-byte aligned; NULL allowed when that size is 0.  Must be
-                                zero-filled once before its first use.  Its first
-                                PA_WORKSPACE_COUNTER_BYTES hold merge counters, at the same
-                                place for every call, and partial results come after them;
-                                every call returns the counters to zero, also when a bounded
-                                wait gave up (PA_EFLAG_WAIT_TIMEOUT).  So one workspace serves
-                                any sequence of calls, whatever their parameters or kernel
-                                family, without clearing it again.  Calls that share a
-                                workspace must not overlap on the device. */
+                                16-byte aligned; NULL allowed when that size is 0.  It holds
+                                the partial results of one call only: nothing in it needs
+                                initialising, and every value a call reads there was written
+                                earlier in the same call.  So one workspace serves any
+                                sequence of calls, whatever their parameters or kernel
+                                family.  Calls that share a workspace must not overlap on
+                                the device. */
     size_t workspace_bytes;
     int flags;               /* 0, or PA_DECODE_INPUTS_READY and/or PA_DECODE_OUT_F32 */
     int query_len;           /* new tokens per sequence, Q (0 or 1: single-token decode).
@@ -194,18 +192,12 @@ typedef struct pa_decode_params {
  */
 #define PA_DECODE_OUT_F32 2
 
-/* Size of the merge-counter region at the start of every split-K workspace:
- * one int per (sequence, KV head) row of the tensor-core family's split
- * (num_seqs * num_kv_heads * ceil(Q * G / 8) rows at most 65536; beyond that
- * the library runs that family in one pass, or the CUDA-core family). */
-#define PA_WORKSPACE_COUNTER_BYTES (256 * 1024)
-
 /*
  * Bytes of device workspace pa_decode needs for these parameters (0 when the
- * call runs in one pass; else PA_WORKSPACE_COUNTER_BYTES plus the partial
- * results).  Depends only on num_seqs, num_q_heads, num_kv_heads, head_dim,
- * query_len, max_seq_len, max_blocks_per_seq, the dtypes, algo and
- * partition_size.  Returns 0 for invalid params.
+ * call runs in one pass; else the partial results).  Depends only on num_seqs,
+ * num_q_heads, num_kv_heads, head_dim, query_len, max_seq_len,
+ * max_blocks_per_seq, the dtypes, algo and partition_size.  Returns 0 for
+ * invalid params.
  */
 size_t pa_decode_workspace_size(const pa_decode_params *p);
 
@@ -216,7 +208,7 @@ size_t pa_decode_workspace_size(const pa_decode_params *p);
  * its alignment: the tensor-core family reads q rows with 16-byte copies, so an
  * unaligned q goes to the CUDA-core family.  Together with
  * pa_decode_workspace_size it also gives the kernel launches of a call: one,
- * plus a merge kernel when the CUDA-core family splits (workspace size > 0).
+ * plus a merge kernel whenever the call splits (workspace size > 0).
  */
 int pa_decode_algo(const pa_decode_params *p, const void *q);
 
@@ -254,13 +246,12 @@ int pa_decode(void *out, const void *q, const void *key_cache, const void *value
  *
  *  - Parameters whose pa_decode_workspace_size exceeds PA_FIXED_SCRATCH_BYTES
  *    return PA_ERR_WORKSPACE and launch nothing.
- *  - The first call on a device sets the area up: it looks up its address,
- *    zero-fills it on `stream` and synchronises `stream`.  Make that first call
- *    before any stream capture.
+ *  - The first call on a device looks up the area's address (no stream work:
+ *    the area needs no clearing).  Make that first call before any stream
+ *    capture.
  *  - All calls on one device share the area: calls that overlap on the device
  *    (different streams, or host threads without ordering) race on it.  Issue
- *    them in one stream order.  Calls in order may use any parameters: the
- *    area's merge counters sit at its start, where no partial result goes.
+ *    them in one stream order.  Calls in order may use any parameters.
  *  - The area's address is kept for the life of the process: do not use the
  *    library after cudaDeviceReset.
  */
@@ -279,9 +270,9 @@ int pa_decode_fixed_scratch(void *out, const void *q, const void *key_cache, con
  * (K tile, V tile) stages), so its wait for that stage runs out: no memory is
  * read or written for it, and nothing hangs.  Expected outcome: PA_OK, the
  * error word gains PA_EFLAG_WAIT_TIMEOUT, the rows that worker had not finished
- * hold no valid result, and the workspace is left ready for the next call (the
- * worker waits, again bounded, for its copies in flight, then takes the merge
- * tickets of its remaining partial results with empty partials).
+ * hold no valid result, and the next call may use the same workspace (the
+ * worker waits, again bounded, for its copies in flight, then writes empty
+ * partial results, weight 0 in the merge, for its remaining segments).
  */
 int pa_decode_stall_selftest(void *out, const void *q, const void *key_cache, const void *value_cache,
                              const int32_t *block_tables, const int32_t *seq_lens, float scale,

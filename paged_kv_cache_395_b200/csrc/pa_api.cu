@@ -140,12 +140,9 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
     // of all (sequence, KV head) rows with 32-bit integers
     const int64_t stream_blocks =
         (int64_t)p->num_seqs * kh.Hkv * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
-    // a split on the tensor-core family keeps one merge counter per row in the
-    // workspace's fixed counter region
-    const bool rows_fit = (int64_t)p->num_seqs * kh.Hkv <= kCounterRows;
     const bool tc_ok = decode_tc_supported(p->q_dtype, p->kv_dtype, p->head_dim, G, p->num_seqs) &&
                        p->num_blocks * p->num_kv_heads * PA_BLOCK_SIZE <= 2147483647LL &&
-                       stream_blocks <= (1LL << 30) && (rows_fit || p->partition_size <= 0);
+                       stream_blocks <= (1LL << 30);
     if (p->algo == PA_ALGO_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
     // several new tokens per sequence, or padded columns: the tensor-core family only
     if ((kh.qlen > 1 || kh.padded) && !tc_ok) return PA_ERR_UNSUPPORTED;
@@ -158,10 +155,8 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
         pl->bytes = decode_workspace_bytes(p->num_seqs, p->num_q_heads, kh.Hkv, p->head_dim, max_len, part);
         return PA_OK;
     }
-    if (p->partition_size == 0 || max_len == 0 || !rows_fit) {
-        // one warp per (sequence, KV head) row, no workspace (with more rows than
-        // counters, rows far outnumber the warps and balance without a split)
-        pl->tc_chunk = -1;
+    if (p->partition_size == 0 || max_len == 0) {
+        pl->tc_chunk = -1;  // one warp per (sequence, KV head) row, no workspace
         return PA_OK;
     }
     const int64_t tmax = (int64_t)p->num_seqs * kh.Hkv * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
@@ -174,10 +169,19 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
         pl->tc_chunk = 0;
         nchunks = tmax < kTcMaxChunks ? tmax : kTcMaxChunks;
     }
+    if (decode_coop_eligible(p->q_dtype, p->kv_dtype, p->head_dim, G, kh.ngroups, kh.qlen, kh.padded, 1)) {
+        // one CTA per chunk of cache rows, 8 * ngroups columns per row
+        const int64_t cmax = (int64_t)p->num_seqs * p->num_kv_heads * ((max_len + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE);
+        const int64_t cn = p->partition_size > 0 ? (cmax + pl->tc_chunk - 1) / pl->tc_chunk
+                                                 : (cmax < kTcMaxChunks ? cmax : kTcMaxChunks);
+        pl->tc_slots = 2 * cn;
+        pl->bytes = up256((size_t)pl->tc_slots * G * kh.ngroups * p->head_dim * sizeof(float)) +
+                    up256((size_t)pl->tc_slots * G * kh.ngroups * sizeof(float));
+        return PA_OK;
+    }
     pl->tc_slots = 2 * nchunks;
-    // the merge counters' fixed region, then partial outputs and lse of two
-    // segments per chunk
-    pl->bytes = kCounterBytes + up256((size_t)pl->tc_slots * G * p->head_dim * sizeof(float)) +
+    // partial outputs and lse of two segments per chunk
+    pl->bytes = up256((size_t)pl->tc_slots * G * p->head_dim * sizeof(float)) +
                 up256((size_t)pl->tc_slots * G * sizeof(float));
     return PA_OK;
 }
@@ -358,17 +362,19 @@ static int decode_impl(void *out, const void *q, const void *key_cache, const vo
                            wait_ns);
     }
     if (stall_at >= 0 && !pl.tc) return PA_ERR_UNSUPPORTED;
-    // workspace: the merge counters' fixed region, then the partial outputs, then their lse
-    if (pl.bytes > 0) a.counters = reinterpret_cast<int *>(ws);
+    // workspace: the partial outputs, then their lse
     if (pl.tc) {
         a.part = 0;
         a.max_parts = 1;
         a.tc_chunk = pl.tc_chunk;
         a.early = (p->flags & PA_DECODE_INPUTS_READY) ? 1 : 0;
         if (pl.bytes > 0) {
-            const size_t o_bytes = up256((size_t)pl.tc_slots * a.G * a.D * sizeof(float));
-            a.ws_o = reinterpret_cast<float *>(ws + kCounterBytes);
-            a.ws_lse = reinterpret_cast<float *>(ws + kCounterBytes + o_bytes);
+            // the cooperative mode keeps all 8 * ngroups columns of a cache row per slot
+            const bool coop = decode_coop_eligible(a.q_dtype, a.kv_dtype, a.D, a.G, a.ngroups, a.qlen,
+                                                   (int64_t)a.G * a.ngroups != a.gcols, 1);
+            const size_t o_bytes = up256((size_t)pl.tc_slots * a.G * (coop ? a.ngroups : 1) * a.D * sizeof(float));
+            a.ws_o = reinterpret_cast<float *>(ws);
+            a.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
         }
         return launch_decode_tc(a, (cudaStream_t)stream);
     }
@@ -376,8 +382,8 @@ static int decode_impl(void *out, const void *q, const void *key_cache, const vo
     a.max_parts = pl.max_parts;
     if (pl.bytes > 0) {
         const size_t o_bytes = up256((size_t)a.B * a.Hq * pl.max_parts * a.D * sizeof(float));
-        a.ws_o = reinterpret_cast<float *>(ws + kCounterBytes);
-        a.ws_lse = reinterpret_cast<float *>(ws + kCounterBytes + o_bytes);
+        a.ws_o = reinterpret_cast<float *>(ws);
+        a.ws_lse = reinterpret_cast<float *>(ws + o_bytes);
     }
     if (pl.max_len == 0) {
         // every row is zero: the one-pass kernel writes zeros for seq_len <= 0

@@ -350,9 +350,7 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int pa
     const size_t o = (size_t)B * Hq * mp * D * sizeof(float);
     const size_t lse = (size_t)B * Hq * mp * sizeof(float);
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    // the counter region is not used by this family, but kept free so that one
-    // workspace serves calls of either family
-    return kCounterBytes + up(o) + up(lse);
+    return up(o) + up(lse);
 }
 
 template <typename TQ, typename TKV, int D, int G>

@@ -24,19 +24,26 @@
 // (sequence, KV head) rows are laid end to end as one stream of blocks (row
 // order: sequence, then KV head; total = sum_b ceil(L_b / 16) * H_kv blocks).
 // With partition_size == 0 warp w takes whole rows w, w + W, ... (W = warps in
-// the grid).  Otherwise the stream is cut into chunks of c blocks -- by default
-// c = ceil(total / W) (at least 8), so every warp reads the same number of
-// blocks whatever the length mix; partition_size > 0 fixes c = partition/16 --
-// and warp w takes chunks w, w + W, ...  A chunk is walked segment by segment
-// (a segment = the part of one row inside the chunk); the producer side of the
-// warp keeps issuing TMA for the next blocks across segment and chunk ends, so
-// the copy stream does not drain.  A segment that is a whole row writes the
-// output directly.  A cut segment is a partial: its normalised output and
-// log2-sum-exp go to workspace slot 2*chunk (first segment of the chunk) or
-// 2*chunk + 1 (last), and it takes a ticket from a per-row counter; the warp
-// that takes the last ticket merges the row's partials
-//   out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M)
-// and resets the counter to zero.  No warp ever waits for another.
+// the grid).  Otherwise the stream is cut into chunks -- by default W' =
+// min(W, 2048) chunks of equal cost, the cost of a chunk being its blocks plus
+// PA_TC_GAMMA for every row that ends in it (the work of finishing a segment and
+// starting the next, measured at about 1.4 blocks' time), so every warp has the
+// same work whatever the length mix; partition_size > 0 fixes chunks of
+// partition/16 blocks -- and warp w takes chunks w, w + W, ...  A chunk is
+// walked segment by segment (a segment = the part of one row inside the chunk);
+// the producer side of the warp keeps issuing TMA for the next blocks across
+// segment and chunk ends, so the copy stream does not drain.  A segment that is
+// a whole row writes the output directly.  A cut segment is a partial: its
+// normalised output and log2-sum-exp go to workspace slot 2*chunk (first segment
+// of the chunk) or 2*chunk + 1 (last).  merge_tc_kernel, launched right after
+// with programmatic dependent launch, merges every cut row:
+//   out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M).
+// No warp ever waits for another.  (Merging inside the decode kernel, by the
+// warp that finished a row's last partial, put those merges at the end of the
+// slowest warps: a separate merge kernel measured 7% faster on the ragged trace.)
+//
+// Groups of 16, 32 or 64 query heads per KV head run in decode_coop_kernel
+// (one CTA per chunk of cache rows, its warps sharing each staged tile).
 #include <cudaTypedefs.h>
 
 #include <map>
@@ -190,7 +197,7 @@ struct TcCfg {
     static constexpr int OK_OFF = BAR_OFF + NW * S * 8;
     static constexpr int SC_OFF = OK_OFF + NW * S * 4;    // float [NW][S][2]: int8 K, V scales
     static constexpr int CUM_OFF = SC_OFF + NW * S * 8;
-    static int smem_bytes(int B) { return 1024 + CUM_OFF + (2 * B + 2) * 4; }
+    static int smem_bytes(int B) { return 1024 + CUM_OFF + (3 * B + 3) * 4; }
 };
 
 // One contiguous run of blocks of one (sequence, KV head) row.
@@ -221,23 +228,44 @@ struct Win {
 
 // Chunks of the concatenated block stream: n chunks of c blocks (the last one
 // shorter); warp w takes chunks w, w + W, w + 2W, ...
+#ifndef PA_TC_GAMMA
+#define PA_TC_GAMMA 2
+#endif
+// Chunks are cut in a virtual stream in which every non-empty row is followed by
+// gam extra units (the cost of finishing one segment and starting the next, in
+// blocks), so a chunk that holds several row ends holds fewer blocks.  cum[b] /
+// cumv[b]: blocks / virtual units of the rows of sequences before b.
 struct Chunks {
-    int total, c, n;
-    __device__ int start(int ch) const { return ch * c; }
-    __device__ int end(int ch) const { return (ch + 1) * c < total ? (ch + 1) * c : total; }
-    __device__ int of(int f) const { return f / c; }
+    int total, vtotal, c, n, gam, Hkv;
+    const int *cum, *cumv;
+    // virtual position of block j of row (b, kvh) of nb blocks
+    __device__ int vpos(int b, int kvh, int nb, int j) const { return cumv[b] + kvh * (nb + gam) + j; }
+    // actual stream position of the first block at or after virtual position v
+    __device__ int at(int v) const {
+        if (v >= vtotal) return total;
+        int l = 0, h = nseq;  // largest b with cumv[b] <= v: sequence b is not empty
+        while (h - l > 1) {
+            const int mid = (l + h) >> 1;
+            if (cumv[mid] <= v) l = mid; else h = mid;
+        }
+        const int nb = cum[l + 1] - cum[l];
+        const int off = v - cumv[l], rl = nb + gam;
+        const int kvh = off / rl, j = off - kvh * rl;
+        return cum[l] * Hkv + kvh * nb + (j < nb ? j : nb);
+    }
+    int nseq;
+    __device__ int start(int ch) const { return at(ch * c); }
+    __device__ int end(int ch) const { return at((ch + 1) * c); }
+    // chunk of block j of row (b, kvh)
+    __device__ int of(int b, int kvh, int nb, int j) const { return vpos(b, kvh, nb, j) / c; }
+    // whether the row (b, kvh) begins after its first chunk's first block, i.e. the
+    // block before it (the previous row's last) lies in the same chunk
+    __device__ bool mid_start(int b, int kvh, int nb) const {
+        const int fr = cum[b] * Hkv + kvh * nb;
+        return fr > 0 && (vpos(b, kvh, nb, 0) - gam - 1) / c == vpos(b, kvh, nb, 0) / c;
+    }
 };
 
-// Ticket increment with release semantics at GPU scope: the warp's
-// partial-result stores (ordered before lane 0 by __syncwarp) are released
-// with it.  The warp that draws a row's last ticket runs fence_acq_rel_gpu
-// before it reads the other segments' partials.
-__device__ __forceinline__ int atom_add_release_gpu(int *p, int v) {
-    int old;
-    asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -430,6 +458,7 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     float *stage_sc = reinterpret_cast<float *>(smem + C::SC_OFF);
     int *cum = reinterpret_cast<int *>(smem + C::CUM_OFF);  // [B + 1] blocks before sequence b
     int *lens = cum + a.B + 1;                                // [B] effective lengths
+    int *cumv = lens + a.B;                                   // [B + 1] virtual units before b
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = a.B, Hkv = a.Hkv;
@@ -452,28 +481,47 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
         __shared__ int wsum[NW];
         const int per = (B + C::THREADS - 1) / C::THREADS;
         const int lo = min(B, tid * per), hi = min(B, lo + per);
-        int s = 0;
+        __shared__ int wsumv[NW];
+        const int gam = a.tc_chunk == 0 ? PA_TC_GAMMA : 0;
+        int s = 0, sv = 0;
         for (int b = lo; b < hi; ++b) {
             const int L = min(min(a.lens[b], a.max_len), a.mbps * kBlockSize);
             lens[b] = L;
-            s += L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
+            const int nb = L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
+            s += nb;
+            sv += nb > 0 ? (nb + gam) * Hkv : 0;
         }
-        int x = s;  // inclusive warp scan
+        int x = s, xv = sv;  // inclusive warp scans
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+            const int y = __shfl_up_sync(0xffffffffu, x, o), yv = __shfl_up_sync(0xffffffffu, xv, o);
+            if (lane >= o) {
+                x += y;
+                xv += yv;
+            }
         }
-        if (lane == 31) wsum[warp] = x;
+        if (lane == 31) {
+            wsum[warp] = x;
+            wsumv[warp] = xv;
+        }
         __syncthreads();
-        int run = x - s;
-        for (int w = 0; w < warp; ++w) run += wsum[w];
+        int run = x - s, runv = xv - sv;
+        for (int w = 0; w < warp; ++w) {
+            run += wsum[w];
+            runv += wsumv[w];
+        }
         for (int b = lo; b < hi; ++b) {
             cum[b] = run;
+            cumv[b] = runv;
             const int L = lens[b];
-            run += L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
+            const int nb = L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
+            run += nb;
+            runv += nb > 0 ? (nb + gam) * Hkv : 0;
         }
-        if (tid == C::THREADS - 1) cum[B] = run;
+        if (tid == C::THREADS - 1) {
+            cum[B] = run;
+            cumv[B] = runv;
+        }
         __syncthreads();
     }
     // blocks of all rows: the host sends this family only streams below 2^31 blocks
@@ -496,16 +544,16 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     // Static schedule: by default one chunk of ceil(total / W) blocks (at least
     // kTcMinChunk) per warp, so every warp reads the same number of blocks;
     // partition_size > 0 fixes the chunk length instead.
-    Chunks ck{total, 1, 0};
+    Chunks ck{total, cumv[B], 1, 0, a.tc_chunk == 0 ? PA_TC_GAMMA : 0, Hkv, cum, cumv, B};
     if (!rows_mode) {
         if (a.tc_chunk > 0) {
             ck.c = a.tc_chunk;
         } else {
             const int wc = min(W, kTcMaxChunks);
-            const int c = (total + wc - 1) / wc;
+            const int c = (ck.vtotal + wc - 1) / wc;
             ck.c = c > kTcMinChunk ? c : kTcMinChunk;
         }
-        ck.n = (total + ck.c - 1) / ck.c;
+        ck.n = (ck.vtotal + ck.c - 1) / ck.c;
     }
 
 
@@ -774,138 +822,6 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     uint32_t bq[C::KSTEPS][2];
     int c_k = 0;
     bool alive = true, drained = false;
-    // Pending ticket: the last partial's ticket is read one segment later, so the
-    // atomic's round trip never stalls the warp.
-    int pend_old = 0;
-    bool pend = false;
-    int pend_b = 0, pend_kvh = 0, pend_nb = 0;
-    int pend_fr = 0;
-    bool due = false;  // a partial is written but its ticket is not taken yet
-    int due_b = 0, due_kvh = 0, due_nb = 0;
-    int due_fr = 0, due_ck = 0;
-    auto merge_row = [&](int b, int kvh, int fr, int nb) {
-        // Last segment of the row to finish: merge all of them,
-        //   out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M).
-        // Pass 1: lane (i, h) reads lse of segment i, head h (32 / G segments
-        // per round) and keeps a running (max, sum); the lanes of a head then
-        // combine theirs.  Pass 2: the partial outputs, NB segments x G heads
-        // per round, all loads issued before they are used.
-        const int ch_first = ck.of(fr), ch_last = ck.of(fr + nb - 1);
-        const int nseg = (int)(ch_last - ch_first + 1);
-        auto slot_of = [&](int i) -> int {  // slot of the row's i-th segment
-            const int ch = ch_first + i;
-            return (int)(2 * ch + ((i == 0 && fr > ck.start(ch)) ? 1 : 0));
-        };
-        constexpr int SPP = 32 / G;                 // segments per round of pass 1
-        // segments per round of pass 2 (16 / G at head_dim <= 128; half that at 256,
-        // whose lanes hold twice the dims)
-        constexpr int NB = (D <= 128 ? 16 : 8) / G > 0 ? (D <= 128 ? 16 : 8) / G : 1;
-        const int li = lane / G, lh = lane % G;
-        using V = FVec<C::DPL>;
-        // the first round's partial outputs do not depend on the weights: their loads
-        // go out with the lse loads, so the merge waits for one round trip, not two
-        typename V::type v[NB][G];
-#pragma unroll
-        for (int jj = 0; jj < NB; ++jj) {
-            if (jj < nseg) {
-                const int sl = slot_of(jj);
-#pragma unroll
-                for (int h = 0; h < G; ++h) v[jj][h] = V::ld(a.ws_o + ((size_t)sl * G + h) * D + lane * C::DPL);
-            }
-        }
-        float x0 = -INFINITY;  // lse of (segment li, head lh), first round
-        if (li < nseg) x0 = __ldcg(a.ws_lse + (size_t)slot_of(li) * G + lh);
-        float mx = x0, sm = x0 == -INFINITY ? 0.f : 1.f;
-        for (int i0 = SPP; i0 < nseg; i0 += SPP) {
-            if (i0 + li < nseg) {
-                const float x = __ldcg(a.ws_lse + (size_t)slot_of(i0 + li) * G + lh);
-                const float mn = fmaxf(mx, x);
-                sm = sm * fast_exp2(mx - mn) + fast_exp2(x - mn);
-                mx = mn;
-            }
-        }
-#pragma unroll
-        for (int o = G; o < 32; o <<= 1) {
-            const float mo = __shfl_xor_sync(0xffffffffu, mx, o);
-            const float so = __shfl_xor_sync(0xffffffffu, sm, o);
-            const float mn = fmaxf(mx, mo);
-            sm = (mx == -INFINITY ? 0.f : sm * fast_exp2(mx - mn)) + (mo == -INFINITY ? 0.f : so * fast_exp2(mo - mn));
-            mx = mn;
-        }
-        const float inv_sum = 1.f / sm;  // lane (., h) now holds head h's max and sum
-        float acc[G][C::DPL];
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int e = 0; e < C::DPL; ++e) acc[h][e] = 0.f;
-        for (int i0 = 0; i0 < nseg; i0 += SPP) {
-            float x = x0;
-            if (i0 > 0) x = i0 + li < nseg ? __ldcg(a.ws_lse + (size_t)slot_of(i0 + li) * G + lh) : -INFINITY;
-            const float wl = x == -INFINITY ? 0.f : fast_exp2(x - mx) * inv_sum;  // weight of (i0 + li, lh)
-            for (int j0 = 0; j0 < SPP && i0 + j0 < nseg; j0 += NB) {
-                if (i0 + j0 > 0) {  // the first round's outputs are already loaded
-#pragma unroll
-                    for (int jj = 0; jj < NB; ++jj) {
-                        if (i0 + j0 + jj < nseg) {
-                            const int sl = slot_of(i0 + j0 + jj);
-#pragma unroll
-                            for (int h = 0; h < G; ++h)
-                                v[jj][h] = V::ld(a.ws_o + ((size_t)sl * G + h) * D + lane * C::DPL);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int jj = 0; jj < NB; ++jj) {
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float w = __shfl_sync(0xffffffffu, wl, (j0 + jj) * G + h);
-                        if (i0 + j0 + jj < nseg) {
-#pragma unroll
-                            for (int e = 0; e < C::DPL; ++e) acc[h][e] = fmaf(w, V::get(v[jj][h], e), acc[h][e]);
-                        }
-                    }
-                }
-            }
-        }
-        const int ncol = ncol_of(kvh);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            if (h < ncol) {
-                const size_t o0 = col_row(b, kvh, h) * D + lane * C::DPL;
-#pragma unroll
-                for (int e = 0; e < C::DPL; ++e) store_out<T>(a.out, a.out_f32, o0 + e, acc[h][e]);
-            }
-        }
-        if (lane == 0) a.counters[(size_t)b * Hkv + kvh] = 0;  // the workspace is left as it was found
-    };
-    auto resolve = [&]() {
-        if (!pend) return;
-        pend = false;
-        const int old = __shfl_sync(0xffffffffu, pend_old, 0);
-        const int nseg = (int)(ck.of(pend_fr + pend_nb - 1) - ck.of(pend_fr) + 1);
-        if (old == nseg - 1) {
-            if (lane == 0) fence_acq_rel_gpu();  // acquire the other segments' partials
-            __syncwarp();
-            merge_row(pend_b, pend_kvh, pend_fr, pend_nb);
-        }
-    };
-    // The ticket of a partial is taken kTicketLag blocks after the partial was
-    // written (or at the next partial's end, or at the end), when its stores have
-    // drained, so that the release does not hold the warp; the ticket's result
-    // is read at the next partial's end.
-    constexpr int kTicketLag = 3;
-    auto take_ticket = [&]() {
-        if (!due) return;
-        due = false;
-        __syncwarp();
-        if (lane == 0) pend_old = atom_add_release_gpu(a.counters + (size_t)due_b * Hkv + due_kvh, 1);
-        pend = true;
-        pend_b = due_b;
-        pend_kvh = due_kvh;
-        pend_fr = due_fr;
-        pend_nb = due_nb;
-    };
-
     while (have) {
         const int len = cs.j1 - cs.j0;
         const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;  // tokens in the row's last block
@@ -1061,8 +977,7 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
                     refill();
                     refill();
                     c_k += 2;
-                    if (due && !pend && c_k >= due_ck + kTicketLag) take_ticket();
-                    ++j;  // with the loop's own increment: two blocks
+                            ++j;  // with the loop's own increment: two blocks
                     continue;
                 }
             }
@@ -1231,7 +1146,6 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             __syncwarp();
             refill();
             ++c_k;
-            if (due && !pend && c_k >= due_ck + kTicketLag) take_ticket();
         }
         if (!alive) {
             // A copy did not land within the limit (PA_EFLAG_WAIT_TIMEOUT is raised).
@@ -1239,8 +1153,7 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             // none lands in shared memory after the warp has moved on or exited.  Then
             // this segment and every later one of the warp finish without data: a whole
             // row writes zeros, a partial writes an empty result (o = 0, lse = -inf,
-            // weight 0 in the merge) and takes its ticket, so every row's merge still
-            // runs and the workspace counters return to zero.
+            // weight 0 in the merge), so every slot the merge kernel reads is written.
             if (!drained) {
                 if (lane == 0)
                     for (int k = c_k; k < p_k; ++k) mbar_wait(&my_bars[k % S], (k / S) & 1, a.wait_ns);
@@ -1278,9 +1191,9 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
         } else {
             // Partial of a row cut by chunk boundaries: chunk ch holds at most two
             // partial segments, its first (slot 2ch) and its last (slot 2ch+1).
-            const int ch_first = ck.of(cs.fr), ch_last = ck.of(cs.fr + cs.nb - 1);
+            const int ch_first = ck.of(cs.b, cs.kvh, cs.nb, 0);
             auto slot_of = [&](int ch) -> int {
-                return (int)(2 * ch + ((ch == ch_first && cs.fr > ck.start(ch)) ? 1 : 0));
+                return (int)(2 * ch + ((ch == ch_first && ck.mid_start(cs.b, cs.kvh, cs.nb)) ? 1 : 0));
             };
             const int sl = slot_of(cs.ch);
 #pragma unroll
@@ -1301,20 +1214,597 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
                 if (h0 < G) a.ws_lse[(size_t)sl * G + h0] = m0 + log2f(l0);
                 if (h1 < G) a.ws_lse[(size_t)sl * G + h1] = m1 + log2f(l1);
             }
-            resolve();
-            take_ticket();
-            due = true;
-            due_ck = c_k;
-            due_b = cs.b;
-            due_kvh = cs.kvh;
-            due_fr = cs.fr;
-            due_nb = cs.nb;
         }
         have = next_seg(cit, cs);
     }
-    resolve();
-    take_ticket();
-    resolve();
+}
+
+// ---------------------------------------------------------------------------
+// log-sum-exp merge of the rows the decode kernel cut into partial segments
+// ---------------------------------------------------------------------------
+// Launched right after decode_tc_kernel (programmatic dependent launch): the
+// prologue (effective lengths, blocks per sequence, their prefix sum) runs
+// while the decode kernel finishes; then every warp takes (row, column) items
+// whose row the decode's schedule cut into several segments and merges
+//   out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M),  M = max_i lse_i
+// over the row's segments i (lse in the log2 domain), all of the row's partial
+// loads issued before their use.  Rows that one segment covered were written
+// by the decode kernel and are skipped.
+template <typename T, int D, int G, bool MQ>
+__global__ void __launch_bounds__(256) merge_tc_kernel(const DecodeArgs a) {
+    constexpr int NWM = 8, DPL = D / 32;
+    extern __shared__ int mcum[];  // [B + 1] blocks, then [B + 1] virtual units
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int B = a.B, Hkv = a.Hkv;
+    {
+        __shared__ int wsum[NWM];
+        const int per = (B + NWM * 32 - 1) / (NWM * 32);
+        const int lo = min(B, tid * per), hi = min(B, lo + per);
+        __shared__ int wsumv[NWM];
+        const int gam = a.tc_chunk == 0 ? PA_TC_GAMMA : 0;
+        int s = 0, sv = 0;
+        for (int b = lo; b < hi; ++b) {
+            const int L = min(min(a.lens[b], a.max_len), a.mbps * kBlockSize);
+            const int nb = L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
+            s += nb;
+            sv += nb > 0 ? (nb + gam) * Hkv : 0;
+        }
+        int x = s, xv = sv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o), yv = __shfl_up_sync(0xffffffffu, xv, o);
+            if (lane >= o) {
+                x += y;
+                xv += yv;
+            }
+        }
+        if (lane == 31) {
+            wsum[warp] = x;
+            wsumv[warp] = xv;
+        }
+        __syncthreads();
+        int run = x - s, runv = xv - sv;
+        for (int w = 0; w < warp; ++w) {
+            run += wsum[w];
+            runv += wsumv[w];
+        }
+        for (int b = lo; b < hi; ++b) {
+            mcum[b] = run;
+            mcum[B + 1 + b] = runv;
+            const int L = min(min(a.lens[b], a.max_len), a.mbps * kBlockSize);
+            const int nb = L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
+            run += nb;
+            runv += nb > 0 ? (nb + gam) * Hkv : 0;
+        }
+        if (tid == NWM * 32 - 1) {
+            mcum[B] = run;
+            mcum[2 * B + 1] = runv;
+        }
+        __syncthreads();
+    }
+    // the decode kernel's chunks (same rule, same numbers)
+    const int total = mcum[B] * Hkv;
+    Chunks ck{total, mcum[2 * B + 1], 1, 0, a.tc_chunk == 0 ? PA_TC_GAMMA : 0, Hkv, mcum, mcum + B + 1, B};
+    if (a.tc_chunk > 0) {
+        ck.c = a.tc_chunk;
+    } else {
+        const int wc = min(a.tc_W, kTcMaxChunks);
+        const int c = (ck.vtotal + wc - 1) / wc;
+        ck.c = c > kTcMinChunk ? c : kTcMinChunk;
+    }
+    ck.n = (ck.vtotal + ck.c - 1) / ck.c;
+    pdl_wait();  // the decode kernel's partial results
+    pdl_release_dependents();
+    const int items = B * Hkv * G;
+    for (int it = blockIdx.x * NWM + warp; it < items; it += gridDim.x * NWM) {
+        const int r = it / G, h = it - r * G;
+        const int b = r / Hkv, kvh = r - b * Hkv;
+        const int nb = mcum[b + 1] - mcum[b];
+        if (nb == 0) continue;
+        const int fr = mcum[b] * Hkv + kvh * nb;
+        const int ch_first = ck.of(b, kvh, nb, 0), ch_last = ck.of(b, kvh, nb, nb - 1);
+        if (ch_first == ch_last) continue;  // written by the decode kernel
+        const int ncol = MQ ? min(G, a.gcols - (kvh % a.ngroups) * G) : G;
+        if (h >= ncol) continue;
+        const int nseg = ch_last - ch_first + 1;
+        auto slot_of = [&](int i) -> int {
+            const int ch = ch_first + i;
+            return 2 * ch + ((i == 0 && ck.mid_start(b, kvh, nb)) ? 1 : 0);
+        };
+        // weights: lane i holds segment i's lse (32 segments per round)
+        float mx = -INFINITY, sm = 0.f;
+        for (int i0 = 0; i0 < nseg; i0 += 32) {
+            const float x = i0 + lane < nseg ? __ldcg(a.ws_lse + (size_t)slot_of(i0 + lane) * G + h) : -INFINITY;
+            const float mn = fmaxf(mx, x);
+            sm = (mx == -INFINITY ? 0.f : sm * fast_exp2(mx - mn)) + (x == -INFINITY ? 0.f : fast_exp2(x - mn));
+            mx = mn;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float mo = __shfl_xor_sync(0xffffffffu, mx, o), so = __shfl_xor_sync(0xffffffffu, sm, o);
+            const float mn = fmaxf(mx, mo);
+            sm = (mx == -INFINITY ? 0.f : sm * fast_exp2(mx - mn)) + (mo == -INFINITY ? 0.f : so * fast_exp2(mo - mn));
+            mx = mn;
+        }
+        const float inv = sm > 0.f ? 1.f / sm : 0.f;
+        float acc[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+        constexpr int NBM = DPL >= 8 ? 4 : 8;  // segments per round, loads issued together
+        for (int i0 = 0; i0 < nseg; i0 += NBM) {
+            float v[NBM][DPL];
+            float wl = 0.f;
+            // lane j < NBM: weight of segment i0 + j
+            if (lane < NBM && i0 + lane < nseg) {
+                const float x = __ldcg(a.ws_lse + (size_t)slot_of(i0 + lane) * G + h);
+                wl = x == -INFINITY ? 0.f : fast_exp2(x - mx) * inv;
+            }
+#pragma unroll
+            for (int j = 0; j < NBM; ++j) {
+                if (i0 + j < nseg) {
+                    // DPL = 2, 4 or 8 consecutive floats of this lane, naturally aligned
+                    const float *src = a.ws_o + ((size_t)slot_of(i0 + j) * G + h) * D + lane * DPL;
+                    const typename FVec<DPL>::type x = FVec<DPL>::ld(src);
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) v[j][e] = FVec<DPL>::get(x, e);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < NBM; ++j) {
+                const float w = __shfl_sync(0xffffffffu, wl, j);
+                if (i0 + j < nseg) {
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, v[j][e], acc[e]);
+                }
+            }
+        }
+        // output row of column h
+        size_t orow;
+        if constexpr (!MQ) {
+            orow = (size_t)b * a.Hq + (size_t)kvh * G + h;
+        } else {
+            const int jg = (kvh % a.ngroups) * G + h;
+            const int qi = jg / a.Greal, hh = jg - qi * a.Greal;
+            orow = ((size_t)b * a.qlen + qi) * a.Hq + (size_t)(kvh / a.ngroups) * a.Greal + hh;
+        }
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) store_out<T>(a.out, a.out_f32, orow * D + lane * DPL + e, acc[e]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-cooperative decode for groups of 16, 32 or 64 query heads per KV head
+// ---------------------------------------------------------------------------
+// With G = 8 * NG query heads per cache KV head (MQA-like groups) every K/V
+// tile feeds NG column groups of 8 heads.  decode_tc_kernel runs them as NG
+// separate rows, each warp staging and walking the tile on its own.  Here one
+// CTA of NG warps takes each cache row once: its tiles go through one ring of S
+// shared stages, warp w computes the 8 heads 8w .. 8w + 7, and only lane 0 of
+// warp 0 issues copies.  A stage is refilled once all NG warps have released it
+// (an mbarrier with NG arrivals); warp 0 refills the stage of block k - 1 right
+// after its own block k, so the ring runs S - 1 blocks ahead of it.  Chunks of
+// the cache-row stream go to CTAs (not warps); cut rows leave partial results
+// for merge_tc_kernel, with GC = 8 NG columns per cache row.
+template <typename T, int D, int NG>
+struct CoopCfg {
+    static constexpr int NW = NG;
+    static constexpr int THREADS = NW * 32;
+    static constexpr int MIN_CTAS = NG == 2 ? 4 : (NG == 4 ? 2 : 1);
+    static constexpr int BOXW = 128 / (int)sizeof(T);
+    static constexpr int BOXES = D / BOXW;
+    static constexpr int BOX_BYTES = 16 * 128;
+    static constexpr int TILE = BOXES * BOX_BYTES;
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int RING_BYTES = NG == 2 ? 48 * 1024 : (NG == 4 ? 64 * 1024 : 128 * 1024);
+    static constexpr int S = RING_BYTES / STAGE;
+    static constexpr int KSTEPS = D / 16, MTILES = D / 16;
+    static constexpr int BAR_OFF = S * STAGE;           // full[S], then empty[S]
+    static constexpr int OK_OFF = BAR_OFF + 2 * S * 8;  // int [S]: the stage's block is in the pool
+    static constexpr int CUM_OFF = OK_OFF + S * 4;
+    static int smem_bytes(int B) { return 1024 + CUM_OFF + (3 * B + 3) * 4; }
+};
+
+template <typename T, int D, int NG>
+__global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>::MIN_CTAS)
+    decode_coop_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const DecodeArgs a) {
+    using C = CoopCfg<T, D, NG>;
+    constexpr int S = C::S, GC = NG * 8;
+    constexpr bool SPLIT_P = !std::is_same<T, __half>::value;  // bf16: P = hi + lo
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *empty = full + S;
+    int *stage_ok = reinterpret_cast<int *>(smem + C::OK_OFF);
+    int *cum = reinterpret_cast<int *>(smem + C::CUM_OFF);  // [B + 1]
+    int *lens = cum + a.B + 1;                                // [B]
+    int *cumv = lens + a.B;                                   // [B + 1]
+    __shared__ int abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int B = a.B, Hc = a.Hkv;  // the launcher passes the cache's KV heads
+    if (tid == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        abort_flag = 0;
+    }
+    if (!a.early) {
+        pdl_wait();
+        pdl_release_dependents();
+    }
+    const int gam = a.tc_chunk == 0 ? PA_TC_GAMMA : 0;
+    {
+        __shared__ int wsum[NG], wsumv[NG];
+        const int per = (B + C::THREADS - 1) / C::THREADS;
+        const int lo = min(B, tid * per), hi = min(B, lo + per);
+        int s = 0, sv = 0;
+        for (int b = lo; b < hi; ++b) {
+            const int L = min(min(a.lens[b], a.max_len), a.mbps * kBlockSize);
+            lens[b] = L;
+            const int nb = L > 0 ? (L + kBlockSize - 1) / kBlockSize : 0;
+            s += nb;
+            sv += nb > 0 ? (nb + gam) * Hc : 0;
+        }
+        int x = s, xv = sv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o), yv = __shfl_up_sync(0xffffffffu, xv, o);
+            if (lane >= o) {
+                x += y;
+                xv += yv;
+            }
+        }
+        if (lane == 31) {
+            wsum[warp] = x;
+            wsumv[warp] = xv;
+        }
+        __syncthreads();
+        int run = x - s, runv = xv - sv;
+        for (int w = 0; w < warp; ++w) {
+            run += wsum[w];
+            runv += wsumv[w];
+        }
+        for (int b = lo; b < hi; ++b) {
+            cum[b] = run;
+            cumv[b] = runv;
+            const int nb = lens[b] > 0 ? (lens[b] + kBlockSize - 1) / kBlockSize : 0;
+            run += nb;
+            runv += nb > 0 ? (nb + gam) * Hc : 0;
+        }
+        if (tid == C::THREADS - 1) {
+            cum[B] = run;
+            cumv[B] = runv;
+        }
+        if (tid == 0) {
+            for (int s2 = 0; s2 < S; ++s2) {
+                mbar_init(&full[s2], 1);
+                mbar_init(&empty[s2], NG);
+            }
+            fence_mbar_init();
+        }
+        __syncthreads();
+    }
+    const int total = cum[B] * Hc;
+    Chunks ck{total, cumv[B], 1, 0, gam, Hc, cum, cumv, B};
+    {
+        if (a.tc_chunk > 0) {
+            ck.c = a.tc_chunk;
+        } else {
+            const int wc = min((int)gridDim.x, kTcMaxChunks);
+            const int c = (ck.vtotal + wc - 1) / wc;
+            ck.c = c > kTcMinChunk ? c : kTcMinChunk;
+        }
+        ck.n = (ck.vtotal + ck.c - 1) / ck.c;
+    }
+    auto locate = [&](int f, Seg &sg) {
+        int lo = 0, hi = B;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (cum[mid] * Hc <= f) lo = mid; else hi = mid;
+        }
+        sg.b = lo;
+        sg.nb = cum[lo + 1] - cum[lo];
+        const int off = f - cum[lo] * Hc;
+        sg.kvh = off / sg.nb;
+        sg.j0 = off - sg.kvh * sg.nb;
+        sg.fr = cum[lo] * Hc + sg.kvh * sg.nb;
+        sg.L = lens[lo];
+    };
+    auto range = [&](SegIter &it) -> bool {
+        const int ch = blockIdx.x + it.k * gridDim.x;
+        if (ch >= ck.n) return false;
+        it.f = ck.start(ch);
+        it.fend = ck.end(ch);
+        it.ch = ch;
+        return true;
+    };
+    auto next_seg = [&](SegIter &it, Seg &sg) -> bool {
+        if (it.done) return false;
+        while (it.f >= it.fend) {
+            ++it.k;
+            if (!range(it)) {
+                it.done = true;
+                return false;
+            }
+        }
+        locate(it.f, sg);
+        const int end = min(it.fend, sg.fr + sg.nb);
+        sg.j1 = sg.j0 + (end - it.f);
+        sg.ch = it.ch;
+        sg.ncol = GC;
+        it.f = end;
+        return true;
+    };
+
+    // ---- producer (warp 0): the CTA's block stream, table entries a window ahead ----
+    SegIter pit{0, 0, 0, -1, false};
+    Win pc{}, pn{};
+    int p_y = -1, p_y_next = -1, p_i = 0, p_k = 0;
+    bool p_alive = true;
+    auto win_first = [&](Win &w) {
+        Seg sg;
+        w.valid = next_seg(pit, sg);
+        if (w.valid) {
+            w.sg = sg;
+            w.o = 0;
+            w.n = min(32, sg.j1 - sg.j0);
+            w.kc = sg.kvh;
+        }
+    };
+    auto win_after = [&](const Win &cur, Win &w) {
+        if (!cur.valid) {
+            w.valid = false;
+            return;
+        }
+        const int len = cur.sg.j1 - cur.sg.j0;
+        if (cur.o + 32 < len) {
+            w = cur;
+            w.o = cur.o + 32;
+            w.n = min(32, len - w.o);
+        } else {
+            win_first(w);
+        }
+    };
+    auto win_load = [&](const Win &w) -> int {
+        if (!w.valid || lane >= w.n) return -1;
+        return a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
+    };
+    // issue the copy of the next block of the stream into its stage (warp 0, all lanes)
+    auto refill = [&]() {
+        if (!pc.valid || !p_alive) return;
+        const int s = p_k % S;
+        if (p_k >= S) {  // the stage's previous block must be released by every warp
+            int ok = lane == 0 ? (int)mbar_wait(&empty[s], ((p_k / S) - 1) & 1, a.wait_ns) : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                p_alive = false;
+                if (lane == 0) atomicExch(&abort_flag, 1);
+                return;
+            }
+        }
+        const int pb = __shfl_sync(0xffffffffu, p_y, p_i);
+        const int y = (pb < 0 || (int64_t)pb >= a.N) ? -1 : (pb * Hc + pc.kc) * kBlockSize;
+        if (lane == 0) {
+            stage_ok[s] = y >= 0;
+            if (y < 0) raise_flag(PA_EFLAG_BAD_BLOCK);
+            const bool stall = p_k == a.stall_at && blockIdx.x == 0;
+            // a releasing arrival: stage_ok is read by the other warps after their wait
+            if (y < 0) {
+                mbar_arrive(&full[s]);
+            } else {
+                mbar_arrive_expect_tx(&full[s], (uint32_t)C::STAGE);
+                if (!stall) {
+                    const uint32_t dst = smem_addr(smem) + s * C::STAGE;
+#pragma unroll
+                    for (int bx = 0; bx < C::BOXES; ++bx) {
+                        tma_load_2d(dst + bx * C::BOX_BYTES, &tmK, bx * C::BOXW, y, smem_addr(&full[s]));
+                        tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * C::BOXW, y, smem_addr(&full[s]));
+                    }
+                }
+            }
+        }
+        ++p_k;
+        if (++p_i == pc.n) {
+            p_i = 0;
+            pc = pn;
+            p_y = p_y_next;
+            win_after(pc, pn);
+            p_y_next = win_load(pn);
+        }
+    };
+    if (warp == 0) {
+        pit.done = !range(pit);
+        win_first(pc);
+        win_after(pc, pn);
+        p_y = win_load(pc);
+        p_y_next = win_load(pn);
+    }
+    if (a.early) {
+        pdl_wait();
+        pdl_release_dependents();
+    }
+    // rows of sequences with no token produce zeros
+    for (int r = blockIdx.x * NG + warp; r < B * Hc; r += gridDim.x * NG) {
+        const int b = r / Hc;
+        if (cum[b + 1] == cum[b]) {
+            const int kvh = r % Hc;
+            for (int j = 0; j < GC; ++j)
+                for (int i = lane; i < D; i += 32)
+                    store_out<T>(a.out, a.out_f32, ((size_t)b * a.Hq + (size_t)kvh * GC + j) * D + i, 0.f);
+        }
+    }
+    if (warp == 0)
+        for (int i = 0; i < S; ++i) refill();
+
+    // ---- consumers: every warp, heads 8 warp .. 8 warp + 7 of each row ----
+    const int g = lane >> 2, c = lane & 3;
+    const int h0 = 2 * c, h1 = 2 * c + 1;
+    const int mi = lane >> 3, r8 = lane & 7;
+    uint32_t koff[4], voff[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int kr = r8 + ((mi & 1) << 3), kc = 2 * i + (mi >> 1);
+        koff[i] = kr * 128 + (((kc & 7) ^ (kr & 7)) << 4);
+        const int vr = r8 + ((mi >> 1) << 3), vc = 2 * i + (mi & 1);
+        voff[i] = C::TILE + vr * 128 + (((vc & 7) ^ (vr & 7)) << 4);
+    }
+    SegIter cit{0, 0, 0, -1, false};
+    cit.done = !range(cit);
+    Seg cs;
+    bool have = next_seg(cit, cs);
+    uint32_t bq[C::KSTEPS][2];
+    int c_k = 0;
+    bool alive = true;
+    const int col0 = warp * 8;  // this warp's first column of the row
+    while (have) {
+        const int len = cs.j1 - cs.j0;
+        const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        float o[C::MTILES][4];
+#pragma unroll
+        for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        if (alive) {
+            // q fragments of the warp's 8 heads: head col0 + g, dims 16 ks + 2c, +1 and +8, +9
+            const uint32_t *q32 = reinterpret_cast<const uint32_t *>(a.q) +
+                                  ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + col0 + g) * (D / 2);
+#pragma unroll
+            for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                bq[ks][0] = __ldg(q32 + ks * 8 + c);
+                bq[ks][1] = __ldg(q32 + ks * 8 + 4 + c);
+            }
+        }
+        for (int j = 0; alive && j < len; ++j) {
+            const int s = c_k % S;
+            const uint32_t parity = (c_k / S) & 1;
+            int ok = lane == 0 ? (int)mbar_wait(&full[s], parity, a.wait_ns) : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok && lane != 0) mbar_wait(&full[s], parity, a.wait_ns);
+            if (!ok || *reinterpret_cast<volatile int *>(&abort_flag)) {
+                if (lane == 0) atomicExch(&abort_flag, 1);
+                alive = false;
+                break;
+            }
+            const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
+            const uint32_t tK = smem_addr(smem) + s * C::STAGE;
+            if (stage_ok[s]) {
+                const uint32_t vm_lo = (2 * c < ntok ? 0x0000ffffu : 0u) | (2 * c + 1 < ntok ? 0xffff0000u : 0u);
+                const uint32_t vm_hi = (2 * c + 8 < ntok ? 0x0000ffffu : 0u) | (2 * c + 9 < ntok ? 0xffff0000u : 0u);
+                uint32_t kf[C::KSTEPS][4], vf[C::MTILES][4];
+#pragma unroll
+                for (int ks = 0; ks < C::KSTEPS; ++ks) ldsm_x4(kf[ks], tK + koff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
+#pragma unroll
+                for (int i = 0; i < C::MTILES; ++i) {
+                    ldsm_x4_t(vf[i], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
+                    vf[i][0] &= vm_lo;
+                    vf[i][1] &= vm_lo;
+                    vf[i][2] &= vm_hi;
+                    vf[i][3] &= vm_hi;
+                }
+                float sa[4][4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) sa[u][0] = sa[u][1] = sa[u][2] = sa[u][3] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < C::KSTEPS; ++ks) Mma<T>::mma(sa[ks & 3], kf[ks], bq[ks][0], bq[ks][1]);
+                float sc[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[e] = (sa[0][e] + sa[1][e]) + (sa[2][e] + sa[3][e]);
+                const bool v0 = g < ntok, v1 = g + 8 < ntok;
+                const float s0 = v0 ? sc[0] * a.scale_log2 : -INFINITY, s1 = v0 ? sc[1] * a.scale_log2 : -INFINITY;
+                const float s2 = v1 ? sc[2] * a.scale_log2 : -INFINITY, s3 = v1 ? sc[3] * a.scale_log2 : -INFINITY;
+                float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+                for (int msk = 4; msk < 32; msk <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
+                }
+                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+                const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
+                const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
+                l0 = l0 * al0 + (p0 + p2);
+                l1 = l1 * al1 + (p1 + p3);
+                m0 = mn0;
+                m1 = mn1;
+                if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+                    for (int i = 0; i < C::MTILES; ++i) {
+                        o[i][0] *= al0;
+                        o[i][1] *= al1;
+                        o[i][2] *= al0;
+                        o[i][3] *= al1;
+                    }
+                }
+                const uint32_t ph01 = Mma<T>::pack(p0, p1), ph23 = Mma<T>::pack(p2, p3);
+                const uint32_t pb0 = movm_t(ph01), pb1 = movm_t(ph23);
+                uint32_t pl0 = 0, pl1 = 0;
+                if constexpr (SPLIT_P) {
+                    const float r0 = __uint_as_float(ph01 << 16), r1 = __uint_as_float(ph01 & 0xffff0000u);
+                    const float r2 = __uint_as_float(ph23 << 16), r3 = __uint_as_float(ph23 & 0xffff0000u);
+                    pl0 = movm_t(Mma<T>::pack(p0 - r0, p1 - r1));
+                    pl1 = movm_t(Mma<T>::pack(p2 - r2, p3 - r3));
+                }
+#pragma unroll
+                for (int i = 0; i < C::MTILES; ++i) {
+                    Mma<T>::mma(o[i], vf[i], pb0, pb1);
+                    if constexpr (SPLIT_P) Mma<T>::mma(o[i], vf[i], pl0, pl1);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
+            ++c_k;
+            if (warp == 0) {
+                // keep the ring S - 1 blocks ahead: the next copy goes into the stage of
+                // block c_k - 2, which every warp has usually released by now
+                while (p_alive && pc.valid && p_k < c_k - 1 + S) refill();
+            }
+        }
+        if (!alive) {
+            m0 = m1 = -INFINITY;
+            l0 = l1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        }
+#pragma unroll
+        for (int msk = 4; msk < 32; msk <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, msk);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, msk);
+        }
+        const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+        if (cs.j0 == 0 && cs.j1 == cs.nb) {
+            const size_t out0 = ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + col0 + h0) * D;
+            const size_t out1 = out0 + D;
+#pragma unroll
+            for (int i = 0; i < C::MTILES; ++i) {
+                const int d0 = 16 * i + g, d1 = d0 + 8;
+                store_out<T>(a.out, a.out_f32, out0 + d0, o[i][0] * inv0);
+                store_out<T>(a.out, a.out_f32, out0 + d1, o[i][2] * inv0);
+                store_out<T>(a.out, a.out_f32, out1 + d0, o[i][1] * inv1);
+                store_out<T>(a.out, a.out_f32, out1 + d1, o[i][3] * inv1);
+            }
+        } else {
+            const int ch_first = ck.of(cs.b, cs.kvh, cs.nb, 0);
+            const int sl = 2 * cs.ch + ((cs.ch == ch_first && ck.mid_start(cs.b, cs.kvh, cs.nb)) ? 1 : 0);
+            float *w0 = a.ws_o + ((size_t)sl * GC + col0 + h0) * D;
+            float *w1 = w0 + D;
+#pragma unroll
+            for (int i = 0; i < C::MTILES; ++i) {
+                const int d0 = 16 * i + g, d1 = d0 + 8;
+                w0[d0] = o[i][0] * inv0;
+                w0[d1] = o[i][2] * inv0;
+                w1[d0] = o[i][1] * inv1;
+                w1[d1] = o[i][3] * inv1;
+            }
+            if (g == 0) {
+                a.ws_lse[(size_t)sl * GC + col0 + h0] = m0 + log2f(l0);
+                a.ws_lse[(size_t)sl * GC + col0 + h1] = m1 + log2f(l1);
+            }
+        }
+        have = next_seg(cit, cs);
+    }
+    // no copy may land after the CTA exits: warp 0 waits (bounded) for the ones it issued
+    if (warp == 0 && lane == 0)
+        for (int k = max(0, p_k - S); k < p_k; ++k) mbar_wait(&full[k % S], (k / S) & 1, a.wait_ns);
 }
 
 // ---------------------------------------------------------------------------
@@ -1438,8 +1928,57 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     const int64_t need = (blocks + C::NW - 1) / C::NW;
     if (need < ctas) ctas = need;
     if (ctas < 1) ctas = 1;
-    return launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), smem, st, tk, tv, a) == cudaSuccess ? PA_OK
-                                                                                             : PA_ERR_CUDA;
+    DecodeArgs a2 = a;
+    a2.tc_W = (int)ctas * C::NW;
+    if (launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), smem, st, tk, tv, a2) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (a.tc_chunk < 0 || a.ws_o == nullptr) return PA_OK;  // one pass: nothing to merge
+    auto mk = merge_tc_kernel<T, D, G, MQ>;
+    const int msmem = 2 * (a.B + 1) * 4;
+    if (!set_smem_attr_once(reinterpret_cast<const void *>(mk), 2 * (kTcMaxB + 1) * 4)) return PA_ERR_CUDA;
+    const int64_t items = (int64_t)a.B * a.Hkv * G;
+    int64_t mctas = (items + 7) / 8;
+    if (mctas > 2 * sms) mctas = 2 * sms;
+    return launch_pdl(mk, dim3((unsigned)mctas), dim3(256), msmem, st, a2) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D, int NG>
+static int launch_coop(const DecodeArgs &a, cudaStream_t st) {
+    using C = CoopCfg<T, D, NG>;
+    auto kern = decode_coop_kernel<T, D, NG>;
+    DecodeArgs a2 = a;
+    a2.Hkv = a.Hkv / a.ngroups;  // cache rows; GC = 8 NG columns each
+    a2.ngroups = 1;
+    a2.G = NG * 8;
+    a2.gcols = NG * 8;
+    const int smem = C::smem_bytes(a.B);
+    if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
+    CUtensorMap tk, tv;
+    const int64_t rows = a.N * a2.Hkv * kBlockSize;
+    if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
+        return PA_ERR_CUDA;
+    int sms = 0, per_sm = 0;
+    if (!launch_shape(reinterpret_cast<const void *>(kern), C::THREADS, smem, &sms, &per_sm)) return PA_ERR_CUDA;
+    const int64_t blocks = (int64_t)a.B * a2.Hkv * ((a.max_len + kBlockSize - 1) / kBlockSize);
+    int64_t ctas = (int64_t)sms * per_sm;
+    const int64_t need = (blocks + kTcMinChunk - 1) / kTcMinChunk;
+    if (need < ctas) ctas = need;
+    if (ctas < 1) ctas = 1;
+    a2.tc_W = (int)ctas;
+    if (launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), smem, st, tk, tv, a2) != cudaSuccess)
+        return PA_ERR_CUDA;
+    auto mk = merge_tc_kernel<T, D, NG * 8, false>;
+    const int msmem = 2 * (a.B + 1) * 4;
+    if (!set_smem_attr_once(reinterpret_cast<const void *>(mk), 2 * (kTcMaxB + 1) * 4)) return PA_ERR_CUDA;
+    const int64_t items = (int64_t)a.B * a2.Hkv * NG * 8;
+    int64_t mctas = (items + 7) / 8;
+    if (mctas > 2 * sms) mctas = 2 * sms;
+    return launch_pdl(mk, dim3((unsigned)mctas), dim3(256), msmem, st, a2) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+bool decode_coop_eligible(int q_dtype, int kv_dtype, int D, int G, int ngroups, int qlen, bool padded, int part) {
+    return (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype && (D == 64 || D == 128) && G == 8 &&
+           (ngroups == 2 || ngroups == 4 || ngroups == 8) && qlen == 1 && !padded && part != 0;
 }
 
 template <typename T, typename TKV, int D, bool MQ>
@@ -1457,6 +1996,15 @@ template <typename T, typename TKV, int D>
 static int launch_tc_g(const DecodeArgs &a, cudaStream_t st) {
     // several new tokens, or padding columns: the general column mapping
     const bool mq = a.qlen > 1 || (int64_t)a.G * a.ngroups != a.gcols;
+    if constexpr (std::is_same<T, TKV>::value && D <= 128) {
+        if (decode_coop_eligible(a.q_dtype, a.kv_dtype, D, a.G, a.ngroups, a.qlen, mq, a.tc_chunk < 0 ? 0 : 1)) {
+            switch (a.ngroups) {
+            case 2: return launch_coop<T, D, 2>(a, st);
+            case 4: return launch_coop<T, D, 4>(a, st);
+            default: return launch_coop<T, D, 8>(a, st);
+            }
+        }
+    }
     return mq ? launch_tc_mq<T, TKV, D, true>(a, st) : launch_tc_mq<T, TKV, D, false>(a, st);
 }
 

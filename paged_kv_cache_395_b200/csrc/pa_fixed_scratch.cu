@@ -1,7 +1,7 @@
 // Split-K decode with a scratch area compiled into the library.
 //
-// pa_decode's split-K modes keep their partial outputs, log-sum-exp values and
-// merge counters in a workspace the caller allocates.  Some callers cannot
+// pa_decode's split-K modes keep their partial outputs and log-sum-exp values
+// in a workspace the caller allocates.  Some callers cannot
 // allocate device memory where they decode: an engine that has handed all free
 // device memory to its KV block pool up front, or a host integration that has
 // no device allocator of its own.  pa_decode_fixed_scratch serves them: it runs
@@ -12,18 +12,16 @@
 // The area is one file-scope __device__ array of PA_FIXED_SCRATCH_BYTES, so each
 // device that loads this module holds one copy.  Because of that:
 //   * the first call on a device does the setup: it looks up the array's device
-//     address (cudaGetSymbolAddress, with that device current), clears it on
-//     the call's stream and waits for the clear; make that first call before
-//     any stream capture;
+//     address (cudaGetSymbolAddress, with that device current); make that first
+//     call before any stream capture.  Nothing in the area needs clearing: every
+//     value a call reads there was written earlier in the same call;
 //   * all calls on one device share the one area, so calls that overlap on the
 //     device (on different streams, or from different host threads without
 //     ordering) race on it: issue them in one stream order;
 //   * parameters whose workspace is larger than PA_FIXED_SCRATCH_BYTES are
 //     rejected with PA_ERR_WORKSPACE before anything is launched;
-//   * calls with different parameters share the area safely: like every
-//     workspace, it keeps the merge counters in a fixed region at its start that
-//     no partial result ever occupies, and every call (one whose bounded wait gave
-//     up included) returns them to zero;
+//   * calls with different parameters share the area safely, for the same
+//     reason;
 //   * the device address is looked up once per device and kept for the process:
 //     after cudaDeviceReset the library must not be used again (its kernel
 //     attributes and encoded copy descriptors are per-context state as well).
@@ -43,10 +41,9 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices];  // device address of g_fixed_scratch per device, once set up
 
-// Device address of the fixed area on the current device; the first call per
-// device looks it up and clears it (the merge counters at its start must start
-// at zero; every decode leaves them at zero again).
-int fixed_scratch(cudaStream_t st, void **out) {
+// Device address of the fixed area on the current device, looked up by the first
+// call per device.
+int fixed_scratch(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
@@ -54,8 +51,6 @@ int fixed_scratch(cudaStream_t st, void **out) {
     if (g_scratch_ptr[dev] == nullptr) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
-        if (cudaMemsetAsync(p, 0, PA_FIXED_SCRATCH_BYTES, st) != cudaSuccess) return PA_ERR_CUDA;
-        if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
         g_scratch_ptr[dev] = p;
     }
     *out = g_scratch_ptr[dev];
@@ -76,7 +71,7 @@ extern "C" int pa_decode_fixed_scratch(void *out, const void *q, const void *key
     if (need > PA_FIXED_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
     if (need > 0) {
         void *ws = nullptr;
-        const int rc = pa::fixed_scratch(reinterpret_cast<cudaStream_t>(stream), &ws);
+        const int rc = pa::fixed_scratch(&ws);
         if (rc != PA_OK) return rc;
         p2.workspace = ws;
         p2.workspace_bytes = PA_FIXED_SCRATCH_BYTES;

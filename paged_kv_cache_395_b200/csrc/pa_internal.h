@@ -57,10 +57,9 @@ struct DecodeArgs {
     int max_parts;           // ceil(max_len / part) when part > 0
     float *ws_o;             // [B][Hq][max_parts][D]
     float *ws_lse;           // [B][Hq][max_parts]  (log2 domain)
-    int *counters;           // [B][Hkv] merge tickets at the start of the workspace, zero
-                             // between calls
     int tc_chunk;            // tensor-core schedule: blocks per chunk, 0 = balanced auto,
                              // -1 = whole rows (one pass)
+    int tc_W;                // warps of the tensor-core decode grid (its merge kernel redoes the schedule)
     int early;               // PA_DECODE_INPUTS_READY: read lengths, tables and q before
                              // the previous kernel on the stream has finished
     int out_f32;             // PA_DECODE_OUT_F32: out is fp32 of q's shape
@@ -69,14 +68,6 @@ struct DecodeArgs {
     unsigned long long wait_ns;  // limit of every bounded wait on a copy
 };
 
-// The tensor-core family's merge counters occupy the first kCounterBytes of every
-// split-K workspace, one int per (sequence, kernel KV head) row, whatever the
-// parameters or the family of the call; partial results always start after them.
-// So a counter never lands on memory that an earlier call with other parameters
-// filled with partial results, and a workspace shared by calls of any shape stays
-// valid.  Split-K on the tensor-core family therefore needs B * H_kv <= kCounterRows.
-constexpr int kCounterRows = PA_WORKSPACE_COUNTER_BYTES / 4;
-constexpr size_t kCounterBytes = PA_WORKSPACE_COUNTER_BYTES;
 // Default limit of a bounded wait: one second.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
@@ -99,10 +90,12 @@ int error_word_decode_tc(unsigned int *flags, bool reset);
 // (kernel, device).  Thread-safe; returns false if CUDA refuses.
 bool set_smem_attr_once(const void *kernel, int bytes);
 
-// Workspace layout for split-K: ws_o | ws_lse | counters, each 256-byte aligned.
+// Workspace layout for split-K: ws_o | ws_lse, each 256-byte aligned.
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int part);
 int launch_decode_tc(const DecodeArgs &a, cudaStream_t st);
 bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B);
+// groups of 16, 32 or 64 query heads per KV head run one CTA per cache row
+bool decode_coop_eligible(int q_dtype, int kv_dtype, int D, int G, int ngroups, int qlen, bool padded, int part);
 int launch_decode_simt(const DecodeArgs &a, cudaStream_t st);
 int launch_merge(const DecodeArgs &a, cudaStream_t st);
 bool decode_simt_supported(int q_dtype, int kv_dtype, int D, int G);

@@ -30,7 +30,6 @@ PA_ALGO_AUTO, PA_ALGO_SIMT, PA_ALGO_TENSOR = 0, 1, 2
 PA_EFLAG_BAD_BLOCK, PA_EFLAG_BAD_SLOT, PA_EFLAG_BAD_PAIR, PA_EFLAG_WAIT_TIMEOUT = 1, 2, 4, 8
 PA_DECODE_INPUTS_READY, PA_DECODE_OUT_F32 = 1, 2
 PA_APPEND_OVERLAP_PREVIOUS = 1
-WORKSPACE_COUNTER_BYTES = 256 * 1024  # PA_WORKSPACE_COUNTER_BYTES
 BLOCK_SIZE = 16
 
 # a uint8 cache tensor [N][H_kv][16][d/2] holds 4-bit values, two per byte
@@ -197,10 +196,10 @@ def pa_decode_workspace_size(q, key_cache, block_tables, max_seq_len, partition_
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor | None:
-    """Split-K workspace; zero-filled, as pa_decode requires before first use."""
+    """Split-K workspace (left uninitialised: pa_decode needs none)."""
     if nbytes == 0:
         return None
-    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
 def _out_flag(out, q) -> int:

@@ -191,14 +191,12 @@ class StepCalls:
                     p = pa.make_params(q, kc, bt, mx, ks, vs, partition_size, self.workspace, algo,
                                        flags)
                     self.keep.append(p)
+                    # a split decode is followed by its merge kernel (both families)
                     split = pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
-                    # the tensor-core family merges inside its decode kernel; the
-                    # CUDA-core family launches a merge kernel after a split decode
-                    tc = pa.lib.pa_decode_algo(ctypes.byref(p), ptr(q)) == pa.PA_ALGO_TENSOR
                     args = (ptr(out), ptr(q), ptr(kc), ptr(vc), ptr(bt), ptr(sl),
                             ctypes.c_float(w.scale), ctypes.byref(p), sp)
                     calls.append(("decode", pa.lib.pa_decode, args))
-                    launches += 2 if (split and not tc) else 1
+                    launches += 2 if split else 1
             self.calls[i] = calls
             self.launches[i] = launches
 

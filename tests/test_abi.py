@@ -95,29 +95,27 @@ def test_decode_null_and_workspace_checks():
     assert rc == pa.PA_ERR_NULL
     p = params(partition_size=16, algo=pa.PA_ALGO_SIMT)  # split-K without a workspace
     need = pa.lib.pa_decode_workspace_size(ctypes.byref(p))
-    # CUDA-core family: the fixed merge-counter region (kept free in every workspace),
-    # then 2 seqs x 8 heads x 4 partitions x 128 floats and their 64 lse floats,
-    # each region rounded up to 256 B
-    C = pa.WORKSPACE_COUNTER_BYTES
-    assert need == C + 2 * 8 * 4 * 128 * 4 + 256
+    # CUDA-core family: 2 seqs x 8 heads x 4 partitions x 128 floats and their 64
+    # lse floats, each region rounded up to 256 B
+    assert need == 2 * 8 * 4 * 128 * 4 + 256
     rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
     assert rc == pa.PA_ERR_WORKSPACE
     p.workspace, p.workspace_bytes = 0x1000, need - 1
     rc = pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p), None)
     assert rc == pa.PA_ERR_WORKSPACE
-    # tensor-core family: the counters, then 2 x 2 rows x 4 blocks = 16 blocks in
-    # chunks of 1 block -> 32 partial slots of 4 heads x (128 + 1) floats
+    # tensor-core family: 2 x 2 rows x 4 blocks = 16 blocks in chunks of 1 block ->
+    # 32 partial slots of 4 heads x (128 + 1) floats
     p = params(partition_size=16, algo=pa.PA_ALGO_TENSOR)
-    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == C + 32 * 4 * 128 * 4 + 512
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == 32 * 4 * 128 * 4 + 512
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(params(partition_size=0, algo=pa.PA_ALGO_TENSOR))) == 0
-    # auto schedule on the tensor-core family: the counters, then at most 2048 chunks
-    # (one per warp), two partial slots each
+    # auto schedule on the tensor-core family: at most 2048 chunks (one per warp),
+    # two partial slots each
     p = params(partition_size=-1, algo=pa.PA_ALGO_TENSOR, num_seqs=64, max_blocks_per_seq=264,
                max_seq_len=4224)
     slots = 2 * 2048
     up = lambda x: (x + 255) // 256 * 256
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == \
-        C + up(slots * 4 * 128 * 4) + up(slots * 4 * 4)
+        up(slots * 4 * 128 * 4) + up(slots * 4 * 4)
     # the tensor-core family needs fp16/bf16 q and cache
     p = params(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p),
@@ -223,24 +221,18 @@ def test_decode_algo_reports_the_family():
     assert algo(params(flags=pa.PA_DECODE_OUT_F32 | pa.PA_DECODE_INPUTS_READY)) == pa.PA_ALGO_TENSOR
 
 
-def test_counter_region_bounds_the_tensor_core_split():
-    """The tensor-core family's split keeps one merge counter per (sequence, KV
-    head) row in the fixed counter region: beyond its 65536 rows the library-picked
-    schedule runs in one pass (no workspace), an explicit split goes to the
-    CUDA-core family, and the tensor-core family refuses it."""
-    rows = pa.WORKSPACE_COUNTER_BYTES // 4
-    assert rows == 4096 * 16
-    fit = params(num_seqs=4096, num_q_heads=64, num_kv_heads=16, partition_size=-1,
-                 max_blocks_per_seq=64, max_seq_len=1024)
-    over = params(num_seqs=4096, num_q_heads=128, num_kv_heads=32, partition_size=-1,
-                  max_blocks_per_seq=64, max_seq_len=1024)
-    assert pa.lib.pa_decode_workspace_size(ctypes.byref(fit)) > 0
-    assert pa.lib.pa_decode_workspace_size(ctypes.byref(over)) == 0
-    assert pa.lib.pa_decode_algo(ctypes.byref(over), ctypes.c_void_p(0x1000)) == pa.PA_ALGO_TENSOR
-    over.partition_size = 256
-    assert pa.lib.pa_decode_algo(ctypes.byref(over), ctypes.c_void_p(0x1000)) == pa.PA_ALGO_SIMT
-    over.algo = pa.PA_ALGO_TENSOR
-    assert pa.lib.pa_decode_algo(ctypes.byref(over), ctypes.c_void_p(0x1000)) == pa.PA_ERR_UNSUPPORTED
+def test_large_groups_plan_the_cooperative_mode():
+    """Groups of 16, 32 or 64 fp16/bf16 query heads per KV head at head_dim 64/128
+    split in the cooperative mode: one partial slot holds all G columns of a cache
+    row, chunks are cut over cache rows.  Its workspace: 2 slots per chunk of the
+    cache-row stream (at most 2048 chunks) x G x (d + 1) floats."""
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    for hq, hkv in ((16, 1), (32, 1), (64, 1), (32, 2)):
+        p = params(num_seqs=4, num_q_heads=hq, num_kv_heads=hkv, max_blocks_per_seq=64, max_seq_len=1024,
+                   partition_size=-1, algo=pa.PA_ALGO_TENSOR)
+        chunks = min(4 * hkv * 64, 2048)
+        assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) == \
+            up(2 * chunks * (hq // hkv) * 128 * 4) + up(2 * chunks * (hq // hkv) * 4), (hq, hkv)
 
 
 def test_stall_selftest_rejects_bad_args():

@@ -3,9 +3,9 @@ against pa_decode with a caller-allocated workspace, and against the oracle.
 
 The file name sorts last so that, in a full run, these calls come after every
 other test has used the device; the tests also pass when run alone.  Two calls
-in a row check that a call leaves the fixed area ready for the next one (its
-merge counters back at zero); calls with different parameters in a row check
-that the counters' place does not move with the parameters.
+in a row check that a call leaves the fixed area ready for the next one, and
+calls with different parameters in a row that nothing one call leaves there
+matters to the next.
 """
 import numpy as np
 import pytest
@@ -100,8 +100,7 @@ def test_fixed_scratch_alternating_parameter_sets():
     7-sequence batch split into 16-token partitions, then a 3-sequence batch with
     256-token partitions, the CUDA-core family's split (its partial results start
     at the same offset as the tensor-core family's), and the first case again.
-    Each call against pa_decode with a fresh zeroed workspace and against the
-    oracle."""
+    Each call against pa_decode with a fresh workspace and against the oracle."""
     cases = [
         (W.random_case([1, 16, 17, 100, 513, 1000, 2047], num_q_heads=32, num_kv_heads=8, head_dim=128,
                        dtype="float16", seed=60), 16, pa.PA_ALGO_TENSOR),
