@@ -54,8 +54,8 @@ FALLBACK_HBM_GBS = 6650.0
 # It holds only for the kernel code it was taken on (hash of the source without
 # comments); after any code change the bench reports null until it is taken again.
 NCU_TRAFFIC = {
-    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "8c024d7969aaa774",
-               "per_alg_byte": (475635968 + 4611328 + 462733312 + 4428800) / (472969728 + 459894508)},
+    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "1435942a2a2a7598",
+               "per_alg_byte": (474932736 + 5912064 + 462019840 + 4562944) / (472969728 + 459894508)},
 }
 
 

@@ -1312,8 +1312,23 @@ __global__ void __launch_bounds__(256) merge_tc_kernel(const DecodeArgs a) {
             return 2 * ch + ((i == 0 && ck.mid_start(b, kvh, nb)) ? 1 : 0);
         };
         // weights: lane i holds segment i's lse (32 segments per round)
-        float mx = -INFINITY, sm = 0.f;
-        for (int i0 = 0; i0 < nseg; i0 += 32) {
+        constexpr int NBM = DPL >= 8 ? 4 : 8;  // segments per round, loads issued together
+        // The first round's partial outputs do not depend on the weights: they are
+        // loaded together with the lse values, so a row of up to NBM segments costs one
+        // round trip.  Lane i holds segment i's lse (32 per round).
+        float v[NBM][DPL];
+#pragma unroll
+        for (int j = 0; j < NBM; ++j) {
+            if (j < nseg) {
+                // DPL = 2, 4 or 8 consecutive floats of this lane, naturally aligned
+                const typename FVec<DPL>::type x = FVec<DPL>::ld(a.ws_o + ((size_t)slot_of(j) * G + h) * D + lane * DPL);
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) v[j][e] = FVec<DPL>::get(x, e);
+            }
+        }
+        const float x0 = lane < nseg ? __ldcg(a.ws_lse + (size_t)slot_of(lane) * G + h) : -INFINITY;
+        float mx = x0, sm = x0 == -INFINITY ? 0.f : 1.f;
+        for (int i0 = 32; i0 < nseg; i0 += 32) {
             const float x = i0 + lane < nseg ? __ldcg(a.ws_lse + (size_t)slot_of(i0 + lane) * G + h) : -INFINITY;
             const float mn = fmaxf(mx, x);
             sm = (mx == -INFINITY ? 0.f : sm * fast_exp2(mx - mn)) + (x == -INFINITY ? 0.f : fast_exp2(x - mn));
@@ -1327,31 +1342,31 @@ __global__ void __launch_bounds__(256) merge_tc_kernel(const DecodeArgs a) {
             mx = mn;
         }
         const float inv = sm > 0.f ? 1.f / sm : 0.f;
+        const float w0 = x0 == -INFINITY ? 0.f : fast_exp2(x0 - mx) * inv;  // weight of segment lane
         float acc[DPL];
 #pragma unroll
         for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-        constexpr int NBM = DPL >= 8 ? 4 : 8;  // segments per round, loads issued together
         for (int i0 = 0; i0 < nseg; i0 += NBM) {
-            float v[NBM][DPL];
             float wl = 0.f;
-            // lane j < NBM: weight of segment i0 + j
-            if (lane < NBM && i0 + lane < nseg) {
-                const float x = __ldcg(a.ws_lse + (size_t)slot_of(i0 + lane) * G + h);
-                wl = x == -INFINITY ? 0.f : fast_exp2(x - mx) * inv;
-            }
+            if (i0 > 0) {
 #pragma unroll
-            for (int j = 0; j < NBM; ++j) {
-                if (i0 + j < nseg) {
-                    // DPL = 2, 4 or 8 consecutive floats of this lane, naturally aligned
-                    const float *src = a.ws_o + ((size_t)slot_of(i0 + j) * G + h) * D + lane * DPL;
-                    const typename FVec<DPL>::type x = FVec<DPL>::ld(src);
+                for (int j = 0; j < NBM; ++j) {
+                    if (i0 + j < nseg) {
+                        const typename FVec<DPL>::type x =
+                            FVec<DPL>::ld(a.ws_o + ((size_t)slot_of(i0 + j) * G + h) * D + lane * DPL);
 #pragma unroll
-                    for (int e = 0; e < DPL; ++e) v[j][e] = FVec<DPL>::get(x, e);
+                        for (int e = 0; e < DPL; ++e) v[j][e] = FVec<DPL>::get(x, e);
+                    }
+                }
+                // segments past the first 32: their weights from their lse, lane j < NBM
+                if (i0 >= 32 && lane < NBM && i0 + lane < nseg) {
+                    const float x = __ldcg(a.ws_lse + (size_t)slot_of(i0 + lane) * G + h);
+                    wl = x == -INFINITY ? 0.f : fast_exp2(x - mx) * inv;
                 }
             }
 #pragma unroll
             for (int j = 0; j < NBM; ++j) {
-                const float w = __shfl_sync(0xffffffffu, wl, j);
+                const float w = i0 < 32 ? __shfl_sync(0xffffffffu, w0, i0 + j) : __shfl_sync(0xffffffffu, wl, j);
                 if (i0 + j < nseg) {
 #pragma unroll
                     for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, v[j][e], acc[e]);

@@ -76,7 +76,7 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 // blocks; the per-CTA prefix sum holds at most kTcMaxB sequences.
 constexpr int kTcMaxChunks = 2048;
 #ifndef PA_TC_MIN_CHUNK
-#define PA_TC_MIN_CHUNK 8
+#define PA_TC_MIN_CHUNK 4
 #endif
 constexpr int kTcMinChunk = PA_TC_MIN_CHUNK;
 constexpr int kTcMaxB = 4096;
