@@ -94,6 +94,32 @@ __device__ __forceinline__ void store_out(void *out, int f32, size_t idx, float 
         reinterpret_cast<T *>(out)[idx] = Cvt<T>::from_f(v);
 }
 
+// Elements idx, idx + 1 (idx even) of a decode output, as one 4- or 8-byte store
+// when the buffer's base allows it.
+template <typename T>
+__device__ __forceinline__ void store_out2(void *out, int f32, size_t idx, float v0, float v1) {
+    if (f32) {
+        float *o = reinterpret_cast<float *>(out) + idx;
+        if (((uintptr_t)out & 7) == 0) {
+            *reinterpret_cast<float2 *>(o) = make_float2(v0, v1);
+        } else {
+            o[0] = v0;
+            o[1] = v1;
+        }
+    } else {
+        T *o = reinterpret_cast<T *>(out) + idx;
+        const T h0 = Cvt<T>::from_f(v0), h1 = Cvt<T>::from_f(v1);
+        if (((uintptr_t)out & 3) == 0) {
+            const uint32_t w = (uint32_t)*reinterpret_cast<const uint16_t *>(&h0) |
+                               ((uint32_t)*reinterpret_cast<const uint16_t *>(&h1) << 16);
+            *reinterpret_cast<uint32_t *>(o) = w;
+        } else {
+            o[0] = h0;
+            o[1] = h1;
+        }
+    }
+}
+
 // Convert N consecutive elements held in registers (as raw 32-bit words) to float.
 template <typename T, int N>
 __device__ __forceinline__ void to_float(const uint32_t *w, float *f);

@@ -43,7 +43,8 @@
 // slowest warps: a separate merge kernel measured 7% faster on the ragged trace.)
 //
 // Groups of 16, 32 or 64 query heads per KV head run in decode_coop_kernel
-// (one CTA per chunk of cache rows, its warps sharing each staged tile).
+// (one CTA per chunk of cache rows, its warps sharing each staged tile, with
+// the heads on the M side of the MMA).
 #include <cudaTypedefs.h>
 
 #include <map>
@@ -1390,41 +1391,57 @@ __global__ void __launch_bounds__(256) merge_tc_kernel(const DecodeArgs a) {
 // ---------------------------------------------------------------------------
 // CTA-cooperative decode for groups of 16, 32 or 64 query heads per KV head
 // ---------------------------------------------------------------------------
-// With G = 8 * NG query heads per cache KV head (MQA-like groups) every K/V
-// tile feeds NG column groups of 8 heads.  decode_tc_kernel runs them as NG
-// separate rows, each warp staging and walking the tile on its own.  Here one
-// CTA of NG warps takes each cache row once: its tiles go through one ring of S
-// shared stages, warp w computes the 8 heads 8w .. 8w + 7, and only lane 0 of
-// warp 0 issues copies.  A stage is refilled once all NG warps have released it
-// (an mbarrier with NG arrivals); warp 0 refills the stage of block k - 1 right
-// after its own block k, so the ring runs S - 1 blocks ahead of it.  Chunks of
-// the cache-row stream go to CTAs (not warps); cut rows leave partial results
-// for merge_tc_kernel, with GC = 8 NG columns per cache row.
+// With G = 16 * NG query heads per cache KV head (MQA-like groups) the group is
+// wide enough to fill the M side of the MMA, so the contraction is laid out the
+// other way round from decode_tc_kernel, with the heads as rows:
+//   S[16 heads x 16 tokens]  = Q[16 x d] . K^T[d x 16]   (A = q, kept in registers
+//                                                          for the whole segment)
+//   O[16 heads x d]         += P[16 x 16] . V[16 x d]     (A = P, taken straight from
+//                                                          the S accumulators)
+// so one ldmatrix of K or V feeds 16 heads and P needs no transpose.  One CTA of
+// NG warps takes each cache row once: its tiles go through one ring of S shared
+// stages, warp w computes the 16 heads 16w .. 16w + 15, and only lane 0 of warp 0
+// issues copies.  A stage is refilled once all NG warps have released it (an
+// mbarrier with NG arrivals); with NG > 1 warp 0 refills the stage of block k - 1
+// right after its own block k (a warp that lags by one block does not hold it
+// up), so the ring runs S - 1 blocks ahead of it.  Chunks of the cache-row stream
+// go to CTAs (not warps); cut rows leave partial results for merge_tc_kernel,
+// with GC = 16 NG columns per cache row.
+//
+// The running maximum moves only when a block's scores exceed it by more than
+// kLazyMax (in log2 units): until then the probabilities are taken against the
+// old maximum (at most 2^kLazyMax, exact in fp32 and rounded to the same
+// relative precision in fp16/bf16), and O and l need no rescale.  The result
+// is the same softmax: numerator and denominator share the reference point.
 template <typename T, int D, int NG>
 struct CoopCfg {
     static constexpr int NW = NG;
     static constexpr int THREADS = NW * 32;
-    static constexpr int MIN_CTAS = NG == 2 ? 4 : (NG == 4 ? 2 : 1);
+    // eight warps per SM: the q fragments (32 registers) and O (64 at d = 128) stay in
+    // registers, ~220 in all
+    static constexpr int MIN_CTAS = 8 / NG;
     static constexpr int BOXW = 128 / (int)sizeof(T);
     static constexpr int BOXES = D / BOXW;
     static constexpr int BOX_BYTES = 16 * 128;
     static constexpr int TILE = BOXES * BOX_BYTES;
     static constexpr int STAGE = 2 * TILE;
-    static constexpr int RING_BYTES = NG == 2 ? 48 * 1024 : (NG == 4 ? 64 * 1024 : 128 * 1024);
+    static constexpr int RING_BYTES = NG == 1 ? 16 * 1024 : (NG == 2 ? 32 * 1024 : 64 * 1024);
     static constexpr int S = RING_BYTES / STAGE;
-    static constexpr int KSTEPS = D / 16, MTILES = D / 16;
+    static constexpr int LAG = NG == 1 ? 0 : 1;  // blocks the refill trails the consumer by
+    static constexpr int KSTEPS = D / 16, NT = D / 8;
     static constexpr int BAR_OFF = S * STAGE;           // full[S], then empty[S]
     static constexpr int OK_OFF = BAR_OFF + 2 * S * 8;  // int [S]: the stage's block is in the pool
     static constexpr int CUM_OFF = OK_OFF + S * 4;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (3 * B + 3) * 4; }
 };
+constexpr float kLazyMax = 8.f;
 
 template <typename T, int D, int NG>
 __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>::MIN_CTAS)
     decode_coop_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const DecodeArgs a) {
     using C = CoopCfg<T, D, NG>;
-    constexpr int S = C::S, GC = NG * 8;
+    constexpr int S = C::S, GC = NG * 16;
     constexpr bool SPLIT_P = !std::is_same<T, __half>::value;  // bf16: P = hi + lo
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem =
@@ -1652,41 +1669,47 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
     if (warp == 0)
         for (int i = 0; i < S; ++i) refill();
 
-    // ---- consumers: every warp, heads 8 warp .. 8 warp + 7 of each row ----
+    // ---- consumers: every warp, heads 16 warp .. 16 warp + 15 of each row ----
+    // Fragment coordinates: thread (g, c) holds rows (heads) g and g + 8 and
+    // columns 2c, 2c + 1 (+ 8) of every 16 x 16 / 16 x 8 tile.
     const int g = lane >> 2, c = lane & 3;
-    const int h0 = 2 * c, h1 = 2 * c + 1;
+    // ldmatrix lane addresses (128-byte swizzle): matrix mi = lane / 8 is token
+    // rows 8 (mi >> 1) .. + 7 and the 16-byte chunk 2i + (mi & 1) of the row.
+    // Non-transposed on K this gives the B fragments of S for both 8-token halves
+    // of k-step i; transposed on V, those of O for dims 16i .. 16i + 15.
     const int mi = lane >> 3, r8 = lane & 7;
-    uint32_t koff[4], voff[4];
+    uint32_t moff[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int kr = r8 + ((mi & 1) << 3), kc = 2 * i + (mi >> 1);
-        koff[i] = kr * 128 + (((kc & 7) ^ (kr & 7)) << 4);
-        const int vr = r8 + ((mi >> 1) << 3), vc = 2 * i + (mi & 1);
-        voff[i] = C::TILE + vr * 128 + (((vc & 7) ^ (vr & 7)) << 4);
+        const int r = r8 + ((mi >> 1) << 3), ch = 2 * i + (mi & 1);
+        moff[i] = r * 128 + (((ch & 7) ^ (r & 7)) << 4);
     }
     SegIter cit{0, 0, 0, -1, false};
     cit.done = !range(cit);
     Seg cs;
     bool have = next_seg(cit, cs);
-    uint32_t bq[C::KSTEPS][2];
+    uint32_t qa[C::KSTEPS][4];
     int c_k = 0;
     bool alive = true;
-    const int col0 = warp * 8;  // this warp's first column of the row
+    const int row0 = warp * 16;  // this warp's first column (head) of the row
     while (have) {
         const int len = cs.j1 - cs.j0;
         const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;
-        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-        float o[C::MTILES][4];
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads g, g + 8
+        float o[C::NT][4];
 #pragma unroll
-        for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        for (int i = 0; i < C::NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
         if (alive) {
-            // q fragments of the warp's 8 heads: head col0 + g, dims 16 ks + 2c, +1 and +8, +9
-            const uint32_t *q32 = reinterpret_cast<const uint32_t *>(a.q) +
-                                  ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + col0 + g) * (D / 2);
+            // A fragments of q: heads row0 + g (+ 8), dims 16 ks + 2c, +1 (+ 8)
+            const uint32_t *q0 = reinterpret_cast<const uint32_t *>(a.q) +
+                                 ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + row0 + g) * (D / 2);
+            const uint32_t *q1 = q0 + 8 * (D / 2);
 #pragma unroll
             for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                bq[ks][0] = __ldg(q32 + ks * 8 + c);
-                bq[ks][1] = __ldg(q32 + ks * 8 + 4 + c);
+                qa[ks][0] = __ldg(q0 + ks * 8 + c);
+                qa[ks][1] = __ldg(q1 + ks * 8 + c);
+                qa[ks][2] = __ldg(q0 + ks * 8 + 4 + c);
+                qa[ks][3] = __ldg(q1 + ks * 8 + 4 + c);
             }
         }
         for (int j = 0; alive && j < len; ++j) {
@@ -1701,118 +1724,147 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
                 break;
             }
             const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
-            const uint32_t tK = smem_addr(smem) + s * C::STAGE;
+            const uint32_t tK = smem_addr(smem) + s * C::STAGE, tV = tK + C::TILE;
             if (stage_ok[s]) {
-                const uint32_t vm_lo = (2 * c < ntok ? 0x0000ffffu : 0u) | (2 * c + 1 < ntok ? 0xffff0000u : 0u);
-                const uint32_t vm_hi = (2 * c + 8 < ntok ? 0x0000ffffu : 0u) | (2 * c + 9 < ntok ? 0xffff0000u : 0u);
-                uint32_t kf[C::KSTEPS][4], vf[C::MTILES][4];
+                // ---- S = Q . K^T: n-tiles of tokens 0-7 and 8-15, two chains each
+                float sa[2][2][4];
 #pragma unroll
-                for (int ks = 0; ks < C::KSTEPS; ++ks) ldsm_x4(kf[ks], tK + koff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
+                for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int i = 0; i < C::MTILES; ++i) {
-                    ldsm_x4_t(vf[i], tK + voff[i & 3] + (i >> 2) * C::BOX_BYTES);
-                    vf[i][0] &= vm_lo;
-                    vf[i][1] &= vm_lo;
-                    vf[i][2] &= vm_hi;
-                    vf[i][3] &= vm_hi;
+                    for (int e = 0; e < 4; ++e) sa[0][u][e] = sa[1][u][e] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                    uint32_t kb[4];
+                    ldsm_x4(kb, tK + moff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
+                    Mma<T>::mma(sa[0][ks & 1], qa[ks], kb[0], kb[1]);
+                    Mma<T>::mma(sa[1][ks & 1], qa[ks], kb[2], kb[3]);
                 }
-                float sa[4][4];
+                // x[nt][e]: head g (e < 2) or g + 8, token 8 nt + 2c + (e & 1), log2 units
+                float x[2][4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) sa[u][0] = sa[u][1] = sa[u][2] = sa[u][3] = 0.f;
+                for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int ks = 0; ks < C::KSTEPS; ++ks) Mma<T>::mma(sa[ks & 3], kf[ks], bq[ks][0], bq[ks][1]);
-                float sc[4];
+                    for (int e = 0; e < 4; ++e) x[nt][e] = (sa[nt][0][e] + sa[nt][1][e]) * a.scale_log2;
+                if (ntok < kBlockSize) {  // the row's last block: slots past the end see nothing
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sc[e] = (sa[0][e] + sa[1][e]) + (sa[2][e] + sa[3][e]);
-                const bool v0 = g < ntok, v1 = g + 8 < ntok;
-                const float s0 = v0 ? sc[0] * a.scale_log2 : -INFINITY, s1 = v0 ? sc[1] * a.scale_log2 : -INFINITY;
-                const float s2 = v1 ? sc[2] * a.scale_log2 : -INFINITY, s3 = v1 ? sc[3] * a.scale_log2 : -INFINITY;
-                float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+                    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int msk = 4; msk < 32; msk <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
+                        for (int e = 0; e < 4; ++e)
+                            if (8 * nt + 2 * c + (e & 1) >= ntok) x[nt][e] = -INFINITY;
                 }
-                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
-                const float p0 = fast_exp2(s0 - mn0), p1 = fast_exp2(s1 - mn1);
-                const float p2 = fast_exp2(s2 - mn0), p3 = fast_exp2(s3 - mn1);
-                l0 = l0 * al0 + (p0 + p2);
-                l1 = l1 * al1 + (p1 + p3);
-                m0 = mn0;
-                m1 = mn1;
-                if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+                float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+                float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                // move the reference point only when a score exceeds it by more than
+                // kLazyMax (always on the segment's first block: m = -inf)
+                if (__any_sync(0xffffffffu, mx0 > m0 + kLazyMax || mx1 > m1 + kLazyMax)) {
+                    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                    const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+                    l0 *= al0;
+                    l1 *= al1;
 #pragma unroll
-                    for (int i = 0; i < C::MTILES; ++i) {
+                    for (int i = 0; i < C::NT; ++i) {
                         o[i][0] *= al0;
-                        o[i][1] *= al1;
-                        o[i][2] *= al0;
+                        o[i][1] *= al0;
+                        o[i][2] *= al1;
                         o[i][3] *= al1;
                     }
+                    m0 = mn0;
+                    m1 = mn1;
                 }
-                const uint32_t ph01 = Mma<T>::pack(p0, p1), ph23 = Mma<T>::pack(p2, p3);
-                const uint32_t pb0 = movm_t(ph01), pb1 = movm_t(ph23);
-                uint32_t pl0 = 0, pl1 = 0;
-                if constexpr (SPLIT_P) {
-                    const float r0 = __uint_as_float(ph01 << 16), r1 = __uint_as_float(ph01 & 0xffff0000u);
-                    const float r2 = __uint_as_float(ph23 << 16), r3 = __uint_as_float(ph23 & 0xffff0000u);
-                    pl0 = movm_t(Mma<T>::pack(p0 - r0, p1 - r1));
-                    pl1 = movm_t(Mma<T>::pack(p2 - r2, p3 - r3));
-                }
+                float p[2][4];
 #pragma unroll
-                for (int i = 0; i < C::MTILES; ++i) {
-                    Mma<T>::mma(o[i], vf[i], pb0, pb1);
-                    if constexpr (SPLIT_P) Mma<T>::mma(o[i], vf[i], pl0, pl1);
+                for (int nt = 0; nt < 2; ++nt) {
+                    p[nt][0] = fast_exp2(x[nt][0] - m0);
+                    p[nt][1] = fast_exp2(x[nt][1] - m0);
+                    p[nt][2] = fast_exp2(x[nt][2] - m1);
+                    p[nt][3] = fast_exp2(x[nt][3] - m1);
+                }
+                l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+                l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+                // ---- A fragments of P (rows heads, k = tokens) straight from S's layout
+                uint32_t pa[4], pl[4];
+                pa[0] = Mma<T>::pack(p[0][0], p[0][1]);
+                pa[1] = Mma<T>::pack(p[0][2], p[0][3]);
+                pa[2] = Mma<T>::pack(p[1][0], p[1][1]);
+                pa[3] = Mma<T>::pack(p[1][2], p[1][3]);
+                if constexpr (SPLIT_P) {
+                    // bf16 keeps 8 significant bits: the remainder goes in a second operand
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const float hi0 = __uint_as_float(pa[r] << 16), hi1 = __uint_as_float(pa[r] & 0xffff0000u);
+                        pl[r] = Mma<T>::pack(p[r >> 1][2 * (r & 1)] - hi0, p[r >> 1][2 * (r & 1) + 1] - hi1);
+                    }
+                }
+                // ---- O += P . V, V fragments masked on the row's last block (stale slots
+                // may hold NaN or Inf; registers 0/1 hold tokens 2c, 2c + 1, 2/3 tokens + 8)
+                const uint32_t vm_lo = ntok < kBlockSize ? (2 * c < ntok ? 0x0000ffffu : 0u) |
+                                                               (2 * c + 1 < ntok ? 0xffff0000u : 0u)
+                                                         : 0xffffffffu;
+                const uint32_t vm_hi = ntok < kBlockSize ? (2 * c + 8 < ntok ? 0x0000ffffu : 0u) |
+                                                               (2 * c + 9 < ntok ? 0xffff0000u : 0u)
+                                                         : 0xffffffffu;
+#pragma unroll
+                for (int i = 0; i < C::KSTEPS; ++i) {
+                    uint32_t vb[4];
+                    ldsm_x4_t(vb, tV + moff[i & 3] + (i >> 2) * C::BOX_BYTES);
+                    if (ntok < kBlockSize) {
+                        vb[0] &= vm_lo;
+                        vb[1] &= vm_lo;
+                        vb[2] &= vm_hi;
+                        vb[3] &= vm_hi;
+                    }
+                    Mma<T>::mma(o[2 * i], pa, vb[0], vb[2]);
+                    Mma<T>::mma(o[2 * i + 1], pa, vb[1], vb[3]);
+                    if constexpr (SPLIT_P) {
+                        Mma<T>::mma(o[2 * i], pl, vb[0], vb[2]);
+                        Mma<T>::mma(o[2 * i + 1], pl, vb[1], vb[3]);
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
             ++c_k;
             if (warp == 0) {
-                // keep the ring S - 1 blocks ahead: the next copy goes into the stage of
-                // block c_k - 2, which every warp has usually released by now
-                while (p_alive && pc.valid && p_k < c_k - 1 + S) refill();
+                // keep the ring S - LAG blocks ahead of warp 0
+                while (p_alive && pc.valid && p_k < c_k - C::LAG + S) refill();
             }
         }
         if (!alive) {
             m0 = m1 = -INFINITY;
             l0 = l1 = 0.f;
 #pragma unroll
-            for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+            for (int i = 0; i < C::NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
         }
-#pragma unroll
-        for (int msk = 4; msk < 32; msk <<= 1) {
-            l0 += __shfl_xor_sync(0xffffffffu, l0, msk);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, msk);
-        }
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
         const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
         if (cs.j0 == 0 && cs.j1 == cs.nb) {
-            const size_t out0 = ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + col0 + h0) * D;
-            const size_t out1 = out0 + D;
+            const size_t out0 = ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + row0 + g) * D + 2 * c;
+            const size_t out1 = out0 + 8 * D;
 #pragma unroll
-            for (int i = 0; i < C::MTILES; ++i) {
-                const int d0 = 16 * i + g, d1 = d0 + 8;
-                store_out<T>(a.out, a.out_f32, out0 + d0, o[i][0] * inv0);
-                store_out<T>(a.out, a.out_f32, out0 + d1, o[i][2] * inv0);
-                store_out<T>(a.out, a.out_f32, out1 + d0, o[i][1] * inv1);
-                store_out<T>(a.out, a.out_f32, out1 + d1, o[i][3] * inv1);
+            for (int i = 0; i < C::NT; ++i) {
+                store_out2<T>(a.out, a.out_f32, out0 + 8 * i, o[i][0] * inv0, o[i][1] * inv0);
+                store_out2<T>(a.out, a.out_f32, out1 + 8 * i, o[i][2] * inv1, o[i][3] * inv1);
             }
         } else {
             const int ch_first = ck.of(cs.b, cs.kvh, cs.nb, 0);
             const int sl = 2 * cs.ch + ((cs.ch == ch_first && ck.mid_start(cs.b, cs.kvh, cs.nb)) ? 1 : 0);
-            float *w0 = a.ws_o + ((size_t)sl * GC + col0 + h0) * D;
-            float *w1 = w0 + D;
+            float *w0 = a.ws_o + ((size_t)sl * GC + row0 + g) * D + 2 * c;
+            float *w1 = w0 + 8 * D;
 #pragma unroll
-            for (int i = 0; i < C::MTILES; ++i) {
-                const int d0 = 16 * i + g, d1 = d0 + 8;
-                w0[d0] = o[i][0] * inv0;
-                w0[d1] = o[i][2] * inv0;
-                w1[d0] = o[i][1] * inv1;
-                w1[d1] = o[i][3] * inv1;
+            for (int i = 0; i < C::NT; ++i) {
+                *reinterpret_cast<float2 *>(w0 + 8 * i) = make_float2(o[i][0] * inv0, o[i][1] * inv0);
+                *reinterpret_cast<float2 *>(w1 + 8 * i) = make_float2(o[i][2] * inv1, o[i][3] * inv1);
             }
-            if (g == 0) {
-                a.ws_lse[(size_t)sl * GC + col0 + h0] = m0 + log2f(l0);
-                a.ws_lse[(size_t)sl * GC + col0 + h1] = m1 + log2f(l1);
+            if (c == 0) {
+                a.ws_lse[(size_t)sl * GC + row0 + g] = m0 + log2f(l0);
+                a.ws_lse[(size_t)sl * GC + row0 + g + 8] = m1 + log2f(l1);
             }
         }
         have = next_seg(cit, cs);
@@ -1964,8 +2016,8 @@ static int launch_coop(const DecodeArgs &a, cudaStream_t st) {
     DecodeArgs a2 = a;
     a2.Hkv = a.Hkv / a.ngroups;  // cache rows; GC = 8 NG columns each
     a2.ngroups = 1;
-    a2.G = NG * 8;
-    a2.gcols = NG * 8;
+    a2.G = NG * 16;
+    a2.gcols = NG * 16;
     const int smem = C::smem_bytes(a.B);
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
     CUtensorMap tk, tv;
@@ -1982,10 +2034,10 @@ static int launch_coop(const DecodeArgs &a, cudaStream_t st) {
     a2.tc_W = (int)ctas;
     if (launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), smem, st, tk, tv, a2) != cudaSuccess)
         return PA_ERR_CUDA;
-    auto mk = merge_tc_kernel<T, D, NG * 8, false>;
+    auto mk = merge_tc_kernel<T, D, NG * 16, false>;
     const int msmem = 2 * (a.B + 1) * 4;
     if (!set_smem_attr_once(reinterpret_cast<const void *>(mk), 2 * (kTcMaxB + 1) * 4)) return PA_ERR_CUDA;
-    const int64_t items = (int64_t)a.B * a2.Hkv * NG * 8;
+    const int64_t items = (int64_t)a.B * a2.Hkv * NG * 16;
     int64_t mctas = (items + 7) / 8;
     if (mctas > 2 * sms) mctas = 2 * sms;
     return launch_pdl(mk, dim3((unsigned)mctas), dim3(256), msmem, st, a2) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -2014,9 +2066,9 @@ static int launch_tc_g(const DecodeArgs &a, cudaStream_t st) {
     if constexpr (std::is_same<T, TKV>::value && D <= 128) {
         if (decode_coop_eligible(a.q_dtype, a.kv_dtype, D, a.G, a.ngroups, a.qlen, mq, a.tc_chunk < 0 ? 0 : 1)) {
             switch (a.ngroups) {
-            case 2: return launch_coop<T, D, 2>(a, st);
-            case 4: return launch_coop<T, D, 4>(a, st);
-            default: return launch_coop<T, D, 8>(a, st);
+            case 2: return launch_coop<T, D, 1>(a, st);
+            case 4: return launch_coop<T, D, 2>(a, st);
+            default: return launch_coop<T, D, 4>(a, st);
             }
         }
     }
