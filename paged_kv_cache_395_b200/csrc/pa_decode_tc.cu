@@ -1417,19 +1417,21 @@ template <typename T, int D, int NG>
 struct CoopCfg {
     static constexpr int NW = NG;
     static constexpr int THREADS = NW * 32;
-    // eight warps per SM: the q fragments (32 registers) and O (64 at d = 128) stay in
-    // registers, ~220 in all
-    static constexpr int MIN_CTAS = 8 / NG;
+    // ten to twelve warps per SM (O, 64 registers at d = 128, stays in registers; q is
+    // read from shared memory)
+    static constexpr int MIN_CTAS = NG == 1 ? 10 : (NG == 2 ? 6 : 3);
     static constexpr int BOXW = 128 / (int)sizeof(T);
     static constexpr int BOXES = D / BOXW;
     static constexpr int BOX_BYTES = 16 * 128;
     static constexpr int TILE = BOXES * BOX_BYTES;
     static constexpr int STAGE = 2 * TILE;
-    static constexpr int RING_BYTES = NG == 1 ? 16 * 1024 : (NG == 2 ? 32 * 1024 : 64 * 1024);
+    static constexpr int RING_BYTES = NG == 1 ? 16 * 1024 : (NG == 2 ? 24 * 1024 : 48 * 1024);
     static constexpr int S = RING_BYTES / STAGE;
     static constexpr int LAG = NG == 1 ? 0 : 1;  // blocks the refill trails the consumer by
     static constexpr int KSTEPS = D / 16, NT = D / 8;
-    static constexpr int BAR_OFF = S * STAGE;           // full[S], then empty[S]
+    static constexpr int QSLOT = 16 * D * 2;            // a warp's 16 q rows (16-byte chunks swizzled)
+    static constexpr int Q_OFF = S * STAGE;
+    static constexpr int BAR_OFF = Q_OFF + NW * QSLOT;  // full[S], then empty[S]
     static constexpr int OK_OFF = BAR_OFF + 2 * S * 8;  // int [S]: the stage's block is in the pool
     static constexpr int CUM_OFF = OK_OFF + S * 4;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (3 * B + 3) * 4; }
@@ -1684,11 +1686,16 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
         const int r = r8 + ((mi >> 1) << 3), ch = 2 * i + (mi & 1);
         moff[i] = r * 128 + (((ch & 7) ^ (r & 7)) << 4);
     }
+    // q rows in the warp's slot: row r, 16-byte chunk ch at r * 2D + ((ch ^ (r & 7)) << 4), so
+    // that the ldmatrix of 8 rows at one chunk hits 8 different bank groups; A fragment of
+    // k-step ks: matrix mi = lane / 8 is rows 8 (mi & 1) .. + 7, chunk 2 ks + (mi >> 1)
+    const uint32_t qslot = smem_addr(smem) + C::Q_OFF + warp * C::QSLOT;
+    const int qr = r8 + ((mi & 1) << 3);
+    auto qaddr = [&](int ks) -> uint32_t { return qslot + qr * (2 * D) + (((2 * ks + (mi >> 1)) ^ (qr & 7)) << 4); };
     SegIter cit{0, 0, 0, -1, false};
     cit.done = !range(cit);
     Seg cs;
     bool have = next_seg(cit, cs);
-    uint32_t qa[C::KSTEPS][4];
     int c_k = 0;
     bool alive = true;
     const int row0 = warp * 16;  // this warp's first column (head) of the row
@@ -1700,17 +1707,19 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
 #pragma unroll
         for (int i = 0; i < C::NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
         if (alive) {
-            // A fragments of q: heads row0 + g (+ 8), dims 16 ks + 2c, +1 (+ 8)
-            const uint32_t *q0 = reinterpret_cast<const uint32_t *>(a.q) +
-                                 ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + row0 + g) * (D / 2);
-            const uint32_t *q1 = q0 + 8 * (D / 2);
+            // the segment's q rows (heads row0 .. row0 + 15, consecutive in q) into the slot
+            const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) +
+                              ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + row0) * (D / 8);
+            __syncwarp();  // the previous segment's fragment reads are done
 #pragma unroll
-            for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                qa[ks][0] = __ldg(q0 + ks * 8 + c);
-                qa[ks][1] = __ldg(q1 + ks * 8 + c);
-                qa[ks][2] = __ldg(q0 + ks * 8 + 4 + c);
-                qa[ks][3] = __ldg(q1 + ks * 8 + 4 + c);
+            for (int i = 0; i < 16 * D / 8 / 32; ++i) {
+                const int id = i * 32 + lane, r = id / (D / 8), ch = id % (D / 8);
+                const uint4 v = __ldg(qg + id);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(qslot + r * (2 * D) + ((ch ^ (r & 7)) << 4)),
+                             "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                             : "memory");
             }
+            __syncwarp();
         }
         for (int j = 0; alive && j < len; ++j) {
             const int s = c_k % S;
@@ -1734,10 +1743,11 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
                     for (int e = 0; e < 4; ++e) sa[0][u][e] = sa[1][u][e] = 0.f;
 #pragma unroll
                 for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                    uint32_t kb[4];
+                    uint32_t kb[4], qa[4];
+                    ldsm_x4(qa, qaddr(ks));
                     ldsm_x4(kb, tK + moff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
-                    Mma<T>::mma(sa[0][ks & 1], qa[ks], kb[0], kb[1]);
-                    Mma<T>::mma(sa[1][ks & 1], qa[ks], kb[2], kb[3]);
+                    Mma<T>::mma(sa[0][ks & 1], qa, kb[0], kb[1]);
+                    Mma<T>::mma(sa[1][ks & 1], qa, kb[2], kb[3]);
                 }
                 // x[nt][e]: head g (e < 2) or g + 8, token 8 nt + 2c + (e & 1), log2 units
                 float x[2][4];
