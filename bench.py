@@ -104,6 +104,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--append", choices=["fused", "plain"], default="fused",
+                    help="fused: a step's new tokens go through pa_decode_append (one kernel with "
+                         "the decode where the library fuses them); plain: pa_reshape_and_cache "
+                         "then pa_decode")
     return ap.parse_args(argv)
 
 
@@ -397,9 +401,18 @@ def main(argv=None):
     elif int8:
         dw.quantize_int8()
     stream = torch.cuda.Stream()
-    # each decode follows this library's own reshape (or decode), which writes none of
-    # q, the tables or the lengths: the decode may read those before it finishes
-    calls = runner.StepCalls(dw, part, int8, algo, stream, flags=pa.PA_DECODE_INPUTS_READY)
+    # each decode follows this library's own reshape, decode or merge kernel, which
+    # writes none of q, the tables, the lengths or the new tokens: the decode may read
+    # those before it finishes
+    fused = args.append == "fused"
+    # the prompts of admitted sequences were computed earlier (a prefill): where the
+    # recipe reuses freed blocks one step late, their append may overlap the kernel
+    # before it
+    pflags = pa.PA_APPEND_OVERLAP_PREVIOUS if getattr(w, "appends_overlap_previous", False) else 0
+    calls = runner.StepCalls(dw, part, int8, algo, stream, flags=pa.PA_DECODE_INPUTS_READY, fused=fused,
+                             prompt_flags=pflags)
+    plain_calls = runner.StepCalls(dw, part, int8, algo, stream, flags=pa.PA_DECODE_INPUTS_READY) \
+        if calls.fused_steps else None
     T = len(w.steps)
     sbytes = step_bytes(w, int8)
     stoks = step_tokens(w)
@@ -468,6 +481,8 @@ def main(argv=None):
         lap_dec_ms, _ = timed(calls.run_decode_only)
         lap_bytes = sum(sbytes[i] for i in idx)
         idx = idx_window
+        # the same window with the plain calls (append kernel, then decode)
+        plain_ms = timed(plain_calls.run)[0] if plain_calls is not None else None
     bytes_rank = sum(sbytes[i] for i in idx)
     toks_rank = sum(stoks[i] for i in idx)
     launches = sum(calls.launches[i] for i in idx)
@@ -496,6 +511,12 @@ def main(argv=None):
                    "timing": ("one CUDA event pair per step, summed" if per_step else
                               "CUDA events around the K steps issued back to back"),
                    "decode_flags": "PA_DECODE_INPUTS_READY",
+                   "step_calls": (("pa_block_copy where a step copies, pa_reshape_and_cache_ex of the "
+                                   "admitted prompts" + (" (PA_APPEND_OVERLAP_PREVIOUS)" if pflags else "") +
+                                   ", pa_decode_append of the new tokens and the decode "
+                                   f"(one kernel in {calls.fused_steps} of {T} steps, plus the merge "
+                                   "where it splits)") if calls.fused_steps else
+                                  "the workload's own calls (pa_block_copy, pa_reshape_and_cache, pa_decode)"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "decode_tokens_per_s": toks_rank * world / (ms_max * 1e-3),
         # the same step repeated for 32 layers: attention-only context for a 7B-class model
@@ -517,6 +538,10 @@ def main(argv=None):
         # window: the sum of its algorithmic bytes over its device time, whole steps and
         # the decode calls alone
         "value_full_trace": lap_value,
+        # the K-step window with the plain calls: pa_reshape_and_cache of all the
+        # step's tokens, then pa_decode
+        "value_plain_append": (replica_throughput(bytes_rank, plain_ms, dist)[0]
+                               if plain_ms is not None else None),
         "decode_full_trace": lap_dec_value,
         "full_trace": {"steps": T, "ms_per_step": lap_ms_max / T, "bytes": lap_bytes * world,
                        "decode_frac_of_" + peak_kind: lap_dec_value / world / peak},
@@ -573,7 +598,9 @@ def time_e2e(dw, w, int8, part, algo, args, T, sbytes, stream, dist):
         views = packs[i][2]
         staged.steps[i] = [tuple(views.get(id(x), x) if isinstance(x, torch.Tensor) else x
                                  for x in op) for op in dw.steps[i]]
-    calls = runner.StepCalls(staged, part, int8, algo, stream, flags=pa.PA_DECODE_INPUTS_READY)
+    pflags = pa.PA_APPEND_OVERLAP_PREVIOUS if getattr(w, "appends_overlap_previous", False) else 0
+    calls = runner.StepCalls(staged, part, int8, algo, stream, flags=pa.PA_DECODE_INPUTS_READY,
+                             fused=args.append == "fused", prompt_flags=pflags)
     K = args.steps
     # Pipelined like a serving loop: step j's inputs are copied in on one copy
     # stream while earlier steps compute on `stream`, and each step's output is

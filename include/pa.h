@@ -71,7 +71,9 @@ enum pa_error_flag {
     PA_EFLAG_BAD_BLOCK = 1,   /* a block table entry read by pa_decode was outside the pool */
     PA_EFLAG_BAD_SLOT = 2,    /* a slot_mapping entry was >= num_blocks * PA_BLOCK_SIZE */
     PA_EFLAG_BAD_PAIR = 4,    /* a pa_block_copy pair was outside the pool */
-    PA_EFLAG_WAIT_TIMEOUT = 8 /* a bounded wait on an asynchronous copy gave up */
+    PA_EFLAG_WAIT_TIMEOUT = 8, /* a bounded wait on an asynchronous copy gave up */
+    PA_EFLAG_APPEND_SLOT = 16  /* pa_decode_append: a new token's slot was not the slot of
+                                  its sequence's position seq_lens[b] - 1 */
 };
 
 #define PA_BLOCK_SIZE 16
@@ -234,6 +236,50 @@ int pa_decode_algo(const pa_decode_params *p, const void *q);
 int pa_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
               const int32_t *block_tables, const int32_t *seq_lens, float scale,
               const pa_decode_params *p, pa_stream_t stream);
+
+/*
+ * Append, then decode, in one call (lqnn.cn/news/235768 section 2.2: the step's
+ * new token goes to the end of its sequence's cache, then the query attends to
+ * the whole sequence).  Result, and cache contents afterwards, are those of
+ *
+ *   pa_reshape_and_cache(k_new, v_new, key_cache, value_cache, slot_mapping,
+ *                        p->num_seqs, p->num_kv_heads, p->head_dim, p->block_size,
+ *                        p->num_blocks, p->kv_dtype, k_token_stride, v_token_stride, stream);
+ *   pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, p, stream);
+ *
+ * for one new token per sequence (query_len 0 or 1; kv_dtype == q_dtype): row b
+ * of k_new / v_new ([num_seqs][num_kv_heads][head_dim] with token strides in
+ * elements) is sequence b's new token and slot_mapping[b] its slot (< 0: none);
+ * seq_lens count it.  Quantised caches: pa_append_int8, then pa_decode.
+ *
+ * Where pa_decode_append_fused says so, the call is one kernel: the decode
+ * writes every new token to its slot itself and uses it in place of what its
+ * copy of that slot held, so no append kernel runs before it.  That relies on
+ * slot_mapping[b] being the slot of position seq_lens[b] - 1 of sequence b
+ * under its block table, as in a decode step; a new token whose slot is another
+ * one sets PA_EFLAG_APPEND_SLOT, is still written to its slot, and leaves the
+ * outputs that read that slot undefined.  A slot >= num_blocks * 16 sets
+ * PA_EFLAG_BAD_SLOT and is skipped, as in pa_reshape_and_cache.  Otherwise the
+ * two calls above run in order.  With PA_DECODE_INPUTS_READY the fused kernel
+ * reads k_new, v_new and slot_mapping early too, so the kernel before it on the
+ * stream must not write them either.
+ */
+int pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                     const int64_t *slot_mapping, int64_t k_token_stride, int64_t v_token_stride,
+                     void *key_cache, void *value_cache, const int32_t *block_tables,
+                     const int32_t *seq_lens, float scale, const pa_decode_params *p,
+                     pa_stream_t stream);
+
+/*
+ * 1 when pa_decode_append with these arguments runs as one kernel -- the
+ * tensor-core family's per-warp decode of single-token fp16 / bf16 rows (not
+ * the cooperative mode of 16-64 query heads per KV head), with q, k_new and
+ * v_new 16-byte aligned and token strides a multiple of 8 elements -- 0 when it
+ * runs pa_reshape_and_cache then pa_decode, or the negative pa_status it would
+ * return.  The pointers are not read.
+ */
+int pa_decode_append_fused(const pa_decode_params *p, const void *q, const void *k_new,
+                           const void *v_new, int64_t k_token_stride, int64_t v_token_stride);
 
 /*
  * pa_decode without a caller workspace.  No counterpart in the paper: it is an

@@ -307,20 +307,51 @@ size_t pa_decode_workspace_size(const pa_decode_params *p) {
 
 namespace pa {
 
-// pa_decode with the two knobs of pa_decode_stall_selftest.
-static int decode_impl(void *out, const void *q, const void *key_cache, const void *value_cache,
-                       const int32_t *block_tables, const int32_t *seq_lens, float scale,
-                       const pa_decode_params *p, pa_stream_t stream, int stall_at,
-                       unsigned long long wait_ns) {
-    Plan pl;
-    const int rc = make_plan(p, &pl);
-    if (rc != PA_OK) return rc;
-    if (p->num_seqs == 0) return PA_OK;
+// The new-token rows of pa_decode_append.
+struct AppendIn {
+    const void *k, *v;
+    const int64_t *slots;
+    int64_t k_stride, v_stride;
+};
+
+// pa_decode's checks of its buffers, after make_plan.
+static int decode_buffers_ok(const void *out, const void *q, const void *key_cache, const void *value_cache,
+                             const int32_t *block_tables, const int32_t *seq_lens, const pa_decode_params *p,
+                             const Plan &pl) {
     if (!out || !q || !key_cache || !value_cache || !block_tables || !seq_lens) return PA_ERR_NULL;
     if ((p->kv_dtype == PA_I8 || p->kv_dtype == PA_I4) && (!p->k_scales || !p->v_scales)) return PA_ERR_NULL;
     if (((uintptr_t)key_cache | (uintptr_t)value_cache) % 16) return PA_ERR_ALIGN;
     if (pl.bytes > 0 && (!p->workspace || p->workspace_bytes < pl.bytes)) return PA_ERR_WORKSPACE;
     if (pl.bytes > 0 && (uintptr_t)p->workspace % 16) return PA_ERR_ALIGN;
+    return PA_OK;
+}
+
+// Whether pa_decode_append runs as one kernel: the per-warp tensor-core decode of
+// single-token fp16 / bf16 rows, with the new-token rows 16-byte aligned.
+static bool append_fusable(const pa_decode_params *p, const Plan &pl, const void *q, const void *k_new,
+                           const void *v_new, int64_t k_stride, int64_t v_stride) {
+    KernelHeads kh;
+    kernel_heads(p, &kh);
+    if (!pl.tc || (uintptr_t)q % 16 || kh.qlen > 1 || kh.padded) return false;
+    if (p->kv_dtype != p->q_dtype || (p->kv_dtype != PA_F16 && p->kv_dtype != PA_BF16)) return false;
+    if (pl.tc_chunk >= 0 &&
+        decode_coop_eligible(p->q_dtype, p->kv_dtype, p->head_dim, kh.G, kh.ngroups, kh.qlen, kh.padded, 1))
+        return false;
+    return ((uintptr_t)k_new | (uintptr_t)v_new) % 16 == 0 && (k_stride * 2) % 16 == 0 && (v_stride * 2) % 16 == 0;
+}
+
+// pa_decode with the two knobs of pa_decode_stall_selftest, and the fused append
+// of pa_decode_append (ap != nullptr: the caller has checked append_fusable).
+static int decode_impl(void *out, const void *q, const void *key_cache, const void *value_cache,
+                       const int32_t *block_tables, const int32_t *seq_lens, float scale,
+                       const pa_decode_params *p, pa_stream_t stream, int stall_at,
+                       unsigned long long wait_ns, const AppendIn *ap = nullptr) {
+    Plan pl;
+    int rc = make_plan(p, &pl);
+    if (rc != PA_OK) return rc;
+    if (p->num_seqs == 0) return PA_OK;
+    rc = decode_buffers_ok(out, q, key_cache, value_cache, block_tables, seq_lens, p, pl);
+    if (rc != PA_OK) return rc;
 
     DecodeArgs a{};
     a.out = out;
@@ -351,6 +382,14 @@ static int decode_impl(void *out, const void *q, const void *key_cache, const vo
     a.out_f32 = (p->flags & PA_DECODE_OUT_F32) ? 1 : 0;
     a.stall_at = stall_at;
     a.wait_ns = wait_ns;
+    if (ap) {
+        a.append = 1;
+        a.k_new = ap->k;
+        a.v_new = ap->v;
+        a.slot_new = ap->slots;
+        a.kn_stride = ap->k_stride;
+        a.vn_stride = ap->v_stride;
+    }
     char *ws = reinterpret_cast<char *>(p->workspace);
     if (pl.tc && (uintptr_t)q % 16) {
         if (p->algo == PA_ALGO_TENSOR || stall_at >= 0) return PA_ERR_ALIGN;
@@ -411,6 +450,45 @@ int pa_decode_stall_selftest(void *out, const void *q, const void *key_cache, co
     if (stall_at < 0 || limit_ns == 0) return PA_ERR_SHAPE;
     return decode_impl(out, q, key_cache, value_cache, block_tables, seq_lens, scale, p, stream, stall_at,
                        (unsigned long long)limit_ns);
+}
+
+int pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                     int64_t k_token_stride, int64_t v_token_stride, void *key_cache, void *value_cache,
+                     const int32_t *block_tables, const int32_t *seq_lens, float scale, const pa_decode_params *p,
+                     pa_stream_t stream) {
+    const int fused = pa_decode_append_fused(p, q, k_new, v_new, k_token_stride, v_token_stride);
+    if (fused < 0) return fused;
+    if (p->num_seqs == 0) return PA_OK;
+    if (!slot_mapping) return PA_ERR_NULL;
+    Plan pl;
+    make_plan(p, &pl);
+    const int rc = decode_buffers_ok(out, q, key_cache, value_cache, block_tables, seq_lens, p, pl);
+    if (rc != PA_OK) return rc;
+    if (fused) {
+        const AppendIn ap{k_new, v_new, slot_mapping, k_token_stride, v_token_stride};
+        return decode_impl(out, q, key_cache, value_cache, block_tables, seq_lens, scale, p, stream, -1,
+                           kWaitLimitNs, &ap);
+    }
+    const int ra = pa_reshape_and_cache(k_new, v_new, key_cache, value_cache, slot_mapping, p->num_seqs,
+                                        p->num_kv_heads, p->head_dim, p->block_size, p->num_blocks, p->kv_dtype,
+                                        k_token_stride, v_token_stride, stream);
+    if (ra != PA_OK) return ra;
+    return decode_impl(out, q, key_cache, value_cache, block_tables, seq_lens, scale, p, stream, -1,
+                       kWaitLimitNs);
+}
+
+int pa_decode_append_fused(const pa_decode_params *p, const void *q, const void *k_new, const void *v_new,
+                           int64_t k_token_stride, int64_t v_token_stride) {
+    Plan pl;
+    const int rc = make_plan(p, &pl);
+    if (rc != PA_OK) return rc;
+    if (p->query_len > 1) return PA_ERR_UNSUPPORTED;
+    if (p->kv_dtype != p->q_dtype) return PA_ERR_DTYPE;
+    if (p->num_seqs > 0 && (!k_new || !v_new)) return PA_ERR_NULL;
+    if (k_token_stride < (int64_t)p->num_kv_heads * p->head_dim ||
+        v_token_stride < (int64_t)p->num_kv_heads * p->head_dim)
+        return PA_ERR_SHAPE;
+    return append_fusable(p, pl, q, k_new, v_new, k_token_stride, v_token_stride) ? 1 : 0;
 }
 
 int pa_decode_algo(const pa_decode_params *p, const void *q) {

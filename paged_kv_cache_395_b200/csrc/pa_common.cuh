@@ -286,7 +286,15 @@ __device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void *src, uint
         : "memory");
 }
 
-__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+// 2^x with the hardware approximation (PTX ex2.approx.ftz: relative error about
+// 2^-22; results below 2^-126 flush to 0, 2^-inf = 0).  Every use weights a
+// probability against a running maximum that some term reaches at 2^0, so a flushed
+// term is below 2^-126 of the sum.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 

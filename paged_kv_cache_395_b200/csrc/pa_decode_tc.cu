@@ -197,7 +197,11 @@ struct TcCfg {
     static constexpr int BAR_OFF = QRING_OFF + NW * S * QSLOT;
     static constexpr int OK_OFF = BAR_OFF + NW * S * 8;
     static constexpr int SC_OFF = OK_OFF + NW * S * 4;    // float [NW][S][2]: int8 K, V scales
-    static constexpr int CUM_OFF = SC_OFF + NW * S * 8;
+    // pa_decode_append: a row end's new K and V rows, and the cache slot its warp writes
+    static constexpr int PATCH = 2 * D * 2;
+    static constexpr int PATCH_OFF = (SC_OFF + NW * S * 8 + 15) / 16 * 16;
+    static constexpr int PSLOT_OFF = PATCH_OFF + NW * S * PATCH;  // int64 [NW][S], -1: none
+    static constexpr int CUM_OFF = PSLOT_OFF + NW * S * 8;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (3 * B + 3) * 4; }
 };
 
@@ -451,6 +455,9 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     constexpr bool kQz = kI8 || kI4;  // quantised cache: per-(block, KV head) scales
     static_assert(!kQz || (std::is_same<T, __half>::value && D == 128),
                   "int8 and 4-bit caches: fp16 q, head_dim 128");
+    // pa_decode_append: single-token rows of an fp16 / bf16 cache
+    constexpr bool kApp = !MQ && !kQz;
+    const bool app = kApp && a.append;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -661,9 +668,17 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     // also load the block's K and V scales, which need the block id at once: an
     // id outside the pool is marked -2 there.
     float p_ks = 0.f, p_vs = 0.f, p_ks_next = 0.f, p_vs_next = 0.f;
-    auto win_load = [&](const Win &w, float &ks, float &vs) -> int {
+    // pa_decode_append: the lane holding a row's last block also loads the sequence's
+    // new-token slot and its length as given (the row's L may have been cut short)
+    long long p_sn = -1, p_sn_next = -1;
+    int p_lr = 0, p_lr_next = 0;
+    auto win_load = [&](const Win &w, float &ks, float &vs, long long &sn, int &lr) -> int {
         if (!w.valid || lane >= w.n) return -1;
         const int pb = a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
+        if (app && w.sg.j0 + w.o + lane == w.sg.nb - 1) {
+            sn = a.slot_new[w.sg.b];
+            lr = a.lens[w.sg.b];
+        }
         if constexpr (kQz) {
             if (pb < 0 || (int64_t)pb >= a.N) return -2;
             ks = a.ks[(size_t)pb * Hc + w.kc];
@@ -674,9 +689,11 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     Win pc, pn;
     win_first(pc);
     win_after(pc, pn);
-    int p_y = win_load(pc, p_ks, p_vs), p_y_next = win_load(pn, p_ks_next, p_vs_next);
+    int p_y = win_load(pc, p_ks, p_vs, p_sn, p_lr), p_y_next = win_load(pn, p_ks_next, p_vs_next, p_sn_next, p_lr_next);
     int p_i = 0, p_k = 0;
     float *my_sc = stage_sc + warp * S * 2;
+    const uint32_t my_patch = smem_addr(smem) + C::PATCH_OFF + warp * S * C::PATCH;
+    long long *my_pslot = reinterpret_cast<long long *>(smem + C::PSLOT_OFF) + warp * S;
     auto refill = [&]() {
         if (!pc.valid) return;
         const int pb = __shfl_sync(0xffffffffu, p_y, p_i);
@@ -687,6 +704,24 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             ksv = __shfl_sync(0xffffffffu, p_ks, p_i);
             vsv = __shfl_sync(0xffffffffu, p_vs, p_i);
         }
+        // pa_decode_append, a row's last block: the new token is patched into the staged
+        // tile when it is the row's last decoded position and its slot is that position's
+        // slot in this block; the row's warp writes it to its cache slot (one warp per
+        // cache KV head) whether or not it is patched
+        bool patch = false;
+        long long psn = -1;
+        if (app && pc.sg.j0 + pc.o + p_i == pc.sg.nb - 1) {
+            const long long sn = __shfl_sync(0xffffffffu, p_sn, p_i);
+            const int lr = __shfl_sync(0xffffffffu, p_lr, p_i);
+            const int L = pc.sg.L;
+            const bool inpool = sn >= 0 && sn < a.N * kBlockSize;
+            const bool cur = lr == L;
+            patch = cur && y >= 0 && sn == (long long)pb * kBlockSize + (L - 1) % kBlockSize;
+            const bool writer = pc.sg.kvh % a.ngroups == 0;
+            psn = inpool && writer ? sn : -1;
+            if (lane == 0 && writer && sn >= 0 && !inpool) raise_flag(PA_EFLAG_BAD_SLOT);
+            if (lane == 0 && writer && cur && sn >= 0 && !patch) raise_flag(PA_EFLAG_APPEND_SLOT);
+        }
         if (lane == 0) {
             const int s = p_k % S;
             uint64_t *bar = &my_bars[s];
@@ -694,8 +729,11 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             // stage's q slot (even when the block itself is skipped)
             const bool seg_first = pc.o == 0 && p_i == 0;
             const int ncol = seg_first ? pc.sg.ncol : 0;
-            const uint32_t tx = (y < 0 ? 0u : (uint32_t)C::STAGE) + (uint32_t)(ncol * D * (int)sizeof(T));
-            my_ok[s] = y >= 0;
+            const bool fetch_new = patch || psn >= 0;
+            const uint32_t tx = (y < 0 ? 0u : (uint32_t)C::STAGE) + (uint32_t)(ncol * D * (int)sizeof(T)) +
+                                (fetch_new ? (uint32_t)C::PATCH : 0u);
+            my_ok[s] = (y >= 0 ? 1 : 0) | (patch ? 2 : 0);
+            if (app) my_pslot[s] = psn;
             if constexpr (kQz) {
                 my_sc[2 * s] = ksv;  // released to the consumer by the arrive below
                 my_sc[2 * s + 1] = vsv;
@@ -722,6 +760,13 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
                     tma_load_2d(dst + C::TILE + bx * C::BOX_BYTES, &tmV, bx * C::BOXW, y, smem_addr(bar));
                 }
             }
+            if (fetch_new && !stall) {
+                const size_t kh = (size_t)(pc.sg.kvh / a.ngroups) * D;
+                const T *kn = reinterpret_cast<const T *>(a.k_new) + (size_t)pc.sg.b * a.kn_stride + kh;
+                const T *vn = reinterpret_cast<const T *>(a.v_new) + (size_t)pc.sg.b * a.vn_stride + kh;
+                bulk_g2s_u32(my_patch + s * C::PATCH, kn, D * 2, smem_addr(bar));
+                bulk_g2s_u32(my_patch + s * C::PATCH + D * 2, vn, D * 2, smem_addr(bar));
+            }
             if (stall) {
             } else if (!MQ && seg_first) {
                 bulk_g2s_u32(qring + s * C::QSLOT, reinterpret_cast<const T *>(a.q) + col_row(pc.sg.b, pc.sg.kvh, 0) * D,
@@ -746,21 +791,41 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             p_y = p_y_next;
             p_ks = p_ks_next;
             p_vs = p_vs_next;
+            p_sn = p_sn_next;
+            p_lr = p_lr_next;
             win_after(pc, pn);
-            p_y_next = win_load(pn, p_ks_next, p_vs_next);
+            p_y_next = win_load(pn, p_ks_next, p_vs_next, p_sn_next, p_lr_next);
         }
     };
     if (a.early) {
         pdl_wait();
         pdl_release_dependents();
     }
-    // rows of sequences with no token produce zeros
+    // rows of sequences with no token produce zeros (and, for pa_decode_append, still
+    // write their new token, if any, to its slot)
     for (int r = gw; r < B * Hkv; r += W) {
         const int b = r / Hkv;
         if (cum[b + 1] == cum[b]) {
             const int kvh = r % Hkv, ncol = ncol_of(kvh);
             for (int j = 0; j < ncol; ++j)
                 for (int i = lane; i < D; i += 32) store_out<T>(a.out, a.out_f32, col_row(b, kvh, j) * D + i, 0.f);
+            if (app && kvh % a.ngroups == 0) {
+                const long long sn = a.slot_new[b];
+                if (sn >= a.N * kBlockSize) {
+                    if (lane == 0) raise_flag(PA_EFLAG_BAD_SLOT);
+                } else if (sn >= 0) {
+                    const int kc = kvh / a.ngroups;
+                    const size_t drow = (((size_t)(sn / kBlockSize) * Hc + kc) * kBlockSize + sn % kBlockSize) * D;
+                    for (int q = lane; q < D / 4; q += 32) {
+                        const bool isv = q >= D / 8;
+                        const int ch = isv ? q - D / 8 : q;
+                        const T *src = reinterpret_cast<const T *>(isv ? a.v_new : a.k_new) +
+                                       (size_t)b * (isv ? a.vn_stride : a.kn_stride) + (size_t)kc * D;
+                        T *dst = reinterpret_cast<T *>(const_cast<void *>(isv ? a.vc : a.kc)) + drow;
+                        reinterpret_cast<uint4 *>(dst)[ch] = reinterpret_cast<const uint4 *>(src)[ch];
+                    }
+                }
+            }
         }
     }
 #pragma unroll
@@ -992,9 +1057,40 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             }
             if (lane != 0) mbar_wait(&my_bars[s], parity, a.wait_ns);
             if (j == 0) load_q(s, bq, ncol);  // the segment's q came with its first block
-            const int ntok = (cs.j0 + j == cs.nb - 1) ? ntok_last : kBlockSize;
+            const bool row_end = cs.j0 + j == cs.nb - 1;
+            const int ntok = row_end ? ntok_last : kBlockSize;
             const uint32_t tK = ring + s * C::STAGE;
-            if (my_ok[s]) {
+            if (app && row_end) {
+                // pa_decode_append: the new token's K and V rows, staged with this block,
+                // replace tile row ntok - 1 (its slot) and go to their cache slot
+                const int okw = my_ok[s];
+                const long long psn = my_pslot[s];
+                if ((okw & 2) || psn >= 0) {
+                    const int r = ntok - 1;
+                    const int kc = cs.kvh / a.ngroups;
+                    const size_t drow =
+                        psn >= 0 ? (((size_t)(psn / kBlockSize) * Hc + kc) * kBlockSize + psn % kBlockSize) * D : 0;
+                    for (int q = lane; q < D / 4; q += 32) {
+                        const bool isv = q >= D / 8;
+                        const int ch = isv ? q - D / 8 : q;  // 16-byte chunk of the row
+                        uint32_t w4[4];
+                        lds_v4(w4, my_patch + s * C::PATCH + q * 16);
+                        if (okw & 2) {
+                            const uint32_t dst = tK + (isv ? C::TILE : 0) + (ch >> 3) * C::BOX_BYTES + r * 128 +
+                                                 (((ch & 7) ^ (r & 7)) << 4);
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w4[0]),
+                                         "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
+                                         : "memory");
+                        }
+                        if (psn >= 0) {
+                            T *cache = reinterpret_cast<T *>(const_cast<void *>(isv ? a.vc : a.kc)) + drow;
+                            reinterpret_cast<uint4 *>(cache)[ch] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+            if (my_ok[s] & 1) {
                 // Slots past the sequence end hold stale data (in fp16/bf16 caches possibly
                 // NaN/Inf); their probabilities are 0, and fp16/bf16 V values are masked
                 // to 0 in the fragments so that they add exactly 0.  V^T fragment registers 0, 1
@@ -1575,6 +1671,8 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
     SegIter pit{0, 0, 0, -1, false};
     Win pc{}, pn{};
     int p_y = -1, p_y_next = -1, p_i = 0, p_k = 0;
+    int p_s = 0;         // stage of block p_k (p_k % S)
+    uint32_t p_ph = 0;   // (p_k / S) & 1
     bool p_alive = true;
     auto win_first = [&](Win &w) {
         Seg sg;
@@ -1607,9 +1705,9 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
     // issue the copy of the next block of the stream into its stage (warp 0, all lanes)
     auto refill = [&]() {
         if (!pc.valid || !p_alive) return;
-        const int s = p_k % S;
+        const int s = p_s;
         if (p_k >= S) {  // the stage's previous block must be released by every warp
-            int ok = lane == 0 ? (int)mbar_wait(&empty[s], ((p_k / S) - 1) & 1, a.wait_ns) : 0;
+            int ok = lane == 0 ? (int)mbar_wait(&empty[s], p_ph ^ 1u, a.wait_ns) : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) {
                 p_alive = false;
@@ -1639,6 +1737,10 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
             }
         }
         ++p_k;
+        if (++p_s == S) {
+            p_s = 0;
+            p_ph ^= 1u;
+        }
         if (++p_i == pc.n) {
             p_i = 0;
             pc = pn;
@@ -1696,7 +1798,8 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
     cit.done = !range(cit);
     Seg cs;
     bool have = next_seg(cit, cs);
-    int c_k = 0;
+    int c_k = 0, c_s = 0;  // blocks consumed; stage of block c_k
+    uint32_t c_ph = 0;     // (c_k / S) & 1
     bool alive = true;
     const int row0 = warp * 16;  // this warp's first column (head) of the row
     while (have) {
@@ -1722,8 +1825,8 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
             __syncwarp();
         }
         for (int j = 0; alive && j < len; ++j) {
-            const int s = c_k % S;
-            const uint32_t parity = (c_k / S) & 1;
+            const int s = c_s;
+            const uint32_t parity = c_ph;
             int ok = lane == 0 ? (int)mbar_wait(&full[s], parity, a.wait_ns) : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (ok && lane != 0) mbar_wait(&full[s], parity, a.wait_ns);
@@ -1838,6 +1941,10 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
             ++c_k;
+            if (++c_s == S) {
+                c_s = 0;
+                c_ph ^= 1u;
+            }
             if (warp == 0) {
                 // keep the ring S - LAG blocks ahead of warp 0
                 while (p_alive && pc.valid && p_k < c_k - C::LAG + S) refill();

@@ -66,6 +66,14 @@ struct DecodeArgs {
     int stall_at;            // -1; else the first worker of the tensor-core family leaves
                              // its stall_at-th copy unissued (pa_decode_stall_selftest)
     unsigned long long wait_ns;  // limit of every bounded wait on a copy
+    // pa_decode_append on the tensor-core family: row b of k_new / v_new ([B][H_kv][D],
+    // token strides in elements) is sequence b's new token, written to cache slot
+    // slot_new[b] (< 0: none) by the kernel, which also uses it in place of what its
+    // copy of that slot's block held
+    int append;
+    const void *k_new, *v_new;
+    const int64_t *slot_new;
+    int64_t kn_stride, vn_stride;
 };
 
 // Default limit of a bounded wait: one second.

@@ -2,7 +2,8 @@
 
 The names mirror the C ABI in ``include/pa.h``:
 
-* ``pa_reshape_and_cache``, ``pa_decode``, ``pa_decode_fixed_scratch``,
+* ``pa_reshape_and_cache``, ``pa_decode``, ``pa_decode_append``,
+  ``pa_decode_append_fused``, ``pa_decode_fixed_scratch``,
   ``pa_decode_stall_selftest``, ``pa_block_copy``, ``pa_quantize_int8``,
   ``pa_quantize_int4``, ``pa_append_int8``, ``pa_decode_workspace_size``,
   ``pa_decode_algo``, ``pa_get_error_flags`` take torch CUDA tensors (or raw device pointers via ``lib``), check device,
@@ -28,6 +29,7 @@ PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_ALIGN = -4, -5, -6, -7
 PA_F32, PA_F16, PA_BF16, PA_I8, PA_I4 = 0, 1, 2, 3, 4
 PA_ALGO_AUTO, PA_ALGO_SIMT, PA_ALGO_TENSOR = 0, 1, 2
 PA_EFLAG_BAD_BLOCK, PA_EFLAG_BAD_SLOT, PA_EFLAG_BAD_PAIR, PA_EFLAG_WAIT_TIMEOUT = 1, 2, 4, 8
+PA_EFLAG_APPEND_SLOT = 16
 PA_DECODE_INPUTS_READY, PA_DECODE_OUT_F32 = 1, 2
 PA_APPEND_OVERLAP_PREVIOUS = 1
 BLOCK_SIZE = 16
@@ -72,6 +74,8 @@ def _load():
     L.pa_reshape_and_cache_ex.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, i64, i64, i32, P]
     L.pa_decode.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), P]
     L.pa_decode_fixed_scratch.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), P]
+    L.pa_decode_append.argtypes = [P, P, P, P, P, i64, i64, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), P]
+    L.pa_decode_append_fused.argtypes = [ctypes.POINTER(PaDecodeParams), P, P, P, i64, i64]
     L.pa_decode_workspace_size.argtypes = [ctypes.POINTER(PaDecodeParams)]
     L.pa_decode_workspace_size.restype = ctypes.c_size_t
     L.pa_decode_algo.argtypes = [ctypes.POINTER(PaDecodeParams), P]
@@ -85,7 +89,8 @@ def _load():
     L.pa_status_string.argtypes = [i32]
     L.pa_status_string.restype = ctypes.c_char_p
     L.pa_version.argtypes = []
-    for n in ("pa_reshape_and_cache", "pa_reshape_and_cache_ex", "pa_append_int8", "pa_decode", "pa_decode_fixed_scratch",
+    for n in ("pa_reshape_and_cache", "pa_reshape_and_cache_ex", "pa_append_int8", "pa_decode", "pa_decode_append",
+              "pa_decode_append_fused", "pa_decode_fixed_scratch",
               "pa_decode_stall_selftest", "pa_decode_algo", "pa_block_copy", "pa_quantize_int8",
               "pa_quantize_int4", "pa_get_error_flags", "pa_version"):
         getattr(L, n).restype = i32
@@ -95,7 +100,8 @@ def _load():
 lib = _load()
 
 # the C-ABI symbols include/pa.h declares
-EXPORTED = ("pa_reshape_and_cache", "pa_reshape_and_cache_ex", "pa_append_int8", "pa_decode_workspace_size", "pa_decode_algo", "pa_decode",
+EXPORTED = ("pa_reshape_and_cache", "pa_reshape_and_cache_ex", "pa_append_int8", "pa_decode_workspace_size",
+            "pa_decode_algo", "pa_decode", "pa_decode_append", "pa_decode_append_fused",
             "pa_decode_fixed_scratch", "pa_decode_stall_selftest", "pa_block_copy", "pa_quantize_int8",
             "pa_quantize_int4", "pa_get_error_flags", "pa_status_string", "pa_version")
 FIXED_SCRATCH_BYTES = 32 << 20  # PA_FIXED_SCRATCH_BYTES
@@ -233,13 +239,60 @@ def pa_decode(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max
                          ctypes.byref(p), _stream(stream)), "pa_decode")
 
 
+def _new_rows(k_new, v_new, slot_mapping, key_cache):
+    """k_new / v_new [B][H_kv][d] (token stride free, heads contiguous rows), int64 slots [B]."""
+    _, H, _, d = key_cache.shape
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        if t.dim() != 3 or t.shape[1:] != (H, d) or t.stride(2) != 1 or t.stride(1) != d:
+            raise ValueError(f"{n} must be [B][H_kv][d] with contiguous head rows")
+        if t.dtype != key_cache.dtype:
+            raise ValueError(f"{n} must have the cache's dtype")
+    if slot_mapping.dtype != torch.int64 or not slot_mapping.is_contiguous():
+        raise ValueError("slot_mapping must be contiguous int64")
+
+
+def pa_decode_append(out, q, k_new, v_new, slot_mapping, key_cache, value_cache, block_tables, seq_lens,
+                     scale, max_seq_len, partition_size=0, workspace=None, algo=PA_ALGO_AUTO, stream=None,
+                     flags=0):
+    """pa_reshape_and_cache of one new token per sequence (k_new / v_new row b,
+    slot_mapping[b]) then pa_decode, as one kernel where pa_decode_append_fused
+    says so (include/pa.h).  seq_lens count the new token."""
+    _dev(out, q, k_new, v_new, slot_mapping, key_cache, value_cache, block_tables, seq_lens, workspace)
+    for t, n in ((out, "out"), (q, "q"), (key_cache, "key_cache"), (value_cache, "value_cache"),
+                 (block_tables, "block_tables"), (seq_lens, "seq_lens")):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_tables and seq_lens must be int32")
+    _new_rows(k_new, v_new, slot_mapping, key_cache)
+    if k_new.shape[0] != q.shape[0] or slot_mapping.numel() != q.shape[0]:
+        raise ValueError("one new token per sequence")
+    flags |= _out_flag(out, q)
+    p = make_params(q, key_cache, block_tables, max_seq_len, None, None, partition_size, workspace, algo,
+                    flags)
+    _check(lib.pa_decode_append(_ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping),
+                                k_new.stride(0), v_new.stride(0), _ptr(key_cache), _ptr(value_cache),
+                                _ptr(block_tables), _ptr(seq_lens), ctypes.c_float(scale), ctypes.byref(p),
+                                _stream(stream)), "pa_decode_append")
+
+
+def pa_decode_append_fused(q, k_new, v_new, key_cache, block_tables, max_seq_len, partition_size=0,
+                           algo=PA_ALGO_AUTO) -> bool:
+    """Whether pa_decode_append with these operands runs as one kernel."""
+    p = make_params(q, key_cache, block_tables, max_seq_len, None, None, partition_size, None, algo)
+    r = int(lib.pa_decode_append_fused(ctypes.byref(p), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                       k_new.stride(0), v_new.stride(0)))
+    _check(min(r, 0), "pa_decode_append_fused")
+    return r == 1
+
+
 def pa_decode_fixed_scratch(out, q, key_cache, value_cache, block_tables, seq_lens, scale,
                             max_seq_len, k_scales=None, v_scales=None, partition_size=-1,
                             algo=PA_ALGO_AUTO, stream=None):
     """pa_decode for callers that cannot allocate a workspace: the split-K
     scratch is the fixed area compiled into the library (FIXED_SCRATCH_BYTES per
     device).  Calls on one device must not overlap; the first call on a device
-    synchronises its stream once and should come before any stream capture."""
+    looks up the area's address and should come before any stream capture."""
     _dev(out, q, key_cache, value_cache, block_tables, seq_lens, k_scales, v_scales)
     for t, n in ((out, "out"), (q, "q"), (key_cache, "key_cache"), (value_cache, "value_cache"),
                  (block_tables, "block_tables"), (seq_lens, "seq_lens")):

@@ -2,8 +2,9 @@
 
 Uploads every operation's arrays once, owns the device KV pool, and runs
 setup / step operations with ``pa_reshape_and_cache``, ``pa_block_copy`` and
-``pa_decode``.  Optionally converts the pool to int8 (``pa_quantize_int8``)
-after setup.
+``pa_decode`` -- or, for a step whose append ends with its sequences' new
+tokens, those tokens and the decode with one ``pa_decode_append`` call.
+Optionally converts the pool to int8 (``pa_quantize_int8``) after setup.
 """
 from __future__ import annotations
 
@@ -40,6 +41,9 @@ class DeviceWorkload:
         self.setup = [self._upload(op) for op in w.setup]
         idx = range(len(w.steps)) if steps is None else steps
         self.steps = {i: [self._upload(op) for op in w.steps[i]] for i in idx}
+        # steps whose append ends with one new token per decoded sequence, at its last
+        # position (pa_decode_append can take those tokens)
+        self.new_tokens = {i: new_token_split(w.steps[i]) for i in idx}
         self.out = {}
 
     def fill(self, nan: bool):
@@ -119,7 +123,24 @@ class DeviceWorkload:
             self.run(op)
 
     def run_step(self, i, partition_size=0, int8=False, algo=pa.PA_ALGO_AUTO, decode=True,
-                 out_f32=False):
+                 out_f32=False, fused=False):
+        """fused: a step whose append ends with its sequences' new tokens runs the
+        rest of the append (if any) with pa_reshape_and_cache, then those tokens and
+        the decode with one pa_decode_append call."""
+        if fused and decode and not int8 and self.new_tokens.get(i) is not None:
+            for op in self.steps[i][:-2]:
+                self.run(op)
+            (_, k, v, s), dec = self.steps[i][-2:]
+            _, q, bt, sl, mx, out = dec
+            T, B = k.shape[0], q.shape[0]
+            if T > B:
+                pa.pa_reshape_and_cache(k[:T - B], v[:T - B], self.kc, self.vc, s[:T - B])
+            if out_f32:
+                out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+            ws = self.workspace_for(dec, partition_size, False, algo) if partition_size != 0 else None
+            pa.pa_decode_append(out, q, k[T - B:], v[T - B:], s[T - B:], self.kc, self.vc, bt, sl, self.w.scale,
+                                mx, partition_size, ws, algo)
+            return out
         out = None
         for op in self.steps[i]:
             if op[0] == "decode":
@@ -135,15 +156,45 @@ class DeviceWorkload:
         return self.run(op, partition_size, None, int8, algo, out_f32=out_f32)
 
 
+def new_token_split(ops):
+    """For a step [..., Reshape, Decode] of single-token decode whose Reshape ends
+    with one token per sequence at its last position (slot of position
+    seq_lens[b] - 1 under the block table; no token for an empty sequence), the
+    number of leading tokens before them; else None."""
+    if len(ops) < 2 or not isinstance(ops[-2], W.Reshape) or not isinstance(ops[-1], W.Decode):
+        return None
+    r, d = ops[-2:]
+    if d.q.ndim != 3:
+        return None
+    B, T = d.q.shape[0], len(r.slot_mapping)
+    if T < B:
+        return None
+    slots = r.slot_mapping[T - B:]
+    L = d.seq_lens.astype(np.int64)
+    for b in range(B):
+        if L[b] <= 0:
+            if slots[b] >= 0:
+                return None
+            continue
+        pos = L[b] - 1
+        if slots[b] != int(d.block_tables[b, pos // W.BLOCK_SIZE]) * W.BLOCK_SIZE + pos % W.BLOCK_SIZE:
+            return None
+    return T - B
+
+
 class StepCalls:
     """Pre-marshalled C-ABI calls for every step, so a timed loop costs one
     ctypes call per library entry point and nothing else on the host."""
 
     def __init__(self, dw: DeviceWorkload, partition_size=-1, int8=False, algo=pa.PA_ALGO_AUTO,
-                 stream=None, flags=0, append_flags=0):
+                 stream=None, flags=0, append_flags=0, fused=False, prompt_flags=0):
         """flags: pa_decode flags; append_flags: pa_reshape_and_cache_ex flags
         (PA_APPEND_OVERLAP_PREVIOUS only for recipes whose appends never touch
-        what the previous step's decode reads, ``appends_overlap_previous``)."""
+        what the previous step's decode reads, ``appends_overlap_previous``).
+        fused: steps whose append ends with their sequences' new tokens issue the
+        leading tokens (prompts of admitted sequences) with pa_reshape_and_cache_ex
+        and prompt_flags, then one pa_decode_append call for the new tokens and the
+        decode (its launches as pa_decode_append_fused reports)."""
         import ctypes
         self.dw = dw
         self.stream = stream if stream is not None else torch.cuda.current_stream()
@@ -153,9 +204,10 @@ class StepCalls:
         ks = dw.k_scales if int8 else None
         vs = dw.v_scales if int8 else None
         ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
-        if append_flags and not getattr(w, "appends_overlap_previous", False):
+        if (append_flags or prompt_flags) and not getattr(w, "appends_overlap_previous", False):
             raise ValueError("this recipe's appends may touch what the previous decode reads")
         aflags = int(append_flags)
+        self.fused_steps = 0
         # one workspace, sized for the largest step
         need = 0
         for ops in dw.steps.values():
@@ -170,6 +222,40 @@ class StepCalls:
         self.launches = {}
         for i, ops in dw.steps.items():
             calls, launches = [], 0
+            lead = dw.new_tokens.get(i) if fused and not int8 else None
+            if lead is not None:
+                N, H, bs, d = dw.kc.shape
+                for op in ops[:-2]:  # copy-on-write copies before the append
+                    if op[0] != "copy":
+                        raise ValueError("a fused step takes only block copies before its append")
+                    n = op[1].numel() // 2
+                    if n:
+                        args = (ptr(dw.kc), ptr(dw.vc), None, None, ptr(op[1]), n, H, d, bs, N,
+                                pa.dtype_code(dw.kc.dtype), sp)
+                        calls.append(("copy", pa.lib.pa_block_copy, args))
+                        launches += 1
+                (_, k, v, s), (_, q, bt, sl, mx, out) = ops[-2:]
+                if lead:
+                    args = (ptr(k), ptr(v), ptr(dw.kc), ptr(dw.vc), ptr(s), lead, H, d, bs, N,
+                            pa.dtype_code(k.dtype), k.stride(0), v.stride(0), int(prompt_flags), sp)
+                    calls.append(("reshape", pa.lib.pa_reshape_and_cache_ex, args))
+                    launches += 1
+                kn, vn, sn = k[lead:], v[lead:], s[lead:]
+                p = pa.make_params(q, kc, bt, mx, None, None, partition_size, self.workspace, algo, flags)
+                self.keep.append(p)
+                split = pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+                one = pa.lib.pa_decode_append_fused(ctypes.byref(p), ptr(q), ptr(kn), ptr(vn), kn.stride(0),
+                                                    vn.stride(0))
+                if one < 0:
+                    raise pa.PaError(one, "pa_decode_append_fused")
+                args = (ptr(out), ptr(q), ptr(kn), ptr(vn), ptr(sn), kn.stride(0), vn.stride(0), ptr(kc),
+                        ptr(vc), ptr(bt), ptr(sl), ctypes.c_float(w.scale), ctypes.byref(p), sp)
+                calls.append(("decode", pa.lib.pa_decode_append, args))
+                launches += (1 if one == 1 else 2) + (1 if split else 0)
+                self.fused_steps += one == 1
+                self.calls[i] = calls
+                self.launches[i] = launches
+                continue
             for op in ops:
                 if op[0] == "reshape":
                     _, k, v, s = op

@@ -251,3 +251,42 @@ def test_stall_selftest_rejects_bad_args():
     p = params(algo=pa.PA_ALGO_SIMT)
     assert L.pa_decode_stall_selftest(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, f, ctypes.byref(p), 0, 1000, None) \
         == pa.PA_ERR_UNSUPPORTED
+
+
+def test_decode_append_reports_when_it_fuses():
+    """pa_decode_append runs as one kernel on the tensor-core family's per-warp
+    decode of single-token fp16/bf16 rows with 16-byte aligned q and new-token
+    rows; otherwise as pa_reshape_and_cache then pa_decode (0); arguments it would
+    reject give their status.  No pointer is read."""
+    A = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced
+    def fused(p, kn=A, vn=A, ks=None, vs=None):
+        row = p.num_kv_heads * p.head_dim
+        return pa.lib.pa_decode_append_fused(ctypes.byref(p), A, kn, vn, row if ks is None else ks,
+                                             row if vs is None else vs)
+    assert fused(params()) == 1
+    assert fused(params(q_dtype=pa.PA_BF16, kv_dtype=pa.PA_BF16, partition_size=-1)) == 1
+    assert fused(params(head_dim=256, partition_size=16)) == 1
+    assert fused(params(head_dim=64, num_q_heads=2, num_kv_heads=2)) == 1
+    assert fused(params(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32)) == 0          # CUDA-core family
+    assert fused(params(algo=pa.PA_ALGO_SIMT)) == 0
+    assert fused(params(num_q_heads=32, num_kv_heads=1, partition_size=-1)) == 0  # cooperative mode
+    assert fused(params(num_q_heads=32, num_kv_heads=1, partition_size=0)) == 1   # rows of 8 heads
+    assert fused(params(), kn=ctypes.c_void_p(0x10008)) == 0                   # k_new not 16-byte aligned
+    assert fused(params(), ks=2 * 128 + 4) == 0                                 # stride not 8 elements
+    assert fused(params(query_len=2)) == pa.PA_ERR_UNSUPPORTED
+    assert fused(params(kv_dtype=pa.PA_I8)) == pa.PA_ERR_DTYPE
+    assert fused(params(), ks=100) == pa.PA_ERR_SHAPE
+    assert fused(params(head_dim=96)) == pa.PA_ERR_UNSUPPORTED
+
+
+def test_decode_append_rejects_before_any_launch():
+    p = params()
+    out = q = kc = vc = bt = sl = FAKE
+    args = lambda slots, **kw: (out, q, FAKE, FAKE, slots, 256, 256, kc, vc, bt, sl,  # noqa: E731
+                                ctypes.c_float(0.1), ctypes.byref(params(**kw)), None)
+    assert pa.lib.pa_decode_append(*args(None)) == pa.PA_ERR_NULL
+    assert pa.lib.pa_decode_append(*args(FAKE, query_len=3)) == pa.PA_ERR_UNSUPPORTED
+    assert pa.lib.pa_decode_append(*args(FAKE, kv_dtype=pa.PA_I8, q_dtype=pa.PA_F16)) == pa.PA_ERR_DTYPE
+    # split-K without a workspace
+    assert pa.lib.pa_decode_append(*args(FAKE, partition_size=16)) == pa.PA_ERR_WORKSPACE
+    del p
