@@ -113,6 +113,13 @@ template <> struct Mma<__half> {
             : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
             : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
     }
+    // d = a . b (a zero accumulator)
+    static __device__ __forceinline__ void mma0(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+    }
 };
 template <> struct Mma<__nv_bfloat16> {
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
@@ -125,6 +132,12 @@ template <> struct Mma<__nv_bfloat16> {
             "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
             : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
             : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    static __device__ __forceinline__ void mma0(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
     }
 };
 
@@ -1802,6 +1815,12 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
     uint32_t c_ph = 0;     // (c_k / S) & 1
     bool alive = true;
     const int row0 = warp * 16;  // this warp's first column (head) of the row
+    // Scores stay unscaled: p = 2^((s - m) |scale| log2 e) with m the (lazy) maximum of
+    // the unscaled scores, kLazyMax of slack in log2 units being lazy_raw unscaled.
+    // (a zero scale is taken as 1e-30: every probability 1 to within 1e-26 relative,
+    // and the slots past a row's end still weigh exactly 0)
+    const float sl = fmaxf(fabsf(a.scale_log2), 1e-30f);
+    const float lazy_raw = kLazyMax / sl;
     while (have) {
         const int len = cs.j1 - cs.j0;
         const int ntok_last = cs.L - (cs.nb - 1) * kBlockSize;
@@ -1814,10 +1833,17 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
             const uint4 *qg = reinterpret_cast<const uint4 *>(a.q) +
                               ((size_t)cs.b * a.Hq + (size_t)cs.kvh * GC + row0) * (D / 8);
             __syncwarp();  // the previous segment's fragment reads are done
+            // a negative scale goes into q (sign bits flipped, exact), so that the scores
+            // below are scaled by |scale| and their maximum is taken before scaling
+            const uint32_t sflip = a.scale_log2 < 0.f ? 0x80008000u : 0u;
 #pragma unroll
             for (int i = 0; i < 16 * D / 8 / 32; ++i) {
                 const int id = i * 32 + lane, r = id / (D / 8), ch = id % (D / 8);
-                const uint4 v = __ldg(qg + id);
+                uint4 v = __ldg(qg + id);
+                v.x ^= sflip;
+                v.y ^= sflip;
+                v.z ^= sflip;
+                v.w ^= sflip;
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(qslot + r * (2 * D) + ((ch ^ (r & 7)) << 4)),
                              "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                              : "memory");
@@ -1827,10 +1853,10 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
         for (int j = 0; alive && j < len; ++j) {
             const int s = c_s;
             const uint32_t parity = c_ph;
-            int ok = lane == 0 ? (int)mbar_wait(&full[s], parity, a.wait_ns) : 0;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (ok && lane != 0) mbar_wait(&full[s], parity, a.wait_ns);
-            if (!ok || *reinterpret_cast<volatile int *>(&abort_flag)) {
+            // every lane polls the stage's barrier; the CTA's abort flag (the producer gave
+            // up) is looked at every 16 blocks and after a failed wait
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], parity, a.wait_ns));
+            if (!ok || ((c_k & 15) == 15 && *reinterpret_cast<volatile int *>(&abort_flag))) {
                 if (lane == 0) atomicExch(&abort_flag, 1);
                 alive = false;
                 break;
@@ -1841,23 +1867,24 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
                 // ---- S = Q . K^T: n-tiles of tokens 0-7 and 8-15, two chains each
                 float sa[2][2][4];
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) sa[0][u][e] = sa[1][u][e] = 0.f;
-#pragma unroll
                 for (int ks = 0; ks < C::KSTEPS; ++ks) {
                     uint32_t kb[4], qa[4];
                     ldsm_x4(qa, qaddr(ks));
                     ldsm_x4(kb, tK + moff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
-                    Mma<T>::mma(sa[0][ks & 1], qa, kb[0], kb[1]);
-                    Mma<T>::mma(sa[1][ks & 1], qa, kb[2], kb[3]);
+                    if (ks < 2) {
+                        Mma<T>::mma0(sa[0][ks & 1], qa, kb[0], kb[1]);
+                        Mma<T>::mma0(sa[1][ks & 1], qa, kb[2], kb[3]);
+                    } else {
+                        Mma<T>::mma(sa[0][ks & 1], qa, kb[0], kb[1]);
+                        Mma<T>::mma(sa[1][ks & 1], qa, kb[2], kb[3]);
+                    }
                 }
-                // x[nt][e]: head g (e < 2) or g + 8, token 8 nt + 2c + (e & 1), log2 units
+                // x[nt][e]: head g (e < 2) or g + 8, token 8 nt + 2c + (e & 1), unscaled
                 float x[2][4];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) x[nt][e] = (sa[nt][0][e] + sa[nt][1][e]) * a.scale_log2;
+                    for (int e = 0; e < 4; ++e) x[nt][e] = sa[nt][0][e] + sa[nt][1][e];
                 if (ntok < kBlockSize) {  // the row's last block: slots past the end see nothing
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt)
@@ -1873,9 +1900,9 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
                 // move the reference point only when a score exceeds it by more than
                 // kLazyMax (always on the segment's first block: m = -inf)
-                if (__any_sync(0xffffffffu, mx0 > m0 + kLazyMax || mx1 > m1 + kLazyMax)) {
+                if (__any_sync(0xffffffffu, mx0 > m0 + lazy_raw || mx1 > m1 + lazy_raw)) {
                     const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                    const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+                    const float al0 = fast_exp2((m0 - mn0) * sl), al1 = fast_exp2((m1 - mn1) * sl);
                     l0 *= al0;
                     l1 *= al1;
 #pragma unroll
@@ -1889,12 +1916,13 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
                     m1 = mn1;
                 }
                 float p[2][4];
+                const float ms0 = m0 * sl, ms1 = m1 * sl;
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    p[nt][0] = fast_exp2(x[nt][0] - m0);
-                    p[nt][1] = fast_exp2(x[nt][1] - m0);
-                    p[nt][2] = fast_exp2(x[nt][2] - m1);
-                    p[nt][3] = fast_exp2(x[nt][3] - m1);
+                    p[nt][0] = fast_exp2(fmaf(x[nt][0], sl, -ms0));
+                    p[nt][1] = fast_exp2(fmaf(x[nt][1], sl, -ms0));
+                    p[nt][2] = fast_exp2(fmaf(x[nt][2], sl, -ms1));
+                    p[nt][3] = fast_exp2(fmaf(x[nt][3], sl, -ms1));
                 }
                 l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
                 l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
@@ -1971,8 +1999,8 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
             }
         } else {
             const int ch_first = ck.of(cs.b, cs.kvh, cs.nb, 0);
-            const int sl = 2 * cs.ch + ((cs.ch == ch_first && ck.mid_start(cs.b, cs.kvh, cs.nb)) ? 1 : 0);
-            float *w0 = a.ws_o + ((size_t)sl * GC + row0 + g) * D + 2 * c;
+            const int slot = 2 * cs.ch + ((cs.ch == ch_first && ck.mid_start(cs.b, cs.kvh, cs.nb)) ? 1 : 0);
+            float *w0 = a.ws_o + ((size_t)slot * GC + row0 + g) * D + 2 * c;
             float *w1 = w0 + 8 * D;
 #pragma unroll
             for (int i = 0; i < C::NT; ++i) {
@@ -1980,8 +2008,8 @@ __global__ void __launch_bounds__(CoopCfg<T, D, NG>::THREADS, CoopCfg<T, D, NG>:
                 *reinterpret_cast<float2 *>(w1 + 8 * i) = make_float2(o[i][2] * inv1, o[i][3] * inv1);
             }
             if (c == 0) {
-                a.ws_lse[(size_t)sl * GC + row0 + g] = m0 + log2f(l0);
-                a.ws_lse[(size_t)sl * GC + row0 + g + 8] = m1 + log2f(l1);
+                a.ws_lse[(size_t)slot * GC + row0 + g] = m0 * sl + log2f(l0);
+                a.ws_lse[(size_t)slot * GC + row0 + g + 8] = m1 * sl + log2f(l1);
             }
         }
         have = next_seg(cit, cs);

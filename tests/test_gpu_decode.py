@@ -437,6 +437,20 @@ def test_large_groups(hq, hkv, part, algo):
     assert_close(got[0], ref[0], "float16", f"G={hq // hkv} part={part}")
 
 
+@pytest.mark.parametrize("scale", [-0.07, 0.0, 0.5])
+@pytest.mark.parametrize("hq", [32, 64])
+def test_large_groups_any_scale(hq, scale):
+    """The cooperative mode keeps scores unscaled and folds the scale into the
+    exponent: a negative scale (flipped into q), a zero scale (uniform weights) and a
+    sharp one, against the oracle."""
+    w = W.random_case([3, 40, 301], num_q_heads=hq, num_kv_heads=1, head_dim=128, dtype="float16",
+                      seed=hq + 5)
+    w.scale = scale
+    ref, _, _ = replay(w)
+    got, _ = run_gpu(w, -1)
+    assert_close(got[0], ref[0], "float16", f"G={hq} scale={scale}")
+
+
 @pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
 def test_large_group_bf16_and_int8(qdt):
     w = W.random_case([7, 129, 640], num_q_heads=64, num_kv_heads=1, head_dim=128, dtype=qdt, seed=77)
