@@ -186,7 +186,10 @@ struct TcCfg {
     // for.  A head_dim-256 stage is 16 KB (K and V tiles of 8 KB), so two stages per
     // warp and three warps per CTA keep two CTAs (six warps, 192 KB in flight) on an SM.
     static constexpr int NW = D == 256 ? 3 : PA_TC_WARPS;
-    static constexpr int MIN_CTAS = D == 256 ? 2 : PA_TC_MIN_CTAS;
+    // 4-bit tiles are 2 KB: their conversion chains keep a warp busy far longer than its
+    // copies take, so three CTAs (twelve warps, 168 registers) share an SM
+    static constexpr int MIN_CTAS = D == 256 ? 2 : (I4 ? 3 : PA_TC_MIN_CTAS);
+    static constexpr int BUDGET = MIN_CTAS >= 3 ? 200 * 1024 / MIN_CTAS - 8 * 1024 : PA_TC_RING_BUDGET;
     static constexpr int THREADS = NW * 32;
     static constexpr int ROW_BYTES = I4 ? D / 2 : 128;              // bytes per box row
     static constexpr int BOXW = I4 ? D / 2 : 128 / (int)sizeof(TKV);  // TMA elements per box row
@@ -198,7 +201,7 @@ struct TcCfg {
     static constexpr int stages() {
         int s = PA_TC_INFLIGHT / STAGE;
         s = s < 2 ? 2 : (s > 8 ? 8 : s);
-        while (s > 2 && NW * s * (STAGE + QSLOT) > PA_TC_RING_BUDGET) --s;
+        while (s > 2 && NW * s * (STAGE + QSLOT) > BUDGET) --s;
         return s;
     }
     static constexpr int S = stages();            // ring stages per warp
@@ -210,8 +213,9 @@ struct TcCfg {
     static constexpr int BAR_OFF = QRING_OFF + NW * S * QSLOT;
     static constexpr int OK_OFF = BAR_OFF + NW * S * 8;
     static constexpr int SC_OFF = OK_OFF + NW * S * 4;    // float [NW][S][2]: int8 K, V scales
-    // pa_decode_append: a row end's new K and V rows, and the cache slot its warp writes
-    static constexpr int PATCH = 2 * D * 2;
+    // pa_decode_append (fp16 / bf16 caches): a row end's new K and V rows, and the cache
+    // slot its warp writes
+    static constexpr int PATCH = std::is_same<TKV, __half>::value || std::is_same<TKV, __nv_bfloat16>::value ? 2 * D * 2 : 0;
     static constexpr int PATCH_OFF = (SC_OFF + NW * S * 8 + 15) / 16 * 16;
     static constexpr int PSLOT_OFF = PATCH_OFF + NW * S * PATCH;  // int64 [NW][S], -1: none
     static constexpr int CUM_OFF = PSLOT_OFF + NW * S * 8;
