@@ -217,8 +217,8 @@ struct TcCfg {
     // slot its warp writes
     static constexpr int PATCH = std::is_same<TKV, __half>::value || std::is_same<TKV, __nv_bfloat16>::value ? 2 * D * 2 : 0;
     static constexpr int PATCH_OFF = (SC_OFF + NW * S * 8 + 15) / 16 * 16;
-    static constexpr int PSLOT_OFF = PATCH_OFF + NW * S * PATCH;  // int64 [NW][S], -1: none
-    static constexpr int CUM_OFF = PSLOT_OFF + NW * S * 8;
+    static constexpr int PSLOT_OFF = PATCH_OFF + NW * S * PATCH;  // int [NW][S], -1: none
+    static constexpr int CUM_OFF = PSLOT_OFF + NW * S * 4;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (3 * B + 3) * 4; }
 };
 
@@ -459,7 +459,7 @@ __device__ __forceinline__ void vfrag_i4(const uint32_t (&r)[4][2], int i, uint3
 // MQ: the general column mapping (several new tokens per sequence, causal among
 // them, or padding columns); without it every row's G columns are the G query
 // heads of one single-token decode, and the kernel keeps the plain addressing.
-template <typename T, typename TKV, int D, int G, bool MQ>
+template <typename T, typename TKV, int D, int G, bool MQ, bool APP>
 __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::MIN_CTAS)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
@@ -472,9 +472,9 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     constexpr bool kQz = kI8 || kI4;  // quantised cache: per-(block, KV head) scales
     static_assert(!kQz || (std::is_same<T, __half>::value && D == 128),
                   "int8 and 4-bit caches: fp16 q, head_dim 128");
-    // pa_decode_append: single-token rows of an fp16 / bf16 cache
-    constexpr bool kApp = !MQ && !kQz;
-    const bool app = kApp && a.append;
+    // APP (pa_decode_append): single-token rows of an fp16 / bf16 cache
+    static_assert(!APP || (!MQ && !kQz), "the fused append takes single-token fp16 / bf16 rows");
+    constexpr bool app = APP;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -686,15 +686,15 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     // id outside the pool is marked -2 there.
     float p_ks = 0.f, p_vs = 0.f, p_ks_next = 0.f, p_vs_next = 0.f;
     // pa_decode_append: the lane holding a row's last block also loads the sequence's
-    // new-token slot and its length as given (the row's L may have been cut short)
-    long long p_sn = -1, p_sn_next = -1;
-    int p_lr = 0, p_lr_next = 0;
-    auto win_load = [&](const Win &w, float &ks, float &vs, long long &sn, int &lr) -> int {
+    // new-token slot (as an int: this family's pools hold fewer than 2^31 slots, so a
+    // larger slot is marked 2^31 - 1, outside the pool)
+    int p_sn = -1, p_sn_next = -1;
+    auto win_load = [&](const Win &w, float &ks, float &vs, int &sn) -> int {
         if (!w.valid || lane >= w.n) return -1;
         const int pb = a.tables[(size_t)w.sg.b * a.mbps + w.sg.j0 + w.o + lane];
         if (app && w.sg.j0 + w.o + lane == w.sg.nb - 1) {
-            sn = a.slot_new[w.sg.b];
-            lr = a.lens[w.sg.b];
+            const long long s64 = a.slot_new[w.sg.b];
+            sn = s64 > 0x7fffffffLL ? 0x7fffffff : (int)s64;
         }
         if constexpr (kQz) {
             if (pb < 0 || (int64_t)pb >= a.N) return -2;
@@ -706,11 +706,11 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     Win pc, pn;
     win_first(pc);
     win_after(pc, pn);
-    int p_y = win_load(pc, p_ks, p_vs, p_sn, p_lr), p_y_next = win_load(pn, p_ks_next, p_vs_next, p_sn_next, p_lr_next);
+    int p_y = win_load(pc, p_ks, p_vs, p_sn), p_y_next = win_load(pn, p_ks_next, p_vs_next, p_sn_next);
     int p_i = 0, p_k = 0;
     float *my_sc = stage_sc + warp * S * 2;
     const uint32_t my_patch = smem_addr(smem) + C::PATCH_OFF + warp * S * C::PATCH;
-    long long *my_pslot = reinterpret_cast<long long *>(smem + C::PSLOT_OFF) + warp * S;
+    int *my_pslot = reinterpret_cast<int *>(smem + C::PSLOT_OFF) + warp * S;
     auto refill = [&]() {
         if (!pc.valid) return;
         const int pb = __shfl_sync(0xffffffffu, p_y, p_i);
@@ -722,22 +722,18 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             vsv = __shfl_sync(0xffffffffu, p_vs, p_i);
         }
         // pa_decode_append, a row's last block: the new token is patched into the staged
-        // tile when it is the row's last decoded position and its slot is that position's
-        // slot in this block; the row's warp writes it to its cache slot (one warp per
-        // cache KV head) whether or not it is patched
+        // tile when its slot is the slot of the row's last decoded position (then the
+        // append before the decode would have put it exactly there); the row's warp
+        // writes it to its cache slot (one warp per cache KV head) in any case
         bool patch = false;
-        long long psn = -1;
+        int psn = -1;
         if (app && pc.sg.j0 + pc.o + p_i == pc.sg.nb - 1) {
-            const long long sn = __shfl_sync(0xffffffffu, p_sn, p_i);
-            const int lr = __shfl_sync(0xffffffffu, p_lr, p_i);
-            const int L = pc.sg.L;
-            const bool inpool = sn >= 0 && sn < a.N * kBlockSize;
-            const bool cur = lr == L;
-            patch = cur && y >= 0 && sn == (long long)pb * kBlockSize + (L - 1) % kBlockSize;
+            const int sn = __shfl_sync(0xffffffffu, p_sn, p_i);
+            const bool inpool = sn >= 0 && (int64_t)sn < a.N * kBlockSize;
+            patch = y >= 0 && sn == pb * kBlockSize + (pc.sg.L - 1) % kBlockSize;
             const bool writer = pc.sg.kvh % a.ngroups == 0;
             psn = inpool && writer ? sn : -1;
             if (lane == 0 && writer && sn >= 0 && !inpool) raise_flag(PA_EFLAG_BAD_SLOT);
-            if (lane == 0 && writer && cur && sn >= 0 && !patch) raise_flag(PA_EFLAG_APPEND_SLOT);
         }
         if (lane == 0) {
             const int s = p_k % S;
@@ -809,9 +805,8 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             p_ks = p_ks_next;
             p_vs = p_vs_next;
             p_sn = p_sn_next;
-            p_lr = p_lr_next;
             win_after(pc, pn);
-            p_y_next = win_load(pn, p_ks_next, p_vs_next, p_sn_next, p_lr_next);
+            p_y_next = win_load(pn, p_ks_next, p_vs_next, p_sn_next);
         }
     };
     if (a.early) {
@@ -1081,7 +1076,10 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
                 // pa_decode_append: the new token's K and V rows, staged with this block,
                 // replace tile row ntok - 1 (its slot) and go to their cache slot
                 const int okw = my_ok[s];
-                const long long psn = my_pslot[s];
+                const int psn = my_pslot[s];
+                // a new token written elsewhere although this row's length counts it: the
+                // slot is not its position's (rare: looked up only here)
+                if (!(okw & 2) && psn >= 0 && lane == 0 && a.lens[cs.b] == cs.L) raise_flag(PA_EFLAG_APPEND_SLOT);
                 if ((okw & 2) || psn >= 0) {
                     const int r = ntok - 1;
                     const int kc = cs.kvh / a.ngroups;
@@ -2127,7 +2125,11 @@ bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
 template <typename T, typename TKV, int D, int G, bool MQ>
 static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     using C = TcCfg<TKV, D, G>;
-    auto kern = decode_tc_kernel<T, TKV, D, G, MQ>;
+    auto kern = decode_tc_kernel<T, TKV, D, G, MQ, false>;
+    if constexpr (!MQ && std::is_same<T, TKV>::value) {
+        if (a.append) kern = decode_tc_kernel<T, TKV, D, G, MQ, true>;
+    }
+    if (a.append && kern == decode_tc_kernel<T, TKV, D, G, MQ, false>) return PA_ERR_UNSUPPORTED;
     const int smem = C::smem_bytes(a.B);
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
     if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are read as aligned 32-bit pairs
