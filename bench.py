@@ -50,12 +50,13 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of the decode kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum of the two captured launches, trace steps 8 and 9 of the
-# ragged workload), per algorithmic byte.
+# ragged workload, the kernel of pa_decode_append that the bench's step runs), per
+# algorithmic byte.
 # It holds only for the kernel code it was taken on (hash of the source without
 # comments); after any code change the bench reports null until it is taken again.
 NCU_TRAFFIC = {
-    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "1435942a2a2a7598",
-               "per_alg_byte": (474932736 + 5912064 + 462019840 + 4562944) / (472969728 + 459894508)},
+    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "cbb6898759f164bf",
+               "per_alg_byte": (475200512 + 4807424 + 462293248 + 4693760) / (472969728 + 459894508)},
 }
 
 
@@ -66,9 +67,10 @@ def code_hash(path):
     return hashlib.sha256(" ".join(s.split()).encode()).hexdigest()[:16]
 
 
-def traffic_per_launch(workload, algo, partition, mean_alg_bytes):
+def traffic_per_launch(workload, algo, partition, mean_alg_bytes, fused=True):
     t = NCU_TRAFFIC.get(workload)
-    if t is None or algo == "simt" or partition != -1 or code_hash(os.path.join(ROOT, t["source"])) != t["code"]:
+    if t is None or algo == "simt" or partition != -1 or not fused or \
+            code_hash(os.path.join(ROOT, t["source"])) != t["code"]:
         return None
     return t["per_alg_byte"] * mean_alg_bytes
 
@@ -525,9 +527,12 @@ def main(argv=None):
         "hbm_frac_of_" + peak_kind: value / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": traffic_per_launch(args.workload, args.algo, part, bytes_rank / K),
+                     "traffic": traffic_per_launch(args.workload, args.algo, part, bytes_rank / K,
+                                                   calls.fused_steps > 0),
                      "traffic_unit": "bytes per decode launch (ncu DRAM read + write, scaled)",
-                     "kernel": "pa_decode: the K steps' decode calls issued back to back",
+                     "kernel": ("pa_decode_append (new tokens + decode, one kernel) and its merge: the K "
+                                "steps' calls issued back to back" if calls.fused_steps else
+                                "pa_decode: the K steps' decode calls issued back to back"),
                      "peak_kind": peak_kind},
         "gpu_launches": launches,
         "host_enqueue_ms": host_ms,
