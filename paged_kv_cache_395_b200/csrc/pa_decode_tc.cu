@@ -1061,13 +1061,10 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
             }
             const int s = c_k % S;
             const uint32_t parity = (c_k / S) & 1;
-            int ok = lane == 0 ? (int)mbar_wait(&my_bars[s], parity, a.wait_ns) : 0;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&my_bars[s], parity, a.wait_ns))) {
                 alive = false;
                 break;
             }
-            if (lane != 0) mbar_wait(&my_bars[s], parity, a.wait_ns);
             if (j == 0) load_q(s, bq, ncol);  // the segment's q came with its first block
             const bool row_end = cs.j0 + j == cs.nb - 1;
             const int ntok = row_end ? ntok_last : kBlockSize;
@@ -1153,21 +1150,26 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
                 }
                 // ---- S^T = K . Q^T, four independent accumulator chains
                 float sa[4][4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) sa[u][0] = sa[u][1] = sa[u][2] = sa[u][3] = 0.f;
+                // the first product of each chain starts from a zero accumulator
+                auto qk = [&](int ks, const uint32_t (&f)[4]) {
+                    if (ks < 4)
+                        Mma<T>::mma0(sa[ks & 3], f, bq[ks][0], bq[ks][1]);
+                    else
+                        Mma<T>::mma(sa[ks & 3], f, bq[ks][0], bq[ks][1]);
+                };
 #pragma unroll
                 for (int ks = 0; ks < C::KSTEPS; ++ks) {
                     if constexpr (kI4) {
                         kfrag_i4(kw4, ks, kf[0]);
-                        Mma<T>::mma(sa[ks & 3], kf[0], bq[ks][0], bq[ks][1]);
+                        qk(ks, kf[0]);
                     } else if constexpr (kI8) {
                         kfrag_i8(kw, ks, kf[0]);
-                        Mma<T>::mma(sa[ks & 3], kf[0], bq[ks][0], bq[ks][1]);
+                        qk(ks, kf[0]);
                     } else if constexpr (kHoistK) {
-                        Mma<T>::mma(sa[ks & 3], kf[ks], bq[ks][0], bq[ks][1]);
+                        qk(ks, kf[ks]);
                     } else {
                         ldsm_x4(kf[0], tK + koff[ks & 3] + (ks >> 2) * C::BOX_BYTES);
-                        Mma<T>::mma(sa[ks & 3], kf[0], bq[ks][0], bq[ks][1]);
+                        qk(ks, kf[0]);
                     }
                 }
                 float sc[4];
