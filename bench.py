@@ -55,8 +55,8 @@ FALLBACK_HBM_GBS = 6650.0
 # It holds only for the kernel code it was taken on (hash of the source without
 # comments); after any code change the bench reports null until it is taken again.
 NCU_TRAFFIC = {
-    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "cbb6898759f164bf",
-               "per_alg_byte": (475200512 + 4807424 + 462293248 + 4693760) / (472969728 + 459894508)},
+    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "7c3c95cd8e684b52",
+               "per_alg_byte": (475201024 + 4691968 + 462296576 + 4716544) / (472969728 + 459894508)},
 }
 
 
