@@ -89,6 +89,8 @@ WORKLOADS = {
                   "copy-on-write + private suffix U[64,1048]",
     "mqa": "MQA: 32 q heads / 1 KV head, head_dim 128, fp16, batch 128, all lengths 4096",
     "d256": "head_dim 256: 16 q / 8 KV heads, fp16, batch 16, all lengths 4096",
+    "d256_int8": "head_dim 256: 16 q / 8 KV heads, int8 KV (per-(block, KV head) scales), fp16 q/out, "
+                 "batch 16, all lengths 4096",
     "specdec": "speculative verification: 7B-GQA 32 q / 8 KV heads, head_dim 128, fp16, batch 64, "
                "lengths U[512,4096], 2 new tokens per sequence per step (causal), 16 steps",
 }
@@ -141,6 +143,8 @@ def make_workload(name):
         return W.mqa(), False, -1
     if name == "d256":
         return W.d256(), False, -1
+    if name == "d256_int8":
+        return W.d256(), "i8", -1
     if name == "specdec":
         return W.specdec(), False, -1
     raise ValueError(name)

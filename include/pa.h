@@ -132,8 +132,8 @@ typedef struct pa_decode_params {
                                 other than 1, 2, 4, 8 or multiples of 8 are padded, on the
                                 tensor-core family only; the CUDA-core family takes
                                 single-token decode with G in 1, 2, 4, 8, 16, 32, 64. */
-    int head_dim;            /* 64, 128 or 256 (256 not with PA_F32; PA_I4 and the
-                                tensor-core int8 path take 128 only) */
+    int head_dim;            /* 64, 128 or 256 (256 not with PA_F32; PA_I4 takes 128
+                                only, and the tensor-core int8 path 128 or 256) */
     int block_size;          /* must be PA_BLOCK_SIZE */
     int max_blocks_per_seq;  /* row stride of block_tables */
     int64_t num_blocks;      /* physical blocks in the pool */

@@ -470,8 +470,8 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     constexpr bool kI8 = std::is_same<TKV, int8_t>::value;
     constexpr bool kI4 = C::I4;
     constexpr bool kQz = kI8 || kI4;  // quantised cache: per-(block, KV head) scales
-    static_assert(!kQz || (std::is_same<T, __half>::value && D == 128),
-                  "int8 and 4-bit caches: fp16 q, head_dim 128");
+    static_assert(!kQz || (std::is_same<T, __half>::value && (D == 128 || (kI8 && D == 256))),
+                  "int8 caches: fp16 q, head_dim 128 or 256; 4-bit caches: fp16 q, head_dim 128");
     // APP (pa_decode_append): single-token rows of an fp16 / bf16 cache
     static_assert(!APP || (!MQ && !kQz), "the fused append takes single-token fp16 / bf16 rows");
     constexpr bool app = APP;
@@ -849,7 +849,8 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
     // O^T row (m-tile i, row g; row g + 8 is dim + 8) -> head dim: m-tile i holds
     // dims 16i .. 16i + 15 for fp16/bf16 tiles; the int8 path gives thread row g
     // the 16 dims 16g .. 16g + 15 instead (see vfrag_i8)
-    auto dmap = [&](int i, int gg) -> int { return kQz ? 16 * gg + i : 16 * i + gg; };
+    // (head_dim 256: m-tiles 8 .. 15 are the second 128-dim box, in the same order)
+    auto dmap = [&](int i, int gg) -> int { return kQz ? (i >> 3) * 128 + 16 * gg + (i & 7) : 16 * i + gg; };
     const int h0 = 2 * c, h1 = 2 * c + 1;  // heads of this thread's S^T / O^T columns
     // B fragments of q (n = heads, k = dims) from the q slot of stage s.  The
     // int8 path orders the contraction's dims differently (see kfrag_i8): k-step
@@ -873,8 +874,9 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
 #pragma unroll
         for (int ks = 0; ks < C::KSTEPS; ++ks) {
             if (g < ncol) {
-                bq[ks][0] = lds_u32(qs + (kI8 ? ks * 8 : ks * 32));
-                bq[ks][1] = lds_u32(qs + (kI8 ? ks * 8 + 4 : ks * 32 + 16));
+                // (int8 at head_dim 256: k-steps 8 .. 15 are dims 128 .. 255, in the same order)
+                bq[ks][0] = lds_u32(qs + (kI8 ? (ks >> 3) * 256 + (ks & 7) * 8 : ks * 32));
+                bq[ks][1] = lds_u32(qs + (kI8 ? (ks >> 3) * 256 + (ks & 7) * 8 + 4 : ks * 32 + 16));
             } else {
                 bq[ks][0] = bq[ks][1] = 0u;
             }
@@ -914,7 +916,7 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
         for (int i = 0; i < C::MTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
         for (int j = 0; alive && j < len; ++j) {
-            if constexpr (kQz && PA_TC_PAIRS) {
+            if constexpr (kQz && PA_TC_PAIRS && D == 128) {
                 if (j + 1 < len) {
                     // ---- two blocks (stages sA, sB) at once: one max/sum reduction and
                     // one rescale for both, two independent MMA streams
@@ -1131,6 +1133,8 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
                     // keeps the unscaled ones)
                     slog *= my_sc[2 * s];
                     vsc = my_sc[2 * s + 1];
+                    // (head_dim 256: the second box's words are read when its k-steps and
+                    // m-tiles come up)
                     kload_i8(kw, tK, g, c);
                     vload_i8(vw, tK + C::TILE, g, c);
                 } else if constexpr (kHoistK) {
@@ -1163,7 +1167,8 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
                         kfrag_i4(kw4, ks, kf[0]);
                         qk(ks, kf[0]);
                     } else if constexpr (kI8) {
-                        kfrag_i8(kw, ks, kf[0]);
+                        if (C::BOXES > 1 && ks == 8) kload_i8(kw, tK + C::BOX_BYTES, g, c);
+                        kfrag_i8(kw, ks & 7, kf[0]);
                         qk(ks, kf[0]);
                     } else if constexpr (kHoistK) {
                         qk(ks, kf[ks]);
@@ -1240,10 +1245,12 @@ __global__ void __launch_bounds__(TcCfg<TKV, D, G>::THREADS, TcCfg<TKV, D, G>::M
                 for (int i = 0; i < C::MTILES; ++i) {
                     const int vi = kHoist ? i : 0;
                     if constexpr (kQz) {
-                        if constexpr (kI4)
+                        if constexpr (kI4) {
                             vfrag_i4(vw4, i, vf[0]);
-                        else
-                            vfrag_i8(vw, i, vf[0]);
+                        } else {
+                            if (C::BOXES > 1 && i == 8) vload_i8(vw, tK + C::TILE + C::BOX_BYTES, g, c);
+                            vfrag_i8(vw, i & 7, vf[0]);
+                        }
                         // no mask: an int8 or 4-bit slot past the sequence end holds a finite
                         // value, and its probability is exactly 0
                     } else if constexpr (!kHoist) {
@@ -2120,7 +2127,8 @@ static bool launch_shape(const void *kernel, int threads, int smem, int *sms, in
 bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B) {
     const bool same = (q_dtype == PA_F16 || q_dtype == PA_BF16) && kv_dtype == q_dtype &&
                       (D == 64 || D == 128 || D == 256);
-    const bool quant = q_dtype == PA_F16 && (kv_dtype == PA_I8 || kv_dtype == PA_I4) && D == 128;
+    const bool quant = q_dtype == PA_F16 &&
+                       ((kv_dtype == PA_I8 && (D == 128 || D == 256)) || (kv_dtype == PA_I4 && D == 128));
     return (same || quant) && (G == 1 || G == 2 || G == 4 || G == 8) && B <= kTcMaxB;
 }
 
@@ -2230,6 +2238,7 @@ static int launch_tc_g(const DecodeArgs &a, cudaStream_t st) {
 
 int launch_decode_tc(const DecodeArgs &a, cudaStream_t st) {
     if (a.q_dtype == PA_F16 && a.kv_dtype == PA_I8) {
+        if (a.D == 256) return launch_tc_g<__half, int8_t, 256>(a, st);
         if (a.D != 128) return PA_ERR_UNSUPPORTED;
         return launch_tc_g<__half, int8_t, 128>(a, st);
     }

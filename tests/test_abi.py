@@ -175,10 +175,12 @@ def test_large_groups_and_head_dim_256_are_planned():
         assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
     p = params(head_dim=256, partition_size=16, algo=pa.PA_ALGO_SIMT)
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
-    # the tensor-core family takes fp16/bf16 head_dim 256 too (not int8 or 4-bit caches)
+    # the tensor-core family takes fp16/bf16 and int8 head_dim 256 too (not 4-bit caches)
     p = params(head_dim=256, partition_size=16, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
-    p = params(head_dim=256, kv_dtype=pa.PA_I8, algo=pa.PA_ALGO_TENSOR)
+    p = params(head_dim=256, kv_dtype=pa.PA_I8, partition_size=16, algo=pa.PA_ALGO_TENSOR)
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+    p = params(head_dim=256, kv_dtype=pa.PA_I4, algo=pa.PA_ALGO_TENSOR)
     assert pa.lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(0.1), ctypes.byref(p),
                             None) == pa.PA_ERR_UNSUPPORTED
 
@@ -211,7 +213,8 @@ def test_decode_algo_reports_the_family():
     assert algo(params(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32)) == pa.PA_ALGO_SIMT
     assert algo(params(head_dim=256)) == pa.PA_ALGO_TENSOR
     assert algo(params(head_dim=256, q_dtype=pa.PA_BF16, kv_dtype=pa.PA_BF16)) == pa.PA_ALGO_TENSOR
-    assert algo(params(head_dim=256, kv_dtype=pa.PA_I8)) == pa.PA_ALGO_SIMT
+    assert algo(params(head_dim=256, kv_dtype=pa.PA_I8)) == pa.PA_ALGO_TENSOR
+    assert algo(params(head_dim=256, kv_dtype=pa.PA_I8, q_dtype=pa.PA_BF16)) == pa.PA_ALGO_SIMT
     assert algo(params(kv_dtype=pa.PA_I8, q_dtype=pa.PA_BF16)) == pa.PA_ALGO_SIMT
     assert algo(params(kv_dtype=pa.PA_I8)) == pa.PA_ALGO_TENSOR
     # a q that is not 16-byte aligned goes to the CUDA-core family, or is refused

@@ -492,15 +492,36 @@ def test_head_dim_256_multi_query(Q):
     assert_close(got[0], ref[0], "float16", f"d=256 Q={Q}")
 
 
-def test_head_dim_256_int8():
-    w = W.random_case([3, 100, 700], num_q_heads=16, num_kv_heads=4, head_dim=256, dtype="float16",
-                      seed=256)
-    got, dw = run_gpu(w, -1, int8=True, dw=runner.DeviceWorkload(w))
+@pytest.mark.parametrize("algo", [pa.PA_ALGO_SIMT, pa.PA_ALGO_TENSOR])
+@pytest.mark.parametrize("hq,hkv", [(16, 4), (8, 8), (32, 4), (64, 1)])
+@pytest.mark.parametrize("part", [0, 16, -1])
+def test_head_dim_256_int8(hq, hkv, part, algo):
+    """int8 caches at head_dim 256 on both families (the tensor-core family reads
+    each 256-byte row as two 128-byte boxes), against the oracle dequantising the
+    same int8 values; one-pass, one-block and library-picked partitions."""
+    if algo == pa.PA_ALGO_SIMT and hq // hkv > 8:
+        pytest.skip("int8 on the CUDA-core family: G in 1, 2, 4, 8")
+    w = W.random_case([3, 16, 100, 700], num_q_heads=hq, num_kv_heads=hkv, head_dim=256, dtype="float16",
+                      seed=256 + hq + hkv)
+    got, dw = run_gpu(w, part, algo, int8=True, dw=runner.DeviceWorkload(w))
     kc8, vc8 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
     ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
     op = w.steps[0][0]
     ref = oracle.decode(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
-    assert_close(got[0], ref, "float16", "d=256 int8")
+    assert_close(got[0], ref, "float16", f"d=256 int8 G={hq // hkv} part={part} algo={algo}")
+
+
+@pytest.mark.parametrize("Q", [2, 3])
+def test_head_dim_256_int8_multi_query(Q):
+    """Several new tokens per sequence over an int8 cache at head_dim 256."""
+    w = W.random_multi_case([Q, 40, 300], Q, num_q_heads=16, num_kv_heads=4, head_dim=256,
+                            dtype="float16", seed=512 + Q)
+    got, dw = run_gpu(w, -1, pa.PA_ALGO_TENSOR, int8=True, dw=runner.DeviceWorkload(w))
+    kc8, vc8 = dw.kc8.cpu().numpy(), dw.vc8.cpu().numpy()
+    ks, vs = dw.k_scales.cpu().numpy(), dw.v_scales.cpu().numpy()
+    op = w.steps[0][0]
+    ref = oracle.decode_multi(op.q, kc8, vc8, op.block_tables, op.seq_lens, w.scale, ks, vs)
+    assert_close(got[0], ref, "float16", f"d=256 int8 Q={Q}")
 
 
 @pytest.mark.slow
