@@ -104,7 +104,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ragged")
     ap.add_argument("--partition", type=int, default=-1)
-    ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--algo", choices=["auto", "simt", "tensor", "tcgen05"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -397,7 +397,8 @@ def main(argv=None):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    algo = {"auto": pa.PA_ALGO_AUTO, "simt": pa.PA_ALGO_SIMT, "tensor": pa.PA_ALGO_TENSOR}[args.algo]
+    algo = {"auto": pa.PA_ALGO_AUTO, "simt": pa.PA_ALGO_SIMT, "tensor": pa.PA_ALGO_TENSOR,
+            "tcgen05": pa.PA_ALGO_TCGEN05}[args.algo]
     w, int8, default_part = make_workload(args.workload)
     part = args.partition
     dw = runner.DeviceWorkload(w, fill_nan=False)

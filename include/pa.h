@@ -64,7 +64,12 @@ enum pa_status {
 enum pa_dtype { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_I8 = 3, PA_I4 = 4 };
 
 /* Kernel family for pa_decode.  AUTO picks the fastest built one. */
-enum pa_algo { PA_ALGO_AUTO = 0, PA_ALGO_SIMT = 1, PA_ALGO_TENSOR = 2 };
+/* PA_ALGO_TCGEN05: the tcgen05 kernel (5th-generation tensor cores, accumulators in
+ * tensor memory) for groups of 32 or 64 fp16/bf16 query heads per KV head at head_dim
+ * 128, split-K (partition_size != 0), num_seqs <= 2048; PA_ERR_UNSUPPORTED elsewhere.
+ * Only on request: for these groups PA_ALGO_AUTO and PA_ALGO_TENSOR run the faster
+ * mma.sync kernel that shares each staged tile across a CTA's warps. */
+enum pa_algo { PA_ALGO_AUTO = 0, PA_ALGO_SIMT = 1, PA_ALGO_TENSOR = 2, PA_ALGO_TCGEN05 = 3 };
 
 /* Bits of the per-device error word (pa_get_error_flags). */
 enum pa_error_flag {
@@ -206,7 +211,7 @@ size_t pa_decode_workspace_size(const pa_decode_params *p);
 
 /*
  * The kernel family pa_decode runs for these parameters and this q:
- * PA_ALGO_TENSOR or PA_ALGO_SIMT, or a negative pa_status for parameters
+ * PA_ALGO_TENSOR, PA_ALGO_SIMT or PA_ALGO_TCGEN05, or a negative pa_status for parameters
  * pa_decode would reject.  q (a device pointer, not read) matters only through
  * its alignment: the tensor-core family reads q rows with 16-byte copies, so an
  * unaligned q goes to the CUDA-core family.  Together with

@@ -99,7 +99,11 @@ static int check_decode_params(const pa_decode_params *p, int *part, int *max_pa
     if (!simt_ok && !tc_ok) return PA_ERR_UNSUPPORTED;
     if (p->algo == PA_ALGO_SIMT && !simt_ok) return PA_ERR_UNSUPPORTED;
     if (p->num_seqs > 65535 || kh.Hkv > 65535) return PA_ERR_UNSUPPORTED;
-    if (p->algo < PA_ALGO_AUTO || p->algo > PA_ALGO_TENSOR) return PA_ERR_UNSUPPORTED;
+    if (p->algo < PA_ALGO_AUTO || p->algo > PA_ALGO_TCGEN05) return PA_ERR_UNSUPPORTED;
+    if (p->algo == PA_ALGO_TCGEN05 &&
+        !decode_umma_eligible(p->q_dtype, p->kv_dtype, p->head_dim, kh.G, kh.ngroups, kh.qlen, kh.padded,
+                              p->partition_size, p->num_seqs))
+        return PA_ERR_UNSUPPORTED;
     if (p->flags & ~(PA_DECODE_INPUTS_READY | PA_DECODE_OUT_F32)) return PA_ERR_UNSUPPORTED;
     int ps = p->partition_size;
     if (ps < -1 || (ps > 0 && ps % PA_BLOCK_SIZE)) return PA_ERR_SHAPE;
@@ -143,12 +147,12 @@ static int make_plan(const pa_decode_params *p, Plan *pl) {
     const bool tc_ok = decode_tc_supported(p->q_dtype, p->kv_dtype, p->head_dim, G, p->num_seqs) &&
                        p->num_blocks * p->num_kv_heads * PA_BLOCK_SIZE <= 2147483647LL &&
                        stream_blocks <= (1LL << 30);
-    if (p->algo == PA_ALGO_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
+    if ((p->algo == PA_ALGO_TENSOR || p->algo == PA_ALGO_TCGEN05) && !tc_ok) return PA_ERR_UNSUPPORTED;
     // several new tokens per sequence, or padded columns: the tensor-core family only
     if ((kh.qlen > 1 || kh.padded) && !tc_ok) return PA_ERR_UNSUPPORTED;
     *pl = Plan{};
     pl->max_len = max_len;
-    pl->tc = p->algo == PA_ALGO_TENSOR || (p->algo == PA_ALGO_AUTO && tc_ok);
+    pl->tc = p->algo == PA_ALGO_TENSOR || p->algo == PA_ALGO_TCGEN05 || (p->algo == PA_ALGO_AUTO && tc_ok);
     if (!pl->tc) {
         pl->part = part;
         pl->max_parts = mp;
@@ -382,6 +386,7 @@ static int decode_impl(void *out, const void *q, const void *key_cache, const vo
     a.out_f32 = (p->flags & PA_DECODE_OUT_F32) ? 1 : 0;
     a.stall_at = stall_at;
     a.wait_ns = wait_ns;
+    a.umma = p->algo == PA_ALGO_TCGEN05 ? 1 : 0;
     if (ap) {
         a.append = 1;
         a.k_new = ap->k;
@@ -392,7 +397,7 @@ static int decode_impl(void *out, const void *q, const void *key_cache, const vo
     }
     char *ws = reinterpret_cast<char *>(p->workspace);
     if (pl.tc && (uintptr_t)q % 16) {
-        if (p->algo == PA_ALGO_TENSOR || stall_at >= 0) return PA_ERR_ALIGN;
+        if (p->algo == PA_ALGO_TENSOR || p->algo == PA_ALGO_TCGEN05 || stall_at >= 0) return PA_ERR_ALIGN;
         // the tensor-core family reads q rows with 16-byte bulk copies; a q that is not
         // 16-byte aligned goes to the CUDA-core family, which needs its own plan
         pa_decode_params p2 = *p;
@@ -495,15 +500,16 @@ int pa_decode_algo(const pa_decode_params *p, const void *q) {
     Plan pl;
     const int rc = make_plan(p, &pl);
     if (rc != PA_OK) return rc;
-    if (pl.tc && (uintptr_t)q % 16) return p->algo == PA_ALGO_TENSOR ? PA_ERR_ALIGN : PA_ALGO_SIMT;
-    return pl.tc ? PA_ALGO_TENSOR : PA_ALGO_SIMT;
+    if (pl.tc && (uintptr_t)q % 16)
+        return p->algo == PA_ALGO_TENSOR || p->algo == PA_ALGO_TCGEN05 ? PA_ERR_ALIGN : PA_ALGO_SIMT;
+    return p->algo == PA_ALGO_TCGEN05 ? PA_ALGO_TCGEN05 : pl.tc ? PA_ALGO_TENSOR : PA_ALGO_SIMT;
 }
 
 int pa_get_error_flags(unsigned int *flags, int reset, pa_stream_t stream) {
     if (!flags) return PA_ERR_NULL;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
     int (*const words[])(unsigned int *, bool) = {error_word_cache_ops, error_word_decode_simt,
-                                                  error_word_decode_tc};
+                                                  error_word_decode_tc, error_word_decode_umma};
     unsigned int all = 0;
     for (auto w : words) {
         unsigned int f = 0;

@@ -55,6 +55,7 @@
 
 #include "pa_common.cuh"
 #include "pa_internal.h"
+#include "pa_tc_shared.cuh"
 
 namespace pa {
 
@@ -88,18 +89,6 @@ __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
     asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
     return y;
 }
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
 template <typename T> struct Mma;
 template <> struct Mma<__half> {
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
@@ -172,6 +161,7 @@ template <> struct Mma<__nv_bfloat16> {
 #define PA_TC_MIN_CTAS 1
 #endif
 
+
 // TKV: the cache element: the q/out type T, int8_t, or U4x2 (two 4-bit values
 // per byte).  fp16/bf16 and int8 tile rows come as 128-byte boxes (64 or 128
 // elements) with 128-byte swizzle; a 4-bit tile row is D / 2 bytes, one box, no
@@ -221,73 +211,6 @@ struct TcCfg {
     static constexpr int CUM_OFF = PSLOT_OFF + NW * S * 4;
     static int smem_bytes(int B) { return 1024 + CUM_OFF + (3 * B + 3) * 4; }
 };
-
-// One contiguous run of blocks of one (sequence, KV head) row.
-struct Seg {
-    int b, kvh, L, nb;  // row: sequence, KV head, tokens, blocks
-    int j0, j1;         // this segment: blocks [j0, j1) of the row
-    int fr;             // index of the row's first block in the concatenated stream
-    int ch;             // chunk that holds the segment (-1: whole-row mode)
-    int ncol;           // the row's real (not padding) columns
-};
-
-// Walks the ranges of one warp and cuts them into segments at row boundaries.
-struct SegIter {
-    int k;              // range counter
-    int f, fend;        // position and end in the concatenated stream
-    int ch;
-    bool done;
-};
-
-// Consecutive table entries of one segment, read 32 at a time (lane l holds
-// entry o + l as a TMA row coordinate, -2 for a block id outside the pool).
-struct Win {
-    Seg sg;
-    int o, n;
-    int kc;  // the cache's KV head of the window's row
-    bool valid;
-};
-
-// Chunks of the concatenated block stream: n chunks of c blocks (the last one
-// shorter); warp w takes chunks w, w + W, w + 2W, ...
-#ifndef PA_TC_GAMMA
-#define PA_TC_GAMMA 2
-#endif
-// Chunks are cut in a virtual stream in which every non-empty row is followed by
-// gam extra units (the cost of finishing one segment and starting the next, in
-// blocks), so a chunk that holds several row ends holds fewer blocks.  cum[b] /
-// cumv[b]: blocks / virtual units of the rows of sequences before b.
-struct Chunks {
-    int total, vtotal, c, n, gam, Hkv;
-    const int *cum, *cumv;
-    // virtual position of block j of row (b, kvh) of nb blocks
-    __device__ int vpos(int b, int kvh, int nb, int j) const { return cumv[b] + kvh * (nb + gam) + j; }
-    // actual stream position of the first block at or after virtual position v
-    __device__ int at(int v) const {
-        if (v >= vtotal) return total;
-        int l = 0, h = nseq;  // largest b with cumv[b] <= v: sequence b is not empty
-        while (h - l > 1) {
-            const int mid = (l + h) >> 1;
-            if (cumv[mid] <= v) l = mid; else h = mid;
-        }
-        const int nb = cum[l + 1] - cum[l];
-        const int off = v - cumv[l], rl = nb + gam;
-        const int kvh = off / rl, j = off - kvh * rl;
-        return cum[l] * Hkv + kvh * nb + (j < nb ? j : nb);
-    }
-    int nseq;
-    __device__ int start(int ch) const { return at(ch * c); }
-    __device__ int end(int ch) const { return at((ch + 1) * c); }
-    // chunk of block j of row (b, kvh)
-    __device__ int of(int b, int kvh, int nb, int j) const { return vpos(b, kvh, nb, j) / c; }
-    // whether the row (b, kvh) begins after its first chunk's first block, i.e. the
-    // block before it (the previous row's last) lies in the same chunk
-    __device__ bool mid_start(int b, int kvh, int nb) const {
-        const int fr = cum[b] * Hkv + kvh * nb;
-        return fr > 0 && (vpos(b, kvh, nb, 0) - gam - 1) / c == vpos(b, kvh, nb, 0) / c;
-    }
-};
-
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -2049,7 +1972,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D map over a cache viewed as [rows = N*H_kv*16][D] with boxes of 16 rows
 // of 128 bytes (64 fp16/bf16 or 128 int8 elements) and 128-byte swizzle.  Encoded maps are cached by (address,
 // rows, D, dtype): the encode is a host call of a few microseconds.
-static bool cache_tensor_map(CUtensorMap *m, const void *base, int64_t rows, int D, int dtype) {
+bool tc_cache_tensor_map(CUtensorMap *m, const void *base, int64_t rows, int D, int dtype) {
     struct Key {
         const void *p;
         int64_t rows;
@@ -2097,7 +2020,7 @@ static bool cache_tensor_map(CUtensorMap *m, const void *base, int64_t rows, int
 
 // SM count and resident CTAs per SM for (kernel, device, dynamic shared memory),
 // queried once: the occupancy query costs microseconds of host time per call.
-static bool launch_shape(const void *kernel, int threads, int smem, int *sms, int *per_sm) {
+bool tc_launch_shape(const void *kernel, int threads, int smem, int *sms, int *per_sm) {
     static std::mutex mu;
     static std::map<std::tuple<const void *, int, int>, std::pair<int, int>> cache;
     int dev = 0;
@@ -2145,10 +2068,10 @@ static int launch_tc(const DecodeArgs &a, cudaStream_t st) {
     if ((uintptr_t)a.q % 16) return PA_ERR_ALIGN;  // q rows are read as aligned 32-bit pairs
     CUtensorMap tk, tv;
     const int64_t rows = a.N * (a.Hkv / a.ngroups) * kBlockSize;  // the cache's rows
-    if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
+    if (!tc_cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !tc_cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
         return PA_ERR_CUDA;
     int sms = 0, per_sm = 0;
-    if (!launch_shape(reinterpret_cast<const void *>(kern), C::THREADS, smem, &sms, &per_sm)) return PA_ERR_CUDA;
+    if (!tc_launch_shape(reinterpret_cast<const void *>(kern), C::THREADS, smem, &sms, &per_sm)) return PA_ERR_CUDA;
     // persistent grid: every resident warp is a worker, but no more warps than
     // there are blocks to read (every sequence at max_len)
     const int64_t blocks = (int64_t)a.B * a.Hkv * ((a.max_len + kBlockSize - 1) / kBlockSize);
@@ -2183,10 +2106,10 @@ static int launch_coop(const DecodeArgs &a, cudaStream_t st) {
     if (!set_smem_attr_once(reinterpret_cast<const void *>(kern), C::smem_bytes(kTcMaxB))) return PA_ERR_CUDA;
     CUtensorMap tk, tv;
     const int64_t rows = a.N * a2.Hkv * kBlockSize;
-    if (!cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
+    if (!tc_cache_tensor_map(&tk, a.kc, rows, D, a.kv_dtype) || !tc_cache_tensor_map(&tv, a.vc, rows, D, a.kv_dtype))
         return PA_ERR_CUDA;
     int sms = 0, per_sm = 0;
-    if (!launch_shape(reinterpret_cast<const void *>(kern), C::THREADS, smem, &sms, &per_sm)) return PA_ERR_CUDA;
+    if (!tc_launch_shape(reinterpret_cast<const void *>(kern), C::THREADS, smem, &sms, &per_sm)) return PA_ERR_CUDA;
     const int64_t blocks = (int64_t)a.B * a2.Hkv * ((a.max_len + kBlockSize - 1) / kBlockSize);
     int64_t ctas = (int64_t)sms * per_sm;
     const int64_t need = (blocks + kTcMinChunk - 1) / kTcMinChunk;
@@ -2195,13 +2118,38 @@ static int launch_coop(const DecodeArgs &a, cudaStream_t st) {
     a2.tc_W = (int)ctas;
     if (launch_pdl(kern, dim3((unsigned)ctas), dim3(C::THREADS), smem, st, tk, tv, a2) != cudaSuccess)
         return PA_ERR_CUDA;
-    auto mk = merge_tc_kernel<T, D, NG * 16, false>;
-    const int msmem = 2 * (a.B + 1) * 4;
+    return launch_merge_rows(a2, sms, st);
+}
+
+template <typename T, int D, int GC>
+static int launch_merge_rows_t(const DecodeArgs &a2, int sms, cudaStream_t st) {
+    auto mk = merge_tc_kernel<T, D, GC, false>;
+    const int msmem = 2 * (a2.B + 1) * 4;
     if (!set_smem_attr_once(reinterpret_cast<const void *>(mk), 2 * (kTcMaxB + 1) * 4)) return PA_ERR_CUDA;
-    const int64_t items = (int64_t)a.B * a2.Hkv * NG * 16;
+    const int64_t items = (int64_t)a2.B * a2.Hkv * GC;
     int64_t mctas = (items + 7) / 8;
     if (mctas > 2 * sms) mctas = 2 * sms;
     return launch_pdl(mk, dim3((unsigned)mctas), dim3(256), msmem, st, a2) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D>
+static int launch_merge_rows_d(const DecodeArgs &a2, int sms, cudaStream_t st) {
+    switch (a2.G) {
+    case 16: return launch_merge_rows_t<T, D, 16>(a2, sms, st);
+    case 32: return launch_merge_rows_t<T, D, 32>(a2, sms, st);
+    case 64: return launch_merge_rows_t<T, D, 64>(a2, sms, st);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+int launch_merge_rows(const DecodeArgs &a2, int sms, cudaStream_t st) {
+    if (a2.D != 64 && a2.D != 128) return PA_ERR_UNSUPPORTED;
+    if (a2.q_dtype == PA_F16)
+        return a2.D == 64 ? launch_merge_rows_d<__half, 64>(a2, sms, st) : launch_merge_rows_d<__half, 128>(a2, sms, st);
+    if (a2.q_dtype == PA_BF16)
+        return a2.D == 64 ? launch_merge_rows_d<__nv_bfloat16, 64>(a2, sms, st)
+                          : launch_merge_rows_d<__nv_bfloat16, 128>(a2, sms, st);
+    return PA_ERR_DTYPE;
 }
 
 bool decode_coop_eligible(int q_dtype, int kv_dtype, int D, int G, int ngroups, int qlen, bool padded, int part) {
@@ -2225,6 +2173,7 @@ static int launch_tc_g(const DecodeArgs &a, cudaStream_t st) {
     // several new tokens, or padding columns: the general column mapping
     const bool mq = a.qlen > 1 || (int64_t)a.G * a.ngroups != a.gcols;
     if constexpr (std::is_same<T, TKV>::value && D <= 128) {
+        if (a.umma && a.tc_chunk >= 0) return launch_decode_umma(a, st);
         if (decode_coop_eligible(a.q_dtype, a.kv_dtype, D, a.G, a.ngroups, a.qlen, mq, a.tc_chunk < 0 ? 0 : 1)) {
             switch (a.ngroups) {
             case 2: return launch_coop<T, D, 1>(a, st);

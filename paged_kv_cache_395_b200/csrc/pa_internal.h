@@ -66,6 +66,7 @@ struct DecodeArgs {
     int stall_at;            // -1; else the first worker of the tensor-core family leaves
                              // its stall_at-th copy unissued (pa_decode_stall_selftest)
     unsigned long long wait_ns;  // limit of every bounded wait on a copy
+    int umma;                // PA_ALGO_TCGEN05: the tcgen05 kernel (pa_decode_umma.cu)
     // pa_decode_append on the tensor-core family: row b of k_new / v_new ([B][H_kv][D],
     // token strides in elements) is sequence b's new token, written to cache slot
     // slot_new[b] (< 0: none) by the kernel, which also uses it in place of what its
@@ -93,6 +94,7 @@ constexpr int kTcMaxB = 4096;
 int error_word_cache_ops(unsigned int *flags, bool reset);
 int error_word_decode_simt(unsigned int *flags, bool reset);
 int error_word_decode_tc(unsigned int *flags, bool reset);
+int error_word_decode_umma(unsigned int *flags, bool reset);
 
 // Raise a kernel's dynamic shared-memory limit on the current device, once per
 // (kernel, device).  Thread-safe; returns false if CUDA refuses.
@@ -104,6 +106,10 @@ int launch_decode_tc(const DecodeArgs &a, cudaStream_t st);
 bool decode_tc_supported(int q_dtype, int kv_dtype, int D, int G, int B);
 // groups of 16, 32 or 64 query heads per KV head run one CTA per cache row
 bool decode_coop_eligible(int q_dtype, int kv_dtype, int D, int G, int ngroups, int qlen, bool padded, int part);
+// groups of 32 or 64 fp16/bf16 query heads per KV head at head_dim 128 on tcgen05
+bool decode_umma_eligible(int q_dtype, int kv_dtype, int D, int G, int ngroups, int qlen, bool padded, int part,
+                          int B);
+int launch_decode_umma(const DecodeArgs &a, cudaStream_t st);
 int launch_decode_simt(const DecodeArgs &a, cudaStream_t st);
 int launch_merge(const DecodeArgs &a, cudaStream_t st);
 bool decode_simt_supported(int q_dtype, int kv_dtype, int D, int G);

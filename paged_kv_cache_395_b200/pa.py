@@ -27,7 +27,7 @@ LIB_PATH = os.path.join(_HERE, "libpa.so")
 PA_OK, PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_DTYPE = 0, -1, -2, -3
 PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_ALIGN = -4, -5, -6, -7
 PA_F32, PA_F16, PA_BF16, PA_I8, PA_I4 = 0, 1, 2, 3, 4
-PA_ALGO_AUTO, PA_ALGO_SIMT, PA_ALGO_TENSOR = 0, 1, 2
+PA_ALGO_AUTO, PA_ALGO_SIMT, PA_ALGO_TENSOR, PA_ALGO_TCGEN05 = 0, 1, 2, 3
 PA_EFLAG_BAD_BLOCK, PA_EFLAG_BAD_SLOT, PA_EFLAG_BAD_PAIR, PA_EFLAG_WAIT_TIMEOUT = 1, 2, 4, 8
 PA_EFLAG_APPEND_SLOT = 16
 PA_DECODE_INPUTS_READY, PA_DECODE_OUT_F32 = 1, 2
@@ -186,7 +186,7 @@ def make_params(q, key_cache, block_tables, max_seq_len, k_scales=None, v_scales
 def pa_decode_algo(q, key_cache, block_tables, max_seq_len, partition_size=0, k_scales=None,
                    v_scales=None, algo=PA_ALGO_AUTO) -> int:
     """The kernel family pa_decode runs for these operands, as the library
-    reports it: PA_ALGO_TENSOR or PA_ALGO_SIMT."""
+    reports it: PA_ALGO_TENSOR, PA_ALGO_SIMT or PA_ALGO_TCGEN05."""
     p = make_params(q, key_cache, block_tables, max_seq_len, k_scales, v_scales, partition_size,
                     None, algo)
     r = int(lib.pa_decode_algo(ctypes.byref(p), _ptr(q)))
@@ -308,14 +308,15 @@ def pa_decode_fixed_scratch(out, q, key_cache, value_cache, block_tables, seq_le
 
 
 def pa_decode_stall_selftest(out, q, key_cache, value_cache, block_tables, seq_lens, scale, max_seq_len,
-                             stall_at, limit_ns, partition_size=-1, workspace=None, stream=None):
-    """pa_decode on the tensor-core family with the failure path exercised: the
-    first worker leaves its stall_at-th copy unissued, so its bounded wait runs
-    out after limit_ns (see include/pa.h).  Returns after the launch; the error
-    word then holds PA_EFLAG_WAIT_TIMEOUT."""
+                             stall_at, limit_ns, partition_size=-1, workspace=None, stream=None,
+                             algo=PA_ALGO_TENSOR):
+    """pa_decode on the tensor-core family (algo PA_ALGO_TENSOR or PA_ALGO_TCGEN05)
+    with the failure path exercised: the first worker leaves its stall_at-th copy
+    unissued, so its bounded wait runs out after limit_ns (see include/pa.h).
+    Returns after the launch; the error word then holds PA_EFLAG_WAIT_TIMEOUT."""
     _dev(out, q, key_cache, value_cache, block_tables, seq_lens, workspace)
     p = make_params(q, key_cache, block_tables, max_seq_len, None, None, partition_size, workspace,
-                    PA_ALGO_TENSOR, _out_flag(out, q))
+                    algo, _out_flag(out, q))
     _check(lib.pa_decode_stall_selftest(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache),
                                         _ptr(block_tables), _ptr(seq_lens), ctypes.c_float(scale),
                                         ctypes.byref(p), int(stall_at), int(limit_ns), _stream(stream)),

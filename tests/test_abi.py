@@ -293,3 +293,22 @@ def test_decode_append_rejects_before_any_launch():
     # split-K without a workspace
     assert pa.lib.pa_decode_append(*args(FAKE, partition_size=16)) == pa.PA_ERR_WORKSPACE
     del p
+
+
+def test_tcgen05_is_planned_only_for_its_groups():
+    """PA_ALGO_TCGEN05 takes groups of 32 or 64 fp16/bf16 query heads per KV head at
+    head_dim 128 in split-K mode (the cooperative workspace layout), and nothing else."""
+    algo = lambda p: pa.lib.pa_decode_algo(ctypes.byref(p), ctypes.c_void_p(0x1000))  # noqa: E731
+    ok = dict(num_q_heads=32, num_kv_heads=1, partition_size=-1, algo=pa.PA_ALGO_TCGEN05)
+    assert algo(params(**ok)) == pa.PA_ALGO_TCGEN05
+    assert algo(params(**dict(ok, num_q_heads=64))) == pa.PA_ALGO_TCGEN05
+    assert algo(params(**dict(ok, num_q_heads=64, num_kv_heads=2, q_dtype=pa.PA_BF16,
+                              kv_dtype=pa.PA_BF16))) == pa.PA_ALGO_TCGEN05
+    a = params(**ok)
+    b = params(**dict(ok, algo=pa.PA_ALGO_TENSOR))
+    assert pa.lib.pa_decode_workspace_size(ctypes.byref(a)) == pa.lib.pa_decode_workspace_size(ctypes.byref(b)) > 0
+    for kw in (dict(num_q_heads=16), dict(num_q_heads=8), dict(head_dim=64), dict(partition_size=0),
+               dict(q_dtype=pa.PA_F32, kv_dtype=pa.PA_F32), dict(kv_dtype=pa.PA_I8), dict(query_len=2),
+               dict(num_seqs=4096, max_blocks_per_seq=1)):
+        assert algo(params(**dict(ok, **kw))) == pa.PA_ERR_UNSUPPORTED, kw
+    assert algo(params(algo=4)) == pa.PA_ERR_UNSUPPORTED

@@ -741,3 +741,78 @@ def test_wait_timeout_reported_and_workspace_left_ready(stall_at):
     pa.pa_decode(out2, q, dw.kc, dw.vc, bt, sl, w.scale, mx, partition_size=-1, workspace=ws,
                  algo=pa.PA_ALGO_TENSOR)
     assert_close(out2, ref, "float16", "next call")
+
+
+# -- the tcgen05 kernel (PA_ALGO_TCGEN05, groups of 32 or 64 heads per KV head) ----------
+@pytest.mark.parametrize("qdt", ["float16", "bfloat16"])
+@pytest.mark.parametrize("hq,hkv", [(32, 1), (64, 1), (64, 2), (128, 4)])
+@pytest.mark.parametrize("part", [16, 48, -1])
+def test_tcgen05_large_groups(hq, hkv, part, qdt):
+    """The tcgen05 kernel against the oracle: lengths of 1 token, a block, a block plus
+    one, ragged tails; one-block, three-block and library-picked partitions (groups of
+    1-4 blocks, rows cut anywhere); bf16 through its fp32 result."""
+    w = W.random_case([1, 16, 17, 40, 300, 901], num_q_heads=hq, num_kv_heads=hkv, head_dim=128, dtype=qdt,
+                      seed=hq * 3 + hkv + part)
+    ref, _, _ = replay(w)
+    got, dw = run_gpu(w, part, pa.PA_ALGO_TCGEN05)
+    check(got[0], ref[0], qdt, f"tcgen05 G={hq // hkv} part={part}", dw, part, pa.PA_ALGO_TCGEN05)
+
+
+@pytest.mark.parametrize("scale", [-0.07, 0.0, 0.5])
+def test_tcgen05_any_scale(scale):
+    w = W.random_case([3, 40, 301], num_q_heads=64, num_kv_heads=1, head_dim=128, dtype="float16", seed=71)
+    w.scale = scale
+    ref, _, _ = replay(w)
+    got, _ = run_gpu(w, -1, pa.PA_ALGO_TCGEN05)
+    assert_close(got[0], ref[0], "float16", f"tcgen05 scale={scale}")
+
+
+def test_tcgen05_skips_blocks_outside_the_pool():
+    """A table entry outside the pool: PA_EFLAG_BAD_BLOCK; the block's scores are masked
+    and its V rows zeroed, every other token counts.  Expected: dense fp64 attention over
+    the workload's own K/V without that block's tokens."""
+    w = W.random_case([40, 300], num_q_heads=32, num_kv_heads=1, head_dim=128, seed=72)
+    op = w.steps[0][0]
+    op.block_tables[1, 3] = w.num_blocks + 5
+    got, _ = run_gpu(w, -1, pa.PA_ALGO_TCGEN05)
+    assert pa.pa_get_error_flags(reset=True) == pa.PA_EFLAG_BAD_BLOCK
+    for b in (0, 1):
+        k, v = (x.astype(np.float64)[:, 0] for x in w.logical[b])
+        keep = [t for t in range(int(op.seq_lens[b])) if b == 0 or t // 16 != 3]
+        s_ = op.q[b].astype(np.float64) @ k[keep].T * w.scale
+        p_ = np.exp(s_ - s_.max(axis=1, keepdims=True))
+        ref = (p_ / p_.sum(axis=1, keepdims=True)) @ v[keep]
+        g = got[0][b].double().cpu().numpy()
+        assert np.all(np.abs(g - ref) <= 2e-3 + 2e-3 * np.abs(ref)), b
+
+
+@pytest.mark.parametrize("stall_at", [0, 2])
+def test_tcgen05_wait_timeout(stall_at):
+    """The tcgen05 kernel's failure path: the first CTA leaves one group's copies
+    unissued; its producer, MMA and softmax warps give up after 5 ms, write empty
+    results and release the tensor memory.  The flag is raised, the other sequences
+    match the oracle, and the next call on the same workspace matches everywhere."""
+    # long enough that every CTA's chunk spans more than three groups of 8 blocks
+    lens = [40000, 30000, 8000]
+    w = W.random_case(lens, num_q_heads=32, num_kv_heads=1, head_dim=128, seed=93)
+    dw = runner.DeviceWorkload(w)
+    dw.run_setup()
+    ref, _, _ = replay(w)
+    _, q, bt, sl, mx, _ = dw.steps[0][-1]
+    ws = dw.workspace_for(dw.steps[0][-1], -1, algo=pa.PA_ALGO_TCGEN05)
+    ws.fill_(0xFF)
+    out = torch.full_like(q, float("nan"))
+    pa.pa_get_error_flags(reset=True)
+    pa.pa_decode_stall_selftest(out, q, dw.kc, dw.vc, bt, sl, w.scale, mx, stall_at, 5_000_000,
+                                partition_size=-1, workspace=ws, algo=pa.PA_ALGO_TCGEN05)
+    torch.cuda.synchronize()
+    assert pa.pa_get_error_flags(reset=True) == pa.PA_EFLAG_WAIT_TIMEOUT
+    got = out.double().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    # the first CTA's chunk lies in sequence 0; sequences 1 and 2 are untouched
+    rows = [(b, h) for b in (1, 2) for h in range(32)]
+    assert_close(out, ref[0], "float16", "sequences away from the stalled CTA", rows=rows)
+    out2 = torch.full_like(q, float("nan"))
+    pa.pa_decode(out2, q, dw.kc, dw.vc, bt, sl, w.scale, mx, partition_size=-1, workspace=ws,
+                 algo=pa.PA_ALGO_TCGEN05)
+    assert_close(out2, ref[0], "float16", "next call")
