@@ -55,13 +55,14 @@ FALLBACK_HBM_GBS = 6650.0
 # It holds only for the kernel code it was taken on (hash of the source without
 # comments); after any code change the bench reports null until it is taken again.
 NCU_TRAFFIC = {
-    "ragged": {"source": "paged_kv_cache_395_b200/csrc/pa_decode_tc.cu", "code": "7c3c95cd8e684b52",
-               "per_alg_byte": (475201024 + 4691968 + 462296576 + 4716544) / (472969728 + 459894508)},
+    "ragged": {"source": ["paged_kv_cache_395_b200/csrc/pa_decode_tc.cu",
+                          "paged_kv_cache_395_b200/csrc/pa_tc_shared.cuh"], "code": "e113e6a303473e88",
+               "per_alg_byte": (475231488 + 7520256 + 462311424 + 6604800) / (472969728 + 459894508)},
 }
 
 
-def code_hash(path):
-    s = open(path).read()
+def code_hash(paths):
+    s = "\n".join(open(os.path.join(ROOT, p)).read() for p in paths)
     s = re.sub(r"/\*.*?\*/", " ", s, flags=re.S)
     s = re.sub(r"//[^\n]*", " ", s)
     return hashlib.sha256(" ".join(s.split()).encode()).hexdigest()[:16]
@@ -70,7 +71,7 @@ def code_hash(path):
 def traffic_per_launch(workload, algo, partition, mean_alg_bytes, fused=True):
     t = NCU_TRAFFIC.get(workload)
     if t is None or algo == "simt" or partition != -1 or not fused or \
-            code_hash(os.path.join(ROOT, t["source"])) != t["code"]:
+            code_hash(t["source"]) != t["code"]:
         return None
     return t["per_alg_byte"] * mean_alg_bytes
 

@@ -59,22 +59,24 @@ def test_code_hash_ignores_comments_and_layout(tmp_path):
     b = tmp_path / "b.cu"
     a.write_text("int f(int x) {\n  // one\n  return x + 1; /* two */\n}\n")
     b.write_text("int f(int x) { /* changed\n comment */ return x + 1;   // other\n}")
-    assert bench.code_hash(str(a)) == bench.code_hash(str(b))
+    assert bench.code_hash([str(a)]) == bench.code_hash([str(b)])
     b.write_text("int f(int x) { return x + 2; }")
-    assert bench.code_hash(str(a)) != bench.code_hash(str(b))
+    assert bench.code_hash([str(a)]) != bench.code_hash([str(b)])
+    # every listed source counts
+    assert bench.code_hash([str(a), str(a)]) != bench.code_hash([str(a), str(b)])
 
 
 def test_traffic_is_reported_only_for_the_captured_kernel(monkeypatch):
     rec = dict(bench.NCU_TRAFFIC["ragged"])
     monkeypatch.setitem(bench.NCU_TRAFFIC, "ragged", rec)
-    monkeypatch.setattr(bench, "code_hash", lambda path: rec["code"])
+    monkeypatch.setattr(bench, "code_hash", lambda paths: rec["code"])
     t = bench.traffic_per_launch("ragged", "auto", -1, 2.0e8)
     assert t == pytest.approx(rec["per_alg_byte"] * 2.0e8)
     assert 1.0 <= rec["per_alg_byte"] < 1.1  # the capture read about the algorithmic bytes
     # another code, the CUDA-core family, a fixed partition or another workload: no figure
-    monkeypatch.setattr(bench, "code_hash", lambda path: "0" * 16)
+    monkeypatch.setattr(bench, "code_hash", lambda paths: "0" * 16)
     assert bench.traffic_per_launch("ragged", "auto", -1, 2.0e8) is None
-    monkeypatch.setattr(bench, "code_hash", lambda path: rec["code"])
+    monkeypatch.setattr(bench, "code_hash", lambda paths: rec["code"])
     assert bench.traffic_per_launch("ragged", "simt", -1, 2.0e8) is None
     assert bench.traffic_per_launch("ragged", "auto", 512, 2.0e8) is None
     assert bench.traffic_per_launch("long", "auto", -1, 2.0e8) is None
