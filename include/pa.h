@@ -214,11 +214,18 @@ size_t pa_decode_workspace_size(const pa_decode_params *p);
  * PA_ALGO_TENSOR, PA_ALGO_SIMT or PA_ALGO_TCGEN05, or a negative pa_status for parameters
  * pa_decode would reject.  q (a device pointer, not read) matters only through
  * its alignment: the tensor-core family reads q rows with 16-byte copies, so an
- * unaligned q goes to the CUDA-core family.  Together with
- * pa_decode_workspace_size it also gives the kernel launches of a call: one,
- * plus a merge kernel whenever the call splits (workspace size > 0).
+ * unaligned q goes to the CUDA-core family.
  */
 int pa_decode_algo(const pa_decode_params *p, const void *q);
+
+/*
+ * Kernel launches of one pa_decode call with these parameters and this q (1 or
+ * 2), or a negative pa_status for parameters pa_decode would reject: the decode
+ * kernel, followed by a merge kernel when the call splits on the family it
+ * runs (an unaligned q can move a call to the CUDA-core family, whose own plan
+ * decides).
+ */
+int pa_decode_launches(const pa_decode_params *p, const void *q);
 
 /*
  * Single-token decode attention over the paged cache

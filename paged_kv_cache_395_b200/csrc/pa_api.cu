@@ -505,6 +505,22 @@ int pa_decode_algo(const pa_decode_params *p, const void *q) {
     return p->algo == PA_ALGO_TCGEN05 ? PA_ALGO_TCGEN05 : pl.tc ? PA_ALGO_TENSOR : PA_ALGO_SIMT;
 }
 
+int pa_decode_launches(const pa_decode_params *p, const void *q) {
+    const int fam = pa_decode_algo(p, q);
+    if (fam < 0) return fam;
+    Plan pl;
+    if (fam == PA_ALGO_SIMT) {
+        pa_decode_params p2 = *p;
+        p2.algo = PA_ALGO_SIMT;
+        const int rc = make_plan(&p2, &pl);
+        if (rc != PA_OK) return rc;
+        return pl.bytes > 0 && pl.max_len > 0 ? 2 : 1;  // merge_kernel after a split decode
+    }
+    const int rc = make_plan(p, &pl);
+    if (rc != PA_OK) return rc;
+    return pl.bytes > 0 ? 2 : 1;  // merge_tc_kernel after a split decode
+}
+
 int pa_get_error_flags(unsigned int *flags, int reset, pa_stream_t stream) {
     if (!flags) return PA_ERR_NULL;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;

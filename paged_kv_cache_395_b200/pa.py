@@ -79,6 +79,7 @@ def _load():
     L.pa_decode_workspace_size.argtypes = [ctypes.POINTER(PaDecodeParams)]
     L.pa_decode_workspace_size.restype = ctypes.c_size_t
     L.pa_decode_algo.argtypes = [ctypes.POINTER(PaDecodeParams), P]
+    L.pa_decode_launches.argtypes = [ctypes.POINTER(PaDecodeParams), P]
     L.pa_decode_stall_selftest.argtypes = [P, P, P, P, P, P, f32, ctypes.POINTER(PaDecodeParams), i32,
                                            ctypes.c_uint64, P]
     L.pa_block_copy.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, P]
@@ -91,8 +92,8 @@ def _load():
     L.pa_version.argtypes = []
     for n in ("pa_reshape_and_cache", "pa_reshape_and_cache_ex", "pa_append_int8", "pa_decode", "pa_decode_append",
               "pa_decode_append_fused", "pa_decode_fixed_scratch",
-              "pa_decode_stall_selftest", "pa_decode_algo", "pa_block_copy", "pa_quantize_int8",
-              "pa_quantize_int4", "pa_get_error_flags", "pa_version"):
+              "pa_decode_stall_selftest", "pa_decode_algo", "pa_decode_launches", "pa_block_copy",
+              "pa_quantize_int8", "pa_quantize_int4", "pa_get_error_flags", "pa_version"):
         getattr(L, n).restype = i32
     return L
 
@@ -101,7 +102,7 @@ lib = _load()
 
 # the C-ABI symbols include/pa.h declares
 EXPORTED = ("pa_reshape_and_cache", "pa_reshape_and_cache_ex", "pa_append_int8", "pa_decode_workspace_size",
-            "pa_decode_algo", "pa_decode", "pa_decode_append", "pa_decode_append_fused",
+            "pa_decode_algo", "pa_decode_launches", "pa_decode", "pa_decode_append", "pa_decode_append_fused",
             "pa_decode_fixed_scratch", "pa_decode_stall_selftest", "pa_block_copy", "pa_quantize_int8",
             "pa_quantize_int4", "pa_get_error_flags", "pa_status_string", "pa_version")
 FIXED_SCRATCH_BYTES = 32 << 20  # PA_FIXED_SCRATCH_BYTES
@@ -191,6 +192,17 @@ def pa_decode_algo(q, key_cache, block_tables, max_seq_len, partition_size=0, k_
                     None, algo)
     r = int(lib.pa_decode_algo(ctypes.byref(p), _ptr(q)))
     _check(min(r, 0), "pa_decode_algo")
+    return r
+
+
+def pa_decode_launches(q, key_cache, block_tables, max_seq_len, partition_size=0, k_scales=None,
+                       v_scales=None, algo=PA_ALGO_AUTO) -> int:
+    """Kernel launches of one pa_decode call with these operands (1 or 2), as the
+    library reports it."""
+    p = make_params(q, key_cache, block_tables, max_seq_len, k_scales, v_scales, partition_size,
+                    None, algo)
+    r = int(lib.pa_decode_launches(ctypes.byref(p), _ptr(q)))
+    _check(min(r, 0), "pa_decode_launches")
     return r
 
 

@@ -243,7 +243,9 @@ class StepCalls:
                 kn, vn, sn = k[lead:], v[lead:], s[lead:]
                 p = pa.make_params(q, kc, bt, mx, None, None, partition_size, self.workspace, algo, flags)
                 self.keep.append(p)
-                split = pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+                dl = pa.lib.pa_decode_launches(ctypes.byref(p), ptr(q))
+                if dl < 0:
+                    raise pa.PaError(dl, "pa_decode_launches")
                 one = pa.lib.pa_decode_append_fused(ctypes.byref(p), ptr(q), ptr(kn), ptr(vn), kn.stride(0),
                                                     vn.stride(0))
                 if one < 0:
@@ -251,7 +253,8 @@ class StepCalls:
                 args = (ptr(out), ptr(q), ptr(kn), ptr(vn), ptr(sn), kn.stride(0), vn.stride(0), ptr(kc),
                         ptr(vc), ptr(bt), ptr(sl), ctypes.c_float(w.scale), ctypes.byref(p), sp)
                 calls.append(("decode", pa.lib.pa_decode_append, args))
-                launches += (1 if one == 1 else 2) + (1 if split else 0)
+                # the append kernel unless fused, then the decode's own launches
+                launches += (0 if one == 1 else 1) + dl
                 self.fused_steps += one == 1
                 self.calls[i] = calls
                 self.launches[i] = launches
@@ -277,12 +280,13 @@ class StepCalls:
                     p = pa.make_params(q, kc, bt, mx, ks, vs, partition_size, self.workspace, algo,
                                        flags)
                     self.keep.append(p)
-                    # a split decode is followed by its merge kernel (both families)
-                    split = pa.lib.pa_decode_workspace_size(ctypes.byref(p)) > 0
+                    dl = pa.lib.pa_decode_launches(ctypes.byref(p), ptr(q))
+                    if dl < 0:
+                        raise pa.PaError(dl, "pa_decode_launches")
                     args = (ptr(out), ptr(q), ptr(kc), ptr(vc), ptr(bt), ptr(sl),
                             ctypes.c_float(w.scale), ctypes.byref(p), sp)
                     calls.append(("decode", pa.lib.pa_decode, args))
-                    launches += 2 if split else 1
+                    launches += dl
             self.calls[i] = calls
             self.launches[i] = launches
 

@@ -312,3 +312,31 @@ def test_tcgen05_is_planned_only_for_its_groups():
                dict(num_seqs=4096, max_blocks_per_seq=1)):
         assert algo(params(**dict(ok, **kw))) == pa.PA_ERR_UNSUPPORTED, kw
     assert algo(params(algo=4)) == pa.PA_ERR_UNSUPPORTED
+
+
+def test_decode_launches_reports_the_merge_kernel():
+    """pa_decode_launches: one decode kernel, followed by a merge kernel when the
+    call splits on the family it runs."""
+    L = pa.lib
+    aligned, unaligned = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1008)
+
+    def n(q=aligned, **kw):
+        return L.pa_decode_launches(ctypes.byref(params(**kw)), q)
+    assert n(partition_size=0) == 1
+    assert n(partition_size=-1, algo=pa.PA_ALGO_TENSOR) == 2
+    assert n(partition_size=16, algo=pa.PA_ALGO_TENSOR) == 2
+    assert n(partition_size=16, algo=pa.PA_ALGO_SIMT) == 2
+    assert n(partition_size=0, algo=pa.PA_ALGO_SIMT) == 1
+    # an unaligned q leaves the tensor-core family under PA_ALGO_AUTO (the CUDA-core
+    # family's own plan: one partition of 64 tokens is one pass)
+    assert n(q=unaligned, partition_size=16) == 2
+    assert n(q=unaligned, partition_size=64) == 1
+    assert n(partition_size=64) == 2
+    assert n(q=unaligned, partition_size=16, algo=pa.PA_ALGO_TENSOR) == pa.PA_ERR_ALIGN
+    # the cooperative mode
+    big = dict(num_seqs=4, num_q_heads=32, num_kv_heads=1, max_blocks_per_seq=64, max_seq_len=1024)
+    assert n(partition_size=-1, **big) == 2
+    assert n(partition_size=0, **big) == 1
+    assert n(partition_size=-1, algo=pa.PA_ALGO_TCGEN05, **big) == 2
+    # invalid parameters: the status pa_decode would return
+    assert n(head_dim=96) == pa.PA_ERR_UNSUPPORTED
