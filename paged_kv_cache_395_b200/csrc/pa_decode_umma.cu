@@ -12,16 +12,19 @@
 // memory by the softmax warps.  A group of 32 heads fills rows 0-31 (rows 32-63 hold zero q rows,
 // computed and ignored).
 //
-// One CTA per SM (192 KB of shared memory), six warps:
-// * warp 4, producer: per group, TMA for each block's K and V 64-dim boxes into four
-//   box-major rings (K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127; two halves
-//   of 8 blocks), so that a group's 16n token rows sit at one 128-byte pitch as the MMA
-//   descriptors want; a new segment's q rows go to one of two q slots (128-byte swizzle,
-//   the same canonical K-major layout).
-// * warp 5, MMA issuer (it also owns the TMEM allocation): lane 0 issues a group's 8 QK
-//   MMAs into S[g % 2] one group ahead, then, once the softmax has written P, the group's
-//   n P.V MMAs into O; tcgen05.commit signals S ready, P.V done, ring half free and q slot
-//   free on mbarriers.
+// One CTA per SM (~195 KB of shared memory), seven warps:
+// * warp 4, K producer: per group, TMA for each block's two 64-dim K boxes into two
+//   box-major rings (K dims 0-63, K dims 64-127; two halves of 8 blocks), so that a
+//   group's 16n token rows sit at one 128-byte pitch as the MMA descriptors want; a
+//   K half is refilled as soon as the QK products that read it have finished.  It
+//   also copies a new segment's q rows into one of two q slots (128-byte swizzle, the
+//   same canonical K-major layout).
+// * warp 6, V producer: the same for the V boxes, a V half being refilled once the
+//   P.V products that read it have finished.
+// * warp 5, MMA issuer (it also owns the TMEM allocation): lane 0 issues a group's 16
+//   QK MMAs into S[g % 2] one group ahead, then, once the softmax has written P and
+//   the group's V tiles have landed, the group's P.V MMAs into O; tcgen05.commit
+//   signals S ready, K half free, P.V done, V half free and q slot free on mbarriers.
 // * warps 0-3, softmax and epilogue.  An M = 64 accumulator puts rows 16w .. 16w + 15 in
 //   TMEM lanes 32w .. 32w + 15 (lane tile 0) or, one tile over, 32w + 16 .. 32w + 31 (lane
 //   tile 1); S takes a group's blocks 0-3 in tile 0 and 4-7 in tile 1, O dims 0-63 in
@@ -33,7 +36,9 @@
 //   2^8), writes its P row, zeroes the stale V rows of a row's last block (0 x NaN would
 //   poison the product), and at a segment's end reads its O row and writes the output or
 //   the partial result.
-// Every barrier completes once per use of its buffer, so no wait can alias a later phase.
+// Every barrier completes once per use of its buffer, and no buffer is refilled before
+// every wait on its previous phase has returned, so no wait can alias a later phase
+// (which is why the softmax waits for S ready, not for the K tiles).
 // Chunks of the cache-row stream go to CTAs as in decode_coop_kernel; cut rows leave
 // partial results for merge_tc_kernel, GC columns per cache row.
 #include <type_traits>
@@ -48,7 +53,7 @@ namespace {
 
 constexpr int kUD = 128;            // head_dim
 constexpr int kUGroup = 8;          // blocks per MMA group
-constexpr int kUThreads = 192;      // warps 0-3 softmax, 4 producer, 5 MMA
+constexpr int kUThreads = 224;      // warps 0-3 softmax, 4 K producer, 5 MMA, 6 V producer
 constexpr int kUBox = 16 * 128;     // one 64-dim box of one block: 16 rows x 128 bytes
 constexpr int kURegion = 2 * kUGroup * kUBox;  // one box-major ring: two halves of 8 blocks
 constexpr int kUQSlot = 2 * 64 * 128;          // 64 q rows x 2 boxes
@@ -64,10 +69,10 @@ constexpr int kUV1 = kUV0 + kURegion;
 constexpr int kUQ = kUV1 + kURegion;           // two q slots
 constexpr int kUP = kUQ + 2 * kUQSlot;         // two P buffers
 constexpr int kUBar = kUP + 2 * kUPBuf;
-// barriers: full[2], empty[2], s_ready[2], p_ready[2], pv_done[2], qfull[2], qempty[2]
-constexpr int kUNBar = 14;
-constexpr int kUMeta = kUBar + kUNBar * 8;     // int [2][4]: n, bad-block mask, tokens of the last block
-constexpr int kUMisc = kUMeta + 2 * 4 * 4;     // tmem address, abort flag
+// barriers: full_k[2], full_v[2], empty_k[2], empty_v[2], s_ready[2], p_ready[2],
+// pv_done[2], qfull[2], qempty[2]
+constexpr int kUNBar = 18;
+constexpr int kUMisc = kUBar + kUNBar * 8;     // tmem address, abort flag
 constexpr int kUCum = kUMisc + 16;
 inline int umma_smem_bytes(int B) { return 1024 + kUCum + (3 * B + 3) * 4; }
 
@@ -209,9 +214,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kUBar);
-    uint64_t *full = bars, *empty = bars + 2, *s_ready = bars + 4, *p_ready = bars + 6, *pv_done = bars + 8,
-             *qfull = bars + 10, *qempty = bars + 12;
-    int *meta = reinterpret_cast<int *>(smem + kUMeta);  // [2][4]
+    uint64_t *full_k = bars, *full_v = bars + 2, *empty_k = bars + 4, *empty_v = bars + 6, *s_ready = bars + 8,
+             *p_ready = bars + 10, *pv_done = bars + 12, *qfull = bars + 14, *qempty = bars + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kUMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kUMisc + 4);
     int *cum = reinterpret_cast<int *>(smem + kUCum);  // [B + 1]
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
     }
     const int gam = a.tc_chunk == 0 ? PA_TC_GAMMA : 0;
     {
-        __shared__ int wsum[6], wsumv[6];
+        __shared__ int wsum[kUThreads / 32], wsumv[kUThreads / 32];
         const int per = (B + kUThreads - 1) / kUThreads;
         const int lo = min(B, tid * per), hi = min(B, lo + per);
         int s = 0, sv = 0;
@@ -274,8 +278,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
         }
         if (tid == 0) {
             for (int i = 0; i < 2; ++i) {
-                mbar_init(&full[i], 1);
-                mbar_init(&empty[i], 1);
+                mbar_init(&full_k[i], 1);
+                mbar_init(&full_v[i], 1);
+                mbar_init(&empty_k[i], 1);
+                mbar_init(&empty_v[i], 1);
                 mbar_init(&s_ready[i], 1);
                 mbar_init(&p_ready[i], 128);
                 mbar_init(&pv_done[i], 1);
@@ -445,9 +451,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&qfull[qs]);
             }
+            // K half gi % 2 is free once group gi - 2's QK products have finished (its V
+            // half, refilled by warp 6, only once that group's P.V has)
             const int h = gi & 1;
             if (gi >= 2) {
-                int ok = lane == 0 ? (int)mbar_sleep_wait(&empty[h], ((gi >> 1) - 1) & 1, a.wait_ns) : 0;
+                int ok = lane == 0 ? (int)mbar_sleep_wait(&empty_k[h], ((gi >> 1) - 1) & 1, a.wait_ns) : 0;
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     ok_all = false;
                     break;
@@ -459,25 +467,20 @@ __global__ void __launch_bounds__(kUThreads, 1)
             const unsigned bad = want & ~good_mask;
             if (lane == 0) {
                 if (bad) raise_flag(PA_EFLAG_BAD_BLOCK);
-                meta[h * 4 + 0] = g.n;
-                meta[h * 4 + 1] = (int)bad;
-                meta[h * 4 + 2] = (g.j0 + g.n == g.nb) ? g.L - (g.nb - 1) * kBlockSize : kBlockSize;
-                const uint32_t bytes = (uint32_t)__popc(good_mask) * 4u * (uint32_t)kUBox;
+                const uint32_t bytes = (uint32_t)__popc(good_mask) * 2u * (uint32_t)kUBox;
                 if (bytes)
-                    mbar_arrive_expect_tx(&full[h], bytes);
+                    mbar_arrive_expect_tx(&full_k[h], bytes);
                 else
-                    mbar_arrive(&full[h]);
+                    mbar_arrive(&full_k[h]);
             }
             __syncwarp();
             const bool stall = blockIdx.x == 0 && gi == a.stall_at;
             if (good && !stall) {
                 const int y = (pb * Hc + g.kc) * kBlockSize;
                 const uint32_t slot = (uint32_t)((h * kUGroup + lane) * kUBox);
-                const uint32_t bar = smem_addr(&full[h]);
+                const uint32_t bar = smem_addr(&full_k[h]);
                 tma_load_2d(sbase + kUK0 + slot, &tmK, 0, y, bar);
                 tma_load_2d(sbase + kUK1 + slot, &tmK, 64, y, bar);
-                tma_load_2d(sbase + kUV0 + slot, &tmV, 0, y, bar);
-                tma_load_2d(sbase + kUV1 + slot, &tmV, 64, y, bar);
             }
             issued_last = gi;
             ++gi;
@@ -486,7 +489,54 @@ __global__ void __launch_bounds__(kUThreads, 1)
         // no copy may land after the CTA exits: wait (bounded) for the last two groups' copies
         if (lane == 0)
             for (int k = max(0, issued_last - 1); k <= issued_last; ++k)
-                mbar_sleep_wait(&full[k & 1], (k >> 1) & 1, a.wait_ns);
+                mbar_sleep_wait(&full_k[k & 1], (k >> 1) & 1, a.wait_ns);
+    } else if (warp == 6) {
+        // ============================== V producer ==============================
+        // the same groups in the same order: V half gi % 2 once group gi - 2's P.V has finished
+        GIt gi_it;
+        git_init(gi_it);
+        Grp cur;
+        bool hc = next_group(gi_it, cur);
+        int pbn = (hc && lane < cur.n) ? a.tables[(size_t)cur.b * a.mbps + cur.j0 + lane] : -1;
+        int gi = 0, issued_last = -1;
+        bool okv = true;
+        while (hc) {
+            const Grp g = cur;
+            const int pb = pbn;
+            hc = next_group(gi_it, cur);
+            pbn = (hc && lane < cur.n) ? a.tables[(size_t)cur.b * a.mbps + cur.j0 + lane] : -1;
+            const int h = gi & 1;
+            if (gi >= 2) {
+                int ok = lane == 0 ? (int)mbar_sleep_wait(&empty_v[h], ((gi >> 1) - 1) & 1, a.wait_ns) : 0;
+                if (!__shfl_sync(0xffffffffu, ok, 0) || *abort_flag) {
+                    okv = false;
+                    break;
+                }
+            }
+            const bool good = lane < g.n && pb >= 0 && (int64_t)pb < a.N;
+            const unsigned good_mask = __ballot_sync(0xffffffffu, good);
+            if (lane == 0) {
+                const uint32_t bytes = (uint32_t)__popc(good_mask) * 2u * (uint32_t)kUBox;
+                if (bytes)
+                    mbar_arrive_expect_tx(&full_v[h], bytes);
+                else
+                    mbar_arrive(&full_v[h]);
+            }
+            __syncwarp();
+            if (good) {
+                const int y = (pb * Hc + g.kc) * kBlockSize;
+                const uint32_t slot = (uint32_t)((h * kUGroup + lane) * kUBox);
+                const uint32_t bar = smem_addr(&full_v[h]);
+                tma_load_2d(sbase + kUV0 + slot, &tmV, 0, y, bar);
+                tma_load_2d(sbase + kUV1 + slot, &tmV, 64, y, bar);
+            }
+            issued_last = gi;
+            ++gi;
+        }
+        if (!okv && lane == 0) *abort_flag = 1;
+        if (lane == 0)
+            for (int k = max(0, issued_last - 1); k <= issued_last; ++k)
+                mbar_sleep_wait(&full_v[k & 1], (k >> 1) & 1, a.wait_ns);
     } else if (warp == 5) {
         // ================================ MMA issuer ================================
         GIt gi_it;
@@ -502,11 +552,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
             const int h = k & 1;
             int ok;
             if (poll) {
-                ok = lane == 0 ? (int)(mbar_try_wait(&full[h], (k >> 1) & 1) &&
+                ok = lane == 0 ? (int)(mbar_try_wait(&full_k[h], (k >> 1) & 1) &&
                                        (!g.seg_first || mbar_try_wait(&qfull[g.si & 1], (g.si >> 1) & 1)))
                                : 0;
             } else {
-                ok = lane == 0 ? (int)mbar_sleep_wait(&full[h], (k >> 1) & 1, a.wait_ns) : 0;
+                ok = lane == 0 ? (int)mbar_sleep_wait(&full_k[h], (k >> 1) & 1, a.wait_ns) : 0;
                 if (ok && g.seg_first && lane == 0) ok = mbar_sleep_wait(&qfull[g.si & 1], (g.si >> 1) & 1, a.wait_ns);
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -531,6 +581,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
                     }
                 }
                 umma_commit(&s_ready[k & 1]);
+                umma_commit(&empty_k[h]);  // the K half may be refilled once these products finish
             }
             __syncwarp();
             last_qk = k;
@@ -545,7 +596,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
             // already in; P.V of this group never waits for the next group's copies (their
             // ring half is refilled only after an earlier P.V)
             bool qk_next = hc && issue_qk(cur, k + 1, true);
-            int okp = lane == 0 ? (int)mbar_sleep_wait(&p_ready[k & 1], (k >> 1) & 1, a.wait_ns) : 0;
+            int okp = lane == 0 ? (int)(mbar_sleep_wait(&p_ready[k & 1], (k >> 1) & 1, a.wait_ns) &&
+                                        mbar_sleep_wait(&full_v[k & 1], (k >> 1) & 1, a.wait_ns))
+                                : 0;
             okp = __shfl_sync(0xffffffffu, okp, 0);
             if (!okp) {
                 ok = false;
@@ -567,7 +620,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
                     }
                 }
                 umma_commit(&pv_done[k & 1]);
-                umma_commit(&empty[k & 1]);
+                umma_commit(&empty_v[k & 1]);
                 if (g.seg_last) umma_commit(&qempty[g.si & 1]);
             }
             __syncwarp();
@@ -594,19 +647,33 @@ __global__ void __launch_bounds__(kUThreads, 1)
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         GIt gi_it;
         git_init(gi_it);
-        Grp g;
+        Grp g, gn;
+        bool hn = next_group(gi_it, gn);
+        // the group's table entries, loaded a group ahead: which of its blocks lie
+        // outside the pool (their scores are masked and their V rows zeroed)
+        int pbn = (hn && lane < gn.n) ? a.tables[(size_t)gn.b * a.mbps + gn.j0 + lane] : -1;
         int gi = 0;
         float m = -INFINITY, l = 0.f;  // l: this thread's half of the row's sum
         bool alive = true;
-        while (next_group(gi_it, g)) {
+        while (hn) {
+            g = gn;
+            const int pbg = pbn;
+            hn = next_group(gi_it, gn);
+            pbn = (hn && lane < gn.n) ? a.tables[(size_t)gn.b * a.mbps + gn.j0 + lane] : -1;
+            const int n = g.n;
+            const unsigned want = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+            const unsigned bad = want & ~__ballot_sync(0xffffffffu, lane < n && pbg >= 0 && (int64_t)pbg < a.N);
+            const int ntok_last = (g.j0 + n == g.nb) ? g.L - (g.nb - 1) * kBlockSize : kBlockSize;
             if (g.seg_first) {
                 m = -INFINITY;
                 l = 0.f;
             }
             const int h = gi & 1;
             if (alive) {
-                const bool okf = mbar_sleep_wait(&full[h], (gi >> 1) & 1, a.wait_ns) &&
-                                 mbar_sleep_wait(&s_ready[h], (gi >> 1) & 1, a.wait_ns);
+                // S ready implies the group's K tiles landed.  (No wait on the K barrier
+                // itself: it may already have moved on to group gi + 2, whose copies start
+                // as soon as this group's QK products are done.)
+                const bool okf = mbar_sleep_wait(&s_ready[h], (gi >> 1) & 1, a.wait_ns);
                 if (!__all_sync(0xffffffffu, okf) || *abort_flag) {
                     alive = false;
                     *abort_flag = 1;
@@ -614,9 +681,6 @@ __global__ void __launch_bounds__(kUThreads, 1)
             }
             if (alive && warp_on) {
                 tc_fence_after();
-                const int n = meta[h * 4 + 0];
-                const unsigned bad = (unsigned)meta[h * 4 + 1];
-                const int ntok_last = meta[h * 4 + 2];
                 float x[64];
                 tmem_ld64(tmem + lane_base + (uint32_t)h * 64u, x);
                 tmem_wait_ld();
@@ -713,11 +777,14 @@ __global__ void __launch_bounds__(kUThreads, 1)
             if (alive) {
                 // ---- stale V rows of the row's last block and of skipped blocks weigh 0 in
                 // P; zero them, as 0 x NaN would poison the product
-                const int n = meta[h * 4 + 0];
-                const unsigned bad = (unsigned)meta[h * 4 + 1];
-                const int ntok_last = meta[h * 4 + 2];
                 if (bad != 0u || ntok_last != kBlockSize) {
-                    for (int t = 0; t < n; ++t) {
+                    // the V tiles must have landed before their stale rows are zeroed
+                    const bool okv = mbar_sleep_wait(&full_v[h], (gi >> 1) & 1, a.wait_ns);
+                    if (!__all_sync(0xffffffffu, okv)) {
+                        alive = false;
+                        *abort_flag = 1;
+                    }
+                    for (int t = 0; alive && t < n; ++t) {
                         const int r0 = ((bad >> t) & 1u) ? 0 : (t == n - 1 ? ntok_last : kBlockSize);
                         const int nz = (kBlockSize - r0) * 16;  // 16-byte chunks over both boxes
                         for (int i = tid; i < nz; i += 128) {
