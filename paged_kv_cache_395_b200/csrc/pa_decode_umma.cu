@@ -7,7 +7,8 @@
 // query heads per KV head the products of a cache tile are dense contractions, so they
 // run as tcgen05 MMAs over groups of n <= 8 consecutive blocks of one cache row:
 //   S[64 heads x 16n tokens] = Q[64 x 128] . K^T     (M = 64, N = 16n, K = 128)
-//   O[64 heads x 128 dims]  += P[64 x 16n] . V        (M = 64, N = 128, K = 16n)
+//   O[64 heads x 128 dims]  += P[64 x 16n] . V        (M = 64, N = 128, K = 16n; one MMA
+//                                                      of N = 128 per block)
 // S (two buffers) and O live in tensor memory (256 columns); P is written to shared
 // memory by the softmax warps.  A group of 32 heads fills rows 0-31 (rows 32-63 hold zero q rows,
 // computed and ignored).
@@ -23,13 +24,16 @@
 //   P.V products that read it have finished.
 // * warp 5, MMA issuer (it also owns the TMEM allocation): lane 0 issues a group's 16
 //   QK MMAs into S[g % 2] one group ahead, then, once the softmax has written P and
-//   the group's V tiles have landed, the group's P.V MMAs into O; tcgen05.commit
+//   the group's V tiles have landed, the group's 8 P.V MMAs into O (V of a block as one
+//   MN-major operand of 128 dims, its two 64-dim ring regions one leading byte offset
+//   apart: an MMA costs about as much to issue at N = 64 as at 128); tcgen05.commit
 //   signals S ready, K half free, P.V done, V half free and q slot free on mbarriers.
 // * warps 0-3, softmax and epilogue.  An M = 64 accumulator puts rows 16w .. 16w + 15 in
 //   TMEM lanes 32w .. 32w + 15 (lane tile 0) or, one tile over, 32w + 16 .. 32w + 31 (lane
-//   tile 1); S takes a group's blocks 0-3 in tile 0 and 4-7 in tile 1, O dims 0-63 in
-//   tile 0 and 64-127 in tile 1.  Thread (w, l) so owns head row 16w + (l & 15): 64 of its
-//   scores and 64 of its output dims; one shuffle joins the two halves' maxima and sums.
+//   tile 1); S takes a group's blocks 0-3 in tile 0 and 4-7 in tile 1, O all 128 dims in
+//   tile 0.  Thread (w, l) so owns head row 16w + (l & 15) and 64 of its scores; one shuffle
+//   joins the two halves' maxima and sums, and the threads of lane tile 0 write the row's
+//   output.
 //   It reads its scores, masks slots past the row's end (and blocks outside the pool), keeps the
 //   online softmax with the lazy maximum of the cooperative kernel (scores unscaled, the
 //   scale in the exponent, O rescaled in TMEM only when the maximum moves by more than
@@ -544,7 +548,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
         Grp cur;
         bool hc = next_group(gi_it, cur);
         const uint32_t id_qk_half = umma_idesc(kFmt, 64, 64, 0);
-        const uint32_t id_pv = umma_idesc(kFmt, 64, 64, 1);
+        const uint32_t id_pv = umma_idesc(kFmt, 64, 128, 1);
         int gi = 0, last_committed = -1, last_qk = -1;
         // QK of group k: S[k % 2] = Q . K^T over the group's 16 n tokens.  poll: only if
         // its tiles (and q) have landed already, else return false without waiting.
@@ -611,13 +615,12 @@ __global__ void __launch_bounds__(kUThreads, 1)
                     const uint32_t pa = pb + (t >> 2) * 64 * 128 + (t & 3) * 32;
                     const uint32_t slot = (uint32_t)(((k & 1) * kUGroup + t) * kUBox);
                     const uint32_t acc = (g.seg_first && t == 0) ? 0u : 1u;
-#pragma unroll
-                    for (int tile = 0; tile < 2; ++tile) {  // dims 0-63 -> lane tile 0, 64-127 -> tile 1
-                        const uint64_t vd = umma_sdesc(sbase + (tile ? kUV1 : kUV0) + slot, 1024, 1024);
-                        const uint32_t d = tmem + 128u + ((uint32_t)(16 * tile) << 16);
-                        umma_f16(d, umma_sdesc(pa, 16, 1024), vd, id_pv, acc);
-                        if (SPLIT) umma_f16(d, umma_sdesc(pa + kUPBuf, 16, 1024), vd, id_pv, 1u);
-                    }
+                    // block t's V as one MN-major operand of N = 128 dims: 64 dims per 128-byte
+                    // swizzle atom, the atom of dims 64-127 one ring region further (the
+                    // leading byte offset), 8-token groups 1024 bytes apart; O in lane tile 0
+                    const uint64_t vd = umma_sdesc(sbase + kUV0 + slot, kUV1 - kUV0, 1024);
+                    umma_f16(tmem + 128u, umma_sdesc(pa, 16, 1024), vd, id_pv, acc);
+                    if (SPLIT) umma_f16(tmem + 128u, umma_sdesc(pa + kUPBuf, 16, 1024), vd, id_pv, 1u);
                 }
                 umma_commit(&pv_done[k & 1]);
                 umma_commit(&empty_v[k & 1]);
@@ -719,7 +722,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
                         } else {
                             tc_fence_after();
 #pragma unroll
-                            for (int q = 0; q < 2; ++q) {
+                            for (int q = 0; q < 4; ++q) {  // O: 128 columns, rows in lane tile 0
                                 float v[32];
                                 tmem_ld32(tmem + lane_base + 128u + (uint32_t)q * 32u, v);
                                 tmem_wait_ld();
@@ -801,38 +804,56 @@ __global__ void __launch_bounds__(kUThreads, 1)
             // ---- segment end: this thread's 64 dims of its row of O to the output or the
             // workspace
             if (g.seg_last) {
-                float o[64];
-#pragma unroll
-                for (int j = 0; j < 64; ++j) o[j] = 0.f;
-                float lse = -INFINITY;
+                // O rows sit in lane tile 0: threads of half 0 write all 128 dims of their row,
+                // 64 at a time (half 1 reads lanes that hold nothing it uses)
+                float lse = -INFINITY, inv = 0.f;
+                bool have_o = false;
                 if (alive) {
                     const bool okw = mbar_sleep_wait(&pv_done[gi & 1], (gi >> 1) & 1, a.wait_ns);
                     if (!__all_sync(0xffffffffu, okw)) {
                         alive = false;
                         *abort_flag = 1;
                     } else if (warp_on) {
-                        tc_fence_after();
-                        tmem_ld64(tmem + lane_base + 128u, o);
-                        tmem_wait_ld();
                         const float lr = l + __shfl_xor_sync(0xffffffffu, l, 16);  // the row's sum
-                        const float inv = lr > 0.f ? 1.f / lr : 0.f;
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) o[j] *= inv;
+                        inv = lr > 0.f ? 1.f / lr : 0.f;
                         lse = m * sl + log2f(lr);
+                        have_o = true;
                     }
                 }
-                if (warp_on && row < GC) {
-                    if (g.whole) {
-                        const size_t orow = ((size_t)g.b * a.Hq + (size_t)g.kc * GC + row) * kUD + 64 * half;
+                const bool writer = warp_on && row < GC && half == 0;
+                size_t obase = 0;
+                float *wbase = nullptr;
+                if (g.whole) {
+                    obase = ((size_t)g.b * a.Hq + (size_t)g.kc * GC + row) * kUD;
+                } else {
+                    const int ch_first = ck.of(g.b, g.kc, g.nb, 0);
+                    const int slot = 2 * g.ch + ((g.ch == ch_first && ck.mid_start(g.b, g.kc, g.nb)) ? 1 : 0);
+                    wbase = a.ws_o + ((size_t)slot * GC + row) * kUD;
+                    if (writer) a.ws_lse[(size_t)slot * GC + row] = lse;
+                }
+                if (have_o) tc_fence_after();
 #pragma unroll
-                        for (int j = 0; j < 64; j += 2) store_out2<T>(a.out, a.out_f32, orow + j, o[j], o[j + 1]);
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    float o[64];
+                    if (have_o) {
+                        tmem_ld64(tmem + lane_base + 128u + (uint32_t)c2 * 64u, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) o[j] *= inv;
                     } else {
-                        const int ch_first = ck.of(g.b, g.kc, g.nb, 0);
-                        const int slot = 2 * g.ch + ((g.ch == ch_first && ck.mid_start(g.b, g.kc, g.nb)) ? 1 : 0);
-                        float4 *w = reinterpret_cast<float4 *>(a.ws_o + ((size_t)slot * GC + row) * kUD + 64 * half);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) w[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-                        if (half == 0) a.ws_lse[(size_t)slot * GC + row] = lse;
+                        for (int j = 0; j < 64; ++j) o[j] = 0.f;
+                    }
+                    if (writer) {
+                        if (g.whole) {
+#pragma unroll
+                            for (int j = 0; j < 64; j += 2)
+                                store_out2<T>(a.out, a.out_f32, obase + 64 * c2 + j, o[j], o[j + 1]);
+                        } else {
+                            float4 *w = reinterpret_cast<float4 *>(wbase + 64 * c2);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) w[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                        }
                     }
                 }
             }
