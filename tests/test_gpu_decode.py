@@ -529,7 +529,8 @@ def test_head_dim_256_int8_multi_query(Q):
 def test_wide_workloads_full_size_sampled(name):
     """The benchmark's MQA and head_dim-256 workloads at full size, in the bench's
     launch configuration (library-picked partition, inputs-ready flag), against
-    the oracle on sampled (sequence, head) rows."""
+    the oracle on sampled (sequence, head) rows; MQA through the opt-in tcgen05
+    kernel as well."""
     w = W.NAMED[name]()
     B, Hq = w.steps[0][0].q.shape[:2]
     rng = np.random.default_rng(0)
@@ -543,6 +544,13 @@ def test_wide_workloads_full_size_sampled(name):
     torch.cuda.synchronize()
     out = dw.steps[0][-1][-1]
     assert_close(out, ref[0], "float16", name, rows=rows)
+    if name == "mqa":
+        # the opt-in tcgen05 kernel, same launch configuration
+        out.fill_(float("nan"))
+        calls = runner.StepCalls(dw, -1, False, pa.PA_ALGO_TCGEN05, flags=pa.PA_DECODE_INPUTS_READY)
+        calls.run(0)
+        torch.cuda.synchronize()
+        assert_close(out, ref[0], "float16", name + " tcgen05", rows=rows)
 
 
 # -- several new tokens per sequence (causal among them) -----------------------------------
@@ -756,6 +764,21 @@ def test_tcgen05_large_groups(hq, hkv, part, qdt):
     ref, _, _ = replay(w)
     got, dw = run_gpu(w, part, pa.PA_ALGO_TCGEN05)
     check(got[0], ref[0], qdt, f"tcgen05 G={hq // hkv} part={part}", dw, part, pa.PA_ALGO_TCGEN05)
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 6.0])
+@pytest.mark.parametrize("part", [-1, 128, 256])
+def test_tcgen05_edge_lengths(part, q_scale):
+    """Empty sequences (zero rows), rows of exactly one and two 8-block groups and one
+    token past them, rows spanning many groups, chunks of one or two groups (128, 256
+    tokens); a sharpened softmax (q scaled by 6) moves the running maximum past the lazy
+    threshold mid-row, so O is rescaled in tensor memory."""
+    lens = [0, 128, 129, 255, 256, 2049, 0, 5, 1500]
+    w = W.random_case(lens, num_q_heads=64, num_kv_heads=2, head_dim=128, dtype="float16",
+                      seed=17 + part + int(q_scale), q_scale=q_scale)
+    ref, _, _ = replay(w)
+    got, dw = run_gpu(w, part, pa.PA_ALGO_TCGEN05)
+    check(got[0], ref[0], "float16", f"tcgen05 edges part={part} q_scale={q_scale}", dw, part, pa.PA_ALGO_TCGEN05)
 
 
 @pytest.mark.parametrize("scale", [-0.07, 0.0, 0.5])
