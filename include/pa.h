@@ -67,8 +67,9 @@ enum pa_dtype { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_I8 = 3, PA_I4 = 4 };
 /* PA_ALGO_TCGEN05: the tcgen05 kernel (5th-generation tensor cores, accumulators in
  * tensor memory) for groups of 32 or 64 fp16/bf16 query heads per KV head at head_dim
  * 128, split-K (partition_size != 0), num_seqs <= 2048; PA_ERR_UNSUPPORTED elsewhere.
- * Only on request: for these groups PA_ALGO_AUTO and PA_ALGO_TENSOR run the faster
- * mma.sync kernel that shares each staged tile across a CTA's warps. */
+ * PA_ALGO_AUTO runs it for the split groups of 64 (faster there); for groups of 16 and 32,
+ * and under PA_ALGO_TENSOR, the mma.sync kernel that shares each staged tile across a
+ * CTA's warps runs instead (faster for those groups). */
 enum pa_algo { PA_ALGO_AUTO = 0, PA_ALGO_SIMT = 1, PA_ALGO_TENSOR = 2, PA_ALGO_TCGEN05 = 3 };
 
 /* Bits of the per-device error word (pa_get_error_flags). */

@@ -312,6 +312,18 @@ size_t pa_decode_workspace_size(const pa_decode_params *p) {
 namespace pa {
 
 // The new-token rows of pa_decode_append.
+// PA_ALGO_AUTO's kernel for groups of 64 query heads per KV head (eight 8-column rows):
+// the tcgen05 kernel, which measured 5-27 % faster there than the cooperative mma.sync
+// kernel (fp16 and bf16, batches of 16 to 128 sequences of 4096 tokens); for groups of 16
+// and 32 the cooperative kernel stays (faster there).
+static bool auto_tcgen05(const pa_decode_params *p, const Plan &pl) {
+    if (p->algo != PA_ALGO_AUTO || !pl.tc || pl.tc_chunk < 0) return false;
+    KernelHeads kh;
+    kernel_heads(p, &kh);
+    return kh.ngroups == 8 && decode_umma_eligible(p->q_dtype, p->kv_dtype, p->head_dim, kh.G, kh.ngroups, kh.qlen,
+                                                   kh.padded, p->partition_size, p->num_seqs);
+}
+
 struct AppendIn {
     const void *k, *v;
     const int64_t *slots;
@@ -386,7 +398,7 @@ static int decode_impl(void *out, const void *q, const void *key_cache, const vo
     a.out_f32 = (p->flags & PA_DECODE_OUT_F32) ? 1 : 0;
     a.stall_at = stall_at;
     a.wait_ns = wait_ns;
-    a.umma = p->algo == PA_ALGO_TCGEN05 ? 1 : 0;
+    a.umma = (p->algo == PA_ALGO_TCGEN05 || auto_tcgen05(p, pl)) ? 1 : 0;
     if (ap) {
         a.append = 1;
         a.k_new = ap->k;
@@ -502,7 +514,8 @@ int pa_decode_algo(const pa_decode_params *p, const void *q) {
     if (rc != PA_OK) return rc;
     if (pl.tc && (uintptr_t)q % 16)
         return p->algo == PA_ALGO_TENSOR || p->algo == PA_ALGO_TCGEN05 ? PA_ERR_ALIGN : PA_ALGO_SIMT;
-    return p->algo == PA_ALGO_TCGEN05 ? PA_ALGO_TCGEN05 : pl.tc ? PA_ALGO_TENSOR : PA_ALGO_SIMT;
+    if (p->algo == PA_ALGO_TCGEN05 || auto_tcgen05(p, pl)) return PA_ALGO_TCGEN05;
+    return pl.tc ? PA_ALGO_TENSOR : PA_ALGO_SIMT;
 }
 
 int pa_decode_launches(const pa_decode_params *p, const void *q) {

@@ -340,3 +340,25 @@ def test_decode_launches_reports_the_merge_kernel():
     assert n(partition_size=-1, algo=pa.PA_ALGO_TCGEN05, **big) == 2
     # invalid parameters: the status pa_decode would return
     assert n(head_dim=96) == pa.PA_ERR_UNSUPPORTED
+
+
+def test_auto_picks_tcgen05_for_groups_of_64():
+    """PA_ALGO_AUTO runs the tcgen05 kernel for split decodes of 64 fp16/bf16 query heads
+    per KV head (where it measured faster), the cooperative mma.sync kernel for groups of
+    16 and 32, and the tensor-core per-row kernel in one pass; PA_ALGO_TENSOR keeps the
+    mma.sync family."""
+    q = ctypes.c_void_p(0x1000)
+    algo = lambda **kw: pa.lib.pa_decode_algo(ctypes.byref(params(**kw)), q)  # noqa: E731
+    g64 = dict(num_seqs=4, num_q_heads=64, num_kv_heads=1, max_blocks_per_seq=64, max_seq_len=1024)
+    assert algo(partition_size=-1, **g64) == pa.PA_ALGO_TCGEN05
+    assert algo(partition_size=64, **dict(g64, q_dtype=pa.PA_BF16, kv_dtype=pa.PA_BF16)) == pa.PA_ALGO_TCGEN05
+    assert algo(partition_size=-1, **dict(g64, num_q_heads=128, num_kv_heads=2)) == pa.PA_ALGO_TCGEN05
+    assert algo(partition_size=0, **g64) == pa.PA_ALGO_TENSOR
+    assert algo(partition_size=-1, algo=pa.PA_ALGO_TENSOR, **g64) == pa.PA_ALGO_TENSOR
+    assert algo(partition_size=-1, **dict(g64, num_q_heads=32)) == pa.PA_ALGO_TENSOR
+    assert algo(partition_size=-1, **dict(g64, num_q_heads=16)) == pa.PA_ALGO_TENSOR
+    assert algo(partition_size=-1, **dict(g64, head_dim=64)) == pa.PA_ALGO_TENSOR
+    assert algo(partition_size=-1, **dict(g64, query_len=2)) == pa.PA_ALGO_TENSOR
+    # an unaligned q still leaves the tensor-core families
+    assert pa.lib.pa_decode_algo(ctypes.byref(params(partition_size=-1, **g64)), ctypes.c_void_p(0x1008)) == \
+        pa.PA_ALGO_SIMT
