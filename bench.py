@@ -89,6 +89,7 @@ WORKLOADS = {
     "mha_prefix": "MHA 32/32 heads, head_dim 128, fp16, batch 16, shared 1000-token prefix with "
                   "copy-on-write + private suffix U[64,1048]",
     "mqa": "MQA: 32 q heads / 1 KV head, head_dim 128, fp16, batch 128, all lengths 4096",
+    "mqa64": "MQA, groups of 64: 64 q heads / 1 KV head, head_dim 128, fp16, batch 128, all lengths 4096",
     "d256": "head_dim 256: 16 q / 8 KV heads, fp16, batch 16, all lengths 4096",
     "d256_int8": "head_dim 256: 16 q / 8 KV heads, int8 KV (per-(block, KV head) scales), fp16 q/out, "
                  "batch 16, all lengths 4096",
@@ -142,6 +143,8 @@ def make_workload(name):
         return W.mha_prefix(), False, 256
     if name == "mqa":
         return W.mqa(), False, -1
+    if name == "mqa64":
+        return W.mqa64(), False, -1
     if name == "d256":
         return W.d256(), False, -1
     if name == "d256_int8":

@@ -278,6 +278,12 @@ def mqa() -> Workload:
     return uniform("mqa", 6, 128, 4096, 32, 1, 128)
 
 
+def mqa64() -> Workload:
+    """Groups of 64: 64 query heads sharing one KV head, head_dim 128, fp16, batch 128,
+    every sequence 4096 tokens (seed 12)."""
+    return uniform("mqa64", 12, 128, 4096, 64, 1, 128)
+
+
 def d256() -> Workload:
     """head_dim 256 decode: 16 query / 8 KV heads, fp16, batch 16, every
     sequence 4096 tokens (seed 7)."""
@@ -413,7 +419,7 @@ def random_multi_case(lens, query_len, num_q_heads=4, num_kv_heads=2, head_dim=6
 
 
 NAMED = {"tiny": tiny, "gqa_b8": gqa_b8, "ragged": ragged, "long": long,
-         "mha_prefix": mha_prefix, "mqa": mqa, "d256": d256, "specdec": specdec}
+         "mha_prefix": mha_prefix, "mqa": mqa, "mqa64": mqa64, "d256": d256, "specdec": specdec}
 
 
 def decode_kv_bytes(op: Decode, w: Workload, kv_elem: float | None = None) -> int:

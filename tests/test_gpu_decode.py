@@ -525,12 +525,12 @@ def test_head_dim_256_int8_multi_query(Q):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["mqa", "d256"])
+@pytest.mark.parametrize("name", ["mqa", "mqa64", "d256"])
 def test_wide_workloads_full_size_sampled(name):
     """The benchmark's MQA and head_dim-256 workloads at full size, in the bench's
     launch configuration (library-picked partition, inputs-ready flag), against
-    the oracle on sampled (sequence, head) rows; MQA through the opt-in tcgen05
-    kernel as well."""
+    the oracle on sampled (sequence, head) rows; MQA through the tcgen05 kernel as
+    well (which the library itself picks for the groups of 64)."""
     w = W.NAMED[name]()
     B, Hq = w.steps[0][0].q.shape[:2]
     rng = np.random.default_rng(0)
